@@ -1,0 +1,399 @@
+"""Benchmark of the 4-bit MoE expert FFN on B200.
+
+Workload (default, decode_t1): one MoE layer, hidden 2048, expert FFN 512,
+128 experts top-8 plus one always-on shared expert, Q4_0 weights and Q8_0
+activations; 1000 distinct seeded tokens, each a separate T=1 call of
+moe_q4_ffn_forward, issued back to back (captured once as a CUDA graph).  One
+step = those 1000 calls.  value = tokens/s over all ranks.
+
+L2: the layer is replicated at 16 distinct device addresses (3.7 GB) and token
+i uses replica i mod 16, so the weights a token reads were last touched about
+270 MB of traffic earlier (L2 is 126 MB): every step is L2-cold for weights.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle (the reference arm of this build) on a
+bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "decode_t1"
+N_TOKENS = 1000
+REPLICAS = 16
+METRIC = "Q4_0 MoE layer tokens/s (T=1 decode, T=947 prefill); % HBM / int8-TC peak"
+
+
+def physical_cores() -> int:
+    try:
+        out = subprocess.run(["lscpu", "-p=CORE,SOCKET"], capture_output=True, text=True).stdout
+        pairs = {tuple(line.split(",")) for line in out.splitlines() if line and not line.startswith("#")}
+        if pairs:
+            return len(pairs)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def oracle_sample(x, lw, seconds=10.0):
+    """The oracle as it stands on a bounded token sample (tokens are
+    independent): probe, then size the sample to about `seconds` of work."""
+    import oracle
+    cores = oracle.set_threads(physical_cores())
+    t0 = time.perf_counter()
+    oracle.moe_forward(lw, x[:16])
+    rate = 16 / (time.perf_counter() - t0)
+    n = int(min(max(16, rate * seconds), 8000))
+    idx = np.arange(n) % x.shape[0]
+    xs = np.ascontiguousarray(x[idx])
+    t0 = time.perf_counter()
+    oracle.moe_forward(lw, xs)
+    dt = time.perf_counter() - t0
+    return n / dt, n, dt, cores
+
+
+def rank_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def run_reference(args):
+    rank, world, _ = rank_env()
+    if rank != 0:
+        return 0
+    import synth
+    x, lw = synth.workload_inputs(WORKLOAD, seed=0, T=N_TOKENS)
+    for _ in range(args.warmup):
+        oracle_sample(x, lw, seconds=1.0)
+    vals, total_tokens, total_s = [], 0, 0.0
+    for _ in range(args.steps):
+        v, n, dt, cores = oracle_sample(x, lw, seconds=max(1.0, 60.0 / max(1, args.steps)))
+        vals.append(v)
+        total_tokens += n
+        total_s += dt
+    value = total_tokens / total_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "tokens_per_step": N_TOKENS},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{total_tokens} tokens of the {N_TOKENS}-token decode workload over "
+                                   f"{args.steps} steps, OpenMP over tokens on {cores} physical cores "
+                                   f"({cpu_model()})"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            p = [s.strip() for s in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx.append(float(p[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def graph_kernel_nodes(graph) -> int:
+    """Kernel nodes in a captured torch CUDA graph (cudaGraphNodeTypeKernel == 0)."""
+    import torch
+    lib = None
+    for cand in ("libcudart.so.12", "libcudart.so"):
+        try:
+            lib = ctypes.CDLL(cand)
+            break
+        except OSError:
+            continue
+    if lib is None:
+        import glob
+        for c in glob.glob(os.path.join(os.path.dirname(torch.__file__), "..", "nvidia", "cuda_runtime", "lib",
+                                        "libcudart.so*")):
+            lib = ctypes.CDLL(c)
+            break
+    g = ctypes.c_void_p(graph.raw_cuda_graph())
+    n = ctypes.c_size_t(0)
+    assert lib.cudaGraphGetNodes(g, None, ctypes.byref(n)) == 0
+    nodes = (ctypes.c_void_p * n.value)()
+    assert lib.cudaGraphGetNodes(g, nodes, ctypes.byref(n)) == 0
+    kernels = 0
+    for i in range(n.value):
+        t = ctypes.c_int(-1)
+        assert lib.cudaGraphNodeGetType(ctypes.c_void_p(nodes[i]), ctypes.byref(t)) == 0
+        kernels += int(t.value == 0)
+    return kernels
+
+
+def source_digest(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str):
+    """dram bytes per launch from the committed ncu summary, if the kernel's
+    source has not changed since it was captured (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(kernel)
+    if not rec:
+        return None
+    if source_digest(rec["sources"]) != rec["digest"]:
+        return None
+    return rec["bytes_per_launch"]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = rank_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    import quantized_moe_q4_b200 as m
+    import synth
+
+    x_np, lw = synth.workload_inputs(WORKLOAD, seed=0, T=N_TOKENS)
+    base = m.Layer.from_host(lw)
+    layers = [base] + [base.replica() for _ in range(REPLICAS - 1)]
+    H, F, E, k = lw.hidden, lw.ffn, lw.n_experts, lw.top_k
+    x = torch.from_numpy(x_np).cuda()
+    y = torch.empty_like(x)
+    ws = m.alloc_workspace(m.moe_q4_ffn_workspace_bytes(base, 1))
+    stream = torch.cuda.Stream()
+    # every launch, graph replay and event of the run goes to this one stream
+    # (CUDAGraph.replay launches on the current stream)
+    torch.cuda.set_stream(stream)
+
+    def step_calls(path=m.PATH_AUTO, events=None):
+        for i in range(N_TOKENS):
+            L = layers[i % REPLICAS]
+            if events is None and path == m.PATH_AUTO:
+                m.moe_q4_ffn_forward(L, x[i:i + 1], y[i:i + 1], ws, stream=stream)
+            else:
+                e0, e1 = events[i] if events else (None, None)
+                m.moe_q4_ffn_forward_debug(L, x[i:i + 1], y[i:i + 1], ws, path=path, ev_start=e0, ev_stop=e1,
+                                           stream=stream)
+
+    # eager run once (also checks the calls succeed), then capture
+    with torch.cuda.stream(stream):
+        step_calls()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.graph(graph, stream=stream):
+        step_calls()
+    graph.instantiate()
+    kernels_per_step = graph_kernel_nodes(graph)
+
+    for _ in range(max(3, args.warmup)):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    clk = clocks.stop()
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * N_TOKENS * args.steps / (ms / 1000.0)
+
+    # dominant kernel (gate/up projection) timed live with events around each launch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(N_TOKENS)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:  # torch creates the CUDA event on first record
+            a.record(stream)
+            b.record(stream)
+    torch.cuda.synchronize()
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=stream):
+        step_calls(events=evs)
+    for _ in range(2):
+        g2.replay()
+    torch.cuda.synchronize()
+    dom_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    del g2
+
+    # algorithmic bytes of one gate/up launch at T=1: the weights of the k routed
+    # experts and the shared expert (gate and up), the token's Q8_0 row, the
+    # requantised output rows
+    nb, nbF = H // 32, F // 32
+    experts = k + 1
+    gu_bytes = experts * 2 * F * nb * 18 + (H + 2 * nb) + experts * (F + 2 * nbF)
+    peak, peak_src = measured_peaks()
+    achieved = gu_bytes / (dom_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": committed_traffic("gateup"), "kernel": "gate/up projection (T=1)",
+                "algorithmic_bytes_per_launch": gu_bytes, "avg_launch_us": dom_ms * 1e3,
+                "peak_source": f"{peak_src} hbm_gbs"}
+    # whole token against the roofline too
+    tok_bytes = experts * 3 * F * nb * 18 + E * H * 4 + H * 4 * 2
+    tok_frac = (tok_bytes * value / world) / 1e9 / peak
+
+    # end to end through the host entry point: per token H2D copy of x, forward,
+    # D2H copy of y, all captured once and replayed; pinned host buffers
+    xh = torch.from_numpy(x_np).pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    wsh = m.alloc_workspace(m.moe_q4_ffn_host_workspace_bytes(base, 1))
+    g3 = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        for i in range(N_TOKENS):
+            m.moe_q4_ffn_forward_host(layers[i % REPLICAS], xh[i:i + 1], yh[i:i + 1], wsh, stream=stream)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g3, stream=stream):
+        for i in range(N_TOKENS):
+            m.moe_q4_ffn_forward_host(layers[i % REPLICAS], xh[i:i + 1], yh[i:i + 1], wsh, stream=stream)
+    for _ in range(3):
+        g3.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        g3.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * N_TOKENS * args.steps / (e2e_ms / 1000.0)
+    del g3
+
+    cpu = None
+    if rank == 0 and world == 1:
+        v, n, dt, cores = oracle_sample(x_np, lw, seconds=10.0)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} tokens of the decode workload (T=1 each, independent), {dt:.1f} s, "
+                         f"OpenMP over tokens on {cores} physical cores ({cpu_model()})"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens_per_step": N_TOKENS, "T_per_call": 1, "hidden": H, "ffn": F,
+                   "experts": E, "top_k": k, "shared_expert": True, "weights": "Q4_0", "activations": "Q8_0",
+                   "l2": f"weights rotate over {REPLICAS} replicas ({REPLICAS * 228} MB) -> L2-cold",
+                   "parallelism": f"replicas x{world} (tokens independent, no collective)",
+                   "graph": "1000 calls captured as one CUDA graph"},
+        "roofline": roofline,
+        "token_hbm_frac": tok_frac,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": N_TOKENS * H * 4,
+                "d2h_bytes_per_step": N_TOKENS * H * 4, "how": "moe_q4_ffn_forward_host per token (pinned "
+                                                              "host x/y), graph-captured"},
+        "gpu_launches": kernels_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,190 @@
+/*
+ * moe_q4.h -- C ABI of the B200 (sm_100a) 4-bit Mixture-of-Experts expert FFN.
+ *
+ * The layer computed here is the MoE part of the model in "A 35B
+ * Hybrid-Attention Mixture-of-Experts Model on a 6GB 2011 GPU: Hand-Written
+ * 4-bit CUDA Inference for Fermi" (Dutch technical summary,
+ * gist.science/nl/paper/2606.24031):
+ *   - Methodologie 1: the prefill runs a grouped 4-bit GEMM over the routed
+ *     experts; the decode runs a W4A8 integer kernel (4-bit weights, 8-bit
+ *     activations, integer multiply-adds).
+ *   - Methodologie 2: weights are group-wise symmetric 4-bit (Q4_0 family),
+ *     activations 8-bit, 128 experts per layer after pruning.
+ *   - Methodologie 4: the whole prompt in one pass, so each expert's GEMM
+ *     sees all of its tokens at once.
+ *
+ * Formats (the readings of the "Q4_0 family" and "8-bit activations"):
+ *   Q4_0 block = 18 bytes: binary16 scale d (little endian), then qs[16];
+ *     weight i<16 = low nibble of qs[i], weight i+16 = high nibble;
+ *     value = (nibble - 8) * d.
+ *   Q8_0 block = 32 int8 q plus a binary16 scale: d = amax/127 (binary32
+ *     division), q = round-half-away-from-zero(x/d) (binary32 division),
+ *     stored scale = binary16(d), nearest-even; all-zero block -> d = 0, q = 0.
+ *
+ * Layer: y[t] = sum_j w[t,j] * FFN_{idx[t,j]}(x[t]) + FFN_shared(x[t]), where
+ *   logits = x.Wr^T (+ bias), idx = top-k (descending, ties to the lower
+ *   expert index), w = softmax over the k chosen logits, and
+ *   FFN_e(x) = Wd_e . Q8_0( silu(Wg_e . Q8_0(x)) * (Wu_e . Q8_0(x)) ).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers (except the *_host entry),
+ *     row-major, owned by the caller.  The library never allocates, frees or
+ *     synchronises; all work is enqueued on `stream` (NULL = legacy default
+ *     stream) and faults surface at the caller's next synchronisation.
+ *   - Pointers must be 16-byte aligned, workspaces 256-byte aligned.
+ *   - hidden and ffn must be positive multiples of 256; 1 <= top_k <=
+ *     min(n_experts, 16); 1 <= n_experts <= 256; 0 <= T <= 2^24.  T == 0 is
+ *     a no-op that returns MOE_Q4_OK.
+ *   - Inputs must be finite.  A binary16 scale that overflows (block amax >
+ *     65504*127) is reported in the device status word, never by a trap.
+ *   - The device must be compute capability 10.0 (B200, sm_100a).
+ *   - Return value: MOE_Q4_OK (0) or a negative MOE_Q4_ERR_* code; nothing is
+ *     enqueued when an argument check fails.
+ */
+#ifndef MOE_Q4_H
+#define MOE_Q4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_q4_stream_t; /* a cudaStream_t */
+
+enum {
+    MOE_Q4_OK = 0,
+    MOE_Q4_ERR_INVALID_ARG = -1, /* null pointer, T < 0 or too large, bad k/E */
+    MOE_Q4_ERR_SHAPE = -2,       /* hidden or ffn not a positive multiple of 256 */
+    MOE_Q4_ERR_ALIGN = -3,       /* pointer not 16-byte (workspace: 256-byte) aligned */
+    MOE_Q4_ERR_WORKSPACE = -4,   /* workspace smaller than moe_q4_ffn_workspace_bytes() */
+    MOE_Q4_ERR_ARCH = -5,        /* current device is not compute capability 10.0 */
+    MOE_Q4_ERR_CUDA = -6,        /* a CUDA runtime call or kernel launch failed */
+    MOE_Q4_ERR_OVERLAP = -7      /* output buffer overlaps an input */
+};
+
+/* Bits of the device status word (first uint32 of a workspace, or the
+ * optional `status` argument): set with atomicOr, never cleared by the
+ * library except at the start of moe_q4_ffn_forward. */
+#define MOE_Q4_STATUS_SCALE_OVERFLOW 0x1u /* a binary16 Q8_0 scale overflowed */
+#define MOE_Q4_STATUS_SPIN_TIMEOUT 0x2u   /* a bounded device-side wait gave up */
+
+/* One MoE layer.  Expert e's matrices are consecutive Q4_0 blocks:
+ *   w_gate, w_up : [n_experts][ffn][hidden/32] blocks (18 B each)
+ *   w_down       : [n_experts][hidden][ffn/32] blocks
+ *   sh_*         : the always-on shared expert, same layout with one expert;
+ *                  all three NULL iff has_shared == 0.
+ *   w_router     : [n_experts][hidden] fp32;  router_bias: [n_experts] or NULL. */
+typedef struct {
+    int32_t hidden, ffn, n_experts, top_k, has_shared;
+    const float* w_router;
+    const float* router_bias;
+    const uint8_t* w_gate;
+    const uint8_t* w_up;
+    const uint8_t* w_down;
+    const uint8_t* sh_gate;
+    const uint8_t* sh_up;
+    const uint8_t* sh_down;
+} moe_q4_layer;
+
+/* Q8_0 activation quantisation (Methodologie 1 and 2: the 8-bit activations
+ * of the W4A8 kernel).  x [T][H] fp32 -> q [T][H] int8 and d [T][H/32]
+ * binary16 bits.  `status` (device uint32, may be NULL) receives
+ * MOE_Q4_STATUS_SCALE_OVERFLOW.  H must be a positive multiple of 32. */
+int moe_q4_quantize_act(const float* x, int64_t T, int32_t H, int8_t* q, uint16_t* d,
+                        uint32_t* status, moe_q4_stream_t stream);
+
+/* Router (Methodologie 1: "MoE-routing" of the grouped GEMM): logits [T][E]
+ * fp32 = x.Wr^T (+ bias), then per token the top-k experts (descending logit,
+ * ties to the lower index) into topk_idx [T][k] int32 and their softmax
+ * weights into topk_w [T][k] fp32.  `logits` is a caller buffer that
+ * receives the logits (required). */
+int moe_q4_route(const moe_q4_layer* L, const float* x, int64_t T, int32_t* topk_idx,
+                 float* topk_w, float* logits, moe_q4_stream_t stream);
+
+/* Bytes of device workspace moe_q4_ffn_forward needs for up to T_max tokens
+ * (0 on invalid arguments). */
+size_t moe_q4_ffn_workspace_bytes(const moe_q4_layer* L, int64_t T_max);
+
+/* The whole MoE expert FFN layer (Methodologie 1: grouped 4-bit GEMM for
+ * prefill, W4A8 kernel for decode; Methodologie 4: all T tokens in one pass).
+ * x [T][H] fp32 in, y [T][H] fp32 out (overwritten; must not overlap x or the
+ * workspace).  The workspace must hold moe_q4_ffn_workspace_bytes(L, T) bytes;
+ * its first uint32 is the device status word (cleared by this call).
+ * Kernel choice by T is internal; results do not depend on it beyond fp32
+ * summation order. */
+int moe_q4_ffn_forward(const moe_q4_layer* L, const float* x, int64_t T, float* y,
+                       void* workspace, size_t ws_bytes, moe_q4_stream_t stream);
+
+/* Bytes of device workspace moe_q4_ffn_forward_host needs: the forward's
+ * workspace plus device staging for x and y. */
+size_t moe_q4_ffn_host_workspace_bytes(const moe_q4_layer* L, int64_t T_max);
+
+/* moe_q4_ffn_forward with x and y in HOST memory (pinned for asynchronous
+ * copies): enqueues the host-to-device copy of x, the forward, and the
+ * device-to-host copy of y on `stream`.  y is valid after the caller
+ * synchronises the stream. */
+int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t T, float* y_host,
+                            void* workspace, size_t ws_bytes, moe_q4_stream_t stream);
+
+/* Static description of an error code. */
+const char* moe_q4_status_string(int status);
+
+/* ---------------------------------------------------------------------
+ * Inspection entry points used by the parity tests.
+ * --------------------------------------------------------------------- */
+
+/* Byte offsets, inside a forward workspace sized for T tokens, of the
+ * intermediate arrays, in this order (MOE_Q4_WS_* indices):
+ *   status u32[4] | logits f32[T][E] | topk_idx i32[T][k] | topk_w f32[T][k]
+ *   | qa i8[T][H] | da u16[T][H/32] | cnt i32[E+1] | off i32[E+2]
+ *   | tile_off i32[E+2] | chunk_cnt i32[C][E] | chunk_base i32[C][E]
+ *   | sorted i32[P] | pos i32[P] | hq i8[P+S*T][F] | dh u16[P+S*T][F/32]
+ *   | total
+ * with P = T*k routed pairs and S = has_shared.  Slots (rows of hq/dh) are
+ * grouped by expert: routed expert e owns slots off[e]..off[e+1]-1 holding
+ * pairs sorted[...] = t*k+j in increasing (t, j) order; the shared expert
+ * owns slots P..P+T-1 (slot P+t = token t).  pos is the inverse of sorted.
+ * Fills n <= MOE_Q4_WS_COUNT entries of `offsets`; returns MOE_Q4_OK or an
+ * error code. */
+enum {
+    MOE_Q4_WS_STATUS = 0, MOE_Q4_WS_LOGITS, MOE_Q4_WS_TOPK_IDX, MOE_Q4_WS_TOPK_W, MOE_Q4_WS_QA,
+    MOE_Q4_WS_DA, MOE_Q4_WS_CNT, MOE_Q4_WS_OFF, MOE_Q4_WS_TILE_OFF, MOE_Q4_WS_CHUNK_CNT,
+    MOE_Q4_WS_CHUNK_BASE, MOE_Q4_WS_SORTED, MOE_Q4_WS_POS, MOE_Q4_WS_HQ, MOE_Q4_WS_DH,
+    MOE_Q4_WS_TOTAL, MOE_Q4_WS_COUNT
+};
+int moe_q4_workspace_layout(const moe_q4_layer* L, int64_t T, size_t* offsets, int n);
+
+/* Kernel family selectors for moe_q4_ffn_forward_debug. */
+enum {
+    MOE_Q4_PATH_AUTO = 0,     /* what moe_q4_ffn_forward does */
+    MOE_Q4_PATH_GROUPED_DP4A = 1,
+    MOE_Q4_PATH_DECODE = 2,
+    MOE_Q4_PATH_TENSOR_CORE = 3
+};
+
+typedef struct {
+    float* h_out;     /* [P+S*T][F] fp32 SwiGLU output before requantisation, slot order; or NULL */
+    int32_t path;     /* MOE_Q4_PATH_* */
+    void* ev_start;   /* cudaEvent_t recorded just before the dominant (gate/up) kernel, or NULL */
+    void* ev_stop;    /* cudaEvent_t recorded just after it, or NULL */
+} moe_q4_debug;
+
+/* moe_q4_ffn_forward with inspection options (see moe_q4_debug). */
+int moe_q4_ffn_forward_debug(const moe_q4_layer* L, const float* x, int64_t T, float* y,
+                             void* workspace, size_t ws_bytes, const moe_q4_debug* dbg,
+                             moe_q4_stream_t stream);
+
+/* Per-block W4A8 integer dot products through the device routine every
+ * projection kernel uses: out[i] = sum_{j<32} (nibble_j(w[i]) - 8) * qa[32*i+j]
+ * for n Q4_0 blocks w (18 B each, consecutive; n a multiple of 8) and n*32 int8
+ * activations. */
+int moe_q4_block_dots(const uint8_t* w_blocks, const int8_t* qa, int64_t n, int32_t* out,
+                      moe_q4_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_Q4_H */

@@ -1,0 +1,256 @@
+"""Python binding of the B200 4-bit MoE expert FFN library (libmoe_q4.so).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels (sm_100a).  PyTorch provides device memory and streams.  The function
+names are the C ABI's (include/moe_q4.h).  Importing this module fails loudly
+if the CUDA library has not been built; there is no fallback.
+
+The layer is the MoE expert FFN of "A 35B Hybrid-Attention Mixture-of-Experts
+Model on a 6GB 2011 GPU: Hand-Written 4-bit CUDA Inference for Fermi" (Dutch
+technical summary, Methodologie 1 and 2): top-k routing, Q8_0 activations,
+grouped W4A8 gate/up and down projections over Q4_0 expert weights, SwiGLU,
+and the router-weighted combine.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_q4.so")
+
+QK = 32
+Q4_BYTES = 18
+
+MOE_Q4_OK = 0
+ERRORS = {
+    -1: "MOE_Q4_ERR_INVALID_ARG", -2: "MOE_Q4_ERR_SHAPE", -3: "MOE_Q4_ERR_ALIGN",
+    -4: "MOE_Q4_ERR_WORKSPACE", -5: "MOE_Q4_ERR_ARCH", -6: "MOE_Q4_ERR_CUDA", -7: "MOE_Q4_ERR_OVERLAP",
+}
+STATUS_SCALE_OVERFLOW = 0x1
+STATUS_SPIN_TIMEOUT = 0x2
+
+PATH_AUTO, PATH_GROUPED_DP4A, PATH_DECODE, PATH_TENSOR_CORE = 0, 1, 2, 3
+
+WS_NAMES = ["status", "logits", "topk_idx", "topk_w", "qa", "da", "cnt", "off", "tile_off",
+            "chunk_cnt", "chunk_base", "sorted", "pos", "hq", "dh", "total"]
+
+# Every extern "C" symbol of include/moe_q4.h.
+EXPORTS = ["moe_q4_quantize_act", "moe_q4_route", "moe_q4_ffn_workspace_bytes", "moe_q4_ffn_forward",
+           "moe_q4_ffn_host_workspace_bytes", "moe_q4_ffn_forward_host", "moe_q4_status_string",
+           "moe_q4_workspace_layout", "moe_q4_ffn_forward_debug", "moe_q4_block_dots"]
+
+
+class MoeQ4Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {ERRORS.get(code, code)} ({moe_q4_status_string(code)})")
+
+
+class _Layer(ctypes.Structure):
+    _fields_ = [
+        ("hidden", ctypes.c_int32), ("ffn", ctypes.c_int32), ("n_experts", ctypes.c_int32),
+        ("top_k", ctypes.c_int32), ("has_shared", ctypes.c_int32),
+        ("w_router", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
+        ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
+        ("sh_gate", ctypes.c_void_p), ("sh_up", ctypes.c_void_p), ("sh_down", ctypes.c_void_p),
+    ]
+
+
+class _Debug(ctypes.Structure):
+    _fields_ = [("h_out", ctypes.c_void_p), ("path", ctypes.c_int32),
+                ("ev_start", ctypes.c_void_p), ("ev_stop", ctypes.c_void_p)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build the CUDA library first "
+            "(python -m quantized_moe_q4_b200.build, or __graft_entry__.build()). There is no CPU fallback.")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    sigs = {
+        "moe_q4_quantize_act": ([P, i64, i32, P, P, P, P], ctypes.c_int),
+        "moe_q4_route": ([P, P, i64, P, P, P, P], ctypes.c_int),
+        "moe_q4_ffn_workspace_bytes": ([P, i64], sz),
+        "moe_q4_ffn_forward": ([P, P, i64, P, P, sz, P], ctypes.c_int),
+        "moe_q4_ffn_host_workspace_bytes": ([P, i64], sz),
+        "moe_q4_ffn_forward_host": ([P, P, i64, P, P, sz, P], ctypes.c_int),
+        "moe_q4_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "moe_q4_workspace_layout": ([P, i64, P, ctypes.c_int], ctypes.c_int),
+        "moe_q4_ffn_forward_debug": ([P, P, i64, P, P, sz, P, P], ctypes.c_int),
+        "moe_q4_block_dots": ([P, P, i64, P, P], ctypes.c_int),
+    }
+    for name, (args, res) in sigs.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(rc: int, what: str):
+    if rc != MOE_Q4_OK:
+        raise MoeQ4Error(rc, what)
+
+
+def moe_q4_status_string(code: int) -> str:
+    return _lib.moe_q4_status_string(int(code)).decode()
+
+
+class Layer:
+    """One MoE layer's weights on the device and its C descriptor.
+
+    w_router [E,H] fp32, router_bias [E] fp32 or None, w_gate/w_up [E,F,H/32,18]
+    uint8, w_down [E,H,F/32,18] uint8, sh_* the shared expert or None."""
+
+    def __init__(self, hidden, ffn, n_experts, top_k, w_router, router_bias, w_gate, w_up, w_down,
+                 sh_gate=None, sh_up=None, sh_down=None):
+        self.hidden, self.ffn, self.n_experts, self.top_k = int(hidden), int(ffn), int(n_experts), int(top_k)
+        self.tensors = dict(w_router=w_router, router_bias=router_bias, w_gate=w_gate, w_up=w_up,
+                            w_down=w_down, sh_gate=sh_gate, sh_up=sh_up, sh_down=sh_down)
+        for k, v in self.tensors.items():
+            if v is not None and not v.is_contiguous():
+                raise ValueError(f"{k} must be contiguous")
+        self.has_shared = sh_gate is not None
+        self.struct = _Layer(self.hidden, self.ffn, self.n_experts, self.top_k, int(self.has_shared),
+                             *(None if v is None else v.data_ptr() for v in self.tensors.values()))
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+    @classmethod
+    def from_host(cls, w, device="cuda"):
+        """From an object with numpy attributes (hidden, ffn, n_experts, top_k,
+        w_router, router_bias, w_gate, w_up, w_down, sh_gate, sh_up, sh_down)."""
+        def dev(a):
+            return None if a is None else torch.from_numpy(a).to(device).contiguous()
+        return cls(w.hidden, w.ffn, w.n_experts, w.top_k, dev(w.w_router), dev(w.router_bias),
+                   dev(w.w_gate), dev(w.w_up), dev(w.w_down), dev(w.sh_gate), dev(w.sh_up), dev(w.sh_down))
+
+    def replica(self):
+        """A copy of every weight tensor at new device addresses."""
+        t = {k: (None if v is None else v.clone()) for k, v in self.tensors.items()}
+        return Layer(self.hidden, self.ffn, self.n_experts, self.top_k, **t)
+
+
+def moe_q4_quantize_act(x: torch.Tensor, q=None, d=None, status=None, stream=None):
+    T, H = x.shape
+    q = torch.empty((T, H), dtype=torch.int8, device=x.device) if q is None else q
+    d = torch.empty((T, H // QK), dtype=torch.int16, device=x.device) if d is None else d
+    _check(_lib.moe_q4_quantize_act(_p(x), T, H, _p(q), _p(d), _p(status), _stream(stream)), "moe_q4_quantize_act")
+    return q, d
+
+
+def moe_q4_route(layer: Layer, x: torch.Tensor, topk_idx=None, topk_w=None, logits=None, stream=None):
+    T = x.shape[0]
+    k, E = layer.top_k, layer.n_experts
+    topk_idx = torch.empty((T, k), dtype=torch.int32, device=x.device) if topk_idx is None else topk_idx
+    topk_w = torch.empty((T, k), dtype=torch.float32, device=x.device) if topk_w is None else topk_w
+    logits = torch.empty((T, E), dtype=torch.float32, device=x.device) if logits is None else logits
+    _check(_lib.moe_q4_route(layer.ref, _p(x), T, _p(topk_idx), _p(topk_w), _p(logits), _stream(stream)),
+           "moe_q4_route")
+    return topk_idx, topk_w, logits
+
+
+def moe_q4_ffn_workspace_bytes(layer: Layer, T_max: int) -> int:
+    return int(_lib.moe_q4_ffn_workspace_bytes(layer.ref, int(T_max)))
+
+
+def moe_q4_ffn_host_workspace_bytes(layer: Layer, T_max: int) -> int:
+    return int(_lib.moe_q4_ffn_host_workspace_bytes(layer.ref, int(T_max)))
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A 256-byte aligned uint8 device buffer (torch's allocator aligns to 512)."""
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    assert ws.data_ptr() % 256 == 0
+    return ws
+
+
+def moe_q4_ffn_forward(layer: Layer, x: torch.Tensor, y=None, workspace=None, stream=None):
+    T = x.shape[0]
+    y = torch.empty_like(x) if y is None else y
+    if workspace is None:
+        workspace = alloc_workspace(moe_q4_ffn_workspace_bytes(layer, T), x.device)
+    _check(_lib.moe_q4_ffn_forward(layer.ref, _p(x), T, _p(y), _p(workspace), workspace.numel(),
+                                   _stream(stream)), "moe_q4_ffn_forward")
+    return y
+
+
+def moe_q4_ffn_forward_debug(layer: Layer, x: torch.Tensor, y, workspace, h_out=None, path=PATH_AUTO,
+                             ev_start=None, ev_stop=None, stream=None):
+    T = x.shape[0]
+    dbg = _Debug(None if h_out is None else h_out.data_ptr(), int(path),
+                 None if ev_start is None else ev_start.cuda_event,
+                 None if ev_stop is None else ev_stop.cuda_event)
+    _check(_lib.moe_q4_ffn_forward_debug(layer.ref, _p(x), T, _p(y), _p(workspace), workspace.numel(),
+                                         ctypes.byref(dbg), _stream(stream)), "moe_q4_ffn_forward_debug")
+    return y
+
+
+def moe_q4_ffn_forward_host(layer: Layer, x_host: torch.Tensor, y_host: torch.Tensor, workspace, stream=None):
+    """x_host/y_host: CPU tensors (pinned for asynchronous copies)."""
+    T = x_host.shape[0]
+    _check(_lib.moe_q4_ffn_forward_host(layer.ref, _p(x_host), T, _p(y_host), _p(workspace), workspace.numel(),
+                                        _stream(stream)), "moe_q4_ffn_forward_host")
+    return y_host
+
+
+def moe_q4_workspace_layout(layer: Layer, T: int) -> dict:
+    arr = (ctypes.c_size_t * len(WS_NAMES))()
+    _check(_lib.moe_q4_workspace_layout(layer.ref, int(T), arr, len(WS_NAMES)), "moe_q4_workspace_layout")
+    return dict(zip(WS_NAMES, list(arr)))
+
+
+def workspace_views(layer: Layer, T: int, ws: torch.Tensor) -> dict:
+    """Typed views of the intermediates inside a forward workspace (for tests)."""
+    off = moe_q4_workspace_layout(layer, T)
+    E, k, H, F = layer.n_experts, layer.top_k, layer.hidden, layer.ffn
+    P = T * k
+    slots = P + (T if layer.has_shared else 0)
+
+    def v(name, dtype, shape):
+        n = 1
+        for s in shape:
+            n *= s
+        nbytes = n * torch.tensor([], dtype=dtype).element_size()
+        return ws[off[name]:off[name] + nbytes].view(dtype).view(*shape)
+
+    return dict(
+        status=v("status", torch.int32, (4,)), logits=v("logits", torch.float32, (T, E)),
+        topk_idx=v("topk_idx", torch.int32, (T, k)), topk_w=v("topk_w", torch.float32, (T, k)),
+        qa=v("qa", torch.int8, (T, H)), da=v("da", torch.int16, (T, H // QK)),
+        cnt=v("cnt", torch.int32, (E + 1,)), off=v("off", torch.int32, (E + 2,)),
+        tile_off=v("tile_off", torch.int32, (E + 2,)), sorted=v("sorted", torch.int32, (P,)),
+        pos=v("pos", torch.int32, (P,)), hq=v("hq", torch.int8, (slots, F)),
+        dh=v("dh", torch.int16, (slots, F // QK)))
+
+
+def moe_q4_block_dots(w_blocks: torch.Tensor, qa: torch.Tensor, out=None, stream=None):
+    n = w_blocks.numel() // Q4_BYTES
+    out = torch.empty(n, dtype=torch.int32, device=w_blocks.device) if out is None else out
+    _check(_lib.moe_q4_block_dots(_p(w_blocks), _p(qa), n, _p(out), _stream(stream)), "moe_q4_block_dots")
+    return out

@@ -1,0 +1,336 @@
+// abi.cu -- the extern "C" entry points of include/moe_q4.h: argument checks,
+// workspace layout, kernel-family dispatch.  No allocation, no host sync.
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe_q4.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace moeq4 {
+
+static constexpr int64_t T_LIMIT = int64_t(1) << 24;
+static constexpr int MAX_DEVICES = 64;
+
+struct DeviceState {
+    int checked;  // 0 unknown, 1 ok, -1 wrong arch
+    DeviceInfo info;
+};
+static DeviceState g_dev[MAX_DEVICES];
+
+static int current_device(DeviceInfo* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return MOE_Q4_ERR_CUDA;
+    DeviceState& st = g_dev[dev];
+    if (st.checked == 0) {
+        int major = 0, minor = 0, sms = 0, smem = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return MOE_Q4_ERR_CUDA;
+        st.info.sm_count = sms;
+        st.info.max_smem_optin = smem;
+        st.checked = (major == 10 && minor == 0) ? 1 : -1;
+    }
+    if (st.checked < 0) return MOE_Q4_ERR_ARCH;
+    *out = st.info;
+    return MOE_Q4_OK;
+}
+
+struct OccEntry {
+    int dev;
+    const void* kernel;
+    int threads;
+    size_t smem;
+    int per_sm;
+};
+static OccEntry g_occ[256];
+static int g_occ_n = 0;
+static std::mutex g_occ_mu;
+
+cudaError_t kernel_occupancy(const void* kernel, int threads, size_t smem, int* per_sm) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(g_occ_mu);
+    for (int i = 0; i < g_occ_n; ++i) {
+        const OccEntry& o = g_occ[i];
+        if (o.dev == dev && o.kernel == kernel && o.threads == threads && o.smem == smem) {
+            *per_sm = o.per_sm;
+            return cudaSuccess;
+        }
+    }
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem);
+    if (e != cudaSuccess) return e;
+    if (n < 1) n = 1;
+    if (g_occ_n < 256) g_occ[g_occ_n++] = OccEntry{dev, kernel, threads, smem, n};
+    *per_sm = n;
+    return cudaSuccess;
+}
+
+cudaError_t record_event(cudaEvent_t ev, cudaStream_t s) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &st);
+    if (e != cudaSuccess) return e;
+    if (st == cudaStreamCaptureStatusActive) return cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+    return cudaEventRecord(ev, s);
+}
+
+static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+static bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return na && nb && x < y + nb && y < x + na;
+}
+
+static int check_layer(const moe_q4_layer* L) {
+    if (!L) return MOE_Q4_ERR_INVALID_ARG;
+    if (L->n_experts < 1 || L->n_experts > 256 || L->top_k < 1 || L->top_k > 16 || L->top_k > L->n_experts)
+        return MOE_Q4_ERR_INVALID_ARG;
+    if (L->has_shared != 0 && L->has_shared != 1) return MOE_Q4_ERR_INVALID_ARG;
+    if (!L->w_router || !L->w_gate || !L->w_up || !L->w_down) return MOE_Q4_ERR_INVALID_ARG;
+    const bool sh = L->sh_gate || L->sh_up || L->sh_down;
+    if (L->has_shared && !(L->sh_gate && L->sh_up && L->sh_down)) return MOE_Q4_ERR_INVALID_ARG;
+    if (!L->has_shared && sh) return MOE_Q4_ERR_INVALID_ARG;
+    if (L->hidden <= 0 || L->ffn <= 0 || L->hidden % 256 || L->ffn % 256 || L->hidden > 16384 || L->ffn > 16384)
+        return MOE_Q4_ERR_SHAPE;
+    const void* ptrs[] = {L->w_router, L->w_gate, L->w_up, L->w_down, L->sh_gate, L->sh_up, L->sh_down};
+    for (const void* q : ptrs)
+        if (q && !aligned(q, 16)) return MOE_Q4_ERR_ALIGN;
+    if (L->router_bias && !aligned(L->router_bias, 4)) return MOE_Q4_ERR_ALIGN;
+    return MOE_Q4_OK;
+}
+
+static LayerView view(const moe_q4_layer* L) {
+    LayerView v;
+    v.H = L->hidden; v.F = L->ffn; v.E = L->n_experts; v.k = L->top_k; v.S = L->has_shared;
+    v.w_router = L->w_router; v.router_bias = L->router_bias;
+    v.w_gate = L->w_gate; v.w_up = L->w_up; v.w_down = L->w_down;
+    v.sh_gate = L->sh_gate; v.sh_up = L->sh_up; v.sh_down = L->sh_down;
+    return v;
+}
+
+static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+static void layout(const LayerView& L, int64_t T, size_t off[WS_COUNT]) {
+    const int64_t P = T * L.k;
+    const int64_t slots = P + (L.S ? T : 0);
+    const int64_t C = ceil_div(P, PERM_CHUNK);
+    const size_t sz[WS_COUNT - 1] = {
+        16,                                            // status
+        sizeof(float) * (size_t)(T * L.E),             // logits
+        sizeof(int32_t) * (size_t)P,                   // topk_idx
+        sizeof(float) * (size_t)P,                     // topk_w
+        (size_t)(T * L.H),                             // qa
+        sizeof(uint16_t) * (size_t)(T * (L.H / QK)),   // da
+        sizeof(int32_t) * (size_t)(L.E + 1),           // cnt
+        sizeof(int32_t) * (size_t)(L.E + 2),           // off
+        sizeof(int32_t) * (size_t)(L.E + 2),           // tile_off
+        sizeof(int32_t) * (size_t)(C * L.E),           // chunk_cnt
+        sizeof(int32_t) * (size_t)(C * L.E),           // chunk_base
+        sizeof(int32_t) * (size_t)P,                   // sorted
+        sizeof(int32_t) * (size_t)P,                   // pos
+        (size_t)(slots * L.F),                         // hq
+        sizeof(uint16_t) * (size_t)(slots * (L.F / QK)),  // dh
+    };
+    size_t o = 0;
+    for (int i = 0; i < WS_COUNT - 1; ++i) {
+        off[i] = o;
+        o += align256(sz[i]);
+    }
+    off[WS_TOTAL] = o;
+}
+
+static Workspace carve(void* base, const size_t off[WS_COUNT]) {
+    char* b = static_cast<char*>(base);
+    Workspace w;
+    w.status = reinterpret_cast<uint32_t*>(b + off[WS_STATUS]);
+    w.logits = reinterpret_cast<float*>(b + off[WS_LOGITS]);
+    w.topk_idx = reinterpret_cast<int32_t*>(b + off[WS_TOPK_IDX]);
+    w.topk_w = reinterpret_cast<float*>(b + off[WS_TOPK_W]);
+    w.qa = reinterpret_cast<int8_t*>(b + off[WS_QA]);
+    w.da = reinterpret_cast<uint16_t*>(b + off[WS_DA]);
+    w.cnt = reinterpret_cast<int32_t*>(b + off[WS_CNT]);
+    w.off = reinterpret_cast<int32_t*>(b + off[WS_OFF]);
+    w.tile_off = reinterpret_cast<int32_t*>(b + off[WS_TILE_OFF]);
+    w.chunk_cnt = reinterpret_cast<int32_t*>(b + off[WS_CHUNK_CNT]);
+    w.chunk_base = reinterpret_cast<int32_t*>(b + off[WS_CHUNK_BASE]);
+    w.sorted = reinterpret_cast<int32_t*>(b + off[WS_SORTED]);
+    w.pos = reinterpret_cast<int32_t*>(b + off[WS_POS]);
+    w.hq = reinterpret_cast<int8_t*>(b + off[WS_HQ]);
+    w.dh = reinterpret_cast<uint16_t*>(b + off[WS_DH]);
+    return w;
+}
+
+static int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ERR_CUDA; }
+
+#define MOE_TRY(expr)                               \
+    do {                                            \
+        cudaError_t e_ = (expr);                    \
+        if (e_ != cudaSuccess) return MOE_Q4_ERR_CUDA; \
+    } while (0)
+
+static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float* y, void* ws, size_t ws_bytes,
+                        const moe_q4_debug* dbg, cudaStream_t s) {
+    int rc = check_layer(Lp);
+    if (rc) return rc;
+    if (T < 0 || T > T_LIMIT) return MOE_Q4_ERR_INVALID_ARG;
+    if (T == 0) return MOE_Q4_OK;
+    if (!x || !y || !ws) return MOE_Q4_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(ws, 256)) return MOE_Q4_ERR_ALIGN;
+    const LayerView L = view(Lp);
+    size_t off[WS_COUNT];
+    layout(L, T, off);
+    if (ws_bytes < off[WS_TOTAL]) return MOE_Q4_ERR_WORKSPACE;
+    const size_t xy_bytes = sizeof(float) * (size_t)(T * L.H);
+    if (overlap(x, xy_bytes, y, xy_bytes) || overlap(y, xy_bytes, ws, off[WS_TOTAL])) return MOE_Q4_ERR_OVERLAP;
+    if (dbg && dbg->h_out && !aligned(dbg->h_out, 4)) return MOE_Q4_ERR_ALIGN;
+    DeviceInfo dev;
+    rc = current_device(&dev);
+    if (rc) return rc;
+
+    const Workspace w = carve(ws, off);
+    MOE_TRY(launch_router_logits(L, x, T, w.logits, w.status, s));
+    MOE_TRY(launch_topk(w.logits, T, L.E, L.k, w.topk_idx, w.topk_w, s));
+    MOE_TRY(launch_quantize(x, T, L.H, w.qa, w.da, w.status, y, s));
+    MOE_TRY(launch_permute(w.topk_idx, T, L.k, L.E, L.S, DP4A_TT, w, s));
+    cudaEvent_t ev0 = dbg ? static_cast<cudaEvent_t>(dbg->ev_start) : nullptr;
+    cudaEvent_t ev1 = dbg ? static_cast<cudaEvent_t>(dbg->ev_stop) : nullptr;
+    if (ev0) MOE_TRY(record_event(ev0, s));
+    MOE_TRY(launch_gateup_dp4a(L, T, w, dbg ? dbg->h_out : nullptr, dev, s));
+    if (ev1) MOE_TRY(record_event(ev1, s));
+    MOE_TRY(launch_down_dp4a(L, T, w, y, dev, s));
+    return MOE_Q4_OK;
+}
+
+}  // namespace moeq4
+
+using namespace moeq4;
+
+extern "C" {
+
+const char* moe_q4_status_string(int status) {
+    switch (status) {
+        case MOE_Q4_OK: return "ok";
+        case MOE_Q4_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_Q4_ERR_SHAPE: return "hidden and ffn must be positive multiples of 256 (at most 16384)";
+        case MOE_Q4_ERR_ALIGN: return "pointer not 16-byte aligned (workspace: 256-byte)";
+        case MOE_Q4_ERR_WORKSPACE: return "workspace too small";
+        case MOE_Q4_ERR_ARCH: return "device is not compute capability 10.0 (sm_100a)";
+        case MOE_Q4_ERR_CUDA: return "CUDA runtime error";
+        case MOE_Q4_ERR_OVERLAP: return "output overlaps an input or the workspace";
+        default: return "unknown status";
+    }
+}
+
+int moe_q4_quantize_act(const float* x, int64_t T, int32_t H, int8_t* q, uint16_t* d, uint32_t* status,
+                        moe_q4_stream_t stream) {
+    if (T < 0 || T > T_LIMIT || H <= 0 || H % QK) return MOE_Q4_ERR_INVALID_ARG;
+    if (T == 0) return MOE_Q4_OK;
+    if (!x || !q || !d) return MOE_Q4_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(d, 2) || (status && !aligned(status, 4)))
+        return MOE_Q4_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    return cuda_rc(launch_quantize(x, T, H, q, d, status, nullptr, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_q4_route(const moe_q4_layer* L, const float* x, int64_t T, int32_t* topk_idx, float* topk_w, float* logits,
+                 moe_q4_stream_t stream) {
+    int rc = check_layer(L);
+    if (rc) return rc;
+    if (T < 0 || T > T_LIMIT) return MOE_Q4_ERR_INVALID_ARG;
+    if (T == 0) return MOE_Q4_OK;
+    if (!x || !topk_idx || !topk_w || !logits) return MOE_Q4_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) || !aligned(logits, 4))
+        return MOE_Q4_ERR_ALIGN;
+    DeviceInfo dev;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    const LayerView v = view(L);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    MOE_TRY(launch_router_logits(v, x, T, logits, nullptr, s));
+    MOE_TRY(launch_topk(logits, T, v.E, v.k, topk_idx, topk_w, s));
+    return MOE_Q4_OK;
+}
+
+size_t moe_q4_ffn_workspace_bytes(const moe_q4_layer* L, int64_t T_max) {
+    if (check_layer(L) || T_max < 0 || T_max > T_LIMIT) return 0;
+    size_t off[WS_COUNT];
+    layout(view(L), std::max<int64_t>(T_max, 1), off);
+    return off[WS_TOTAL];
+}
+
+int moe_q4_workspace_layout(const moe_q4_layer* L, int64_t T, size_t* offsets, int n) {
+    int rc = check_layer(L);
+    if (rc) return rc;
+    if (T < 0 || T > T_LIMIT || !offsets || n < 0) return MOE_Q4_ERR_INVALID_ARG;
+    size_t off[WS_COUNT];
+    layout(view(L), std::max<int64_t>(T, 1), off);
+    for (int i = 0; i < n && i < WS_COUNT; ++i) offsets[i] = off[i];
+    return MOE_Q4_OK;
+}
+
+int moe_q4_ffn_forward(const moe_q4_layer* L, const float* x, int64_t T, float* y, void* workspace,
+                       size_t ws_bytes, moe_q4_stream_t stream) {
+    return forward_impl(L, x, T, y, workspace, ws_bytes, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_q4_ffn_forward_debug(const moe_q4_layer* L, const float* x, int64_t T, float* y, void* workspace,
+                             size_t ws_bytes, const moe_q4_debug* dbg, moe_q4_stream_t stream) {
+    if (dbg && (dbg->path < MOE_Q4_PATH_AUTO || dbg->path > MOE_Q4_PATH_TENSOR_CORE)) return MOE_Q4_ERR_INVALID_ARG;
+    return forward_impl(L, x, T, y, workspace, ws_bytes, dbg, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moe_q4_ffn_host_workspace_bytes(const moe_q4_layer* L, int64_t T_max) {
+    const size_t base = moe_q4_ffn_workspace_bytes(L, T_max);
+    if (!base) return 0;
+    const size_t xy = align256(sizeof(float) * (size_t)(std::max<int64_t>(T_max, 1) * L->hidden));
+    return base + 2 * xy;
+}
+
+int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t T, float* y_host, void* workspace,
+                            size_t ws_bytes, moe_q4_stream_t stream) {
+    int rc = check_layer(L);
+    if (rc) return rc;
+    if (T < 0 || T > T_LIMIT) return MOE_Q4_ERR_INVALID_ARG;
+    if (T == 0) return MOE_Q4_OK;
+    if (!x_host || !y_host || !workspace) return MOE_Q4_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return MOE_Q4_ERR_ALIGN;
+    size_t off[WS_COUNT];
+    layout(view(L), T, off);
+    const size_t xy = align256(sizeof(float) * (size_t)(T * L->hidden));
+    if (ws_bytes < off[WS_TOTAL] + 2 * xy) return MOE_Q4_ERR_WORKSPACE;
+    char* base = static_cast<char*>(workspace);
+    float* x_dev = reinterpret_cast<float*>(base + off[WS_TOTAL]);
+    float* y_dev = reinterpret_cast<float*>(base + off[WS_TOTAL] + xy);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t bytes = sizeof(float) * (size_t)(T * L->hidden);
+    DeviceInfo dev;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    MOE_TRY(cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s));
+    rc = forward_impl(L, x_dev, T, y_dev, workspace, off[WS_TOTAL], nullptr, s);
+    if (rc) return rc;
+    MOE_TRY(cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, s));
+    return MOE_Q4_OK;
+}
+
+int moe_q4_block_dots(const uint8_t* w_blocks, const int8_t* qa, int64_t n, int32_t* out, moe_q4_stream_t stream) {
+    if (n < 0 || n > (int64_t(1) << 31) || (n % 8)) return MOE_Q4_ERR_INVALID_ARG;
+    if (n == 0) return MOE_Q4_OK;
+    if (!w_blocks || !qa || !out) return MOE_Q4_ERR_INVALID_ARG;
+    if (!aligned(w_blocks, 16) || !aligned(qa, 16) || !aligned(out, 4)) return MOE_Q4_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    return cuda_rc(launch_block_dots(w_blocks, qa, n, out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,80 @@
+// launch.h -- host-side launchers of the kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moeq4 {
+
+// Shapes and device pointers of one layer as the kernels see them.
+struct LayerView {
+    int H, F, E, k, S;
+    const float* w_router;
+    const float* router_bias;
+    const uint8_t* w_gate;
+    const uint8_t* w_up;
+    const uint8_t* w_down;
+    const uint8_t* sh_gate;
+    const uint8_t* sh_up;
+    const uint8_t* sh_down;
+};
+
+// Pointers into a forward workspace.
+struct Workspace {
+    uint32_t* status;
+    float* logits;
+    int32_t* topk_idx;
+    float* topk_w;
+    int8_t* qa;
+    uint16_t* da;
+    int32_t* cnt;
+    int32_t* off;
+    int32_t* tile_off;
+    int32_t* chunk_cnt;
+    int32_t* chunk_base;
+    int32_t* sorted;
+    int32_t* pos;
+    int8_t* hq;
+    uint16_t* dh;
+};
+
+struct DeviceInfo {
+    int sm_count;
+    int max_smem_optin;
+};
+
+// k_route.cu
+// status_clear (may be NULL): a status word the first thread zeroes.
+cudaError_t launch_router_logits(const LayerView& L, const float* x, int64_t T, float* logits,
+                                 uint32_t* status_clear, cudaStream_t s);
+cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* idx, float* w,
+                        cudaStream_t s);
+
+// k_quant_perm.cu
+cudaError_t launch_quantize(const float* x, int64_t T, int H, int8_t* q, uint16_t* d,
+                            uint32_t* status, float* y_zero, cudaStream_t s);
+cudaError_t launch_permute(const int32_t* idx, int64_t T, int k, int E, int S, int tile_tokens,
+                           const Workspace& ws, cudaStream_t s);
+
+// k_grouped_dp4a.cu
+cudaError_t launch_gateup_dp4a(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg,
+                               const DeviceInfo& dev, cudaStream_t s);
+cudaError_t launch_down_dp4a(const LayerView& L, int64_t T, const Workspace& ws, float* y,
+                             const DeviceInfo& dev, cudaStream_t s);
+cudaError_t launch_block_dots(const uint8_t* w, const int8_t* qa, int64_t n, int32_t* out,
+                              cudaStream_t s);
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Resident CTAs per SM of `kernel` at `threads` and `smem` dynamic bytes, with
+// the dynamic shared-memory limit raised to `smem` first.  Cached per device,
+// kernel and size, so the CUDA attribute calls happen on the first (eager)
+// launch only, never while a stream is being captured.  At least 1.
+cudaError_t kernel_occupancy(const void* kernel, int threads, size_t smem, int* per_sm);
+
+// cudaEventRecord that also works inside stream capture (as an external event
+// record node whose timestamp can be read after each graph launch).
+cudaError_t record_event(cudaEvent_t ev, cudaStream_t s);
+
+}  // namespace moeq4

@@ -1,0 +1,153 @@
+"""Host-side checks of the C-ABI library, no GPU needed: it loads, it exports
+every function include/moe_q4.h declares, the Python binding wraps them all,
+and argument checks reject bad calls before any CUDA call is made."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from quantized_moe_q4_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "moe_q4.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_q4_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_three_core_calls():
+    names = header_functions()
+    for n in ("moe_q4_quantize_act", "moe_q4_route", "moe_q4_ffn_forward"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_wraps_every_declared_symbol(lib):
+    import quantized_moe_q4_b200 as m
+    assert sorted(m.EXPORTS) == header_functions()
+    for name in header_functions():
+        assert callable(getattr(m, name, None)), name
+
+
+def test_status_strings(lib):
+    lib.moe_q4_status_string.restype = ctypes.c_char_p
+    assert lib.moe_q4_status_string(0) == b"ok"
+    for code in range(-7, 0):
+        assert lib.moe_q4_status_string(code) not in (b"", b"unknown status")
+
+
+class _L(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("hidden", "ffn", "n_experts", "top_k", "has_shared")] + \
+               [(n, ctypes.c_void_p) for n in ("w_router", "router_bias", "w_gate", "w_up", "w_down",
+                                                "sh_gate", "sh_up", "sh_down")]
+
+
+FAKE = 0x7F0000000000  # a 256-byte aligned address that is never dereferenced
+
+
+def make(**kw):
+    d = dict(hidden=2048, ffn=512, n_experts=128, top_k=8, has_shared=1, w_router=FAKE, router_bias=None,
+             w_gate=FAKE, w_up=FAKE, w_down=FAKE, sh_gate=FAKE, sh_up=FAKE, sh_down=FAKE)
+    d.update(kw)
+    return _L(**d)
+
+
+def fwd(lib, L, x=FAKE + 0x1000000, T=4, y=FAKE + 0x2000000, ws=FAKE + 0x3000000, nbytes=1 << 40):
+    f = lib.moe_q4_ffn_forward
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_size_t, ctypes.c_void_p]
+    return f(ctypes.byref(L), x, T, y, ws, nbytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(top_k=0), -1), (dict(top_k=17, n_experts=32), -1), (dict(top_k=9, n_experts=8), -1),
+    (dict(n_experts=0), -1), (dict(n_experts=257), -1), (dict(has_shared=2), -1),
+    (dict(w_gate=None), -1), (dict(sh_up=None), -1), (dict(has_shared=0), -1),
+    (dict(hidden=2000), -2), (dict(ffn=500), -2), (dict(hidden=0), -2), (dict(ffn=128), -2),
+    (dict(hidden=32768), -2), (dict(w_up=FAKE + 8), -3), (dict(sh_down=FAKE + 2), -3),
+])
+def test_forward_rejects_bad_layers(lib, kw, code):
+    assert fwd(lib, make(**kw)) == code
+
+
+def test_forward_rejects_bad_calls(lib):
+    L = make()
+    assert fwd(lib, L, T=-1) == -1
+    assert fwd(lib, L, T=(1 << 24) + 1) == -1
+    assert fwd(lib, L, T=0) == 0                           # no-op, nothing touched
+    assert fwd(lib, L, x=None) == -1
+    assert fwd(lib, L, y=FAKE + 0x2000004) == -3
+    assert fwd(lib, L, ws=FAKE + 0x3000010) == -3
+    assert fwd(lib, L, nbytes=1000) == -4
+    assert fwd(lib, L, y=FAKE + 0x1000000) == -7             # y == x
+    assert fwd(lib, L, y=FAKE + 0x3000000, ws=FAKE + 0x3000000) == -7
+
+
+def test_workspace_bytes_and_layout(lib):
+    L = make()
+    lib.moe_q4_ffn_workspace_bytes.restype = ctypes.c_size_t
+    lib.moe_q4_ffn_workspace_bytes.argtypes = [ctypes.c_void_p, ctypes.c_int64]
+    n1 = lib.moe_q4_ffn_workspace_bytes(ctypes.byref(L), 1)
+    n947 = lib.moe_q4_ffn_workspace_bytes(ctypes.byref(L), 947)
+    assert 0 < n1 < n947
+    assert lib.moe_q4_ffn_workspace_bytes(ctypes.byref(make(top_k=0)), 4) == 0
+    offs = (ctypes.c_size_t * 16)()
+    lib.moe_q4_workspace_layout.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int]
+    assert lib.moe_q4_workspace_layout(ctypes.byref(L), 947, offs, 16) == 0
+    o = list(offs)
+    assert o[0] == 0 and all(b > a for a, b in zip(o, o[1:])) and all(v % 256 == 0 for v in o)
+    assert o[-1] == n947
+    T, k, H, F = 947, 8, 2048, 512
+    P = T * k
+    # hq spans (P + T) slots of F bytes
+    assert o[14] - o[13] >= (P + T) * F
+
+
+def test_other_entry_points_reject_bad_args(lib):
+    q = lib.moe_q4_quantize_act
+    q.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p]
+    assert q(FAKE, 4, 48, FAKE, FAKE, None, None) == -1      # H not a multiple of 32
+    assert q(FAKE + 4, 4, 64, FAKE, FAKE, None, None) == -3
+    assert q(FAKE, 0, 64, None, None, None, None) == 0
+    r = lib.moe_q4_route
+    r.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p]
+    L = make()
+    assert r(ctypes.byref(L), FAKE, 4, FAKE, FAKE, None, None) == -1
+    b = lib.moe_q4_block_dots
+    b.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+    assert b(FAKE, FAKE, 7, FAKE, None) == -1                # n not a multiple of 8
+    assert b(FAKE + 2, FAKE, 8, FAKE, None) == -3
+    d = lib.moe_q4_ffn_forward_debug
+    d.argtypes = [ctypes.c_void_p] * 2 + [ctypes.c_int64] + [ctypes.c_void_p] * 2 + [ctypes.c_size_t] + \
+                 [ctypes.c_void_p] * 2
+
+    class _D(ctypes.Structure):
+        _fields_ = [("h_out", ctypes.c_void_p), ("path", ctypes.c_int32), ("ev_start", ctypes.c_void_p),
+                    ("ev_stop", ctypes.c_void_p)]
+    dbg = _D(None, 9, None, None)
+    assert d(ctypes.byref(L), FAKE, 4, FAKE + 0x1000000, FAKE + 0x2000000, 1 << 40, ctypes.byref(dbg), None) == -1
+
+
+def test_product_package_does_not_use_the_oracle():
+    pkg = os.path.join(ROOT, "quantized_moe_q4_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f
+                assert "libmoe_q4_oracle" not in src and "moe_q4_oracle" not in src, f

@@ -128,6 +128,32 @@ size_t moe_q4_ffn_host_workspace_bytes(const moe_q4_layer* L, int64_t T_max);
 int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t T, float* y_host,
                             void* workspace, size_t ws_bytes, moe_q4_stream_t stream);
 
+/* The paper has no counterpart of this entry point; it exists for callers
+ * that cannot allocate device memory.  Examples: a host runtime or plugin
+ * whose device memory is reserved up front by someone else, a latency-critical
+ * decode loop that cannot pay for cudaMalloc's implicit device
+ * synchronisation, and code that may not allocate while it records a CUDA
+ * graph.
+ * moe_q4_ffn_forward with the workspace replaced by a static device array of
+ * MOE_Q4_NOALLOC_SCRATCH_BYTES held by the library on every GPU that loads
+ * it, until the process exits.  Nothing is allocated or freed.
+ *   - x, y: as for moe_q4_ffn_forward (caller-owned device buffers).
+ *   - A problem whose workspace (moe_q4_ffn_workspace_bytes(L, T)) exceeds
+ *     the scratch returns MOE_Q4_ERR_WORKSPACE and enqueues nothing; for a
+ *     layer with hidden 2048, ffn 512, 128 experts, top-8 and a shared expert
+ *     that allows T up to 542 tokens.
+ *   - The first call on a device looks up the scratch's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls share the one array, which keeps the last call's contents.
+ *     Each call writes every scratch value it later reads (the status word,
+ *     the first uint32 of the scratch, is cleared at the start), so nothing
+ *     needs clearing between calls.  Calls that overlap on the GPU (other
+ *     streams, other host threads) race on the scratch: serialise them. */
+#define MOE_Q4_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+int moe_q4_ffn_forward_noalloc(const moe_q4_layer* L, const float* x, int64_t T, float* y,
+                               moe_q4_stream_t stream);
+
 /* Static description of an error code. */
 const char* moe_q4_status_string(int status);
 

@@ -41,7 +41,8 @@ WS_NAMES = ["status", "logits", "topk_idx", "topk_w", "qa", "da", "cnt", "off", 
 # Every extern "C" symbol of include/moe_q4.h.
 EXPORTS = ["moe_q4_quantize_act", "moe_q4_route", "moe_q4_ffn_workspace_bytes", "moe_q4_ffn_forward",
            "moe_q4_ffn_host_workspace_bytes", "moe_q4_ffn_forward_host", "moe_q4_status_string",
-           "moe_q4_workspace_layout", "moe_q4_ffn_forward_debug", "moe_q4_block_dots"]
+           "moe_q4_workspace_layout", "moe_q4_ffn_forward_debug", "moe_q4_block_dots",
+           "moe_q4_ffn_forward_noalloc"]
 
 
 class MoeQ4Error(RuntimeError):
@@ -83,6 +84,7 @@ def _load() -> ctypes.CDLL:
         "moe_q4_workspace_layout": ([P, i64, P, ctypes.c_int], ctypes.c_int),
         "moe_q4_ffn_forward_debug": ([P, P, i64, P, P, sz, P, P], ctypes.c_int),
         "moe_q4_block_dots": ([P, P, i64, P, P], ctypes.c_int),
+        "moe_q4_ffn_forward_noalloc": ([P, P, i64, P, P], ctypes.c_int),
     }
     for name, (args, res) in sigs.items():
         f = getattr(lib, name)
@@ -254,3 +256,14 @@ def moe_q4_block_dots(w_blocks: torch.Tensor, qa: torch.Tensor, out=None, stream
     out = torch.empty(n, dtype=torch.int32, device=w_blocks.device) if out is None else out
     _check(_lib.moe_q4_block_dots(_p(w_blocks), _p(qa), n, _p(out), _stream(stream)), "moe_q4_block_dots")
     return out
+
+
+def moe_q4_ffn_forward_noalloc(layer: Layer, x: torch.Tensor, y=None, stream=None):
+    """The layer with the library's static device scratch instead of a
+    caller workspace (for callers that cannot allocate device memory; see
+    include/moe_q4.h).  Calls that overlap on the GPU race on the scratch."""
+    T = x.shape[0]
+    y = torch.empty_like(x) if y is None else y
+    _check(_lib.moe_q4_ffn_forward_noalloc(layer.ref, _p(x), T, _p(y), _stream(stream)),
+           "moe_q4_ffn_forward_noalloc")
+    return y

@@ -157,6 +157,10 @@ int moe_q4_ffn_forward_noalloc(const moe_q4_layer* L, const float* x, int64_t T,
 /* Static description of an error code. */
 const char* moe_q4_status_string(int status);
 
+/* Description of the CUDA runtime error behind the last MOE_Q4_ERR_CUDA that
+ * an entry point returned on the calling thread ("no CUDA error" if none). */
+const char* moe_q4_last_cuda_error(void);
+
 /* ---------------------------------------------------------------------
  * Inspection entry points used by the parity tests.
  * --------------------------------------------------------------------- */

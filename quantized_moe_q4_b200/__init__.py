@@ -42,13 +42,16 @@ WS_NAMES = ["status", "logits", "topk_idx", "topk_w", "qa", "da", "cnt", "off", 
 EXPORTS = ["moe_q4_quantize_act", "moe_q4_route", "moe_q4_ffn_workspace_bytes", "moe_q4_ffn_forward",
            "moe_q4_ffn_host_workspace_bytes", "moe_q4_ffn_forward_host", "moe_q4_status_string",
            "moe_q4_workspace_layout", "moe_q4_ffn_forward_debug", "moe_q4_block_dots",
-           "moe_q4_ffn_forward_noalloc"]
+           "moe_q4_ffn_forward_noalloc", "moe_q4_last_cuda_error"]
 
 
 class MoeQ4Error(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
-        super().__init__(f"{what}: {ERRORS.get(code, code)} ({moe_q4_status_string(code)})")
+        detail = moe_q4_status_string(code)
+        if code == -6:
+            detail += ": " + moe_q4_last_cuda_error()
+        super().__init__(f"{what}: {ERRORS.get(code, code)} ({detail})")
 
 
 class _Layer(ctypes.Structure):
@@ -85,6 +88,7 @@ def _load() -> ctypes.CDLL:
         "moe_q4_ffn_forward_debug": ([P, P, i64, P, P, sz, P, P], ctypes.c_int),
         "moe_q4_block_dots": ([P, P, i64, P, P], ctypes.c_int),
         "moe_q4_ffn_forward_noalloc": ([P, P, i64, P, P], ctypes.c_int),
+        "moe_q4_last_cuda_error": ([], ctypes.c_char_p),
     }
     for name, (args, res) in sigs.items():
         f = getattr(lib, name)
@@ -119,6 +123,10 @@ def _check(rc: int, what: str):
 
 def moe_q4_status_string(code: int) -> str:
     return _lib.moe_q4_status_string(int(code)).decode()
+
+
+def moe_q4_last_cuda_error() -> str:
+    return _lib.moe_q4_last_cuda_error().decode()
 
 
 class Layer:

@@ -4,7 +4,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/moe_q4.h"
+#include "moe_q4.h"
 #include "common.cuh"
 #include "launch.h"
 
@@ -50,20 +50,41 @@ static OccEntry g_occ[256];
 static int g_occ_n = 0;
 static std::mutex g_occ_mu;
 
+static size_t kernel_static_smem(const void* kernel) {
+    cudaFuncAttributes a;
+    if (cudaFuncGetAttributes(&a, kernel) != cudaSuccess) return 0;
+    return a.sharedSizeBytes;
+}
+
+// Last CUDA error seen by an entry point of this thread (for error messages).
+static thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
 cudaError_t kernel_occupancy(const void* kernel, int threads, size_t smem, int* per_sm) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(g_occ_mu);
+    bool kernel_seen = false;
     for (int i = 0; i < g_occ_n; ++i) {
         const OccEntry& o = g_occ[i];
-        if (o.dev == dev && o.kernel == kernel && o.threads == threads && o.smem == smem) {
+        if (o.dev != dev || o.kernel != kernel) continue;
+        kernel_seen = true;
+        if (o.threads == threads && o.smem == smem) {
             *per_sm = o.per_sm;
             return cudaSuccess;
         }
     }
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    // The dynamic shared-memory limit is one attribute per function: raise it
+    // once to the device's opt-in maximum, so launches of every size (cached
+    // or not) stay within it.
+    if (!kernel_seen) {
+        int max_optin = 0;
+        e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return e;
+        const int dyn_max = max_optin - (int)kernel_static_smem(kernel);
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max);
+        if (e != cudaSuccess) return e;
+    }
     int n = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem);
     if (e != cudaSuccess) return e;
@@ -167,12 +188,16 @@ static Workspace carve(void* base, const size_t off[WS_COUNT]) {
     return w;
 }
 
-static int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ERR_CUDA; }
+static int cuda_rc(cudaError_t e) {
+    if (e == cudaSuccess) return MOE_Q4_OK;
+    g_last_cuda_error = e;
+    return MOE_Q4_ERR_CUDA;
+}
 
-#define MOE_TRY(expr)                               \
-    do {                                            \
-        cudaError_t e_ = (expr);                    \
-        if (e_ != cudaSuccess) return MOE_Q4_ERR_CUDA; \
+#define MOE_TRY(expr)                          \
+    do {                                       \
+        cudaError_t e_ = (expr);               \
+        if (e_ != cudaSuccess) return cuda_rc(e_); \
     } while (0)
 
 static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float* y, void* ws, size_t ws_bytes,
@@ -195,12 +220,16 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
     if (rc) return rc;
 
     const Workspace w = carve(ws, off);
+    cudaEvent_t ev0 = dbg ? static_cast<cudaEvent_t>(dbg->ev_start) : nullptr;
+    cudaEvent_t ev1 = dbg ? static_cast<cudaEvent_t>(dbg->ev_stop) : nullptr;
+    const int path = dbg ? dbg->path : MOE_Q4_PATH_AUTO;
+    if ((path == MOE_Q4_PATH_AUTO || path == MOE_Q4_PATH_DECODE) && decode_eligible(L, T, dev))
+        return cuda_rc(launch_decode(L, x, y, w, dbg ? dbg->h_out : nullptr, dev, ev0, ev1, s));
+
     MOE_TRY(launch_router_logits(L, x, T, w.logits, w.status, s));
     MOE_TRY(launch_topk(w.logits, T, L.E, L.k, w.topk_idx, w.topk_w, s));
     MOE_TRY(launch_quantize(x, T, L.H, w.qa, w.da, w.status, y, s));
     MOE_TRY(launch_permute(w.topk_idx, T, L.k, L.E, L.S, DP4A_TT, w, s));
-    cudaEvent_t ev0 = dbg ? static_cast<cudaEvent_t>(dbg->ev_start) : nullptr;
-    cudaEvent_t ev1 = dbg ? static_cast<cudaEvent_t>(dbg->ev_stop) : nullptr;
     if (ev0) MOE_TRY(record_event(ev0, s));
     MOE_TRY(launch_gateup_dp4a(L, T, w, dbg ? dbg->h_out : nullptr, dev, s));
     if (ev1) MOE_TRY(record_event(ev1, s));
@@ -213,6 +242,10 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
 using namespace moeq4;
 
 extern "C" {
+
+const char* moe_q4_last_cuda_error(void) {
+    return g_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(g_last_cuda_error);
+}
 
 const char* moe_q4_status_string(int status) {
     switch (status) {

@@ -62,6 +62,13 @@ cudaError_t launch_gateup_dp4a(const LayerView& L, int64_t T, const Workspace& w
                                const DeviceInfo& dev, cudaStream_t s);
 cudaError_t launch_down_dp4a(const LayerView& L, int64_t T, const Workspace& ws, float* y,
                              const DeviceInfo& dev, cudaStream_t s);
+// k_decode.cu: the fused T=1 path (router kernel + cooperative FFN kernel,
+// chained with programmatic dependent launch).  Events, if given, bracket the
+// FFN kernel.
+bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev);
+cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Workspace& ws, float* h_dbg,
+                          const DeviceInfo& dev, cudaEvent_t ev_start, cudaEvent_t ev_stop, cudaStream_t s);
+
 cudaError_t launch_block_dots(const uint8_t* w, const int8_t* qa, int64_t n, int32_t* out,
                               cudaStream_t s);
 

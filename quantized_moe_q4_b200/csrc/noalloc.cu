@@ -12,7 +12,7 @@
 // of device memory until the process exits.
 #include <mutex>
 
-#include "../../include/moe_q4.h"
+#include "moe_q4.h"
 
 namespace {
 

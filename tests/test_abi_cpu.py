@@ -13,7 +13,11 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def lib():
-    from quantized_moe_q4_b200 import build
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "moe_q4_cuda_build", os.path.join(ROOT, "quantized_moe_q4_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
     path = build.build()
     return ctypes.CDLL(path)
 

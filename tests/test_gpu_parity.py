@@ -24,7 +24,7 @@ if not torch.cuda.is_available():  # collected on CPU hosts only with -m gpu
 
 import quantized_moe_q4_b200 as m  # noqa: E402  (loads the CUDA library; fails loudly if missing)
 
-PATHS = [m.PATH_AUTO, m.PATH_GROUPED_DP4A]
+PATHS = [m.PATH_AUTO, m.PATH_GROUPED_DP4A, m.PATH_DECODE]
 
 
 # --------------------------------------------------------------- building blocks
@@ -146,6 +146,11 @@ def test_zipf_16384_full_size_sampled(path):
     (9, 256, 256, 4, 4, True),        # k = E, ragged token tile
     (3, 512, 768, 5, 2, True),        # F = 3*256
     (40, 768, 256, 256, 16, False),   # E = 256, k = 16
+    (1, 768, 768, 5, 2, True),        # decode path: odd H and F
+    (1, 4096, 512, 16, 4, True),      # decode path: wide H
+    (1, 512, 1024, 8, 8, True),       # decode path: more gate/up items than CTAs
+    (1, 2048, 2048, 64, 8, True),     # too large for the decode path: falls back
+    (1, 256, 512, 256, 16, False),    # decode path: E = 256, k = 16
     (17, 4096, 256, 8, 2, True),      # wide H
 ])
 def test_shapes_and_degenerate_cases(path, T, H, F, E, k, shared):
@@ -154,6 +159,17 @@ def test_shapes_and_degenerate_cases(path, T, H, F, E, k, shared):
     check_routing(lw, x, v)
     check_permutation(lw, v)
     teacher_forced_check(lw, x, v, np.arange(T))
+
+
+def test_kernel_shared_memory_sizes_in_any_order():
+    # the same kernels at a large, a small and again the large shared-memory
+    # size: the per-kernel dynamic shared-memory limit must cover all of them
+    cases = [(1, 4096, 512, 16, 4, True), (1, 256, 256, 4, 2, True), (1, 4096, 512, 16, 4, True),
+             (9, 4096, 256, 8, 2, True), (9, 256, 256, 4, 2, True), (9, 4096, 256, 8, 2, True)]
+    for T, H, F, E, k, shared in cases:
+        x, lw = synth.random_layer(seed=H + T, H=H, F=F, E=E, k=k, shared=shared, T=T)
+        v = run_forward(lw, x)
+        teacher_forced_check(lw, x, v, np.arange(T))
 
 
 def test_zero_tokens_is_a_noop():

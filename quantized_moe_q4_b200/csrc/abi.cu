@@ -11,6 +11,8 @@
 namespace moeq4 {
 
 static constexpr int64_t T_LIMIT = int64_t(1) << 24;
+// Token count from which the automatic choice uses the tensor-core kernels.
+static constexpr int64_t TC_MIN_TOKENS = 32;
 static constexpr int MAX_DEVICES = 64;
 
 struct DeviceState {
@@ -226,14 +228,22 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
     if ((path == MOE_Q4_PATH_AUTO || path == MOE_Q4_PATH_DECODE) && decode_eligible(L, T, dev))
         return cuda_rc(launch_decode(L, x, y, w, dbg ? dbg->h_out : nullptr, dev, ev0, ev1, s));
 
+    // grouped paths: tensor cores once experts see tens of tokens, else dp4a
+    const bool tc = (path == MOE_Q4_PATH_TENSOR_CORE) || (path == MOE_Q4_PATH_AUTO && T >= TC_MIN_TOKENS);
     MOE_TRY(launch_router_logits(L, x, T, w.logits, w.status, s));
     MOE_TRY(launch_topk(w.logits, T, L.E, L.k, w.topk_idx, w.topk_w, s));
     MOE_TRY(launch_quantize(x, T, L.H, w.qa, w.da, w.status, y, s));
-    MOE_TRY(launch_permute(w.topk_idx, T, L.k, L.E, L.S, DP4A_TT, w, s));
+    MOE_TRY(launch_permute(w.topk_idx, T, L.k, L.E, L.S, tc ? TC_TILE_TOKENS : DP4A_TT, w, s));
     if (ev0) MOE_TRY(record_event(ev0, s));
-    MOE_TRY(launch_gateup_dp4a(L, T, w, dbg ? dbg->h_out : nullptr, dev, s));
+    if (tc)
+        MOE_TRY(launch_gateup_tc(L, T, w, dbg ? dbg->h_out : nullptr, dev, s));
+    else
+        MOE_TRY(launch_gateup_dp4a(L, T, w, dbg ? dbg->h_out : nullptr, dev, s));
     if (ev1) MOE_TRY(record_event(ev1, s));
-    MOE_TRY(launch_down_dp4a(L, T, w, y, dev, s));
+    if (tc)
+        MOE_TRY(launch_down_tc(L, T, w, y, dev, s));
+    else
+        MOE_TRY(launch_down_dp4a(L, T, w, y, dev, s));
     return MOE_Q4_OK;
 }
 

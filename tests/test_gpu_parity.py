@@ -24,7 +24,7 @@ if not torch.cuda.is_available():  # collected on CPU hosts only with -m gpu
 
 import quantized_moe_q4_b200 as m  # noqa: E402  (loads the CUDA library; fails loudly if missing)
 
-PATHS = [m.PATH_AUTO, m.PATH_GROUPED_DP4A, m.PATH_DECODE]
+PATHS = [m.PATH_AUTO, m.PATH_GROUPED_DP4A, m.PATH_DECODE, m.PATH_TENSOR_CORE]
 
 
 # --------------------------------------------------------------- building blocks

@@ -214,6 +214,55 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def int8_peak_tops():
+    """Dense int8 tensor peak: the measured bf16 GEMM peak x the nominal
+    int8/bf16 ratio (4.5 / 2.25 PFLOP/s)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        return float(json.load(open(path))["bf16_tflops"]) * 2.0, "measured bf16 x nominal int8/bf16 ratio 2"
+    return 1590.0 * 2.0, "fallback bf16 x nominal int8/bf16 ratio 2"
+
+
+def prefill_lines(m, torch, stream):
+    """Single-pass prefill of the two prefill workloads on the automatic path
+    (tensor cores at these sizes): tokens/s over whole forwards and the int8
+    ops/s of the gate/up kernel, L2 flushed (256 MB written) before each rep."""
+    import synth
+    out = {}
+    peak, peak_src = int8_peak_tops()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for name in ("prefill_t947", "zipf_t16384"):
+        x_np, lw = synth.workload_inputs(name, seed=0)
+        L = m.Layer.from_host(lw)
+        x = torch.from_numpy(x_np).cuda()
+        T = x.shape[0]
+        y = torch.empty_like(x)
+        ws = m.alloc_workspace(m.moe_q4_ffn_workspace_bytes(L, T))
+        tot, gu = [], []
+        for rep in range(8):
+            flush.zero_()
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            for e in evs[2:]:
+                e.record(stream)  # torch creates the CUDA event on first record
+            evs[0].record(stream)
+            m.moe_q4_ffn_forward_debug(L, x, y, ws, ev_start=evs[2], ev_stop=evs[3], stream=stream)
+            evs[1].record(stream)
+            torch.cuda.synchronize()
+            if rep >= 3:
+                tot.append(evs[0].elapsed_time(evs[1]))
+                gu.append(evs[2].elapsed_time(evs[3]))
+        ms, gu_ms = float(np.median(tot)), float(np.median(gu))
+        pairs = T * (lw.top_k + 1)
+        gu_ops = 2.0 * pairs * 2 * lw.ffn * lw.hidden
+        out[name] = {"tokens_per_s": T / (ms * 1e-3), "ms": ms, "gateup_ms": gu_ms,
+                     "gateup_int8_tops": gu_ops / (gu_ms * 1e-3) / 1e12, "int8_peak_tops": peak,
+                     "gateup_frac_of_int8_peak": gu_ops / (gu_ms * 1e-3) / 1e12 / peak, "peak_source": peak_src,
+                     "l2": "256 MB flush before each rep"}
+        del L, x, y, ws
+    del flush
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -350,6 +399,8 @@ def run_ours(args):
     e2e_value = world * N_TOKENS * args.steps / (e2e_ms / 1000.0)
     del g3
 
+    prefill = prefill_lines(m, torch, stream) if rank == 0 else None
+
     cpu = None
     if rank == 0 and world == 1:
         v, n, dt, cores = oracle_sample(x_np, lw, seconds=10.0)
@@ -374,6 +425,7 @@ def run_ours(args):
                                                               "host x/y), graph-captured"},
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clk,
+        "prefill": prefill,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -1,31 +1,51 @@
 // k_tc_grouped.cu -- grouped W4A8 projections on the 5th-generation tensor
-// cores (tcgen05.mma kind::i8, accumulators in TMEM).
+// cores (tcgen05.mma, accumulators in TMEM), warp-specialised and pipelined.
 //
 // The grouped 4-bit GEMM of the prefill ("A 35B Hybrid-Attention
 // Mixture-of-Experts Model on a 6GB 2011 GPU", Dutch technical summary,
 // Methodologie 1), with the page's single-pass prefill (Methodologie 4): every
-// expert sees all of its tokens at once, so its weights are read once per
-// token tile.
+// expert sees all of its tokens at once.
 //
-// Orientation: the MMA's M dimension is 128 weight rows (gate/up: 64 gate rows
-// + the same 64 up rows; down: 128 rows of H), N is a tile of 64 slots of one
-// expert, K runs over Q4_0 blocks.  Each 32-wide block is one MMA (K = 32)
-// into its own TMEM buffer, because every block has its own pair of binary16
-// scales: the epilogue reads the exact int32 block sums and accumulates
-// dW[row,b] * dA[slot,b] * I_b in fp32 registers (lane = row).
+// Arithmetic.  Every Q4_0 block (32 weights along K) carries its own binary16
+// scale, and so does every Q8_0 block of the activations, so the sum over K is
+// sum_b dW[row,b] * dA[slot,b] * I_b with I_b the exact integer block dot
+// product.  The tensor core computes I_b: operands hold the exact small
+// integers (nibble - 8 in [-8, 7], q in [-127, 127]) as binary16, products and
+// 32-term sums are exact in the fp32 accumulator, so each 32-wide block is two
+// K=16 MMAs into its own TMEM buffer.  The epilogue then accumulates
+// acc += I_b * (dW * dA) in fp32 registers (packed f32x2 FMUL + FFMA; the
+// product of two binary16 scales is exact in binary32).  Binary16 rather than
+// int8 operands spare an int32 -> fp32 conversion per accumulator element per
+// block, which on B200 issues at about a quarter of the FMA rate and would
+// bound the kernel.
 //
-// Per K chunk of 8 blocks:
-//   1. bulk copies of the 128 packed weight rows (144 B each) into staging;
-//      16-byte cp.async gathers of the 64 slots' int8 activations straight
-//      into the K-major operand layout (8-row x 16-byte core matrices);
-//   2. each thread unpacks one weight row: nibbles -> signed int8 (nib - 8)
-//      into the same operand layout, scales -> shared memory;
-//   3. one thread issues the 8 MMAs and commits them to an mbarrier;
-//   4. the four warps read their 32 TMEM lanes and rescale.
-// After the last chunk: gate/up -> SwiGLU and Q8_0 requantisation of h
-// (a warp's 32 lanes are the 32 rows of one Q8_0 block); down -> y[t] +=
-// w_slot * o (fp32 atomics).
+// Tile: 128 weight rows (gate/up: 64 gate rows + the same 64 up rows; down:
+// 128 rows of H) x 64 slots of one expert (MMA M = 128, N = 64).
+//
+// Warp roles (14 warps):
+//   0      producer: 2D tensor copies (TMA) of the packed weight rows (a box
+//          of 64 or 128 rows x 144 B = 8 blocks) and 16-byte cp.async gathers
+//          of the slots' int8 activations and their scales, two input stages;
+//   1..4   converters: nibbles -> binary16 (nib - 8) and int8 -> binary16 into
+//          the K-major operand layout (8-row x 16-byte core matrices), two
+//          operand stages of 4 blocks; block scales into a ring shared with
+//          the epilogue;
+//   5      MMA issuer (one thread): two MMAs per block, one commit per block,
+//          descriptors precomputed (the issue path is a handful of instructions);
+//   6..13  epilogue: 4 TMEM lane quarters x 2 column halves; per block one
+//          TMEM load of 32 columns, rescale-accumulate; after the last block of
+//          a tile gate/up -> SwiGLU + Q8_0 requantisation, down ->
+//          y += w_slot * o (fp32 atomics).
+// Eight TMEM buffers of 64 columns and a 16-entry scale ring (so the converters
+// run up to four operand stages ahead of the epilogue); full/empty mbarriers between every pair of
+// roles; every wait bounded, and one that runs out makes every role leave its
+// loop and records STATUS_SPIN_TIMEOUT.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "launch.h"
@@ -34,21 +54,50 @@
 
 namespace moeq4 {
 
-constexpr int TC_M = 128;
-constexpr int TC_N = 64;
-constexpr int TC_KB = 8;                     // Q4_0 blocks per K chunk
-constexpr int TC_THREADS = 128;              // one thread per TMEM lane
-constexpr uint32_t TC_TMEM_COLS = TC_KB * TC_N;  // one 64-column buffer per block
-constexpr int TC_STAGE_ROW = TC_KB * Q4_BYTES;   // 144 packed bytes per row per chunk
+namespace {
 
-constexpr size_t TC_SMEM_A = (size_t)TC_KB * TC_M * QK;     // 32 KB
-constexpr size_t TC_SMEM_B = (size_t)TC_KB * TC_N * QK;     // 16 KB
-constexpr size_t TC_SMEM_STAGE = (size_t)TC_M * TC_STAGE_ROW;  // 18 KB
-// more than half of an SM's shared memory: one CTA per SM, so the 512 TMEM
-// columns one CTA allocates are always free
-constexpr size_t TC_SMEM_TOTAL = 120 * 1024;
+constexpr int TM = 128;            // MMA M: weight rows per tile
+constexpr int TN = TC_TILE_TOKENS; // MMA N: slots per tile
+constexpr int IN_KB = 8;           // Q4_0 blocks per input stage (144-byte rows: a 16-byte multiple)
+constexpr int OP_KB = 4;           // blocks per operand stage
+constexpr int NIN = 2, NOP = 2, NTM = 8, NSC = 16;  // input, operand, TMEM and scale ring depths
+constexpr int IN_ROW = IN_KB * Q4_BYTES;          // 144
+constexpr int THREADS = 14 * 32;  // 4 warps on some SM sub-partitions: at most 128 registers a thread
+constexpr int W_PROD = 0, W_CONV0 = 1, W_MMA = 5, W_EPI0 = 6;
+constexpr int N_CONV = 128, N_EPI = 256;
+constexpr uint32_t TMEM_COLS = NTM * TN;          // 512
+constexpr uint32_t LIMIT = 1u << 22;
+static_assert(TN == 64, "the epilogue maps two warps of 32 columns onto a tile");
 
-enum { TC_GATEUP = 0, TC_DOWN = 1 };
+// dynamic shared memory map (bytes)
+constexpr size_t SZ_IN_W = (size_t)TM * IN_ROW;           // one input stage of packed weight rows
+constexpr size_t SZ_IN_B = (size_t)TN * IN_KB * QK;       // int8 activations, [16-byte chunk][slot]
+constexpr size_t SZ_IN_DA = (size_t)TN * IN_KB * 2;       // activation scale bits, [slot][block]
+constexpr size_t SZ_KSTEP_A = (size_t)TM * 32;            // 128 rows x 16 binary16
+constexpr size_t SZ_KSTEP_B = (size_t)TN * 32;
+constexpr size_t SZ_OP_A = (size_t)OP_KB * 2 * SZ_KSTEP_A;
+constexpr size_t SZ_OP_B = (size_t)OP_KB * 2 * SZ_KSTEP_B;
+constexpr int XCH_LD = TN + 1;
+constexpr size_t OFF_IN_W = 0;
+constexpr size_t OFF_IN_B = OFF_IN_W + NIN * SZ_IN_W;
+constexpr size_t OFF_IN_DA = OFF_IN_B + NIN * SZ_IN_B;
+constexpr size_t OFF_OP_A = (OFF_IN_DA + NIN * SZ_IN_DA + 1023) & ~size_t(1023);
+constexpr size_t OFF_OP_B = OFF_OP_A + NOP * SZ_OP_A;
+constexpr size_t OFF_DW = OFF_OP_B + NOP * SZ_OP_B;
+constexpr size_t OFF_DA = OFF_DW + (size_t)NSC * TM * 4;
+constexpr size_t OFF_XCH = OFF_DA + (size_t)NSC * TN * 4;
+constexpr size_t SMEM_BYTES = OFF_XCH + (size_t)TM * XCH_LD * 4;
+constexpr size_t SMEM_ALLOC = SMEM_BYTES + 1024;          // slack to align the map to 1024 B
+static_assert(SMEM_ALLOC <= 220 * 1024, "shared memory map too large");
+
+enum { GATEUP = 0, DOWN = 1 };
+
+// Tensor maps of the weight matrices, rows of 18-byte blocks viewed as bytes:
+// gate/up: [0] all experts' gate rows, [1] up rows, [2] shared gate, [3]
+// shared up; down: [0] all experts' down rows, [2] shared down.
+struct TcMaps {
+    CUtensorMap m[4];
+};
 
 struct TcParams {
     int H, F, E, k, P;
@@ -71,21 +120,105 @@ struct TcParams {
     uint32_t* status;
 };
 
-// nibble bytes (0..15) -> signed int8 bytes (nib - 8): for nib >= 8 the value
-// is nib ^ 8; for nib < 8 it is 0xF8 | nib, i.e. nib ^ 8 with the top four bits
-// set, and (~nib & 8) * 0x1E supplies exactly those bits without carries.
-__device__ __forceinline__ uint32_t nib_to_s8(uint32_t n) {
-    return (n ^ 0x08080808u) | ((~n & 0x08080808u) * 0x1Eu);
+// ---------------------------------------------------------------- helpers
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Offset of the 16-byte piece kc (0: K bytes 0..15, 1: 16..31) of row r of
-// block kb in a K-major operand tile of `rows` rows (8-row x 16-byte core
-// matrices; K core matrices 128 B apart, 8-row groups 256 B apart).
-__device__ __forceinline__ uint32_t op_offset(int kb, int rows, int r, int kc) {
-    return (uint32_t)(kb * rows * QK + (r >> 3) * 256 + kc * 128 + (r & 7) * 16);
+// Arrive on `bar` once this thread's earlier cp.async copies complete; the
+// arrival counts towards the barrier's expected count.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ int find_group_tc(const int* tile_off, int ngroups, int tile) {
+
+// Bounded wait shared by all roles: once any wait of the CTA has run out,
+// `abort` is set and every later wait returns false soon after.
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    for (uint32_t i = 0; i < LIMIT; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *abort) return false;
+    }
+    *abort = 1;
+    return false;
+}
+
+// Barrier of the epilogue warps (one arrival per warp), bounded like every
+// other wait so that a role that gave up cannot strand the others.
+__device__ __forceinline__ bool epi_sync(uint64_t* bar, uint32_t use, volatile int* abort) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+    return wait_phase(bar, use & 1, abort);
+}
+
+// 2D tiled tensor copy global -> shared (no multicast), completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// acc[slot pair j] += I (32 columns of one block) * dW * dA[slot].
+__device__ __forceinline__ void rescale_acc(float2 (&acc)[16], const uint32_t (&r)[32], float dwv, const float* da) {
+    const float4* da4 = reinterpret_cast<const float4*>(da);
+    const float2 dw2 = make_float2(dwv, dwv);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float4 d = da4[j];
+        const float2 s0 = __fmul2_rn(dw2, make_float2(d.x, d.y));
+        const float2 s1 = __fmul2_rn(dw2, make_float2(d.z, d.w));
+        acc[2 * j] = __ffma2_rn(make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), s0, acc[2 * j]);
+        acc[2 * j + 1] =
+            __ffma2_rn(make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), s1, acc[2 * j + 1]);
+    }
+}
+
+// D[tmem] (=|+=) A x B^T, binary16 operands, fp32 accumulator.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+// kind::f16 instruction descriptor: binary16 A and B, fp32 accumulator, both
+// operands K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+    return (1u << 4)                        // accumulator format: F32
+           | ((uint32_t)(N >> 3) << 17)     // N / 8
+           | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+// Four unsigned bytes u_i of w -> binary16 (1024 + u_i) - bias, two per word:
+// 1024 + u has the bit pattern 0x6400 | u for u < 256, and the subtraction of
+// two exact small integers is exact.
+__device__ __forceinline__ uint2 bytes_to_f16(uint32_t w, uint32_t bias2) {
+    const uint32_t lo = __byte_perm(w, 0x64646464u, 0x4140);
+    const uint32_t hi = __byte_perm(w, 0x64646464u, 0x4342);
+    const __half2 b = *reinterpret_cast<const __half2*>(&bias2);
+    const __half2 a0 = __hsub2(*reinterpret_cast<const __half2*>(&lo), b);
+    const __half2 a1 = __hsub2(*reinterpret_cast<const __half2*>(&hi), b);
+    return make_uint2(*reinterpret_cast<const uint32_t*>(&a0), *reinterpret_cast<const uint32_t*>(&a1));
+}
+
+constexpr uint32_t BIAS_NIB = 0x64086408u;   // binary16 1032, twice: 1024 + n - 1032 = n - 8
+constexpr uint32_t BIAS_ACT = 0x64806480u;   // binary16 1152, twice: 1024 + (q ^ 0x80) - 1152 = q
+
+// Byte offset of the 16-byte core-matrix piece `core` (0/1) of row r in K-step
+// `ks` of block `kb` of an operand stage with `rows` rows: K-steps are 32-byte
+// (16 x binary16) slabs; inside one, 8-row groups are 256 B apart and the two
+// pieces of a row 128 B apart (the descriptor's SBO and LBO).
+__device__ __forceinline__ uint32_t op_off(int kb, int ks, int rows, int r, int core) {
+    return (uint32_t)((kb * 2 + ks) * rows * 32 + (r >> 3) * 256 + core * 128 + (r & 7) * 16);
+}
+
+__device__ __forceinline__ int find_group(const int* tile_off, int ngroups, int tile) {
     int lo = 0, hi = ngroups;
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -94,45 +227,90 @@ __device__ __forceinline__ int find_group_tc(const int* tile_off, int ngroups, i
     return lo;
 }
 
+struct Tile {
+    int g, slot0, nslots, rb;
+};
+
+// Work item -> (group, first slot, slots in the tile, row block).
+__device__ __forceinline__ Tile tile_of(int item, int n_rb, const int* tile_off_s, const int* off_s, int ngroups) {
+    Tile t;
+    const int tile = item / n_rb;
+    t.rb = item - tile * n_rb;
+    t.g = find_group(tile_off_s, ngroups, tile);
+    t.slot0 = off_s[t.g] + (tile - tile_off_s[t.g]) * TN;
+    t.nslots = min(TN, off_s[t.g + 1] - t.slot0);
+    return t;
+}
+
+// Token and routing weight of slot s of group g (group E: the shared expert,
+// slot P + t is token t with weight 1).
+__device__ __forceinline__ void slot_info(const TcParams& p, int g, int s, int& tok, float& w) {
+    if (g < p.E) {
+        const int pair = __ldg(p.sorted + s);
+        tok = pair / p.k;
+        w = __ldg(p.topk_w + pair);
+    } else {
+        tok = s - p.P;
+        w = 1.0f;
+    }
+}
+
+}  // namespace
+
 template <int MODE>
-__global__ void __launch_bounds__(TC_THREADS, 1) tc_grouped_kernel(TcParams p) {
-    extern __shared__ __align__(1024) unsigned char smem[];
-    __shared__ __align__(8) uint64_t bar_w, bar_mma;
+__global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, const __grid_constant__ TcMaps maps) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    __shared__ __align__(8) uint64_t in_full[NIN], in_empty[NIN], op_full[NOP], op_empty[NOP], tm_full[NTM],
+        tm_empty[NTM], sc_full[NSC], sc_empty[NSC], epi_bar;
     __shared__ uint32_t tmem_base_s;
-    __shared__ int tile_off_s[258];
-    __shared__ int off_s[258];
-    __shared__ int tok_s[TC_N];
-    __shared__ float wgt_s[TC_N];
-    __shared__ const int8_t* act_row_s[TC_N];
-    __shared__ const uint16_t* act_scale_s[TC_N];
+    __shared__ int abort_s;
+    __shared__ int tile_off_s[258], off_s[258];
 
-    uint8_t* A = smem;
-    uint8_t* B = A + TC_SMEM_A;
-    uint8_t* stage = B + TC_SMEM_B;
-    float* dw_s = reinterpret_cast<float*>(stage + TC_SMEM_STAGE);
-    float* da_s = dw_s + TC_M * TC_KB;
-    float* xch = reinterpret_cast<float*>(A);  // 128 x 65 floats, reuses A and B after the K loop
+    uint8_t* in_w = smem + OFF_IN_W;
+    int8_t* in_b = reinterpret_cast<int8_t*>(smem + OFF_IN_B);
+    uint16_t* in_da = reinterpret_cast<uint16_t*>(smem + OFF_IN_DA);
+    uint8_t* op_a = smem + OFF_OP_A;
+    uint8_t* op_b = smem + OFF_OP_B;
+    float* dw_ring = reinterpret_cast<float*>(smem + OFF_DW);
+    float* da_ring = reinterpret_cast<float*>(smem + OFF_DA);
+    float* xch = reinterpret_cast<float*>(smem + OFF_XCH);
+    volatile int* abort = &abort_s;
 
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = p.H, F = p.F, E = p.E;
-    const int K = (MODE == TC_GATEUP) ? H : F;
-    const int nbK = K / QK, nchunks = nbK / TC_KB;
+    const int K = (MODE == GATEUP) ? H : F;
+    const int nbK = K / QK;
     const int nbF = F / QK;
-    const size_t wrow = (size_t)nbK * Q4_BYTES;  // bytes per weight row
-    const size_t mat_stride = (MODE == TC_GATEUP) ? (size_t)F * wrow : (size_t)H * wrow;
-    const int n_rb = (MODE == TC_GATEUP) ? F / 64 : H / TC_M;
+    const int n_rb = (MODE == GATEUP) ? F / 64 : H / TM;
     const int ngroups = E + 1;
 
-    if (warp == 0) {
-        tmem_alloc(&tmem_base_s, TC_TMEM_COLS);
+    if (warp == W_PROD) {
+        tmem_alloc(&tmem_base_s, TMEM_COLS);
         tmem_relinquish();
     }
-    if (t == 0) {
-        mbar_init(&bar_w, TC_THREADS);
-        mbar_init(&bar_mma, 1);
+    if (tid == 32) {
+        abort_s = 0;
+        for (int i = 0; i < NIN; ++i) {
+            mbar_init(&in_full[i], 64);   // 32 producer-lane arrivals + 32 cp.async arrivals
+            mbar_init(&in_empty[i], N_CONV);
+        }
+        for (int i = 0; i < NOP; ++i) {
+            mbar_init(&op_full[i], N_CONV);
+            mbar_init(&op_empty[i], 1);
+        }
+        for (int i = 0; i < NTM; ++i) {
+            mbar_init(&tm_full[i], 1);
+            mbar_init(&tm_empty[i], N_EPI / 32);
+        }
+        for (int i = 0; i < NSC; ++i) {
+            mbar_init(&sc_full[i], N_CONV / 32);
+            mbar_init(&sc_empty[i], N_EPI / 32);
+        }
+        mbar_init(&epi_bar, N_EPI / 32);
         mbar_fence_init();
     }
-    for (int i = t; i <= ngroups; i += TC_THREADS) {
+    for (int i = tid; i <= ngroups; i += THREADS) {
         tile_off_s[i] = p.tile_off[i];
         off_s[i] = p.off[i];
     }
@@ -140,174 +318,301 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_grouped_kernel(TcParams p) {
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = tmem_base_s;
-    const uint32_t idesc = idesc_i8(TC_M, TC_N);
     const int n_items = tile_off_s[ngroups] * n_rb;
-    uint32_t phase = 0;
-    bool timed_out = false;
 
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int tile = item / n_rb, rb = item - tile * n_rb;
-        const int g = find_group_tc(tile_off_s, ngroups, tile);
-        const int slot0 = off_s[g] + (tile - tile_off_s[g]) * TC_N;
-        const int nslots = min(TC_N, off_s[g + 1] - slot0);
-        if (t < TC_N) {
-            int tok = 0;
-            float w = 0.0f;
-            if (t < nslots) {
-                const int s = slot0 + t;
-                if (g < E) {
-                    const int pair = __ldg(p.sorted + s);
-                    tok = pair / p.k;
-                    w = __ldg(p.topk_w + pair);
-                } else {
-                    tok = s - p.P;
-                    w = 1.0f;
-                }
-                if (MODE == TC_GATEUP) {
-                    act_row_s[t] = p.qa + (size_t)tok * H;
-                    act_scale_s[t] = p.da + (size_t)tok * (H / QK);
-                } else {
-                    act_row_s[t] = p.hq + (size_t)s * F;
-                    act_scale_s[t] = p.dh + (size_t)s * nbF;
-                }
-            }
-            tok_s[t] = tok;
-            wgt_s[t] = w;
-        }
-        // this thread's weight row
-        const uint8_t* wsrc;
-        if (MODE == TC_GATEUP) {
-            const int f = rb * 64 + (t & 63);
-            const uint8_t* base = (t < 64) ? ((g < E) ? p.w_gate + g * mat_stride : p.sh_gate)
-                                           : ((g < E) ? p.w_up + g * mat_stride : p.sh_up);
-            wsrc = base + (size_t)f * wrow;
-        } else {
-            wsrc = ((g < E) ? p.w_down + g * mat_stride : p.sh_down) + (size_t)(rb * TC_M + t) * wrow;
-        }
-        __syncthreads();
-
-        float acc[TC_N];
+    if (warp == W_PROD) {
+        // ------------------------------------------------------------ producer
+        uint32_t i_in = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+            const Tile T = tile_of(item, n_rb, tile_off_s, off_s, ngroups);
+            // weight rows of this item: one box of 64 gate + one of 64 up rows, or 128 down rows
+            const bool shared_g = T.g >= E;
+            const CUtensorMap* map0 = &maps.m[shared_g ? 2 : 0];
+            const CUtensorMap* map1 = &maps.m[shared_g ? 3 : 1];
+            const int wy = (shared_g ? 0 : T.g * ((MODE == GATEUP) ? F : H)) + T.rb * ((MODE == GATEUP) ? 64 : TM);
+            const int8_t* arow[2];
+            const uint16_t* ascale[2];
 #pragma unroll
-        for (int n = 0; n < TC_N; ++n) acc[n] = 0.0f;
-
-        for (int c = 0; c < nchunks; ++c) {
-            // 1. packed weight rows -> staging; activations -> operand B
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&bar_w, (uint32_t)TC_STAGE_ROW);
-            bulk_g2s(stage + t * TC_STAGE_ROW, wsrc + (size_t)c * TC_STAGE_ROW, (uint32_t)TC_STAGE_ROW, &bar_w);
-            for (int i = t; i < TC_N * TC_KB * 2; i += TC_THREADS) {
-                const int n = i / (TC_KB * 2), kb = (i >> 1) % TC_KB, kc = i & 1;
-                uint8_t* dst = B + op_offset(kb, TC_N, n, kc);
-                if (n < nslots)
-                    cp_async16(dst, act_row_s[n] + (size_t)(c * TC_KB + kb) * QK + kc * 16);
-                else
-                    *reinterpret_cast<int4*>(dst) = make_int4(0, 0, 0, 0);
-            }
-            for (int i = t; i < TC_N * TC_KB; i += TC_THREADS) {
-                const int n = i / TC_KB, kb = i % TC_KB;
-                da_s[i] = (n < nslots) ? half_bits_to_float(__ldg(act_scale_s[n] + c * TC_KB + kb)) : 0.0f;
-            }
-            cp_async_wait_all();
-            if (!mbar_wait_bounded(&bar_w, phase & 1, 1u << 20)) timed_out = true;
-
-            // 2. unpack this thread's row: nibbles -> signed int8 operand A
-            const uint8_t* srow = stage + t * TC_STAGE_ROW;
-#pragma unroll
-            for (int kb = 0; kb < TC_KB; ++kb) {
-                uint32_t qs[4], dbits;
-                load_q4_block_smem(srow + kb * Q4_BYTES, qs, dbits);
-                dw_s[t * TC_KB + kb] = half_bits_to_float(dbits);
-                int4 lo, hi;
-                lo.x = (int)nib_to_s8(qs[0] & 0x0f0f0f0fu);
-                lo.y = (int)nib_to_s8(qs[1] & 0x0f0f0f0fu);
-                lo.z = (int)nib_to_s8(qs[2] & 0x0f0f0f0fu);
-                lo.w = (int)nib_to_s8(qs[3] & 0x0f0f0f0fu);
-                hi.x = (int)nib_to_s8((qs[0] >> 4) & 0x0f0f0f0fu);
-                hi.y = (int)nib_to_s8((qs[1] >> 4) & 0x0f0f0f0fu);
-                hi.z = (int)nib_to_s8((qs[2] >> 4) & 0x0f0f0f0fu);
-                hi.w = (int)nib_to_s8((qs[3] >> 4) & 0x0f0f0f0fu);
-                *reinterpret_cast<int4*>(A + op_offset(kb, TC_M, t, 0)) = lo;
-                *reinterpret_cast<int4*>(A + op_offset(kb, TC_M, t, 1)) = hi;
-            }
-            fence_proxy_async_smem();  // operand writes -> visible to the tensor core
-            tc_fence_before_sync();
-            __syncthreads();
-            tc_fence_after_sync();
-
-            // 3. one MMA per block into its own TMEM buffer
-            if (t == 0) {
-#pragma unroll
-                for (int kb = 0; kb < TC_KB; ++kb) {
-                    const uint64_t da = smem_desc_kmajor(A + (size_t)kb * TC_M * QK, 128, 256);
-                    const uint64_t db = smem_desc_kmajor(B + (size_t)kb * TC_N * QK, 128, 256);
-                    mma_i8(tmem + kb * TC_N, da, db, idesc, false);
-                }
-                mma_commit(&bar_mma);
-            }
-            if (!mbar_wait_bounded(&bar_mma, phase & 1, 1u << 20)) timed_out = true;
-            tc_fence_after_sync();
-
-            // 4. rescale: lane = row t, 64 slot columns per block
-            const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll 1
-            for (int kb = 0; kb < TC_KB; ++kb) {
-                const float dw = dw_s[t * TC_KB + kb];
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32];
-                    tmem_ld32(lane_addr + kb * TC_N + half * 32, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int n = half * 32 + j;
-                        acc[n] = fmaf((float)(int)r[j], dw * da_s[n * TC_KB + kb], acc[n]);
+            for (int j = 0; j < 2; ++j) {
+                const int n = lane + 32 * j;
+                arow[j] = nullptr;
+                ascale[j] = nullptr;
+                if (n < T.nslots) {
+                    const int s = T.slot0 + n;
+                    int tok;
+                    float w;
+                    slot_info(p, T.g, s, tok, w);
+                    if (MODE == GATEUP) {
+                        arow[j] = p.qa + (size_t)tok * H;
+                        ascale[j] = p.da + (size_t)tok * (H / QK);
+                    } else {
+                        arow[j] = p.hq + (size_t)s * F;
+                        ascale[j] = p.dh + (size_t)s * nbF;
                     }
                 }
             }
-            tc_fence_before_sync();
-            __syncthreads();  // staging, operands and TMEM buffers are free again
-            phase ^= 1u;
-        }
-
-        if (MODE == TC_GATEUP) {
-            // rows t < 64: gate row f0 + t; rows 64 + t: up row f0 + t
-            const int f0 = rb * 64;
+            for (int c = 0; c < nbK / IN_KB; ++c, ++i_in) {
+                const int s = i_in % NIN;
+                if (!wait_phase(&in_empty[s], ((i_in / NIN) & 1) ^ 1, abort)) { ok = false; break; }
+                uint8_t* dw = in_w + (size_t)s * SZ_IN_W;
+                int8_t* db = in_b + (size_t)s * SZ_IN_B;
+                uint16_t* dda = in_da + (size_t)s * TN * IN_KB;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&in_full[s], (uint32_t)(TM * IN_ROW));
+                    tma_load_2d(dw, map0, c * IN_ROW, wy, &in_full[s]);
+                    if (MODE == GATEUP) tma_load_2d(dw + 64 * IN_ROW, map1, c * IN_ROW, wy, &in_full[s]);
+                } else {
+                    mbar_arrive(&in_full[s]);
+                }
 #pragma unroll
-            for (int n = 0; n < TC_N; ++n) xch[t * 65 + n] = acc[n];
-            __syncthreads();
-            if (t < 64) {
+                for (int j = 0; j < 2; ++j) {
+                    if (arow[j]) {
+                        const int n = lane + 32 * j;
+                        const int8_t* src = arow[j] + (size_t)c * IN_KB * QK;
+#pragma unroll
+                        for (int q = 0; q < IN_KB * 2; ++q) cp_async16(db + ((size_t)q * TN + n) * 16, src + q * 16);
+                        cp_async16(dda + n * IN_KB, ascale[j] + c * IN_KB);   // 8 binary16 scales
+                    }
+                }
+                cp_async_arrive_noinc(&in_full[s]);
+            }
+        }
+        // let the copies in flight land before the CTA can exit
+        cp_async_wait_all();
+        if (i_in > 0) mbar_wait_bounded(&in_full[(i_in - 1) % NIN], ((i_in - 1) / NIN) & 1, LIMIT);
+    } else if (warp >= W_CONV0 && warp < W_CONV0 + 4) {
+        // ------------------------------------------------------------ converters
+        const int ct = tid - W_CONV0 * 32;  // weight row of this thread; slot column ct & 63
+        uint32_t i_op = 0, gb = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+            const Tile T = tile_of(item, n_rb, tile_off_s, off_s, ngroups);
+            for (int c = 0; c < nbK / OP_KB && ok; ++c, ++i_op, gb += OP_KB) {
+                const uint32_t i_in = i_op >> 1;
+                const int s = i_in % NIN, sub = i_op & 1;
+                if (sub == 0 && !wait_phase(&in_full[s], (i_in / NIN) & 1, abort)) { ok = false; break; }
+                const int o = i_op % NOP;
+                if (!wait_phase(&op_empty[o], ((i_op / NOP) & 1) ^ 1, abort)) { ok = false; break; }
+                uint8_t* oa = op_a + (size_t)o * SZ_OP_A;
+                uint8_t* ob = op_b + (size_t)o * SZ_OP_B;
+
+                // weights: this row's 4 blocks, 72 bytes at an 8-byte boundary
+                uint32_t w[18];
+                const uint2* wsrc = reinterpret_cast<const uint2*>(in_w + (size_t)s * SZ_IN_W + (size_t)ct * IN_ROW +
+                                                                   sub * OP_KB * Q4_BYTES);
+#pragma unroll
+                for (int i = 0; i < 9; ++i) {
+                    const uint2 v = wsrc[i];
+                    w[2 * i] = v.x;
+                    w[2 * i + 1] = v.y;
+                }
+                float dws[OP_KB];
+#pragma unroll
+                for (int kb = 0; kb < OP_KB; ++kb) {
+                    // block kb starts at byte 18 kb: scale, then 16 nibble bytes
+                    const int bw = (18 * kb) / 4;
+                    uint32_t qs[4], dbits;
+                    if ((kb & 1) == 0) {
+                        dbits = w[bw] & 0xffffu;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) qs[i] = __funnelshift_r(w[bw + i], w[bw + i + 1], 16);
+                    } else {
+                        dbits = w[bw] >> 16;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) qs[i] = w[bw + 1 + i];
+                    }
+                    dws[kb] = half_bits_to_float(dbits);
+#pragma unroll
+                    for (int core = 0; core < 2; ++core) {
+                        // K-step 0: low nibbles (weights 0..15); K-step 1: high nibbles (16..31)
+                        const uint2 l0 = bytes_to_f16(qs[2 * core] & 0x0f0f0f0fu, BIAS_NIB);
+                        const uint2 l1 = bytes_to_f16(qs[2 * core + 1] & 0x0f0f0f0fu, BIAS_NIB);
+                        const uint2 h0 = bytes_to_f16((qs[2 * core] >> 4) & 0x0f0f0f0fu, BIAS_NIB);
+                        const uint2 h1 = bytes_to_f16((qs[2 * core + 1] >> 4) & 0x0f0f0f0fu, BIAS_NIB);
+                        *reinterpret_cast<uint4*>(oa + op_off(kb, 0, TM, ct, core)) = make_uint4(l0.x, l0.y, l1.x, l1.y);
+                        *reinterpret_cast<uint4*>(oa + op_off(kb, 1, TM, ct, core)) = make_uint4(h0.x, h0.y, h1.x, h1.y);
+                    }
+                }
+                // activations: slot n = ct & 63, blocks (ct >> 6) and (ct >> 6) + 2
+                const int n = ct & 63;
+                const bool valid = n < T.nslots;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int kb = (ct >> 6) + 2 * j;
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        uint4 v = make_uint4(0, 0, 0, 0), u = make_uint4(0, 0, 0, 0);
+                        if (valid) {
+                            const int q = (sub * OP_KB + kb) * 2 + ks;
+                            const uint4 a = *reinterpret_cast<const uint4*>(in_b + (size_t)s * SZ_IN_B +
+                                                                            ((size_t)q * TN + n) * 16);
+                            const uint2 a0 = bytes_to_f16(a.x ^ 0x80808080u, BIAS_ACT);
+                            const uint2 a1 = bytes_to_f16(a.y ^ 0x80808080u, BIAS_ACT);
+                            const uint2 a2 = bytes_to_f16(a.z ^ 0x80808080u, BIAS_ACT);
+                            const uint2 a3 = bytes_to_f16(a.w ^ 0x80808080u, BIAS_ACT);
+                            v = make_uint4(a0.x, a0.y, a1.x, a1.y);
+                            u = make_uint4(a2.x, a2.y, a3.x, a3.y);
+                        }
+                        *reinterpret_cast<uint4*>(ob + op_off(kb, ks, TN, n, 0)) = v;
+                        *reinterpret_cast<uint4*>(ob + op_off(kb, ks, TN, n, 1)) = u;
+                    }
+                }
+                // this slot's activation scales, read before the input stage is released
+                float das[OP_KB];
+#pragma unroll
+                for (int kb = 0; kb < OP_KB; ++kb)
+                    das[kb] = valid ? half_bits_to_float(in_da[(size_t)s * TN * IN_KB + n * IN_KB + sub * OP_KB + kb])
+                                    : 0.0f;
+                fence_proxy_async_smem();
+                mbar_arrive(&op_full[o]);
+                if (sub == 1) mbar_arrive(&in_empty[s]);
+                // scales of these 4 blocks into the ring read by the epilogue; the
+                // epilogue frees entries in order, so the last one being free
+                // means all four are
+                const uint32_t glast = gb + OP_KB - 1, buf0 = gb % NSC;
+                if (!wait_phase(&sc_empty[glast % NSC], ((glast / NSC) & 1) ^ 1, abort)) { ok = false; break; }
+#pragma unroll
+                for (int kb = 0; kb < OP_KB; ++kb) {
+                    dw_ring[(buf0 + kb) * TM + ct] = dws[kb];
+                    if (ct < TN) da_ring[(buf0 + kb) * TN + ct] = das[kb];
+                }
+                __syncwarp();
+                if (lane == 0) {
+#pragma unroll
+                    for (int kb = 0; kb < OP_KB; ++kb) mbar_arrive(&sc_full[buf0 + kb]);
+                }
+            }
+        }
+    } else if (warp == W_MMA) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_f16(TM, TN);
+            // descriptors of the first K-step of each operand stage; a later
+            // K-step adds its byte offset / 16 to the start-address field
+            const uint64_t a0 = smem_desc_kmajor(op_a, 128, 256), a1 = smem_desc_kmajor(op_a + SZ_OP_A, 128, 256);
+            const uint64_t b0 = smem_desc_kmajor(op_b, 128, 256), b1 = smem_desc_kmajor(op_b + SZ_OP_B, 128, 256);
+            static_assert(NOP == 2, "two operand stages");
+            uint32_t i_op = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+                for (int c = 0; c < nbK / OP_KB; ++c, ++i_op) {
+                    const int o = i_op & 1;
+                    // the stage's 4 TMEM buffers are free once the last of them is
+                    const uint32_t glast = i_op * OP_KB + OP_KB - 1, buf0 = (i_op * OP_KB) % NTM;
+                    if (!wait_phase(&op_full[o], (i_op / NOP) & 1, abort) ||
+                        !wait_phase(&tm_empty[glast % NTM], ((glast / NTM) & 1) ^ 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint64_t ad = o ? a1 : a0, bd = o ? b1 : b0;
+#pragma unroll
+                    for (int kb = 0; kb < OP_KB; ++kb) {
+                        const uint32_t d = tmem + (buf0 + kb) * TN;
+                        mma_f16(d, ad + (uint64_t)((kb * 2) * (SZ_KSTEP_A >> 4)), bd + (uint64_t)((kb * 2) * (SZ_KSTEP_B >> 4)),
+                                idesc, false);
+                        mma_f16(d, ad + (uint64_t)((kb * 2 + 1) * (SZ_KSTEP_A >> 4)),
+                                bd + (uint64_t)((kb * 2 + 1) * (SZ_KSTEP_B >> 4)), idesc, true);
+                        mma_commit(&tm_full[buf0 + kb]);
+                    }
+                    mma_commit(&op_empty[o]);
+                }
+            }
+            // the last commit's arrival must land before the CTA can exit
+            if (i_op > 0) mbar_wait_bounded(&op_empty[(i_op - 1) % NOP], ((i_op - 1) / NOP) & 1, LIMIT);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                   // TMEM lane quarter this warp may access
+        const int hcol = (warp - W_EPI0) >> 2;    // column half: slots 32 hcol .. 32 hcol + 31
+        const int row = 32 * q + lane;            // weight row (TMEM lane) of this thread
+        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + 32 * hcol;
+        uint32_t gb = 0, epi_phase = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+            const Tile T = tile_of(item, n_rb, tile_off_s, off_s, ngroups);
+            float2 acc[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] = make_float2(0.0f, 0.0f);
+            // two blocks per pass: both TMEM loads in flight before either is used
+            for (int b = 0; b < nbK; b += 2, gb += 2) {
+                const uint32_t b0 = gb % NTM, b1 = b0 + 1, par = (gb / NTM) & 1;
+                const uint32_t s0 = gb % NSC, s1 = s0 + 1, spar = (gb / NSC) & 1;
+                if (!wait_phase(&tm_full[b0], par, abort) || !wait_phase(&sc_full[s0], spar, abort) ||
+                    !wait_phase(&tm_full[b1], par, abort) || !wait_phase(&sc_full[s1], spar, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                uint32_t r0[32], r1[32];
+                tmem_ld32(taddr + b0 * TN, r0);
+                tmem_ld32(taddr + b1 * TN, r1);
+                tmem_wait_ld();
+                rescale_acc(acc, r0, dw_ring[s0 * TM + row], da_ring + s0 * TN + 32 * hcol);
+                rescale_acc(acc, r1, dw_ring[s1 * TM + row], da_ring + s1 * TN + 32 * hcol);
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&tm_empty[b0]);
+                    mbar_arrive(&tm_empty[b1]);
+                    mbar_arrive(&sc_empty[s0]);
+                    mbar_arrive(&sc_empty[s1]);
+                }
+            }
+            if (!ok) break;
+            if (MODE == GATEUP) {
+                float* xr = xch + (size_t)row * XCH_LD + 32 * hcol;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    xr[2 * j] = acc[j].x;
+                    xr[2 * j + 1] = acc[j].y;
+                }
+                if (!epi_sync(&epi_bar, epi_phase++, abort)) break;
+                // 2 Q8_0 blocks of h (gate rows 0..31 and 32..63) x 64 slots,
+                // 16 slots per warp; lane = f within the block
+                const int ew = warp - W_EPI0;
+                const int fb = ew & 1, r0 = 32 * fb + lane;
+                const int f0 = T.rb * 64;
 #pragma unroll 1
-                for (int n = 0; n < TC_N; ++n) {
-                    // all 32 lanes of the warp take every column: the Q8_0
-                    // block of h is the warp's 32 rows
-                    const float h = swiglu(xch[t * 65 + n], xch[(t + 64) * 65 + n]);
-                    uint16_t db;
+                for (int j = 0; j < 16; ++j) {
+                    const int n = (ew >> 1) * 16 + j;
+                    const float h = swiglu(xch[(size_t)r0 * XCH_LD + n], xch[(size_t)(64 + r0) * XCH_LD + n]);
+                    uint16_t dbits;
                     bool ov;
-                    const int q = q8_0_lane(h, db, ov);
-                    if (n < nslots) {
-                        const int s = slot0 + n;
-                        if (p.h_dbg) p.h_dbg[(size_t)s * F + f0 + t] = h;
-                        p.hq[(size_t)s * F + f0 + t] = (int8_t)q;
+                    const int qv = q8_0_lane(h, dbits, ov);
+                    if (n < T.nslots) {
+                        const int s = T.slot0 + n;
+                        if (p.h_dbg) p.h_dbg[(size_t)s * F + f0 + r0] = h;
+                        p.hq[(size_t)s * F + f0 + r0] = (int8_t)qv;
                         if (lane == 0) {
-                            p.dh[(size_t)s * nbF + (f0 >> 5) + warp] = db;
+                            p.dh[(size_t)s * nbF + (f0 >> 5) + fb] = dbits;
                             if (ov) atomicOr(p.status, STATUS_SCALE_OVERFLOW);
                         }
                     }
                 }
-            }
-        } else {
-            const int h0 = rb * TC_M;
+                if (!epi_sync(&epi_bar, epi_phase++, abort)) break;  // xch is free for the next tile
+            } else {
+                int tok = 0;
+                float w = 0.0f;
+                const int n_me = 32 * hcol + lane;
+                if (n_me < T.nslots) slot_info(p, T.g, T.slot0 + n_me, tok, w);
+                const int h0 = T.rb * TM;
 #pragma unroll
-            for (int n = 0; n < TC_N; ++n)
-                if (n < nslots) atomicAdd(p.y + (size_t)tok_s[n] * H + h0 + t, wgt_s[n] * acc[n]);
+                for (int j = 0; j < 32; ++j) {
+                    const int tj = __shfl_sync(0xffffffffu, tok, j);
+                    const float wj = __shfl_sync(0xffffffffu, w, j);
+                    const float v = (j & 1) ? acc[j >> 1].y : acc[j >> 1].x;
+                    if (32 * hcol + j < T.nslots) atomicAdd(p.y + (size_t)tj * H + h0 + row, wj * v);
+                }
+            }
         }
-        __syncthreads();
     }
 
-    if (timed_out) atomicOr(p.status, STATUS_SPIN_TIMEOUT);
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, TC_TMEM_COLS);
+    if (tid == 0 && abort_s) atomicOr(p.status, STATUS_SPIN_TIMEOUT);
+    if (warp == W_PROD) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 static TcParams make_tc_params(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, float* y) {
@@ -322,31 +627,85 @@ static TcParams make_tc_params(const LayerView& L, int64_t T, const Workspace& w
 
 static int64_t tc_max_tiles(const LayerView& L, int64_t T) {
     const int64_t P = T * L.k;
-    return ceil_div(P, TC_N) + std::min<int64_t>(L.E, P) + (L.S ? ceil_div(T, TC_N) : 0);
+    return ceil_div(P, TN) + std::min<int64_t>(L.E, P) + (L.S ? ceil_div(T, TN) : 0);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on the driver library).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// `rows` rows of `row_bytes` bytes at `base` (16-byte aligned, row_bytes a
+// multiple of 16), copied as boxes of `box_rows` rows x 144 bytes.
+static cudaError_t encode_rows(CUtensorMap* map, const uint8_t* base, uint64_t rows, uint64_t row_bytes,
+                               uint32_t box_rows) {
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {row_bytes, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)IN_ROW, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int MODE>
+static cudaError_t make_maps(const LayerView& L, TcMaps* maps) {
+    std::memset(maps, 0, sizeof(TcMaps));
+    const uint64_t E = (uint64_t)L.E, F = (uint64_t)L.F, H = (uint64_t)L.H;
+    cudaError_t e = cudaSuccess;
+    if (MODE == GATEUP) {
+        const uint64_t rb = H / QK * Q4_BYTES;
+        if (e == cudaSuccess) e = encode_rows(&maps->m[0], L.w_gate, E * F, rb, 64);
+        if (e == cudaSuccess) e = encode_rows(&maps->m[1], L.w_up, E * F, rb, 64);
+        if (L.S && e == cudaSuccess) e = encode_rows(&maps->m[2], L.sh_gate, F, rb, 64);
+        if (L.S && e == cudaSuccess) e = encode_rows(&maps->m[3], L.sh_up, F, rb, 64);
+    } else {
+        const uint64_t rb = F / QK * Q4_BYTES;
+        if (e == cudaSuccess) e = encode_rows(&maps->m[0], L.w_down, E * H, rb, TM);
+        if (L.S && e == cudaSuccess) e = encode_rows(&maps->m[2], L.sh_down, H, rb, TM);
+    }
+    return e;
 }
 
 template <int MODE>
 static cudaError_t launch_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, float* y,
                              const DeviceInfo& dev, cudaStream_t s) {
     int per_sm = 0;
-    cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(tc_grouped_kernel<MODE>), TC_THREADS,
-                                     TC_SMEM_TOTAL, &per_sm);
+    cudaError_t e =
+        kernel_occupancy(reinterpret_cast<const void*>(tc_grouped_kernel<MODE>), THREADS, SMEM_ALLOC, &per_sm);
     if (e != cudaSuccess) return e;
-    const int n_rb = (MODE == TC_GATEUP) ? L.F / 64 : L.H / TC_M;
+    TcMaps maps;
+    e = make_maps<MODE>(L, &maps);
+    if (e != cudaSuccess) return e;
+    const int n_rb = (MODE == GATEUP) ? L.F / 64 : L.H / TM;
     const int64_t items = tc_max_tiles(L, T) * n_rb;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, dev.sm_count));
-    tc_grouped_kernel<MODE><<<(unsigned)grid, TC_THREADS, TC_SMEM_TOTAL, s>>>(make_tc_params(L, T, ws, h_dbg, y));
+    tc_grouped_kernel<MODE><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(make_tc_params(L, T, ws, h_dbg, y), maps);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gateup_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, const DeviceInfo& dev,
                              cudaStream_t s) {
-    return launch_tc<TC_GATEUP>(L, T, ws, h_dbg, nullptr, dev, s);
+    return launch_tc<GATEUP>(L, T, ws, h_dbg, nullptr, dev, s);
 }
 
 cudaError_t launch_down_tc(const LayerView& L, int64_t T, const Workspace& ws, float* y, const DeviceInfo& dev,
                            cudaStream_t s) {
-    return launch_tc<TC_DOWN>(L, T, ws, nullptr, y, dev, s);
+    return launch_tc<DOWN>(L, T, ws, nullptr, y, dev, s);
 }
 
 }  // namespace moeq4

@@ -62,7 +62,7 @@ cudaError_t launch_gateup_dp4a(const LayerView& L, int64_t T, const Workspace& w
                                const DeviceInfo& dev, cudaStream_t s);
 cudaError_t launch_down_dp4a(const LayerView& L, int64_t T, const Workspace& ws, float* y,
                              const DeviceInfo& dev, cudaStream_t s);
-// k_tc_grouped.cu: grouped projections on tcgen05 (kind::i8, TMEM); the
+// k_tc_grouped.cu: grouped projections on tcgen05 (kind::f16, TMEM); the
 // permutation must have been built with TC_TILE_TOKENS slots per tile.
 constexpr int TC_TILE_TOKENS = 64;
 cudaError_t launch_gateup_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, const DeviceInfo& dev,

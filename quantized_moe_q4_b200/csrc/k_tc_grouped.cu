@@ -26,17 +26,21 @@
 //   0      producer: 2D tensor copies (TMA) of the packed weight rows (a box
 //          of 64 or 128 rows x 144 B = 8 blocks) and 16-byte cp.async gathers
 //          of the slots' int8 activations and their scales, two input stages;
-//   1..4   converters: nibbles -> binary16 (nib - 8) and int8 -> binary16 into
-//          the K-major operand layout (8-row x 16-byte core matrices), two
-//          operand stages of 4 blocks; block scales into a ring shared with
-//          the epilogue;
-//   5      MMA issuer (one thread): two MMAs per block, one commit per block,
+//   1..4   converters: nibbles -> binary16 (nib - 8) written straight into
+//          TMEM (tcgen05.st; A is read by the MMA from there, so the weight
+//          operand never touches shared memory), int8 -> binary16 activations
+//          into the K-major shared-memory layout (8-row x 16-byte core
+//          matrices); two operand stages of 4 blocks; block scales into a ring
+//          shared with the epilogue;
+//   5      MMA issuer (one thread): two MMAs per block (A from TMEM, B from
+//          shared memory), one commit per block,
 //          descriptors precomputed (the issue path is a handful of instructions);
 //   6..13  epilogue: 4 TMEM lane quarters x 2 column halves; per block one
 //          TMEM load of 32 columns, rescale-accumulate; after the last block of
 //          a tile gate/up -> SwiGLU + Q8_0 requantisation, down ->
 //          y += w_slot * o (fp32 atomics).
-// Eight TMEM buffers of 64 columns and a 16-entry scale ring (so the converters
+// TMEM: six accumulators of 64 columns, then the A ring (2 stages x 4 blocks x
+// 16 columns); a 16-entry scale ring (so the converters
 // run up to four operand stages ahead of the epilogue); full/empty mbarriers between every pair of
 // roles; every wait bounded, and one that runs out makes every role leave its
 // loop and records STATUS_SPIN_TIMEOUT.
@@ -60,12 +64,15 @@ constexpr int TM = 128;            // MMA M: weight rows per tile
 constexpr int TN = TC_TILE_TOKENS; // MMA N: slots per tile
 constexpr int IN_KB = 8;           // Q4_0 blocks per input stage (144-byte rows: a 16-byte multiple)
 constexpr int OP_KB = 4;           // blocks per operand stage
-constexpr int NIN = 2, NOP = 2, NTM = 8, NSC = 16;  // input, operand, TMEM and scale ring depths
+constexpr int NIN = 2, NOP = 2, NTM = 6, NSC = 16;  // input, operand, accumulator and scale ring depths
 constexpr int IN_ROW = IN_KB * Q4_BYTES;          // 144
 constexpr int THREADS = 14 * 32;  // 4 warps on some SM sub-partitions: at most 128 registers a thread
 constexpr int W_PROD = 0, W_CONV0 = 1, W_MMA = 5, W_EPI0 = 6;
 constexpr int N_CONV = 128, N_EPI = 256;
-constexpr uint32_t TMEM_COLS = NTM * TN;          // 512
+constexpr uint32_t A_COL0 = NTM * TN;             // TMEM columns of the A ring (after the accumulators)
+constexpr uint32_t A_COLS_PER_BLOCK = QK / 2;      // 32 binary16 per row = 16 columns
+constexpr uint32_t TMEM_COLS = 512;
+static_assert(A_COL0 + NOP * OP_KB * A_COLS_PER_BLOCK <= TMEM_COLS, "TMEM budget");
 constexpr uint32_t LIMIT = 1u << 22;
 static_assert(TN == 64, "the epilogue maps two warps of 32 columns onto a tile");
 
@@ -73,16 +80,13 @@ static_assert(TN == 64, "the epilogue maps two warps of 32 columns onto a tile")
 constexpr size_t SZ_IN_W = (size_t)TM * IN_ROW;           // one input stage of packed weight rows
 constexpr size_t SZ_IN_B = (size_t)TN * IN_KB * QK;       // int8 activations, [16-byte chunk][slot]
 constexpr size_t SZ_IN_DA = (size_t)TN * IN_KB * 2;       // activation scale bits, [slot][block]
-constexpr size_t SZ_KSTEP_A = (size_t)TM * 32;            // 128 rows x 16 binary16
 constexpr size_t SZ_KSTEP_B = (size_t)TN * 32;
-constexpr size_t SZ_OP_A = (size_t)OP_KB * 2 * SZ_KSTEP_A;
 constexpr size_t SZ_OP_B = (size_t)OP_KB * 2 * SZ_KSTEP_B;
 constexpr int XCH_LD = TN + 1;
 constexpr size_t OFF_IN_W = 0;
 constexpr size_t OFF_IN_B = OFF_IN_W + NIN * SZ_IN_W;
 constexpr size_t OFF_IN_DA = OFF_IN_B + NIN * SZ_IN_B;
-constexpr size_t OFF_OP_A = (OFF_IN_DA + NIN * SZ_IN_DA + 1023) & ~size_t(1023);
-constexpr size_t OFF_OP_B = OFF_OP_A + NOP * SZ_OP_A;
+constexpr size_t OFF_OP_B = (OFF_IN_DA + NIN * SZ_IN_DA + 1023) & ~size_t(1023);
 constexpr size_t OFF_DW = OFF_OP_B + NOP * SZ_OP_B;
 constexpr size_t OFF_DA = OFF_DW + (size_t)NSC * TM * 4;
 constexpr size_t OFF_XCH = OFF_DA + (size_t)NSC * TN * 4;
@@ -176,16 +180,29 @@ __device__ __forceinline__ void rescale_acc(float2 (&acc)[16], const uint32_t (&
     }
 }
 
-// D[tmem] (=|+=) A x B^T, binary16 operands, fp32 accumulator.
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                        bool accumulate) {
+// D[tmem] (=|+=) A[tmem] x B[smem]^T, binary16 operands, fp32 accumulator;
+// A holds row m in TMEM lane m, K along the columns (two binary16 a column).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           bool accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
         : "memory");
 }
+
+// 16 consecutive 32-bit columns of this warp's 32 TMEM lanes (lane = row).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // kind::f16 instruction descriptor: binary16 A and B, fp32 accumulator, both
 // operands K-major, M x N.
@@ -270,7 +287,6 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
     uint8_t* in_w = smem + OFF_IN_W;
     int8_t* in_b = reinterpret_cast<int8_t*>(smem + OFF_IN_B);
     uint16_t* in_da = reinterpret_cast<uint16_t*>(smem + OFF_IN_DA);
-    uint8_t* op_a = smem + OFF_OP_A;
     uint8_t* op_b = smem + OFF_OP_B;
     float* dw_ring = reinterpret_cast<float*>(smem + OFF_DW);
     float* da_ring = reinterpret_cast<float*>(smem + OFF_DA);
@@ -383,7 +399,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
         if (i_in > 0) mbar_wait_bounded(&in_full[(i_in - 1) % NIN], ((i_in - 1) / NIN) & 1, LIMIT);
     } else if (warp >= W_CONV0 && warp < W_CONV0 + 4) {
         // ------------------------------------------------------------ converters
-        const int ct = tid - W_CONV0 * 32;  // weight row of this thread; slot column ct & 63
+        const int ct = tid - W_CONV0 * 32;        // slot column ct & 63 of the activation work
+        const int crow = 32 * (warp & 3) + lane;  // weight row = the TMEM lane this warp may write
         uint32_t i_op = 0, gb = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -394,12 +411,13 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                 if (sub == 0 && !wait_phase(&in_full[s], (i_in / NIN) & 1, abort)) { ok = false; break; }
                 const int o = i_op % NOP;
                 if (!wait_phase(&op_empty[o], ((i_op / NOP) & 1) ^ 1, abort)) { ok = false; break; }
-                uint8_t* oa = op_a + (size_t)o * SZ_OP_A;
+                tc_fence_after_sync();
+                const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + A_COL0 + o * OP_KB * A_COLS_PER_BLOCK;
                 uint8_t* ob = op_b + (size_t)o * SZ_OP_B;
 
                 // weights: this row's 4 blocks, 72 bytes at an 8-byte boundary
                 uint32_t w[18];
-                const uint2* wsrc = reinterpret_cast<const uint2*>(in_w + (size_t)s * SZ_IN_W + (size_t)ct * IN_ROW +
+                const uint2* wsrc = reinterpret_cast<const uint2*>(in_w + (size_t)s * SZ_IN_W + (size_t)crow * IN_ROW +
                                                                    sub * OP_KB * Q4_BYTES);
 #pragma unroll
                 for (int i = 0; i < 9; ++i) {
@@ -423,16 +441,18 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                         for (int i = 0; i < 4; ++i) qs[i] = w[bw + 1 + i];
                     }
                     dws[kb] = half_bits_to_float(dbits);
+                    // columns 0..7: low nibbles (weights 0..15), 8..15: high nibbles (16..31)
+                    uint32_t v[16];
 #pragma unroll
-                    for (int core = 0; core < 2; ++core) {
-                        // K-step 0: low nibbles (weights 0..15); K-step 1: high nibbles (16..31)
-                        const uint2 l0 = bytes_to_f16(qs[2 * core] & 0x0f0f0f0fu, BIAS_NIB);
-                        const uint2 l1 = bytes_to_f16(qs[2 * core + 1] & 0x0f0f0f0fu, BIAS_NIB);
-                        const uint2 h0 = bytes_to_f16((qs[2 * core] >> 4) & 0x0f0f0f0fu, BIAS_NIB);
-                        const uint2 h1 = bytes_to_f16((qs[2 * core + 1] >> 4) & 0x0f0f0f0fu, BIAS_NIB);
-                        *reinterpret_cast<uint4*>(oa + op_off(kb, 0, TM, ct, core)) = make_uint4(l0.x, l0.y, l1.x, l1.y);
-                        *reinterpret_cast<uint4*>(oa + op_off(kb, 1, TM, ct, core)) = make_uint4(h0.x, h0.y, h1.x, h1.y);
+                    for (int i = 0; i < 4; ++i) {
+                        const uint2 lo = bytes_to_f16(qs[i] & 0x0f0f0f0fu, BIAS_NIB);
+                        const uint2 hi = bytes_to_f16((qs[i] >> 4) & 0x0f0f0f0fu, BIAS_NIB);
+                        v[2 * i] = lo.x;
+                        v[2 * i + 1] = lo.y;
+                        v[8 + 2 * i] = hi.x;
+                        v[8 + 2 * i + 1] = hi.y;
                     }
+                    tmem_st16(ta + kb * A_COLS_PER_BLOCK, v);
                 }
                 // activations: slot n = ct & 63, blocks (ct >> 6) and (ct >> 6) + 2
                 const int n = ct & 63;
@@ -464,7 +484,9 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                 for (int kb = 0; kb < OP_KB; ++kb)
                     das[kb] = valid ? half_bits_to_float(in_da[(size_t)s * TN * IN_KB + n * IN_KB + sub * OP_KB + kb])
                                     : 0.0f;
+                tmem_wait_st();
                 fence_proxy_async_smem();
+                tc_fence_before_sync();
                 mbar_arrive(&op_full[o]);
                 if (sub == 1) mbar_arrive(&in_empty[s]);
                 // scales of these 4 blocks into the ring read by the epilogue; the
@@ -474,7 +496,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                 if (!wait_phase(&sc_empty[glast % NSC], ((glast / NSC) & 1) ^ 1, abort)) { ok = false; break; }
 #pragma unroll
                 for (int kb = 0; kb < OP_KB; ++kb) {
-                    dw_ring[(buf0 + kb) * TM + ct] = dws[kb];
+                    dw_ring[(buf0 + kb) * TM + crow] = dws[kb];
                     if (ct < TN) da_ring[(buf0 + kb) * TN + ct] = das[kb];
                 }
                 __syncwarp();
@@ -490,7 +512,6 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
             constexpr uint32_t idesc = idesc_f16(TM, TN);
             // descriptors of the first K-step of each operand stage; a later
             // K-step adds its byte offset / 16 to the start-address field
-            const uint64_t a0 = smem_desc_kmajor(op_a, 128, 256), a1 = smem_desc_kmajor(op_a + SZ_OP_A, 128, 256);
             const uint64_t b0 = smem_desc_kmajor(op_b, 128, 256), b1 = smem_desc_kmajor(op_b + SZ_OP_B, 128, 256);
             static_assert(NOP == 2, "two operand stages");
             uint32_t i_op = 0;
@@ -498,25 +519,31 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 for (int c = 0; c < nbK / OP_KB; ++c, ++i_op) {
                     const int o = i_op & 1;
-                    // the stage's 4 TMEM buffers are free once the last of them is
-                    const uint32_t glast = i_op * OP_KB + OP_KB - 1, buf0 = (i_op * OP_KB) % NTM;
-                    if (!wait_phase(&op_full[o], (i_op / NOP) & 1, abort) ||
-                        !wait_phase(&tm_empty[glast % NTM], ((glast / NTM) & 1) ^ 1, abort)) {
+                    const uint32_t g0 = i_op * OP_KB;
+                    if (!wait_phase(&op_full[o], (i_op / NOP) & 1, abort)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after_sync();
-                    const uint64_t ad = o ? a1 : a0, bd = o ? b1 : b0;
+                    const uint64_t bd = o ? b1 : b0;
+                    const uint32_t ta = tmem + A_COL0 + o * OP_KB * A_COLS_PER_BLOCK;
 #pragma unroll
                     for (int kb = 0; kb < OP_KB; ++kb) {
-                        const uint32_t d = tmem + (buf0 + kb) * TN;
-                        mma_f16(d, ad + (uint64_t)((kb * 2) * (SZ_KSTEP_A >> 4)), bd + (uint64_t)((kb * 2) * (SZ_KSTEP_B >> 4)),
-                                idesc, false);
-                        mma_f16(d, ad + (uint64_t)((kb * 2 + 1) * (SZ_KSTEP_A >> 4)),
-                                bd + (uint64_t)((kb * 2 + 1) * (SZ_KSTEP_B >> 4)), idesc, true);
-                        mma_commit(&tm_full[buf0 + kb]);
+                        // each block waits only for its own accumulator
+                        const uint32_t g = g0 + kb, buf = g % NTM;
+                        if (!wait_phase(&tm_empty[buf], ((g / NTM) & 1) ^ 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        const uint32_t d = tmem + buf * TN;
+                        mma_f16_ts(d, ta + kb * A_COLS_PER_BLOCK, bd + (uint64_t)((kb * 2) * (SZ_KSTEP_B >> 4)), idesc,
+                                   false);
+                        mma_f16_ts(d, ta + kb * A_COLS_PER_BLOCK + A_COLS_PER_BLOCK / 2,
+                                   bd + (uint64_t)((kb * 2 + 1) * (SZ_KSTEP_B >> 4)), idesc, true);
+                        mma_commit(&tm_full[buf]);
                     }
                     mma_commit(&op_empty[o]);
+                    if (!ok) break;
                 }
             }
             // the last commit's arrival must land before the CTA can exit
@@ -537,6 +564,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
             for (int j = 0; j < 16; ++j) acc[j] = make_float2(0.0f, 0.0f);
             // two blocks per pass: both TMEM loads in flight before either is used
             for (int b = 0; b < nbK; b += 2, gb += 2) {
+                static_assert(NTM % 2 == 0, "pairs of accumulators never wrap");
                 const uint32_t b0 = gb % NTM, b1 = b0 + 1, par = (gb / NTM) & 1;
                 const uint32_t s0 = gb % NSC, s1 = s0 + 1, spar = (gb / NSC) & 1;
                 if (!wait_phase(&tm_full[b0], par, abort) || !wait_phase(&sc_full[s0], spar, abort) ||

@@ -25,7 +25,8 @@
 // Warp roles (14 warps):
 //   0      producer: 2D tensor copies (TMA) of the packed weight rows (a box
 //          of 64 or 128 rows x 144 B = 8 blocks) and 16-byte cp.async gathers
-//          of the slots' int8 activations and their scales, two input stages;
+//          of the slots' int8 activations and their scales, four input stages
+//          in flight (a stage takes about 2 us to land under load);
 //   1..4   converters: nibbles -> binary16 (nib - 8) written straight into
 //          TMEM (tcgen05.st; A is read by the MMA from there, so the weight
 //          operand never touches shared memory), int8 -> binary16 activations
@@ -64,7 +65,7 @@ constexpr int TM = 128;            // MMA M: weight rows per tile
 constexpr int TN = TC_TILE_TOKENS; // MMA N: slots per tile
 constexpr int IN_KB = 8;           // Q4_0 blocks per input stage (144-byte rows: a 16-byte multiple)
 constexpr int OP_KB = 4;           // blocks per operand stage
-constexpr int NIN = 2, NOP = 2, NTM = 6, NSC = 16;  // input, operand, accumulator and scale ring depths
+constexpr int NIN = 4, NOP = 2, NTM = 6, NSC = 16;  // input, operand, accumulator and scale ring depths
 constexpr int IN_ROW = IN_KB * Q4_BYTES;          // 144
 constexpr int THREADS = 14 * 32;  // 4 warps on some SM sub-partitions: at most 128 registers a thread
 constexpr int W_PROD = 0, W_CONV0 = 1, W_MMA = 5, W_EPI0 = 6;
@@ -597,26 +598,43 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                     xr[2 * j + 1] = acc[j].y;
                 }
                 if (!epi_sync(&epi_bar, epi_phase++, abort)) break;
-                // 2 Q8_0 blocks of h (gate rows 0..31 and 32..63) x 64 slots,
-                // 16 slots per warp; lane = f within the block
-                const int ew = warp - W_EPI0;
-                const int fb = ew & 1, r0 = 32 * fb + lane;
+                // SwiGLU + Q8_0 of h.  A unit is one 32-row block of h (gate rows
+                // 32 fb .. 32 fb + 31) of one slot n; two lanes share a unit, 16
+                // rows each, so every value is independent of the others and a
+                // single shuffle gives the block's absolute maximum.  Both
+                // divisions of the Q8_0 rule stay IEEE (div.rn).
+                const int u = ((warp - W_EPI0) * 32 + lane) >> 1;   // 0..127
+                const int n = u & 63, fb = u >> 6, half = lane & 1;
+                const int r0 = 32 * fb + 16 * half;
                 const int f0 = T.rb * 64;
-#pragma unroll 1
+                float h[16];
+                float amax = 0.0f;
+#pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const int n = (ew >> 1) * 16 + j;
-                    const float h = swiglu(xch[(size_t)r0 * XCH_LD + n], xch[(size_t)(64 + r0) * XCH_LD + n]);
-                    uint16_t dbits;
-                    bool ov;
-                    const int qv = q8_0_lane(h, dbits, ov);
-                    if (n < T.nslots) {
-                        const int s = T.slot0 + n;
-                        if (p.h_dbg) p.h_dbg[(size_t)s * F + f0 + r0] = h;
-                        p.hq[(size_t)s * F + f0 + r0] = (int8_t)qv;
-                        if (lane == 0) {
-                            p.dh[(size_t)s * nbF + (f0 >> 5) + fb] = dbits;
-                            if (ov) atomicOr(p.status, STATUS_SCALE_OVERFLOW);
-                        }
+                    h[j] = swiglu(xch[(size_t)(r0 + j) * XCH_LD + n], xch[(size_t)(64 + r0 + j) * XCH_LD + n]);
+                    amax = fmaxf(amax, fabsf(h[j]));
+                }
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                const float d = __fdiv_rn(amax, 127.0f);
+                const uint16_t dbits = __half_as_ushort(__float2half_rn(d));
+                uint32_t packed[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    int qv = 0;
+                    if (d != 0.0f) qv = max(-127, min(127, round_half_away(__fdiv_rn(h[j], d))));
+                    packed[j >> 2] |= (uint32_t)(qv & 0xff) << (8 * (j & 3));
+                }
+                if (n < T.nslots) {
+                    const int sl = T.slot0 + n;
+                    *reinterpret_cast<uint4*>(p.hq + (size_t)sl * F + f0 + r0) =
+                        make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                    if (p.h_dbg) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) p.h_dbg[(size_t)sl * F + f0 + r0 + j] = h[j];
+                    }
+                    if (half == 0) {
+                        p.dh[(size_t)sl * nbF + (f0 >> 5) + fb] = dbits;
+                        if ((dbits & 0x7fffu) == 0x7c00u) atomicOr(p.status, STATUS_SCALE_OVERFLOW);
                     }
                 }
                 if (!epi_sync(&epi_bar, epi_phase++, abort)) break;  // xch is free for the next tile

@@ -57,6 +57,8 @@ def _load():
         lib.orc_permute.argtypes = [P, i64, i32, i32, P, P, P, P]
         lib.orc_moe_forward.argtypes = [P, P, i64, P, P, P, P, P, P]
         lib.orc_moe_forward.restype = ctypes.c_int
+        lib.orc_rmsnorm.argtypes = [P, i64, i32, ctypes.c_float, P]
+        lib.orc_residual_add.argtypes = [P, P, i64]
         lib.orc_set_threads.argtypes = [i32]
         lib.orc_set_threads.restype = ctypes.c_int
         _lib = lib
@@ -247,3 +249,33 @@ def moe_forward(layer, x: np.ndarray, *, forced_idx=None, forced_w=None, forced_
             arrays["logits"] = None
         return y, arrays
     return y
+
+
+# ---------------------------------------------------------------- stack glue
+
+
+def rmsnorm(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """Unit-gain RMSNorm of each row (the stack's reading of the inter-layer
+    glue): mean of squares in binary64, xn = binary32(x / sqrt(mean + eps))."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    T, H = x.shape
+    out = np.empty_like(x)
+    _load().orc_rmsnorm(_ptr(x), T, H, float(eps), _ptr(out))
+    return out
+
+
+def residual_add(x: np.ndarray, y: np.ndarray) -> np.ndarray:
+    """binary32(x + y), the exact sum rounded once."""
+    out = np.array(x, dtype=np.float32, order="C", copy=True)
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    assert y.shape == out.shape
+    _load().orc_residual_add(_ptr(out), _ptr(y), out.size)
+    return out
+
+
+def stack_forward(layers, x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """x_{l+1} = x_l + MoE_l(RMSNorm(x_l)) through `layers` (free running)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    for lw in layers:
+        x = residual_add(x, moe_forward(lw, rmsnorm(x, eps)))
+    return x

@@ -375,6 +375,33 @@ int orc_moe_forward(const orc_layer* L, const float* x, int64_t T, float* y,
     return 0;
 }
 
+/* ------------------------------------------------------------------ */
+/* Glue between the layers of a stack                                  */
+/* ------------------------------------------------------------------ */
+
+/* The page runs the MoE layers one after another (Methodologie 1: expert
+ * weights are streamed layer by layer) but fixes no step between them; the
+ * multi-layer workload joins them by a residual add.  Without a normalisation
+ * the activations grow by about 25x per layer and the binary16 Q8_0 scales
+ * overflow within a few layers, so the reading taken is
+ * x_{l+1} = x_l + MoE_l(RMSNorm(x_l)) with a unit-gain RMSNorm over H:
+ * rms = sqrt(mean_h x^2 + eps), the mean taken in binary64;
+ * xn = binary32(x / rms). */
+void orc_rmsnorm(const float* x, int64_t T, int H, float eps, float* xn) {
+    for (int64_t t = 0; t < T; ++t) {
+        const float* r = x + t * H;
+        double ss = 0.0;
+        for (int h = 0; h < H; ++h) ss += (double)r[h] * (double)r[h];
+        const double rms = sqrt(ss / (double)H + (double)eps);
+        for (int h = 0; h < H; ++h) xn[t * H + h] = (float)((double)r[h] / rms);
+    }
+}
+
+/* x <- binary32(x + y): the exact sum rounded once. */
+void orc_residual_add(float* x, const float* y, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) x[i] = (float)((double)x[i] + (double)y[i]);
+}
+
 /* Thread count used by the OpenMP loops (timing only); returns the count. */
 int orc_set_threads(int n) {
 #ifdef _OPENMP

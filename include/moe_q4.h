@@ -154,6 +154,41 @@ int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t 
 int moe_q4_ffn_forward_noalloc(const moe_q4_layer* L, const float* x, int64_t T, float* y,
                                moe_q4_stream_t stream);
 
+/* ---------------------------------------------------------------------
+ * Stacks of layers.
+ *
+ * The page runs the MoE layers one after another (Methodologie 1: expert
+ * weights are streamed layer by layer) but fixes no step between them.  The
+ * multi-layer workload joins them by a residual add; without a normalisation
+ * the activations grow by about 25x per layer and the binary16 Q8_0 scales
+ * overflow within a few layers.  The step taken between layers is
+ *     x_{l+1} = x_l + MoE_l(RMSNorm(x_l)),
+ * RMSNorm with unit gain over H: rms = sqrt(mean_h x^2 + eps) with the mean
+ * of squares accumulated in binary64, xn = binary32(x / rms) (binary64
+ * division, one rounding).
+ * --------------------------------------------------------------------- */
+
+/* x [T][H] fp32 (in place), y [T][H] fp32 or NULL, xn [T][H] fp32 or NULL:
+ *   if y: x <- binary32(x + y);  then if xn: xn = RMSNorm(x).
+ * H a positive multiple of 256, eps finite and >= 0, 0 <= T <= 2^24;
+ * 16-byte aligned pointers; xn must not overlap x or y (x and y must not
+ * overlap either).  Returns MOE_Q4_OK or an error code; T == 0 is a no-op. */
+int moe_q4_residual_rmsnorm(float* x, const float* y, int64_t T, int32_t H, float eps, float* xn,
+                            moe_q4_stream_t stream);
+
+/* Workspace of moe_q4_stack_forward for layers shaped like *L and up to T_max
+ * tokens: RMSNorm output and layer output [T_max][H] fp32 each, then one layer
+ * workspace.  0 for an invalid layer or T_max. */
+size_t moe_q4_stack_workspace_bytes(const moe_q4_layer* L, int64_t T_max);
+
+/* n_layers >= 1 layers (an array of descriptors, all with the same hidden,
+ * ffn, n_experts, top_k and has_shared) applied in order to x [T][H] fp32 in
+ * place: for each layer, x <- x + MoE_l(RMSNorm(x)).  Same conventions and
+ * errors as moe_q4_ffn_forward; MOE_Q4_ERR_SHAPE if the layers differ in
+ * shape.  The device status word of the workspace accumulates over layers. */
+int moe_q4_stack_forward(const moe_q4_layer* layers, int32_t n_layers, float* x, int64_t T, float eps,
+                         void* workspace, size_t ws_bytes, moe_q4_stream_t stream);
+
 /* Static description of an error code. */
 const char* moe_q4_status_string(int status);
 

@@ -42,7 +42,8 @@ WS_NAMES = ["status", "logits", "topk_idx", "topk_w", "qa", "da", "cnt", "off", 
 EXPORTS = ["moe_q4_quantize_act", "moe_q4_route", "moe_q4_ffn_workspace_bytes", "moe_q4_ffn_forward",
            "moe_q4_ffn_host_workspace_bytes", "moe_q4_ffn_forward_host", "moe_q4_status_string",
            "moe_q4_workspace_layout", "moe_q4_ffn_forward_debug", "moe_q4_block_dots",
-           "moe_q4_ffn_forward_noalloc", "moe_q4_last_cuda_error"]
+           "moe_q4_ffn_forward_noalloc", "moe_q4_last_cuda_error", "moe_q4_residual_rmsnorm",
+           "moe_q4_stack_workspace_bytes", "moe_q4_stack_forward"]
 
 
 class MoeQ4Error(RuntimeError):
@@ -89,6 +90,9 @@ def _load() -> ctypes.CDLL:
         "moe_q4_block_dots": ([P, P, i64, P, P], ctypes.c_int),
         "moe_q4_ffn_forward_noalloc": ([P, P, i64, P, P], ctypes.c_int),
         "moe_q4_last_cuda_error": ([], ctypes.c_char_p),
+        "moe_q4_residual_rmsnorm": ([P, P, i64, i32, ctypes.c_float, P, P], ctypes.c_int),
+        "moe_q4_stack_workspace_bytes": ([P, i64], sz),
+        "moe_q4_stack_forward": ([P, i32, P, i64, ctypes.c_float, P, sz, P], ctypes.c_int),
     }
     for name, (args, res) in sigs.items():
         f = getattr(lib, name)
@@ -275,3 +279,30 @@ def moe_q4_ffn_forward_noalloc(layer: Layer, x: torch.Tensor, y=None, stream=Non
     _check(_lib.moe_q4_ffn_forward_noalloc(layer.ref, _p(x), T, _p(y), _stream(stream)),
            "moe_q4_ffn_forward_noalloc")
     return y
+
+
+# ---------------------------------------------------------------- stacks of layers
+
+def moe_q4_residual_rmsnorm(x: torch.Tensor, y=None, eps: float = 1e-6, xn=None, stream=None):
+    """x <- x + y (if y is given, in place), then returns xn = RMSNorm(x) (unit
+    gain over the last dimension), written into `xn` if given."""
+    T, H = x.shape
+    xn = torch.empty_like(x) if xn is None else xn
+    _check(_lib.moe_q4_residual_rmsnorm(_p(x), _p(y), T, H, float(eps), _p(xn), _stream(stream)),
+           "moe_q4_residual_rmsnorm")
+    return xn
+
+
+def moe_q4_stack_workspace_bytes(layer: Layer, T_max: int) -> int:
+    return int(_lib.moe_q4_stack_workspace_bytes(layer.ref, int(T_max)))
+
+
+def moe_q4_stack_forward(layers, x: torch.Tensor, eps: float = 1e-6, workspace=None, stream=None):
+    """x <- x + MoE_l(RMSNorm(x)) for every layer in order, in place on x."""
+    T = x.shape[0]
+    arr = (_Layer * len(layers))(*[l.struct for l in layers])
+    if workspace is None:
+        workspace = alloc_workspace(moe_q4_stack_workspace_bytes(layers[0], T), x.device)
+    _check(_lib.moe_q4_stack_forward(arr, len(layers), _p(x), T, float(eps), _p(workspace), workspace.numel(),
+                                     _stream(stream)), "moe_q4_stack_forward")
+    return x

@@ -1,6 +1,7 @@
 // abi.cu -- the extern "C" entry points of include/moe_q4.h: argument checks,
 // workspace layout, kernel-family dispatch.  No allocation, no host sync.
 #include <algorithm>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
@@ -363,6 +364,66 @@ int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t 
     if (rc) return rc;
     MOE_TRY(cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, s));
     return MOE_Q4_OK;
+}
+
+int moe_q4_residual_rmsnorm(float* x, const float* y, int64_t T, int32_t H, float eps, float* xn,
+                            moe_q4_stream_t stream) {
+    if (T < 0 || T > T_LIMIT || H <= 0 || H % 256 || !(eps >= 0.0f) || !(eps < INFINITY))
+        return MOE_Q4_ERR_INVALID_ARG;
+    if (T == 0) return MOE_Q4_OK;
+    if (!x) return MOE_Q4_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || (y && !aligned(y, 16)) || (xn && !aligned(xn, 16))) return MOE_Q4_ERR_ALIGN;
+    const size_t bytes = sizeof(float) * (size_t)T * (size_t)H;
+    if ((y && overlap(x, bytes, y, bytes)) || (xn && overlap(x, bytes, xn, bytes)) ||
+        (xn && y && overlap(y, bytes, xn, bytes)))
+        return MOE_Q4_ERR_OVERLAP;
+    DeviceInfo dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    return cuda_rc(launch_residual_rmsnorm(x, y, T, H, eps, xn, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_q4_stack_workspace_bytes(const moe_q4_layer* L, int64_t T_max) {
+    const size_t base = moe_q4_ffn_workspace_bytes(L, T_max);
+    if (!base) return 0;
+    const size_t xy = align256(sizeof(float) * (size_t)(std::max<int64_t>(T_max, 1) * L->hidden));
+    return 2 * xy + base;
+}
+
+int moe_q4_stack_forward(const moe_q4_layer* layers, int32_t n_layers, float* x, int64_t T, float eps,
+                         void* workspace, size_t ws_bytes, moe_q4_stream_t stream) {
+    if (!layers || n_layers < 1 || !(eps >= 0.0f) || !(eps < INFINITY)) return MOE_Q4_ERR_INVALID_ARG;
+    for (int32_t l = 0; l < n_layers; ++l) {
+        const int rc = check_layer(&layers[l]);
+        if (rc) return rc;
+        const moe_q4_layer& a = layers[0];
+        const moe_q4_layer& b = layers[l];
+        if (a.hidden != b.hidden || a.ffn != b.ffn || a.n_experts != b.n_experts || a.top_k != b.top_k ||
+            (a.has_shared != 0) != (b.has_shared != 0))
+            return MOE_Q4_ERR_SHAPE;
+    }
+    if (T < 0 || T > T_LIMIT) return MOE_Q4_ERR_INVALID_ARG;
+    if (T == 0) return MOE_Q4_OK;
+    if (!x || !workspace) return MOE_Q4_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(workspace, 256)) return MOE_Q4_ERR_ALIGN;
+    const int32_t H = layers[0].hidden;
+    const size_t xy = align256(sizeof(float) * (size_t)(T * H));
+    size_t off[WS_COUNT];
+    layout(view(&layers[0]), T, off);
+    if (ws_bytes < 2 * xy + off[WS_TOTAL]) return MOE_Q4_ERR_WORKSPACE;
+    if (overlap(x, sizeof(float) * (size_t)(T * H), workspace, 2 * xy + off[WS_TOTAL])) return MOE_Q4_ERR_OVERLAP;
+    char* base = static_cast<char*>(workspace);
+    float* xn = reinterpret_cast<float*>(base);
+    float* y = reinterpret_cast<float*>(base + xy);
+    void* lws = base + 2 * xy;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    for (int32_t l = 0; l < n_layers; ++l) {
+        int rc = moe_q4_residual_rmsnorm(x, l ? y : nullptr, T, H, eps, xn, stream);
+        if (rc) return rc;
+        rc = forward_impl(&layers[l], xn, T, y, lws, off[WS_TOTAL], nullptr, s);
+        if (rc) return rc;
+    }
+    return moe_q4_residual_rmsnorm(x, y, T, H, eps, nullptr, stream);
 }
 
 int moe_q4_block_dots(const uint8_t* w_blocks, const int8_t* qa, int64_t n, int32_t* out, moe_q4_stream_t stream) {

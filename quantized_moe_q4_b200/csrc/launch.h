@@ -80,6 +80,10 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
 cudaError_t launch_block_dots(const uint8_t* w, const int8_t* qa, int64_t n, int32_t* out,
                               cudaStream_t s);
 
+// k_stack.cu: x += y (if y), then xn = RMSNorm(x) (if xn); H a multiple of 128.
+cudaError_t launch_residual_rmsnorm(float* x, const float* y, int64_t T, int H, float eps, float* xn,
+                                    cudaStream_t s);
+
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Resident CTAs per SM of `kernel` at `threads` and `smem` dynamic bytes, with

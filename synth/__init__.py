@@ -126,6 +126,13 @@ def stack_layer(layer_index: int, H: int, F: int, E: int, k: int, shared: bool, 
     return make_layer(rng, H, F, E, k, shared, None)
 
 
+def stack_inputs(T: int, H: int, seed: int = 0) -> np.ndarray:
+    """Input activations x [T,H] of a multi-layer stack (first draw of
+    PCG64(seed); the layers come from stack_layer)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return rng.standard_normal((T, H), dtype=np.float32)
+
+
 def random_layer(seed: int, H: int, F: int, E: int, k: int, shared: bool, zipf=None, T: int = 1):
     """Small random case for property tests: same recipe, any shape."""
     return make_inputs(T, H, F, E, k, shared, zipf, seed)

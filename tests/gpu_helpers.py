@@ -25,11 +25,12 @@ def device_layer(lw):
     return _CACHE[key][1]
 
 
-def run_forward(lw, x_np, path=0, want_h=True):
+def run_forward(lw, x_np, path=0, want_h=True, L=None):
     """One forward on the device; returns numpy copies of y, h and the
-    workspace intermediates (slot-ordered)."""
+    workspace intermediates (slot-ordered).  `L`: the layer's device copy
+    (default: a cached upload of lw)."""
     import quantized_moe_q4_b200 as m
-    L = device_layer(lw)
+    L = device_layer(lw) if L is None else L
     x = torch.from_numpy(np.ascontiguousarray(x_np)).cuda()
     T = x.shape[0]
     y = torch.empty_like(x)

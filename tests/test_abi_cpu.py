@@ -147,6 +147,43 @@ def test_other_entry_points_reject_bad_args(lib):
     assert d(ctypes.byref(L), FAKE, 4, FAKE + 0x1000000, FAKE + 0x2000000, 1 << 40, ctypes.byref(dbg), None) == -1
 
 
+def test_stack_entry_points_reject_bad_args(lib):
+    n = lib.moe_q4_residual_rmsnorm
+    n.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float,
+                  ctypes.c_void_p, ctypes.c_void_p]
+    X, Y, XN = FAKE, FAKE + 0x1000000, FAKE + 0x2000000
+    assert n(X, Y, 4, 2000, 1e-6, XN, None) == -1            # H not a multiple of 256
+    assert n(X, Y, 4, 2048, -1.0, XN, None) == -1            # negative eps
+    assert n(X, Y, 4, 2048, float("nan"), XN, None) == -1
+    assert n(None, Y, 4, 2048, 1e-6, XN, None) == -1
+    assert n(X + 4, Y, 4, 2048, 1e-6, XN, None) == -3
+    assert n(X, Y, 4, 2048, 1e-6, X + 4096, None) == -7      # xn overlaps x
+    assert n(X, X, 4, 2048, 1e-6, XN, None) == -7            # y is x
+    assert n(X, None, 0, 2048, 1e-6, None, None) == 0        # T == 0: no-op
+    wb = lib.moe_q4_stack_workspace_bytes
+    wb.argtypes, wb.restype = [ctypes.c_void_p, ctypes.c_int64], ctypes.c_size_t
+    lib.moe_q4_ffn_workspace_bytes.argtypes = [ctypes.c_void_p, ctypes.c_int64]
+    lib.moe_q4_ffn_workspace_bytes.restype = ctypes.c_size_t
+    L = make()
+    assert wb(ctypes.byref(L), 64) == lib.moe_q4_ffn_workspace_bytes(ctypes.byref(L), 64) + 2 * 64 * 2048 * 4
+    assert wb(ctypes.byref(make(top_k=0)), 64) == 0
+    f = lib.moe_q4_stack_forward
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64, ctypes.c_float,
+                  ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    arr = (_L * 3)(make(), make(), make())
+    WS = FAKE + 0x10000000
+    assert f(arr, 0, X, 4, 1e-6, WS, 1 << 40, None) == -1      # no layers
+    assert f(None, 3, X, 4, 1e-6, WS, 1 << 40, None) == -1
+    bad = (_L * 3)(make(), make(ffn=768), make())
+    assert f(bad, 3, X, 4, 1e-6, WS, 1 << 40, None) == -2      # layers differ in shape
+    bad = (_L * 2)(make(), make(top_k=0))
+    assert f(bad, 2, X, 4, 1e-6, WS, 1 << 40, None) == -1      # an invalid layer
+    assert f(arr, 3, X, 4, 1e-6, WS, 1000, None) == -4
+    assert f(arr, 3, X + 8, 4, 1e-6, WS, 1 << 40, None) == -3
+    assert f(arr, 3, WS, 4, 1e-6, WS, 1 << 40, None) == -7     # x inside the workspace
+    assert f(arr, 3, X, 0, 1e-6, WS, 1 << 40, None) == 0       # T == 0: no-op
+
+
 def test_product_package_does_not_use_the_oracle():
     pkg = os.path.join(ROOT, "quantized_moe_q4_b200")
     for dirpath, _, files in os.walk(pkg):

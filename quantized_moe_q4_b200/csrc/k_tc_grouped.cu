@@ -193,13 +193,22 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
         : "memory");
 }
 
-// 16 consecutive 32-bit columns of this warp's 32 TMEM lanes (lane = row).
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+// 64 consecutive 32-bit columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&v)[64]) {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
-        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,"
+        "%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
+        "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31]), "r"(v[32]),
+        "r"(v[33]), "r"(v[34]), "r"(v[35]), "r"(v[36]), "r"(v[37]), "r"(v[38]), "r"(v[39]), "r"(v[40]),
+        "r"(v[41]), "r"(v[42]), "r"(v[43]), "r"(v[44]), "r"(v[45]), "r"(v[46]), "r"(v[47]), "r"(v[48]),
+        "r"(v[49]), "r"(v[50]), "r"(v[51]), "r"(v[52]), "r"(v[53]), "r"(v[54]), "r"(v[55]), "r"(v[56]),
+        "r"(v[57]), "r"(v[58]), "r"(v[59]), "r"(v[60]), "r"(v[61]), "r"(v[62]), "r"(v[63])
         : "memory");
 }
 
@@ -427,6 +436,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                     w[2 * i + 1] = v.y;
                 }
                 float dws[OP_KB];
+                uint32_t v[OP_KB * 16];  // the 4 blocks' binary16 pairs, 64 consecutive TMEM columns
 #pragma unroll
                 for (int kb = 0; kb < OP_KB; ++kb) {
                     // block kb starts at byte 18 kb: scale, then 16 nibble bytes
@@ -442,19 +452,20 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                         for (int i = 0; i < 4; ++i) qs[i] = w[bw + 1 + i];
                     }
                     dws[kb] = half_bits_to_float(dbits);
-                    // columns 0..7: low nibbles (weights 0..15), 8..15: high nibbles (16..31)
-                    uint32_t v[16];
+                    // columns 0..7 of a block: low nibbles (weights 0..15), 8..15: high nibbles (16..31)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const uint2 lo = bytes_to_f16(qs[i] & 0x0f0f0f0fu, BIAS_NIB);
                         const uint2 hi = bytes_to_f16((qs[i] >> 4) & 0x0f0f0f0fu, BIAS_NIB);
-                        v[2 * i] = lo.x;
-                        v[2 * i + 1] = lo.y;
-                        v[8 + 2 * i] = hi.x;
-                        v[8 + 2 * i + 1] = hi.y;
+                        v[16 * kb + 2 * i] = lo.x;
+                        v[16 * kb + 2 * i + 1] = lo.y;
+                        v[16 * kb + 8 + 2 * i] = hi.x;
+                        v[16 * kb + 8 + 2 * i + 1] = hi.y;
                     }
-                    tmem_st16(ta + kb * A_COLS_PER_BLOCK, v);
                 }
+                // one asynchronous TMEM store of all four blocks; the activation
+                // work below overlaps it, tcgen05.wait::st before the hand-off
+                tmem_st64(ta, v);
                 // activations: slot n = ct & 63, blocks (ct >> 6) and (ct >> 6) + 2
                 const int n = ct & 63;
                 const bool valid = n < T.nslots;

@@ -344,7 +344,8 @@ def run_ours(args):
 
     x_np, lw = synth.workload_inputs(WORKLOAD, seed=0, T=N_TOKENS)
     base = m.Layer.from_host(lw)
-    layers = [base] + [base.replica() for _ in range(REPLICAS - 1)]
+    replicas = args.replicas
+    layers = [base] + [base.replica() for _ in range(replicas - 1)]
     H, F, E, k = lw.hidden, lw.ffn, lw.n_experts, lw.top_k
     x = torch.from_numpy(x_np).cuda()
     y = torch.empty_like(x)
@@ -356,7 +357,7 @@ def run_ours(args):
 
     def step_calls(path=m.PATH_AUTO, events=None):
         for i in range(N_TOKENS):
-            L = layers[i % REPLICAS]
+            L = layers[i % replicas]
             if events is None and path == m.PATH_AUTO:
                 m.moe_q4_ffn_forward(L, x[i:i + 1], y[i:i + 1], ws, stream=stream)
             else:
@@ -442,11 +443,11 @@ def run_ours(args):
     g3 = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         for i in range(N_TOKENS):
-            m.moe_q4_ffn_forward_host(layers[i % REPLICAS], xh[i:i + 1], yh[i:i + 1], wsh, stream=stream)
+            m.moe_q4_ffn_forward_host(layers[i % replicas], xh[i:i + 1], yh[i:i + 1], wsh, stream=stream)
     torch.cuda.synchronize()
     with torch.cuda.graph(g3, stream=stream):
         for i in range(N_TOKENS):
-            m.moe_q4_ffn_forward_host(layers[i % REPLICAS], xh[i:i + 1], yh[i:i + 1], wsh, stream=stream)
+            m.moe_q4_ffn_forward_host(layers[i % replicas], xh[i:i + 1], yh[i:i + 1], wsh, stream=stream)
     for _ in range(3):
         g3.replay()
     torch.cuda.synchronize()
@@ -465,11 +466,12 @@ def run_ours(args):
     e2e_value = world * N_TOKENS * args.steps / (e2e_ms / 1000.0)
     del g3
 
-    prefill = prefill_lines(m, torch, stream) if rank == 0 else None
-    stack = stack_lines(m, torch, stream) if rank == 0 else None
+    extras = set(args.extras.split(",")) if args.extras != "none" else set()
+    prefill = prefill_lines(m, torch, stream) if rank == 0 and "prefill" in extras else None
+    stack = stack_lines(m, torch, stream) if rank == 0 and "stack" in extras else None
 
     cpu = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and "cpu" in extras:
         v, n, dt, cores = oracle_sample(x_np, lw, seconds=10.0)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{n} tokens of the decode workload (T=1 each, independent), {dt:.1f} s, "
@@ -481,7 +483,7 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "i8", "data": "synthetic",
         "config": {"workload": WORKLOAD, "tokens_per_step": N_TOKENS, "T_per_call": 1, "hidden": H, "ffn": F,
                    "experts": E, "top_k": k, "shared_expert": True, "weights": "Q4_0", "activations": "Q8_0",
-                   "l2": f"weights rotate over {REPLICAS} replicas ({REPLICAS * 228} MB) -> L2-cold",
+                   "l2": f"weights rotate over {replicas} replicas ({replicas * 228} MB) -> L2-cold",
                    "parallelism": f"replicas x{world} (tokens independent, no collective)",
                    "graph": "1000 calls captured as one CUDA graph"},
         "roofline": roofline,
@@ -510,6 +512,10 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--replicas", type=int, default=REPLICAS,
+                    help="device copies of the decode layer the tokens rotate over (16: L2-cold)")
+    ap.add_argument("--extras", default="prefill,stack,cpu",
+                    help="comma list of the extra lines to run (prefill, stack, cpu) or 'none'")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

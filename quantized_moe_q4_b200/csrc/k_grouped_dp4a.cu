@@ -1,74 +1,76 @@
-// k_grouped_dp4a.cu -- grouped W4A8 projections on the integer dp4a pipe.
+// k_grouped_dp4a.cu -- grouped W4A8 projections for few tokens per expert, on
+// the integer dp4a pipe, streaming the weights.
 //
 // The grouped 4-bit GEMM of "A 35B Hybrid-Attention Mixture-of-Experts Model
-// on a 6GB 2011 GPU" (Dutch technical summary, Methodologie 1), computed as
-// per-block exact integer dot products (the W4A8 integer multiply-adds of the
-// same section) scaled by the two binary16 block scales and summed in binary32:
+// on a 6GB 2011 GPU" (Dutch technical summary, Methodologie 1), computed with
+// the W4A8 integer multiply-adds of the same section: per-block exact integer
+// dot products scaled by the two binary16 block scales and summed in binary32,
 //   g[s,n] = sum_b dWg[e,n,b] * dA[t,b] * I_b,   I_b = sum_i (nib_i - 8) q_i.
-// Work items are (expert group, tile of up to DP4A_TT of its slots, block of
-// rows), consumed by a persistent grid; the item list is built on the device
-// by the permutation, so the host never learns the per-expert counts.
-//
-//   gate/up item: 32 rows of F of both Wg and Wu, then SwiGLU and the Q8_0
-//                 requantisation of those 32 values per slot (one block).
-//   down item:    64 rows of H of Wd; each slot's result, times its routing
-//                 weight (1 for the shared expert), is added into y[t].
+// When every expert sees only a few tokens (small batches, decode of several
+// sequences) the layer is bound by streaming the active experts' weights, so
+// this kernel is built around that stream:
+//   - a work item is (expert group, tile of up to 8 of its slots, 64 weight
+//     rows: 32 rows of Wg + the same 32 of Wu, or 64 rows of Wd); items come
+//     from the device-built tile list and are consumed by one persistent CTA
+//     per SM;
+//   - a producer warp moves each item's weights in chunks of 64 rows x 32
+//     blocks with one or two 2D tensor copies (TMA; 8-byte elements, so a
+//     box row is a whole 576-byte chunk row), and the tile's int8
+//     activations and scales with 16-byte cp.async, three chunks in flight;
+//   - sixteen compute warps: a lane owns 2 weight rows and every 16th block of
+//     the chunk, keeps its slots' activation blocks in registers and its
+//     2 x 8 (row, slot) sums in registers across the item's chunks; the 16
+//     lanes of a row group add their sums with shuffles once per item;
+//   - epilogue: gate/up -> SwiGLU + Q8_0 requantisation of each slot's 32-row
+//     block of h; down -> y[t] += w * o (fp32 atomics; weight 1 for the
+//     shared expert).
+// Every wait is bounded; a wait that runs out releases every role and records
+// STATUS_SPIN_TIMEOUT.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "launch.h"
+#include "ptx.cuh"
 
 namespace moeq4 {
 
-struct ItemRange {
-    int g;       // group: routed expert 0..E-1, or E = shared expert
-    int slot0;   // first slot of the tile
-    int nslots;  // slots in the tile (1..DP4A_TT)
-    int rb;      // row block
+namespace {
+
+constexpr int SR = 64;                 // weight rows per item
+constexpr int ST = DP4A_TT;            // slots per tile (8)
+constexpr int KCMAX = 32;              // blocks per chunk
+constexpr int NST = 3;                 // chunks in flight
+constexpr int NCW = 16;                // compute warps
+constexpr int RPL = 2;                 // weight rows per lane
+constexpr int THREADS = (NCW + 1) * 32;
+constexpr uint32_t LIMIT = 1u << 22;
+constexpr size_t SZ_W = (size_t)SR * KCMAX * Q4_BYTES;    // 36,864
+constexpr size_t SZ_A = (size_t)ST * KCMAX * QK;          // 8,192
+constexpr size_t SZ_D = (size_t)ST * KCMAX * 2;           // 512
+constexpr size_t SZ_STAGE = SZ_W + SZ_A + SZ_D;           // 45,568 = 356 x 128
+constexpr size_t OFF_RES = NST * SZ_STAGE;
+constexpr size_t SMEM_BYTES = OFF_RES + (size_t)SR * ST * 4;
+constexpr size_t SMEM_ALLOC = SMEM_BYTES + 128;           // slack to align the stages to 128 B
+static_assert(SZ_STAGE % 128 == 0, "TMA destinations need 128-byte alignment");
+static_assert(SMEM_ALLOC <= 200 * 1024, "shared memory map too large");
+
+enum { GATEUP = 0, DOWN = 1 };
+
+// 2D views of the weight matrices for TMA, in 8-byte elements so that one
+// row segment of a box is a whole chunk row (KC blocks x 18 B, up to 576 B)
+// rather than many short ones.  gate/up: [0] gate, [1] up, [2] shared gate,
+// [3] shared up; down: [0] down, [2] shared down.
+struct StreamMaps {
+    CUtensorMap m[4];
 };
 
-// Largest g in [0, ngroups) with tile_off[g] <= tile (tile_off ascending).
-__device__ __forceinline__ int find_group(const int* tile_off, int ngroups, int tile) {
-    int lo = 0, hi = ngroups;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (tile_off[mid] <= tile) lo = mid; else hi = mid;
-    }
-    return lo;
-}
-
-__device__ __forceinline__ ItemRange decode_item(int item, int n_rb, const int* tile_off_s, const int* off_s,
-                                                 int ngroups) {
-    ItemRange r;
-    const int tile = item / n_rb;
-    r.rb = item - tile * n_rb;
-    r.g = find_group(tile_off_s, ngroups, tile);
-    r.slot0 = off_s[r.g] + (tile - tile_off_s[r.g]) * DP4A_TT;
-    r.nslots = min(DP4A_TT, off_s[r.g + 1] - r.slot0);
-    return r;
-}
-
-// Token of a slot and its routing weight.
-__device__ __forceinline__ void slot_token(int s, int g, int E, int k, int P, const int32_t* sorted,
-                                           const float* topk_w, int& t, float& w) {
-    if (g < E) {
-        const int pair = __ldg(sorted + s);
-        t = pair / k;
-        w = __ldg(topk_w + pair);
-    } else {
-        t = s - P;
-        w = 1.0f;
-    }
-}
-
-struct GroupedParams {
+struct StreamParams {
     int H, F, E, k, P;
-    const uint8_t* w_gate;
-    const uint8_t* w_up;
-    const uint8_t* w_down;
-    const uint8_t* sh_gate;
-    const uint8_t* sh_up;
-    const uint8_t* sh_down;
     const int8_t* qa;
     const uint16_t* da;
     const int32_t* off;
@@ -82,242 +84,378 @@ struct GroupedParams {
     uint32_t* status;
 };
 
-// Stage the int8 rows of the tile's slots, their block scales and block sums.
-// src row of slot i is row `rows[i]` of q [*, K] / d [*, K/32].
-__device__ __forceinline__ void stage_q8_rows(const int8_t* __restrict__ q, const uint16_t* __restrict__ d, int K,
-                                              const int* rows, int nslots, int8_t* q_s, float* d_s, int* sum_s) {
+__device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async16_(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all_() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ void cp_async_arrive_noinc_(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Bounded wait; once any wait of the CTA has run out, every later one
+// returns false soon after.
+__device__ __forceinline__ bool wait_phase_s(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    for (uint32_t i = 0; i < LIMIT; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *abort) return false;
+    }
+    *abort = 1;
+    return false;
+}
+
+// Barrier of the compute warps (one arrival per warp), bounded.
+__device__ __forceinline__ bool compute_sync(uint64_t* bar, uint32_t use, volatile int* abort) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive1(bar);
+    return wait_phase_s(bar, use & 1, abort);
+}
+
+__device__ __forceinline__ int find_group_s(const int* tile_off, int ngroups, int tile) {
+    int lo = 0, hi = ngroups;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tile_off[mid] <= tile) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+struct SItem {
+    int g, slot0, nslots, rb;
+};
+
+__device__ __forceinline__ SItem item_of(int item, int n_rb, const int* tile_off_s, const int* off_s, int ngroups) {
+    SItem t;
+    const int tile = item / n_rb;
+    t.rb = item - tile * n_rb;
+    t.g = find_group_s(tile_off_s, ngroups, tile);
+    t.slot0 = off_s[t.g] + (tile - tile_off_s[t.g]) * ST;
+    t.nslots = min(ST, off_s[t.g + 1] - t.slot0);
+    return t;
+}
+
+// Token and routing weight of slot s of group g (group E: the shared expert,
+// slot P + t is token t, weight 1).
+__device__ __forceinline__ void slot_tok(const StreamParams& p, int g, int s, int& tok, float& w) {
+    if (g < p.E) {
+        const int pair = __ldg(p.sorted + s);
+        tok = pair / p.k;
+        w = __ldg(p.topk_w + pair);
+    } else {
+        tok = s - p.P;
+        w = 1.0f;
+    }
+}
+
+// binary32 value of an integer |I| < 2^22, exactly, without the slow int->float
+// conversion: the integer is placed in the mantissa of 1.5 * 2^23.
+__device__ __forceinline__ float int_to_float_exact(int I) {
+    return __fsub_rn(__int_as_float(I + 0x4B400000), 12582912.0f);
+}
+
+}  // namespace
+
+template <int MODE>
+__global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_constant__ StreamMaps maps) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
+    __shared__ __align__(8) uint64_t full[NST], empty[NST], cbar;
+    __shared__ int abort_s;
+    __shared__ int tile_off_s[258], off_s[258];
+    __shared__ const int8_t* arow_s[ST];
+    __shared__ const uint16_t* ascale_s[ST];
+    float* res = reinterpret_cast<float*>(smem + OFF_RES);
+    volatile int* abort = &abort_s;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = p.H, F = p.F, E = p.E;
+    const int K = (MODE == GATEUP) ? H : F;
     const int nb = K / QK;
-    const int chunks = K / 16;  // int4 chunks per row
-    for (int i = threadIdx.x; i < nslots * chunks; i += blockDim.x) {
-        const int r = i / chunks, c = i - r * chunks;
-        reinterpret_cast<int4*>(q_s + (size_t)r * K)[c] =
-            __ldg(reinterpret_cast<const int4*>(q + (size_t)rows[r] * K) + c);
-    }
-    for (int i = threadIdx.x; i < nslots * nb; i += blockDim.x) {
-        const int r = i / nb, b = i - r * nb;
-        d_s[i] = half_bits_to_float(__ldg(d + (size_t)rows[r] * nb + b));
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < nslots * nb; i += blockDim.x) {
-        const int r = i / nb, b = i - r * nb;
-        const int* qw = reinterpret_cast<const int*>(q_s + (size_t)r * K + b * QK);
-        int s = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) s = __dp4a(qw[j], 0x01010101, s);
-        sum_s[i] = s;
-    }
-    __syncthreads();
-}
+    const int KC = min(KCMAX, nb);          // nb is a multiple of 8
+    const int nchunk = nb / KC;
+    const int n_rb = (MODE == GATEUP) ? F / 32 : H / SR;
+    const int ngroups = E + 1;
+    const uint32_t chunk_bytes = (uint32_t)(SR * KC * Q4_BYTES);
 
-// Dot products of one Q4_0 row (nb blocks) with the staged slots; the LPR
-// lanes of a lane group split the blocks and reduce at the end.
-template <int LPR>
-__device__ __forceinline__ void row_dots(const uint8_t* __restrict__ wrow, int nb, int K, int sub, int nslots,
-                                         const int8_t* q_s, const float* d_s, const int* sum_s,
-                                         float acc[DP4A_TT]) {
-#pragma unroll
-    for (int t = 0; t < DP4A_TT; ++t) acc[t] = 0.0f;
-    for (int b = sub; b < nb; b += LPR) {
-        uint32_t qs[4], dbits;
-        load_q4_block(wrow + (size_t)b * Q4_BYTES, qs, dbits);
-        const float dw = half_bits_to_float(dbits);
-#pragma unroll
-        for (int t = 0; t < DP4A_TT; ++t) {
-            if (t < nslots) {
-                const int4* qv = reinterpret_cast<const int4*>(q_s + (size_t)t * K + b * QK);
-                const int4 a0 = qv[0], a1 = qv[1];
-                const int qa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                const int I = q4_q8_dot(qs, qa, sum_s[t * nb + b]);
-                acc[t] = fmaf((float)I, dw * d_s[t * nb + b], acc[t]);
-            }
+    if (tid == 0) {
+        abort_s = 0;
+        for (int i = 0; i < NST; ++i) {
+            mbar_init(&full[i], 64);   // 32 producer arrivals + 32 cp.async arrivals
+            mbar_init(&empty[i], NCW);
         }
+        mbar_init(&cbar, NCW);
+        mbar_fence_init();
     }
-#pragma unroll
-    for (int t = 0; t < DP4A_TT; ++t) {
-#pragma unroll
-        for (int o = LPR / 2; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
-    }
-}
-
-template <int LPR>
-__global__ void __launch_bounds__(256) gateup_dp4a_kernel(GroupedParams p) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ int tile_off_s[258];
-    __shared__ int off_s[258];
-    __shared__ int rows_s[DP4A_TT];
-    __shared__ float gs[GU_ROWS][DP4A_TT];
-    __shared__ float us[GU_ROWS][DP4A_TT];
-    const int H = p.H, F = p.F, nb = H / QK;
-    int8_t* q_s = reinterpret_cast<int8_t*>(smem);
-    float* d_s = reinterpret_cast<float*>(smem + (size_t)DP4A_TT * H);
-    int* sum_s = reinterpret_cast<int*>(d_s + DP4A_TT * nb);
-    const int ngroups = p.E + 1;
-    for (int i = threadIdx.x; i <= ngroups; i += blockDim.x) {
+    for (int i = tid; i <= ngroups; i += THREADS) {
         tile_off_s[i] = p.tile_off[i];
         off_s[i] = p.off[i];
     }
     __syncthreads();
-    const int n_rb = F / GU_ROWS;
     const int n_items = tile_off_s[ngroups] * n_rb;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int sub = lane % LPR, lgrp = lane / LPR;
-    constexpr int ROWS_PER_PASS = 32 / LPR;
-    const size_t gu_stride = (size_t)F * nb * Q4_BYTES;
 
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const ItemRange it = decode_item(item, n_rb, tile_off_s, off_s, ngroups);
-        if (threadIdx.x < it.nslots) {
-            int t;
-            float w;
-            slot_token(it.slot0 + threadIdx.x, it.g, p.E, p.k, p.P, p.sorted, p.topk_w, t, w);
-            rows_s[threadIdx.x] = t;
+    if (warp == NCW) {
+        // ------------------------------------------------------------ producer
+        uint32_t ic = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+            const SItem it = item_of(item, n_rb, tile_off_s, off_s, ngroups);
+            const bool sh = it.g >= E;
+            if (lane < it.nslots) {
+                int tok;
+                float w;
+                const int s = it.slot0 + lane;
+                slot_tok(p, it.g, s, tok, w);
+                if (MODE == GATEUP) {
+                    arow_s[lane] = p.qa + (size_t)tok * H;
+                    ascale_s[lane] = p.da + (size_t)tok * (H / QK);
+                } else {
+                    arow_s[lane] = p.hq + (size_t)s * F;
+                    ascale_s[lane] = p.dh + (size_t)s * (F / QK);
+                }
+            }
+            __syncwarp();
+            const CUtensorMap* m0 = &maps.m[sh ? 2 : 0];
+            const CUtensorMap* m1 = &maps.m[sh ? 3 : 1];
+            const int z = (sh ? 0 : it.g * ((MODE == GATEUP) ? F : H)) + it.rb * ((MODE == GATEUP) ? 32 : SR);
+            for (int c = 0; c < nchunk; ++c, ++ic) {
+                const int st = ic % NST;
+                if (!wait_phase_s(&empty[st], ((ic / NST) & 1) ^ 1, abort)) { ok = false; break; }
+                unsigned char* sw = smem + st * SZ_STAGE;
+                int8_t* sa = reinterpret_cast<int8_t*>(sw + SZ_W);
+                unsigned char* sd = sw + SZ_W + SZ_A;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[st], chunk_bytes);
+                    const int x8 = c * KC * Q4_BYTES / 8;   // chunk start in 8-byte elements (16-B multiple)
+                    if (MODE == GATEUP) {
+                        tma_load_2d_(sw, m0, x8, z, &full[st]);
+                        tma_load_2d_(sw + (size_t)32 * KC * Q4_BYTES, m1, x8, z, &full[st]);
+                    } else {
+                        tma_load_2d_(sw, m0, x8, z, &full[st]);
+                    }
+                } else {
+                    mbar_arrive1(&full[st]);
+                }
+                for (int n = 0; n < it.nslots; ++n) {
+                    const int8_t* src = arow_s[n] + (size_t)c * KC * QK;
+                    int8_t* dst = sa + (size_t)n * KC * QK;
+                    for (int j = lane; j < 2 * KC; j += 32) cp_async16_(dst + j * 16, src + j * 16);   // activations
+                    if (lane < KC / 8)                                                               // binary16 scales
+                        cp_async16_(sd + (size_t)n * KC * 2 + lane * 16, ascale_s[n] + (size_t)c * KC + lane * 8);
+                }
+                cp_async_arrive_noinc_(&full[st]);
+            }
+            __syncwarp();
         }
-        __syncthreads();
-        stage_q8_rows(p.qa, p.da, H, rows_s, it.nslots, q_s, d_s, sum_s);
-
-        const uint8_t* Wg = (it.g < p.E) ? p.w_gate + it.g * gu_stride : p.sh_gate;
-        const uint8_t* Wu = (it.g < p.E) ? p.w_up + it.g * gu_stride : p.sh_up;
-        const int n0 = it.rb * GU_ROWS;
-        // 64 row jobs (32 gate + 32 up), 8 per warp
-        for (int j0 = warp * 8; j0 < warp * 8 + 8; j0 += ROWS_PER_PASS) {
-            const int job = j0 + lgrp;
-            const int mat = job >> 5, rloc = job & 31;
-            const uint8_t* wrow = (mat ? Wu : Wg) + (size_t)(n0 + rloc) * nb * Q4_BYTES;
-            float acc[DP4A_TT];
-            row_dots<LPR>(wrow, nb, H, sub, it.nslots, q_s, d_s, sum_s, acc);
-            if (sub == 0) {
+        cp_async_wait_all_();
+        if (ic > 0) mbar_wait_bounded(&full[(ic - 1) % NST], ((ic - 1) / NST) & 1, LIMIT);
+    } else {
+        // ------------------------------------------------------------ compute
+        const int rg = 2 * warp + (lane >> 4);   // row group: rows RPL rg .. RPL rg + RPL - 1
+        const int ks = lane & 15;                // this lane's blocks: ks, ks + 16, ...
+        uint32_t ic = 0, cuse = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+            const SItem it = item_of(item, n_rb, tile_off_s, off_s, ngroups);
+            float acc[RPL][ST];
 #pragma unroll
-                for (int t = 0; t < DP4A_TT; ++t) (mat ? us : gs)[rloc][t] = acc[t];
+            for (int r = 0; r < RPL; ++r)
+#pragma unroll
+                for (int s = 0; s < ST; ++s) acc[r][s] = 0.0f;
+            for (int c = 0; c < nchunk; ++c, ++ic) {
+                const int st = ic % NST;
+                if (!wait_phase_s(&full[st], (ic / NST) & 1, abort)) { ok = false; break; }
+                const unsigned char* sw = smem + st * SZ_STAGE;
+                const int8_t* sa = reinterpret_cast<const int8_t*>(sw + SZ_W);
+                const uint16_t* sd = reinterpret_cast<const uint16_t*>(sw + SZ_W + SZ_A);
+                for (int b = ks; b < KC; b += 16) {
+#pragma unroll
+                    for (int sp = 0; sp < ST; sp += 4) {
+                        if (sp >= it.nslots) break;
+                        // activation blocks of slots sp..sp+3 for block b
+                        int qa[4][8];
+                        int base[4];
+                        float dA[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int4* av = reinterpret_cast<const int4*>(sa + (size_t)(sp + j) * KC * QK + b * QK);
+                            const int4 a0 = av[0], a1 = av[1];
+                            qa[j][0] = a0.x; qa[j][1] = a0.y; qa[j][2] = a0.z; qa[j][3] = a0.w;
+                            qa[j][4] = a1.x; qa[j][5] = a1.y; qa[j][6] = a1.z; qa[j][7] = a1.w;
+                            int sum = 0;
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) sum = __dp4a(qa[j][i], 0x01010101, sum);
+                            base[j] = -8 * sum;
+                            dA[j] = half_bits_to_float(sd[(sp + j) * KC + b]);
+                        }
+#pragma unroll
+                        for (int r = 0; r < RPL; ++r) {
+                            uint32_t qs[4], dbits;
+                            load_q4_block_smem(sw + (size_t)(RPL * rg + r) * KC * Q4_BYTES + b * Q4_BYTES, qs, dbits);
+                            const float dW = half_bits_to_float(dbits);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                int I = base[j];
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    I = dp4a_u8s8(qs[i] & 0x0f0f0f0fu, qa[j][i], I);
+                                    I = dp4a_u8s8((qs[i] >> 4) & 0x0f0f0f0fu, qa[j][4 + i], I);
+                                }
+                                acc[r][sp + j] = fmaf(int_to_float_exact(I), dW * dA[j], acc[r][sp + j]);
+                            }
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive1(&empty[st]);
             }
-        }
-        __syncthreads();
-        // epilogue: one warp per slot, lane = row of the 32-row block
-        for (int t = warp; t < it.nslots; t += 8) {
-            const int slot = it.slot0 + t;
-            const float h = swiglu(gs[lane][t], us[lane][t]);
-            if (p.h_dbg) p.h_dbg[(size_t)slot * F + n0 + lane] = h;
-            uint16_t db;
-            bool ov;
-            const int q = q8_0_lane(h, db, ov);
-            p.hq[(size_t)slot * F + n0 + lane] = (int8_t)q;
-            if (lane == 0) {
-                p.dh[(size_t)slot * (F / QK) + it.rb] = db;
-                if (ov) atomicOr(p.status, STATUS_SCALE_OVERFLOW);
+            if (!ok) break;
+            // the 16 lanes of a row group hold partial sums over their blocks
+#pragma unroll
+            for (int r = 0; r < RPL; ++r)
+#pragma unroll
+                for (int s = 0; s < ST; ++s) {
+                    if (s < it.nslots) {
+                        float v = acc[r][s];
+                        v += __shfl_xor_sync(0xffffffffu, v, 8);
+                        v += __shfl_xor_sync(0xffffffffu, v, 4);
+                        v += __shfl_xor_sync(0xffffffffu, v, 2);
+                        v += __shfl_xor_sync(0xffffffffu, v, 1);
+                        if (ks == 0) res[(RPL * rg + r) * ST + s] = v;
+                    }
+                }
+            if (!compute_sync(&cbar, cuse++, abort)) break;
+            if (MODE == GATEUP) {
+                // warp w < 8: slot w; lane = row f0 + lane of the 32-row block of h
+                const int s = warp;
+                if (s < it.nslots && s < ST) {
+                    const int slot = it.slot0 + s;
+                    const int f0 = it.rb * 32;
+                    const float h = swiglu(res[lane * ST + s], res[(32 + lane) * ST + s]);
+                    if (p.h_dbg) p.h_dbg[(size_t)slot * F + f0 + lane] = h;
+                    uint16_t db;
+                    bool ov;
+                    const int q = q8_0_lane(h, db, ov);
+                    p.hq[(size_t)slot * F + f0 + lane] = (int8_t)q;
+                    if (lane == 0) {
+                        p.dh[(size_t)slot * (F / QK) + it.rb] = db;
+                        if (ov) atomicOr(p.status, STATUS_SCALE_OVERFLOW);
+                    }
+                }
+            } else {
+                // warp w: slot w & 7, rows 32 (w >> 3) .. + 31 of the 64 rows of H
+                const int s = warp & (ST - 1), r = 32 * (warp / ST) + lane;
+                if (s < it.nslots) {
+                    int tok;
+                    float w;
+                    slot_tok(p, it.g, it.slot0 + s, tok, w);
+                    atomicAdd(p.y + (size_t)tok * H + it.rb * SR + r, w * res[r * ST + s]);
+                }
             }
+            if (!compute_sync(&cbar, cuse++, abort)) break;  // res is free for the next item
         }
-        __syncthreads();
-    }
-}
-
-template <int LPR>
-__global__ void __launch_bounds__(256) down_dp4a_kernel(GroupedParams p) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ int tile_off_s[258];
-    __shared__ int off_s[258];
-    __shared__ int slots_s[DP4A_TT];
-    __shared__ int tok_s[DP4A_TT];
-    __shared__ float wgt_s[DP4A_TT];
-    const int H = p.H, F = p.F, nbF = F / QK;
-    int8_t* q_s = reinterpret_cast<int8_t*>(smem);
-    float* d_s = reinterpret_cast<float*>(smem + (size_t)DP4A_TT * F);
-    int* sum_s = reinterpret_cast<int*>(d_s + DP4A_TT * nbF);
-    const int ngroups = p.E + 1;
-    for (int i = threadIdx.x; i <= ngroups; i += blockDim.x) {
-        tile_off_s[i] = p.tile_off[i];
-        off_s[i] = p.off[i];
     }
     __syncthreads();
-    const int n_rb = H / DN_ROWS;
-    const int n_items = tile_off_s[ngroups] * n_rb;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int sub = lane % LPR, lgrp = lane / LPR;
-    constexpr int ROWS_PER_PASS = 32 / LPR;
-    const size_t dn_stride = (size_t)H * nbF * Q4_BYTES;
-
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const ItemRange it = decode_item(item, n_rb, tile_off_s, off_s, ngroups);
-        if (threadIdx.x < it.nslots) {
-            int t;
-            float w;
-            slot_token(it.slot0 + threadIdx.x, it.g, p.E, p.k, p.P, p.sorted, p.topk_w, t, w);
-            slots_s[threadIdx.x] = it.slot0 + threadIdx.x;
-            tok_s[threadIdx.x] = t;
-            wgt_s[threadIdx.x] = w;
-        }
-        __syncthreads();
-        stage_q8_rows(p.hq, p.dh, F, slots_s, it.nslots, q_s, d_s, sum_s);
-
-        const uint8_t* Wd = (it.g < p.E) ? p.w_down + it.g * dn_stride : p.sh_down;
-        const int n0 = it.rb * DN_ROWS;
-        for (int r0 = warp * 8; r0 < warp * 8 + 8; r0 += ROWS_PER_PASS) {
-            const int n = n0 + r0 + lgrp;
-            const uint8_t* wrow = Wd + (size_t)n * nbF * Q4_BYTES;
-            float acc[DP4A_TT];
-            row_dots<LPR>(wrow, nbF, F, sub, it.nslots, q_s, d_s, sum_s, acc);
-            if (sub == 0) {
-#pragma unroll
-                for (int t = 0; t < DP4A_TT; ++t)
-                    if (t < it.nslots) atomicAdd(p.y + (size_t)tok_s[t] * H + n, wgt_s[t] * acc[t]);
-            }
-        }
-        __syncthreads();
-    }
+    if (tid == 0 && abort_s) atomicOr(p.status, STATUS_SPIN_TIMEOUT);
 }
 
-static int lanes_per_row(int nblocks) { return nblocks >= 32 ? 32 : (nblocks >= 16 ? 16 : 8); }
+namespace {
 
-static GroupedParams make_params(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, float* y) {
-    GroupedParams p;
+PFN_cuTensorMapEncodeTiled_v12000 stream_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// `rows` rows of nb 18-byte blocks at `base` (row bytes a multiple of 144),
+// viewed as [rows][nb * 18 / 8] 8-byte elements, copied as boxes of box_rows
+// rows x KC blocks.
+cudaError_t encode_rows_2d(CUtensorMap* map, const uint8_t* base, uint64_t rows, int nb, int KC, uint32_t box_rows) {
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = stream_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {(cuuint64_t)nb * Q4_BYTES / 8, rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)nb * Q4_BYTES};
+    const cuuint32_t box[2] = {(cuuint32_t)(KC * Q4_BYTES / 8), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+StreamParams make_stream_params(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, float* y) {
+    StreamParams p;
     p.H = L.H; p.F = L.F; p.E = L.E; p.k = L.k; p.P = (int)(T * L.k);
-    p.w_gate = L.w_gate; p.w_up = L.w_up; p.w_down = L.w_down;
-    p.sh_gate = L.sh_gate; p.sh_up = L.sh_up; p.sh_down = L.sh_down;
     p.qa = ws.qa; p.da = ws.da; p.off = ws.off; p.tile_off = ws.tile_off; p.sorted = ws.sorted;
     p.topk_w = ws.topk_w; p.hq = ws.hq; p.dh = ws.dh; p.h_dbg = h_dbg; p.y = y; p.status = ws.status;
     return p;
 }
 
-// Upper bound of the work tiles over all groups: sum_g ceil(c_g / TT).
-static int64_t max_tiles(const LayerView& L, int64_t T) {
+// Upper bound of the work tiles over all groups: sum_g ceil(c_g / ST).
+int64_t stream_max_tiles(const LayerView& L, int64_t T) {
     const int64_t P = T * L.k;
-    return ceil_div(P, DP4A_TT) + std::min<int64_t>(L.E, P) + (L.S ? ceil_div(T, DP4A_TT) : 0);
+    return ceil_div(P, ST) + std::min<int64_t>(L.E, P) + (L.S ? ceil_div(T, ST) : 0);
 }
 
-template <typename K>
-static cudaError_t launch_persistent(K kernel, int64_t items, size_t smem, const DeviceInfo& dev,
-                                     const GroupedParams& p, cudaStream_t s) {
+template <int MODE>
+cudaError_t launch_stream(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, float* y,
+                          const DeviceInfo& dev, cudaStream_t s) {
     int per_sm = 0;
-    cudaError_t err = kernel_occupancy(reinterpret_cast<const void*>(kernel), 256, smem, &per_sm);
-    if (err != cudaSuccess) return err;
-    int64_t grid = std::min<int64_t>(items, (int64_t)dev.sm_count * per_sm);
-    if (grid < 1) grid = 1;
-    kernel<<<(unsigned)grid, 256, smem, s>>>(p);
+    cudaError_t e =
+        kernel_occupancy(reinterpret_cast<const void*>(stream_dp4a_kernel<MODE>), THREADS, SMEM_ALLOC, &per_sm);
+    if (e != cudaSuccess) return e;
+    StreamMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    const uint64_t E = (uint64_t)L.E, F = (uint64_t)L.F, H = (uint64_t)L.H;
+    if (MODE == GATEUP) {
+        const int nb = L.H / QK, KC = std::min(KCMAX, nb);
+        e = encode_rows_2d(&maps.m[0], L.w_gate, E * F, nb, KC, 32);
+        if (e == cudaSuccess) e = encode_rows_2d(&maps.m[1], L.w_up, E * F, nb, KC, 32);
+        if (e == cudaSuccess && L.S) e = encode_rows_2d(&maps.m[2], L.sh_gate, F, nb, KC, 32);
+        if (e == cudaSuccess && L.S) e = encode_rows_2d(&maps.m[3], L.sh_up, F, nb, KC, 32);
+    } else {
+        const int nb = L.F / QK, KC = std::min(KCMAX, nb);
+        e = encode_rows_2d(&maps.m[0], L.w_down, E * H, nb, KC, SR);
+        if (e == cudaSuccess && L.S) e = encode_rows_2d(&maps.m[2], L.sh_down, H, nb, KC, SR);
+    }
+    if (e != cudaSuccess) return e;
+    const int n_rb = (MODE == GATEUP) ? L.F / 32 : L.H / SR;
+    const int64_t items = stream_max_tiles(L, T) * n_rb;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, dev.sm_count));
+    stream_dp4a_kernel<MODE><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(make_stream_params(L, T, ws, h_dbg, y), maps);
     return cudaGetLastError();
 }
 
+}  // namespace
+
 cudaError_t launch_gateup_dp4a(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg,
                                const DeviceInfo& dev, cudaStream_t s) {
-    const GroupedParams p = make_params(L, T, ws, h_dbg, nullptr);
-    const int nb = L.H / QK;
-    const size_t smem = (size_t)DP4A_TT * L.H + (size_t)DP4A_TT * nb * 8;
-    const int64_t items = max_tiles(L, T) * (L.F / GU_ROWS);
-    switch (lanes_per_row(nb)) {
-        case 32: return launch_persistent(gateup_dp4a_kernel<32>, items, smem, dev, p, s);
-        case 16: return launch_persistent(gateup_dp4a_kernel<16>, items, smem, dev, p, s);
-        default: return launch_persistent(gateup_dp4a_kernel<8>, items, smem, dev, p, s);
-    }
+    return launch_stream<GATEUP>(L, T, ws, h_dbg, nullptr, dev, s);
 }
 
 cudaError_t launch_down_dp4a(const LayerView& L, int64_t T, const Workspace& ws, float* y,
                              const DeviceInfo& dev, cudaStream_t s) {
-    const GroupedParams p = make_params(L, T, ws, nullptr, y);
-    const int nbF = L.F / QK;
-    const size_t smem = (size_t)DP4A_TT * L.F + (size_t)DP4A_TT * nbF * 8;
-    const int64_t items = max_tiles(L, T) * (L.H / DN_ROWS);
-    switch (lanes_per_row(nbF)) {
-        case 32: return launch_persistent(down_dp4a_kernel<32>, items, smem, dev, p, s);
-        case 16: return launch_persistent(down_dp4a_kernel<16>, items, smem, dev, p, s);
-        default: return launch_persistent(down_dp4a_kernel<8>, items, smem, dev, p, s);
-    }
+    return launch_stream<DOWN>(L, T, ws, nullptr, y, dev, s);
 }
 
 // ---------------------------------------------------------------------------

@@ -13,30 +13,32 @@
 namespace moeq4 {
 
 // ---------------------------------------------------------------------------
-// Logits, few tokens: one warp per expert row of Wr, float4 loads along H,
-// up to TT tokens per CTA row (x rows are read through L1).
+// Logits, up to a few hundred tokens: one CTA per (expert, tile of RT tokens);
+// its 8 warps split H into 8 slices, and the slices' sums are added in a fixed
+// order (deterministic), so even a handful of tokens spreads over E CTAs.
 // ---------------------------------------------------------------------------
-template <int TT>
-__global__ void __launch_bounds__(128) router_logits_small(const float* __restrict__ x, int T, int H,
+constexpr int RT = 8;
+
+__global__ void __launch_bounds__(256) router_logits_split(const float* __restrict__ x, int T, int H,
                                                             const float* __restrict__ Wr,
                                                             const float* __restrict__ bias, int E,
                                                             float* __restrict__ logits,
                                                             uint32_t* __restrict__ status_clear) {
     if (status_clear && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status_clear = 0u;
+    __shared__ float part[8][RT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = blockIdx.x * 4 + warp;
-    const int t0 = blockIdx.y * TT;
-    if (e >= E) return;
-    float acc[TT];
-#pragma unroll
-    for (int t = 0; t < TT; ++t) acc[t] = 0.0f;
+    const int e = blockIdx.x;
+    const int t0 = blockIdx.y * RT;
+    const int slice = H / 8;                      // a multiple of 32 floats
+    const int h4_0 = warp * (slice >> 2), h4_1 = h4_0 + (slice >> 2);
     const float4* wr = reinterpret_cast<const float4*>(Wr + (size_t)e * H);
-    const int H4 = H >> 2;
-#pragma unroll 4
-    for (int h4 = lane; h4 < H4; h4 += 32) {
+    float acc[RT];
+#pragma unroll
+    for (int t = 0; t < RT; ++t) acc[t] = 0.0f;
+    for (int h4 = h4_0 + lane; h4 < h4_1; h4 += 32) {
         const float4 w = __ldg(wr + h4);
 #pragma unroll
-        for (int t = 0; t < TT; ++t) {
+        for (int t = 0; t < RT; ++t) {
             if (t0 + t < T) {
                 const float4 v = __ldg(reinterpret_cast<const float4*>(x + (size_t)(t0 + t) * H) + h4);
                 acc[t] = fmaf(w.x, v.x, acc[t]);
@@ -46,13 +48,19 @@ __global__ void __launch_bounds__(128) router_logits_small(const float* __restri
             }
         }
     }
-    const float b = bias ? __ldg(bias + e) : 0.0f;
 #pragma unroll
-    for (int t = 0; t < TT; ++t) {
+    for (int t = 0; t < RT; ++t) {
         float a = acc[t];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (lane == 0 && t0 + t < T) logits[(size_t)(t0 + t) * E + e] = a + b;
+        if (lane == 0) part[warp][t] = a;
+    }
+    __syncthreads();
+    if (threadIdx.x < RT && t0 + (int)threadIdx.x < T) {
+        float a = part[0][threadIdx.x];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) a += part[w][threadIdx.x];
+        logits[(size_t)(t0 + threadIdx.x) * E + e] = a + (bias ? __ldg(bias + e) : 0.0f);
     }
 }
 
@@ -169,9 +177,11 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
 
 cudaError_t launch_router_logits(const LayerView& L, const float* x, int64_t T, float* logits,
                                  uint32_t* status_clear, cudaStream_t s) {
-    if (T <= 32) {
-        dim3 grid((unsigned)ceil_div(L.E, 4), (unsigned)ceil_div(T, 8));
-        router_logits_small<8><<<grid, 128, 0, s>>>(x, (int)T, L.H, L.w_router, L.router_bias, L.E, logits, status_clear);
+    if (T <= 512) {
+        // x rows are re-read once per expert from L2 (at most 512 x H x 4 x E bytes)
+        dim3 grid((unsigned)L.E, (unsigned)ceil_div(T, RT));
+        router_logits_split<<<grid, 256, 0, s>>>(x, (int)T, L.H, L.w_router, L.router_bias, L.E, logits,
+                                                 status_clear);
     } else {
         dim3 grid((unsigned)ceil_div(L.E, 64), (unsigned)ceil_div(T, 64));
         router_logits_tiled<<<grid, 256, 0, s>>>(x, (int)T, L.H, L.w_router, L.router_bias, L.E, logits,

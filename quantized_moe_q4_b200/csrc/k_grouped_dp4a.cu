@@ -251,7 +251,10 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
                 for (int n = 0; n < it.nslots; ++n) {
                     const int8_t* src = arow_s[n] + (size_t)c * KC * QK;
                     int8_t* dst = sa + (size_t)n * KC * QK;
-                    for (int j = lane; j < 2 * KC; j += 32) cp_async16_(dst + j * 16, src + j * 16);   // activations
+                    // activations as [half][block][16 B]: the 16 lanes that own
+                    // consecutive blocks read 256 contiguous bytes
+                    for (int j = lane; j < 2 * KC; j += 32)
+                        cp_async16_(dst + (size_t)(j & 1) * KC * 16 + (j >> 1) * 16, src + j * 16);
                     if (lane < KC / 8)                                                               // binary16 scales
                         cp_async16_(sd + (size_t)n * KC * 2 + lane * 16, ascale_s[n] + (size_t)c * KC + lane * 8);
                 }
@@ -281,6 +284,15 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
                 const int8_t* sa = reinterpret_cast<const int8_t*>(sw + SZ_W);
                 const uint16_t* sd = reinterpret_cast<const uint16_t*>(sw + SZ_W + SZ_A);
                 for (int b = ks; b < KC; b += 16) {
+                    // this lane's weight blocks (its RPL rows, block b), loaded once
+                    uint32_t qs[RPL][4];
+                    float dW[RPL];
+#pragma unroll
+                    for (int r = 0; r < RPL; ++r) {
+                        uint32_t dbits;
+                        load_q4_block_smem(sw + (size_t)(RPL * rg + r) * KC * Q4_BYTES + b * Q4_BYTES, qs[r], dbits);
+                        dW[r] = half_bits_to_float(dbits);
+                    }
 #pragma unroll
                     for (int sp = 0; sp < ST; sp += 4) {
                         if (sp >= it.nslots) break;
@@ -290,8 +302,9 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
                         float dA[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            const int4* av = reinterpret_cast<const int4*>(sa + (size_t)(sp + j) * KC * QK + b * QK);
-                            const int4 a0 = av[0], a1 = av[1];
+                            const int8_t* a = sa + (size_t)(sp + j) * KC * QK;
+                            const int4 a0 = *reinterpret_cast<const int4*>(a + b * 16);
+                            const int4 a1 = *reinterpret_cast<const int4*>(a + (size_t)KC * 16 + b * 16);
                             qa[j][0] = a0.x; qa[j][1] = a0.y; qa[j][2] = a0.z; qa[j][3] = a0.w;
                             qa[j][4] = a1.x; qa[j][5] = a1.y; qa[j][6] = a1.z; qa[j][7] = a1.w;
                             int sum = 0;
@@ -302,18 +315,15 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
                         }
 #pragma unroll
                         for (int r = 0; r < RPL; ++r) {
-                            uint32_t qs[4], dbits;
-                            load_q4_block_smem(sw + (size_t)(RPL * rg + r) * KC * Q4_BYTES + b * Q4_BYTES, qs, dbits);
-                            const float dW = half_bits_to_float(dbits);
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 int I = base[j];
 #pragma unroll
                                 for (int i = 0; i < 4; ++i) {
-                                    I = dp4a_u8s8(qs[i] & 0x0f0f0f0fu, qa[j][i], I);
-                                    I = dp4a_u8s8((qs[i] >> 4) & 0x0f0f0f0fu, qa[j][4 + i], I);
+                                    I = dp4a_u8s8(qs[r][i] & 0x0f0f0f0fu, qa[j][i], I);
+                                    I = dp4a_u8s8((qs[r][i] >> 4) & 0x0f0f0f0fu, qa[j][4 + i], I);
                                 }
-                                acc[r][sp + j] = fmaf(int_to_float_exact(I), dW * dA[j], acc[r][sp + j]);
+                                acc[r][sp + j] = fmaf(int_to_float_exact(I), dW[r] * dA[j], acc[r][sp + j]);
                             }
                         }
                     }

@@ -263,6 +263,75 @@ def prefill_lines(m, torch, stream):
     return out
 
 
+def chunked_lines(m, torch, stream):
+    """Single pass against chunked prefill (the page's Methodologie 4 claim):
+    the 947- and 16384-token prompts through moe_q4_ffn_forward in chunks of
+    C tokens (ceil(T/C) calls back to back), tokens/s per C; 256 MB written
+    between reps to flush L2."""
+    import synth
+    out = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for name, sizes in (("prefill_t947", (64, 128, 256, 512, 947)),
+                        ("zipf_t16384", (256, 1024, 4096, 16384))):
+        x_np, lw = synth.workload_inputs(name, seed=0)
+        L = m.Layer.from_host(lw)
+        x = torch.from_numpy(x_np).cuda()
+        T = x.shape[0]
+        y = torch.empty_like(x)
+        rec = {}
+        for C in sizes:
+            ws = m.alloc_workspace(m.moe_q4_ffn_workspace_bytes(L, C))
+            times = []
+            for rep in range(5):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for t0 in range(0, T, C):
+                    m.moe_q4_ffn_forward(L, x[t0:t0 + C], y[t0:t0 + C], ws, stream=stream)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if rep >= 2:
+                    times.append(e0.elapsed_time(e1))
+            ms = float(np.median(times))
+            rec[str(C)] = {"ms": ms, "tokens_per_s": T / (ms * 1e-3), "calls": -(-T // C)}
+            del ws
+        out[name] = rec
+        del L, x, y
+    del flush
+    return out
+
+
+def gemv_lines(m, torch, stream):
+    """The W4A8 LM-head GEMV: one 131072 x 2048 Q4_0 matrix (151 MB, beyond
+    the 126 MB L2; two copies alternate so every rep is L2-cold) against
+    1..8 tokens; HBM GB/s over the matrix + x + y bytes."""
+    import synth
+    hbm, src = measured_peaks()
+    N, H = 131072, 2048
+    rng = np.random.Generator(np.random.PCG64(7))
+    W = torch.from_numpy(synth._q4_0_matrix(rng, N, H // 32)).cuda()
+    Ws = [W, W.clone()]
+    out = {"rows": N, "hidden": H, "peak_source": src}
+    for T in (1, 4, 8):
+        x = torch.from_numpy(np.random.default_rng(T).standard_normal((T, H)).astype(np.float32)).cuda()
+        y = torch.empty((T, N), dtype=torch.float32, device="cuda")
+        ws = m.alloc_workspace(m.moe_q4_gemv_workspace_bytes(T, H))
+        times = []
+        for rep in range(12):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            m.moe_q4_gemv(Ws[rep % 2], x, y, ws, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 4:
+                times.append(e0.elapsed_time(e1))
+        us = float(np.median(times)) * 1000.0
+        nbytes = N * (H // 32) * 18 + T * H * 4 + T * N * 4
+        out[f"T{T}"] = {"us": us, "hbm_gbs": nbytes / (us * 1e-6) / 1e9, "hbm_frac": nbytes / (us * 1e-6) / 1e9 / hbm}
+    del W, Ws
+    return out
+
+
 def stack_lines(m, torch, stream):
     """The 40-layer stack (x <- x + MoE_l(RMSNorm(x)), independently seeded
     layers, 9.1 GB of weights: every step is L2-cold) through the one-call
@@ -469,6 +538,8 @@ def run_ours(args):
     extras = set(args.extras.split(",")) if args.extras != "none" else set()
     prefill = prefill_lines(m, torch, stream) if rank == 0 and "prefill" in extras else None
     stack = stack_lines(m, torch, stream) if rank == 0 and "stack" in extras else None
+    chunked = chunked_lines(m, torch, stream) if rank == 0 and "chunked" in extras else None
+    gemv = gemv_lines(m, torch, stream) if rank == 0 and "gemv" in extras else None
 
     cpu = None
     if rank == 0 and world == 1 and "cpu" in extras:
@@ -496,6 +567,8 @@ def run_ours(args):
         "clocks": clk,
         "prefill": prefill,
         "stack": stack,
+        "chunked_prefill": chunked,
+        "lm_head_gemv": gemv,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -514,8 +587,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--replicas", type=int, default=REPLICAS,
                     help="device copies of the decode layer the tokens rotate over (16: L2-cold)")
-    ap.add_argument("--extras", default="prefill,stack,cpu",
-                    help="comma list of the extra lines to run (prefill, stack, cpu) or 'none'")
+    ap.add_argument("--extras", default="prefill,stack,chunked,gemv,cpu",
+                    help="comma list of the extra lines to run (prefill, stack, chunked, gemv, cpu) or 'none'")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -189,6 +189,26 @@ size_t moe_q4_stack_workspace_bytes(const moe_q4_layer* L, int64_t T_max);
 int moe_q4_stack_forward(const moe_q4_layer* layers, int32_t n_layers, float* x, int64_t T, float eps,
                          void* workspace, size_t ws_bytes, moe_q4_stream_t stream);
 
+/* ---------------------------------------------------------------------
+ * W4A8 GEMV of one large Q4_0 matrix (the LM head).
+ *
+ * The page reports the LM head run on the GPU against the CPU (Resultaten,
+ * 116 -> 139 ms/token on Fermi).  Here it is the decode path's W4A8 GEMV
+ * applied to one vocabulary-sized matrix: x [T][H] fp32 (1 <= T <= 8) is
+ * quantised to Q8_0 exactly as moe_q4_quantize_act does, and
+ *     y[t][n] = sum_b dW[n,b] * dA[t,b] * I_{n,b,t}   (binary32)
+ * with I the exact per-block integer dot product, for the N rows of
+ * W [N][H/32] Q4_0 blocks (18 B each).  y is [T][N] fp32, overwritten.
+ * H a positive multiple of 256 up to 16384, 1 <= N <= 2^30; pointers 16-byte
+ * aligned, the workspace 256-byte aligned and at least
+ * moe_q4_gemv_workspace_bytes(T, H) bytes (status word, Q8_0 of x); y must
+ * not overlap x or the workspace.  The status word (first uint32 of the
+ * workspace) reports a binary16 scale overflow.
+ * --------------------------------------------------------------------- */
+size_t moe_q4_gemv_workspace_bytes(int64_t T, int32_t H);
+int moe_q4_gemv(const uint8_t* W, int64_t N, int32_t H, const float* x, int64_t T, float* y, void* workspace,
+                size_t ws_bytes, moe_q4_stream_t stream);
+
 /* Static description of an error code. */
 const char* moe_q4_status_string(int status);
 

@@ -43,7 +43,7 @@ EXPORTS = ["moe_q4_quantize_act", "moe_q4_route", "moe_q4_ffn_workspace_bytes", 
            "moe_q4_ffn_host_workspace_bytes", "moe_q4_ffn_forward_host", "moe_q4_status_string",
            "moe_q4_workspace_layout", "moe_q4_ffn_forward_debug", "moe_q4_block_dots",
            "moe_q4_ffn_forward_noalloc", "moe_q4_last_cuda_error", "moe_q4_residual_rmsnorm",
-           "moe_q4_stack_workspace_bytes", "moe_q4_stack_forward"]
+           "moe_q4_stack_workspace_bytes", "moe_q4_stack_forward", "moe_q4_gemv_workspace_bytes", "moe_q4_gemv"]
 
 
 class MoeQ4Error(RuntimeError):
@@ -93,6 +93,8 @@ def _load() -> ctypes.CDLL:
         "moe_q4_residual_rmsnorm": ([P, P, i64, i32, ctypes.c_float, P, P], ctypes.c_int),
         "moe_q4_stack_workspace_bytes": ([P, i64], sz),
         "moe_q4_stack_forward": ([P, i32, P, i64, ctypes.c_float, P, sz, P], ctypes.c_int),
+        "moe_q4_gemv_workspace_bytes": ([i64, i32], sz),
+        "moe_q4_gemv": ([P, i64, i32, P, i64, P, P, sz, P], ctypes.c_int),
     }
     for name, (args, res) in sigs.items():
         f = getattr(lib, name)
@@ -306,3 +308,22 @@ def moe_q4_stack_forward(layers, x: torch.Tensor, eps: float = 1e-6, workspace=N
     _check(_lib.moe_q4_stack_forward(arr, len(layers), _p(x), T, float(eps), _p(workspace), workspace.numel(),
                                      _stream(stream)), "moe_q4_stack_forward")
     return x
+
+
+# ---------------------------------------------------------------- LM-head GEMV
+
+def moe_q4_gemv_workspace_bytes(T: int, H: int) -> int:
+    return int(_lib.moe_q4_gemv_workspace_bytes(int(T), int(H)))
+
+
+def moe_q4_gemv(W: torch.Tensor, x: torch.Tensor, y=None, workspace=None, stream=None):
+    """y [T, N] = W4A8 product of the Q4_0 matrix W [N, H/32, 18] (uint8) with
+    the Q8_0 form of x [T, H] (T <= 8)."""
+    T, H = x.shape
+    N = W.shape[0]
+    y = torch.empty((T, N), dtype=torch.float32, device=x.device) if y is None else y
+    if workspace is None:
+        workspace = alloc_workspace(moe_q4_gemv_workspace_bytes(T, H), x.device)
+    _check(_lib.moe_q4_gemv(_p(W), N, H, _p(x), T, _p(y), _p(workspace), workspace.numel(), _stream(stream)),
+           "moe_q4_gemv")
+    return y

@@ -426,6 +426,35 @@ int moe_q4_stack_forward(const moe_q4_layer* layers, int32_t n_layers, float* x,
     return moe_q4_residual_rmsnorm(x, y, T, H, eps, nullptr, stream);
 }
 
+size_t moe_q4_gemv_workspace_bytes(int64_t T, int32_t H) {
+    if (T < 1 || T > 8 || H <= 0 || H % 256 || H > 16384) return 0;
+    return 256 + align256((size_t)T * H) + align256((size_t)T * (H / QK) * 2);
+}
+
+int moe_q4_gemv(const uint8_t* W, int64_t N, int32_t H, const float* x, int64_t T, float* y, void* workspace,
+                size_t ws_bytes, moe_q4_stream_t stream) {
+    if (T < 0 || T > 8 || N < 1 || N > (int64_t(1) << 30)) return MOE_Q4_ERR_INVALID_ARG;
+    if (H <= 0 || H % 256 || H > 16384) return MOE_Q4_ERR_SHAPE;
+    if (T == 0) return MOE_Q4_OK;
+    if (!W || !x || !y || !workspace) return MOE_Q4_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(x, 16) || !aligned(y, 16) || !aligned(workspace, 256)) return MOE_Q4_ERR_ALIGN;
+    const size_t need = moe_q4_gemv_workspace_bytes(T, H);
+    if (ws_bytes < need) return MOE_Q4_ERR_WORKSPACE;
+    const size_t ybytes = sizeof(float) * (size_t)T * (size_t)N, xbytes = sizeof(float) * (size_t)T * H;
+    if (overlap(y, ybytes, x, xbytes) || overlap(y, ybytes, workspace, need)) return MOE_Q4_ERR_OVERLAP;
+    DeviceInfo dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* base = static_cast<char*>(workspace);
+    uint32_t* status = reinterpret_cast<uint32_t*>(base);
+    int8_t* qa = reinterpret_cast<int8_t*>(base + 256);
+    uint16_t* da = reinterpret_cast<uint16_t*>(base + 256 + align256((size_t)T * H));
+    MOE_TRY(cudaMemsetAsync(status, 0, sizeof(uint32_t), s));
+    MOE_TRY(launch_quantize(x, T, H, qa, da, status, nullptr, s));
+    return cuda_rc(launch_gemv_dp4a(W, N, H, qa, da, (int)T, y, status, dev, s));
+}
+
 int moe_q4_block_dots(const uint8_t* w_blocks, const int8_t* qa, int64_t n, int32_t* out, moe_q4_stream_t stream) {
     if (n < 0 || n > (int64_t(1) << 31) || (n % 8)) return MOE_Q4_ERR_INVALID_ARG;
     if (n == 0) return MOE_Q4_OK;

@@ -59,7 +59,7 @@ constexpr size_t SMEM_ALLOC = SMEM_BYTES + 128;           // slack to align the 
 static_assert(SZ_STAGE % 128 == 0, "TMA destinations need 128-byte alignment");
 static_assert(SMEM_ALLOC <= 200 * 1024, "shared memory map too large");
 
-enum { GATEUP = 0, DOWN = 1 };
+enum { GATEUP = 0, DOWN = 1, GEMV = 2 };
 
 // 2D views of the weight matrices for TMA, in 8-byte elements so that one
 // row segment of a box is a whole chunk row (KC blocks x 18 B, up to 576 B)
@@ -71,6 +71,7 @@ struct StreamMaps {
 
 struct StreamParams {
     int H, F, E, k, P;
+    int N, T;  // GEMV: rows of the matrix, tokens (the slots of the one tile)
     const int8_t* qa;
     const uint16_t* da;
     const int32_t* off;
@@ -166,6 +167,43 @@ __device__ __forceinline__ float int_to_float_exact(int I) {
     return __fsub_rn(__int_as_float(I + 0x4B400000), 12582912.0f);
 }
 
+// acc[r][s0 + j] += the W4A8 block term of block b for slots s0 .. s0 + SPW - 1
+// (activations of a slot: [half][block][16 B] at sa + slot * KC * 32).
+template <int SPW, int RPL_, int ST_>
+__device__ __forceinline__ void block_slots(float (&acc)[RPL_][ST_], int s0, const uint32_t (&qs)[RPL_][4],
+                                            const float (&dW)[RPL_], const int8_t* sa, const uint16_t* sd, int KC,
+                                            int b) {
+    int qa[SPW][8];
+    int base[SPW];
+    float dA[SPW];
+#pragma unroll
+    for (int j = 0; j < SPW; ++j) {
+        const int8_t* a = sa + (size_t)(s0 + j) * KC * QK;
+        const int4 a0 = *reinterpret_cast<const int4*>(a + b * 16);
+        const int4 a1 = *reinterpret_cast<const int4*>(a + (size_t)KC * 16 + b * 16);
+        qa[j][0] = a0.x; qa[j][1] = a0.y; qa[j][2] = a0.z; qa[j][3] = a0.w;
+        qa[j][4] = a1.x; qa[j][5] = a1.y; qa[j][6] = a1.z; qa[j][7] = a1.w;
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sum = __dp4a(qa[j][i], 0x01010101, sum);
+        base[j] = -8 * sum;
+        dA[j] = half_bits_to_float(sd[(s0 + j) * KC + b]);
+    }
+#pragma unroll
+    for (int r = 0; r < RPL_; ++r) {
+#pragma unroll
+        for (int j = 0; j < SPW; ++j) {
+            int I = base[j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                I = dp4a_u8s8(qs[r][i] & 0x0f0f0f0fu, qa[j][i], I);
+                I = dp4a_u8s8((qs[r][i] >> 4) & 0x0f0f0f0fu, qa[j][4 + i], I);
+            }
+            acc[r][s0 + j] = fmaf(int_to_float_exact(I), dW[r] * dA[j], acc[r][s0 + j]);
+        }
+    }
+}
+
 }  // namespace
 
 template <int MODE>
@@ -182,11 +220,11 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = p.H, F = p.F, E = p.E;
-    const int K = (MODE == GATEUP) ? H : F;
+    const int K = (MODE == DOWN) ? F : H;
     const int nb = K / QK;
     const int KC = min(KCMAX, nb);          // nb is a multiple of 8
     const int nchunk = nb / KC;
-    const int n_rb = (MODE == GATEUP) ? F / 32 : H / SR;
+    const int n_rb = (MODE == GATEUP) ? F / 32 : ((MODE == DOWN) ? H / SR : (p.N + SR - 1) / SR);
     const int ngroups = E + 1;
     const uint32_t chunk_bytes = (uint32_t)(SR * KC * Q4_BYTES);
 
@@ -199,21 +237,26 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
         mbar_init(&cbar, NCW);
         mbar_fence_init();
     }
-    for (int i = tid; i <= ngroups; i += THREADS) {
-        tile_off_s[i] = p.tile_off[i];
-        off_s[i] = p.off[i];
+    if (MODE != GEMV) {
+        for (int i = tid; i <= ngroups; i += THREADS) {
+            tile_off_s[i] = p.tile_off[i];
+            off_s[i] = p.off[i];
+        }
     }
     __syncthreads();
-    const int n_items = tile_off_s[ngroups] * n_rb;
+    const int n_items = (MODE == GEMV) ? n_rb : tile_off_s[ngroups] * n_rb;
 
     if (warp == NCW) {
         // ------------------------------------------------------------ producer
         uint32_t ic = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-            const SItem it = item_of(item, n_rb, tile_off_s, off_s, ngroups);
-            const bool sh = it.g >= E;
-            if (lane < it.nslots) {
+            const SItem it = (MODE == GEMV) ? SItem{0, 0, p.T, item} : item_of(item, n_rb, tile_off_s, off_s, ngroups);
+            const bool sh = (MODE != GEMV) && it.g >= E;
+            if (MODE == GEMV && lane < it.nslots) {
+                arow_s[lane] = p.qa + (size_t)lane * H;
+                ascale_s[lane] = p.da + (size_t)lane * (H / QK);
+            } else if (MODE != GEMV && lane < it.nslots) {
                 int tok;
                 float w;
                 const int s = it.slot0 + lane;
@@ -229,7 +272,8 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
             __syncwarp();
             const CUtensorMap* m0 = &maps.m[sh ? 2 : 0];
             const CUtensorMap* m1 = &maps.m[sh ? 3 : 1];
-            const int z = (sh ? 0 : it.g * ((MODE == GATEUP) ? F : H)) + it.rb * ((MODE == GATEUP) ? 32 : SR);
+            const int z = (MODE == GEMV) ? it.rb * SR
+                                         : (sh ? 0 : it.g * ((MODE == GATEUP) ? F : H)) + it.rb * ((MODE == GATEUP) ? 32 : SR);
             for (int c = 0; c < nchunk; ++c, ++ic) {
                 const int st = ic % NST;
                 if (!wait_phase_s(&empty[st], ((ic / NST) & 1) ^ 1, abort)) { ok = false; break; }
@@ -271,7 +315,7 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
         uint32_t ic = 0, cuse = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-            const SItem it = item_of(item, n_rb, tile_off_s, off_s, ngroups);
+            const SItem it = (MODE == GEMV) ? SItem{0, 0, p.T, item} : item_of(item, n_rb, tile_off_s, off_s, ngroups);
             float acc[RPL][ST];
 #pragma unroll
             for (int r = 0; r < RPL; ++r)
@@ -293,38 +337,17 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
                         load_q4_block_smem(sw + (size_t)(RPL * rg + r) * KC * Q4_BYTES + b * Q4_BYTES, qs[r], dbits);
                         dW[r] = half_bits_to_float(dbits);
                     }
+                    // slot passes of 4, 2 or 1 as many slots as the tile holds
 #pragma unroll
                     for (int sp = 0; sp < ST; sp += 4) {
-                        if (sp >= it.nslots) break;
-                        // activation blocks of slots sp..sp+3 for block b
-                        int qa[4][8];
-                        int base[4];
-                        float dA[4];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int8_t* a = sa + (size_t)(sp + j) * KC * QK;
-                            const int4 a0 = *reinterpret_cast<const int4*>(a + b * 16);
-                            const int4 a1 = *reinterpret_cast<const int4*>(a + (size_t)KC * 16 + b * 16);
-                            qa[j][0] = a0.x; qa[j][1] = a0.y; qa[j][2] = a0.z; qa[j][3] = a0.w;
-                            qa[j][4] = a1.x; qa[j][5] = a1.y; qa[j][6] = a1.z; qa[j][7] = a1.w;
-                            int sum = 0;
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) sum = __dp4a(qa[j][i], 0x01010101, sum);
-                            base[j] = -8 * sum;
-                            dA[j] = half_bits_to_float(sd[(sp + j) * KC + b]);
-                        }
-#pragma unroll
-                        for (int r = 0; r < RPL; ++r) {
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                int I = base[j];
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    I = dp4a_u8s8(qs[r][i] & 0x0f0f0f0fu, qa[j][i], I);
-                                    I = dp4a_u8s8((qs[r][i] >> 4) & 0x0f0f0f0fu, qa[j][4 + i], I);
-                                }
-                                acc[r][sp + j] = fmaf(int_to_float_exact(I), dW[r] * dA[j], acc[r][sp + j]);
-                            }
+                        const int rem = it.nslots - sp;
+                        if (rem >= 4) {
+                            block_slots<4>(acc, sp, qs, dW, sa, sd, KC, b);
+                        } else if (rem >= 2) {
+                            block_slots<2>(acc, sp, qs, dW, sa, sd, KC, b);
+                            if (rem == 3) block_slots<1>(acc, sp + 2, qs, dW, sa, sd, KC, b);
+                        } else if (rem == 1) {
+                            block_slots<1>(acc, sp, qs, dW, sa, sd, KC, b);
                         }
                     }
                 }
@@ -364,6 +387,11 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
                         if (ov) atomicOr(p.status, STATUS_SCALE_OVERFLOW);
                     }
                 }
+            } else if (MODE == GEMV) {
+                // warp w: token w & 7, rows 32 (w >> 3) .. + 31 of the item's 64 rows
+                const int s = warp & (ST - 1), r = 32 * (warp / ST) + lane;
+                const int n = it.rb * SR + r;
+                if (s < it.nslots && n < p.N) p.y[(size_t)s * p.N + n] = res[r * ST + s];
             } else {
                 // warp w: slot w & 7, rows 32 (w >> 3) .. + 31 of the 64 rows of H
                 const int s = warp & (ST - 1), r = 32 * (warp / ST) + lane;
@@ -416,6 +444,7 @@ cudaError_t encode_rows_2d(CUtensorMap* map, const uint8_t* base, uint64_t rows,
 StreamParams make_stream_params(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, float* y) {
     StreamParams p;
     p.H = L.H; p.F = L.F; p.E = L.E; p.k = L.k; p.P = (int)(T * L.k);
+    p.N = 0; p.T = 0;
     p.qa = ws.qa; p.da = ws.da; p.off = ws.off; p.tile_off = ws.tile_off; p.sorted = ws.sorted;
     p.topk_w = ws.topk_w; p.hq = ws.hq; p.dh = ws.dh; p.h_dbg = h_dbg; p.y = y; p.status = ws.status;
     return p;
@@ -457,6 +486,26 @@ cudaError_t launch_stream(const LayerView& L, int64_t T, const Workspace& ws, fl
 }
 
 }  // namespace
+
+cudaError_t launch_gemv_dp4a(const uint8_t* W, int64_t N, int H, const int8_t* qa, const uint16_t* da, int T,
+                             float* y, uint32_t* status, const DeviceInfo& dev, cudaStream_t s) {
+    int per_sm = 0;
+    cudaError_t e =
+        kernel_occupancy(reinterpret_cast<const void*>(stream_dp4a_kernel<GEMV>), THREADS, SMEM_ALLOC, &per_sm);
+    if (e != cudaSuccess) return e;
+    StreamMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    const int nb = H / QK, KC = std::min(KCMAX, nb);
+    e = encode_rows_2d(&maps.m[0], W, (uint64_t)N, nb, KC, SR);
+    if (e != cudaSuccess) return e;
+    StreamParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.H = H; p.N = (int)N; p.T = T; p.qa = qa; p.da = da; p.y = y; p.status = status;
+    const int64_t items = ceil_div(N, SR);
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, dev.sm_count));
+    stream_dp4a_kernel<GEMV><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(p, maps);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_gateup_dp4a(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg,
                                const DeviceInfo& dev, cudaStream_t s) {

@@ -62,6 +62,10 @@ cudaError_t launch_gateup_dp4a(const LayerView& L, int64_t T, const Workspace& w
                                const DeviceInfo& dev, cudaStream_t s);
 cudaError_t launch_down_dp4a(const LayerView& L, int64_t T, const Workspace& ws, float* y,
                              const DeviceInfo& dev, cudaStream_t s);
+// y[t][n] (t < T <= 8, n < N) = W4A8 product of Q4_0 rows W [N][H/32] with the
+// Q8_0 activations qa/da of T tokens (the streaming kernel's GEMV mode).
+cudaError_t launch_gemv_dp4a(const uint8_t* W, int64_t N, int H, const int8_t* qa, const uint16_t* da, int T,
+                             float* y, uint32_t* status, const DeviceInfo& dev, cudaStream_t s);
 // k_tc_grouped.cu: grouped projections on tcgen05 (kind::f16, TMEM); the
 // permutation must have been built with TC_TILE_TOKENS slots per tile.
 constexpr int TC_TILE_TOKENS = 64;

@@ -184,6 +184,24 @@ def test_stack_entry_points_reject_bad_args(lib):
     assert f(arr, 3, X, 0, 1e-6, WS, 1 << 40, None) == 0       # T == 0: no-op
 
 
+def test_gemv_rejects_bad_args(lib):
+    wb = lib.moe_q4_gemv_workspace_bytes
+    wb.argtypes, wb.restype = [ctypes.c_int64, ctypes.c_int32], ctypes.c_size_t
+    assert wb(1, 2048) == 256 + 2048 + 256 and wb(9, 2048) == 0 and wb(1, 2000) == 0
+    g = lib.moe_q4_gemv
+    g.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    Wp, X, Y, WS = FAKE, FAKE + 0x1000000, FAKE + 0x2000000, FAKE + 0x3000000
+    assert g(Wp, 1000, 2048, X, 9, Y, WS, 1 << 20, None) == -1      # T > 8
+    assert g(Wp, 0, 2048, X, 1, Y, WS, 1 << 20, None) == -1         # no rows
+    assert g(Wp, 1000, 2000, X, 1, Y, WS, 1 << 20, None) == -2      # H not a multiple of 256
+    assert g(None, 1000, 2048, X, 1, Y, WS, 1 << 20, None) == -1
+    assert g(Wp + 8, 1000, 2048, X, 1, Y, WS, 1 << 20, None) == -3
+    assert g(Wp, 1000, 2048, X, 1, Y, WS, 100, None) == -4
+    assert g(Wp, 1000, 2048, X, 1, X, WS, 1 << 20, None) == -7      # y is x
+    assert g(Wp, 1000, 2048, X, 0, Y, WS, 1 << 20, None) == 0       # T == 0: no-op
+
+
 def test_product_package_does_not_use_the_oracle():
     pkg = os.path.join(ROOT, "quantized_moe_q4_b200")
     for dirpath, _, files in os.walk(pkg):

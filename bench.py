@@ -76,6 +76,23 @@ def oracle_sample(x, lw, seconds=10.0):
     return n / dt, n, dt, cores
 
 
+def simd_sample(x, lw, seconds=5.0):
+    """The host SIMD W4A8 decode (the page's own CPU decode method) on a
+    bounded token sample, like the oracle's."""
+    import cpu_simd
+    cores = cpu_simd.set_threads(physical_cores())
+    t0 = time.perf_counter()
+    cpu_simd.moe_forward(lw, x[:64])
+    rate = 64 / (time.perf_counter() - t0)
+    n = int(min(max(64, rate * seconds), 20000))
+    idx = np.arange(n) % x.shape[0]
+    xs = np.ascontiguousarray(x[idx])
+    t0 = time.perf_counter()
+    cpu_simd.moe_forward(lw, xs)
+    dt = time.perf_counter() - t0
+    return n / dt, n, dt, cores
+
+
 def rank_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
@@ -542,7 +559,12 @@ def run_ours(args):
     gemv = gemv_lines(m, torch, stream) if rank == 0 and "gemv" in extras else None
 
     cpu = None
+    simd = None
     if rank == 0 and world == 1 and "cpu" in extras:
+        v2, n2, dt2, cores2 = simd_sample(x_np, lw, seconds=5.0)
+        simd = {"value": v2, "unit": "tokens/s", "cores": cores2, "kind": "simd_w4a8",
+                "sample": f"{n2} tokens of the decode workload, {dt2:.1f} s, AVX2/VNNI integer W4A8 "
+                          f"(cpu_simd/, the page's CPU decode method) on {cores2} physical cores"}
         v, n, dt, cores = oracle_sample(x_np, lw, seconds=10.0)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{n} tokens of the decode workload (T=1 each, independent), {dt:.1f} s, "
@@ -560,6 +582,7 @@ def run_ours(args):
         "roofline": roofline,
         "token_hbm_frac": tok_frac,
         "cpu_baseline": cpu,
+        "cpu_simd_baseline": simd,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": N_TOKENS * H * 4,
                 "d2h_bytes_per_step": N_TOKENS * H * 4, "how": "moe_q4_ffn_forward_host per token (pinned "
                                                               "host x/y), graph-captured"},

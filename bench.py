@@ -349,6 +349,37 @@ def gemv_lines(m, torch, stream):
     return out
 
 
+def streamed_lines(m, torch, stream):
+    """Host-streamed experts (expert matrices in page-locked host memory,
+    the selected experts copied per call): decode T = 1 and the 947-token
+    prefill; link GB/s over the expert bytes that cross per call."""
+    import synth
+    out = {}
+    for name, T in (("decode_t1", 1), ("prefill_t947", 947)):
+        x_np, lw = synth.workload_inputs(name, seed=0, T=T if name == "decode_t1" else None)
+        Lh = m.Layer.from_host_pinned(lw)
+        x = torch.from_numpy(x_np[:T].copy()).cuda()
+        y = torch.empty_like(x)
+        ws = m.alloc_workspace(m.moe_q4_ffn_workspace_bytes(Lh, T))
+        st = m.alloc_workspace(m.moe_q4_staging_bytes(Lh))
+        times = []
+        for rep in range(6):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            m.moe_q4_ffn_forward_streamed(Lh, x, y, ws, st, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 2:
+                times.append(e0.elapsed_time(e1))
+        ms = float(np.median(times))
+        cnt = m.workspace_views(Lh, T, ws)["cnt"][:lw.n_experts].cpu().numpy()
+        staged = (int(np.count_nonzero(cnt)) + 1) * 3 * lw.ffn * (lw.hidden // 32) * 18
+        out[name] = {"T": T, "ms": ms, "tokens_per_s": T / (ms * 1e-3), "expert_bytes_staged": staged,
+                     "link_gbs": staged / (ms * 1e-3) / 1e9}
+        del Lh, x, y, ws, st
+    return out
+
+
 def stack_lines(m, torch, stream):
     """The 40-layer stack (x <- x + MoE_l(RMSNorm(x)), independently seeded
     layers, 9.1 GB of weights: every step is L2-cold) through the one-call
@@ -557,6 +588,7 @@ def run_ours(args):
     stack = stack_lines(m, torch, stream) if rank == 0 and "stack" in extras else None
     chunked = chunked_lines(m, torch, stream) if rank == 0 and "chunked" in extras else None
     gemv = gemv_lines(m, torch, stream) if rank == 0 and "gemv" in extras else None
+    streamed = streamed_lines(m, torch, stream) if rank == 0 and "streamed" in extras else None
 
     cpu = None
     simd = None
@@ -592,6 +624,7 @@ def run_ours(args):
         "stack": stack,
         "chunked_prefill": chunked,
         "lm_head_gemv": gemv,
+        "host_streamed_experts": streamed,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -610,8 +643,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--replicas", type=int, default=REPLICAS,
                     help="device copies of the decode layer the tokens rotate over (16: L2-cold)")
-    ap.add_argument("--extras", default="prefill,stack,chunked,gemv,cpu",
-                    help="comma list of the extra lines to run (prefill, stack, chunked, gemv, cpu) or 'none'")
+    ap.add_argument("--extras", default="prefill,stack,chunked,gemv,streamed,cpu",
+                    help="comma list of the extra lines (prefill, stack, chunked, gemv, streamed, cpu) or 'none'")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -190,6 +190,27 @@ int moe_q4_stack_forward(const moe_q4_layer* layers, int32_t n_layers, float* x,
                          void* workspace, size_t ws_bytes, moe_q4_stream_t stream);
 
 /* ---------------------------------------------------------------------
+ * Host-streamed experts.
+ *
+ * The page keeps its expert weights in page-locked host memory and streams
+ * them to a small GPU layer by layer (Methodologie 1 and 2).  Here the
+ * expert matrices of L (w_gate, w_up, w_down and the shared ones) are
+ * PAGE-LOCKED HOST pointers (cudaHostAlloc / cudaHostRegister; pageable
+ * memory is rejected with MOE_Q4_ERR_INVALID_ARG), while w_router,
+ * router_bias, x, y, the workspace and `staging` are device memory.  Each
+ * call routes the tokens on the device, copies exactly the experts that the
+ * routing selects (and the shared expert) into `staging` (at least
+ * moe_q4_staging_bytes(L) bytes, 256-byte aligned: a device copy laid out
+ * like the layer), with the GPU reading the host pages directly, and then
+ * runs moe_q4_ffn_forward on the staged copy.  No host synchronisation:
+ * the call is stream-ordered and graph-capturable.  Same results as
+ * moe_q4_ffn_forward on a resident copy of the layer.
+ * --------------------------------------------------------------------- */
+size_t moe_q4_staging_bytes(const moe_q4_layer* L);
+int moe_q4_ffn_forward_streamed(const moe_q4_layer* L, const float* x, int64_t T, float* y, void* workspace,
+                                size_t ws_bytes, void* staging, size_t staging_bytes, moe_q4_stream_t stream);
+
+/* ---------------------------------------------------------------------
  * W4A8 GEMV of one large Q4_0 matrix (the LM head).
  *
  * The page reports the LM head run on the GPU against the CPU (Resultaten,

@@ -17,6 +17,7 @@ import ctypes
 import os
 from typing import Optional
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -43,7 +44,8 @@ EXPORTS = ["moe_q4_quantize_act", "moe_q4_route", "moe_q4_ffn_workspace_bytes", 
            "moe_q4_ffn_host_workspace_bytes", "moe_q4_ffn_forward_host", "moe_q4_status_string",
            "moe_q4_workspace_layout", "moe_q4_ffn_forward_debug", "moe_q4_block_dots",
            "moe_q4_ffn_forward_noalloc", "moe_q4_last_cuda_error", "moe_q4_residual_rmsnorm",
-           "moe_q4_stack_workspace_bytes", "moe_q4_stack_forward", "moe_q4_gemv_workspace_bytes", "moe_q4_gemv"]
+           "moe_q4_stack_workspace_bytes", "moe_q4_stack_forward", "moe_q4_gemv_workspace_bytes", "moe_q4_gemv",
+           "moe_q4_staging_bytes", "moe_q4_ffn_forward_streamed"]
 
 
 class MoeQ4Error(RuntimeError):
@@ -95,6 +97,8 @@ def _load() -> ctypes.CDLL:
         "moe_q4_stack_forward": ([P, i32, P, i64, ctypes.c_float, P, sz, P], ctypes.c_int),
         "moe_q4_gemv_workspace_bytes": ([i64, i32], sz),
         "moe_q4_gemv": ([P, i64, i32, P, i64, P, P, sz, P], ctypes.c_int),
+        "moe_q4_staging_bytes": ([P], sz),
+        "moe_q4_ffn_forward_streamed": ([P, P, i64, P, P, sz, P, sz, P], ctypes.c_int),
     }
     for name, (args, res) in sigs.items():
         f = getattr(lib, name)
@@ -165,6 +169,19 @@ class Layer:
             return None if a is None else torch.from_numpy(a).to(device).contiguous()
         return cls(w.hidden, w.ffn, w.n_experts, w.top_k, dev(w.w_router), dev(w.router_bias),
                    dev(w.w_gate), dev(w.w_up), dev(w.w_down), dev(w.sh_gate), dev(w.sh_up), dev(w.sh_down))
+
+    @classmethod
+    def from_host_pinned(cls, w, device="cuda"):
+        """Router weights on the device, expert matrices in page-locked host
+        memory (for moe_q4_ffn_forward_streamed)."""
+        def dev(a):
+            return None if a is None else torch.from_numpy(a).to(device).contiguous()
+
+        def pinned(a):
+            return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+        return cls(w.hidden, w.ffn, w.n_experts, w.top_k, dev(w.w_router), dev(w.router_bias),
+                   pinned(w.w_gate), pinned(w.w_up), pinned(w.w_down), pinned(w.sh_gate), pinned(w.sh_up),
+                   pinned(w.sh_down))
 
     def replica(self):
         """A copy of every weight tensor at new device addresses."""
@@ -326,4 +343,26 @@ def moe_q4_gemv(W: torch.Tensor, x: torch.Tensor, y=None, workspace=None, stream
         workspace = alloc_workspace(moe_q4_gemv_workspace_bytes(T, H), x.device)
     _check(_lib.moe_q4_gemv(_p(W), N, H, _p(x), T, _p(y), _p(workspace), workspace.numel(), _stream(stream)),
            "moe_q4_gemv")
+    return y
+
+
+# ---------------------------------------------------------------- host-streamed experts
+
+def moe_q4_staging_bytes(layer: Layer) -> int:
+    return int(_lib.moe_q4_staging_bytes(layer.ref))
+
+
+def moe_q4_ffn_forward_streamed(layer: Layer, x: torch.Tensor, y=None, workspace=None, staging=None, stream=None):
+    """The layer with its expert matrices in page-locked host memory (see
+    Layer.from_host_pinned): the experts the routing selects are copied into
+    `staging` on the device, then the layer runs there."""
+    T = x.shape[0]
+    y = torch.empty_like(x) if y is None else y
+    if workspace is None:
+        workspace = alloc_workspace(moe_q4_ffn_workspace_bytes(layer, T), x.device)
+    if staging is None:
+        staging = alloc_workspace(moe_q4_staging_bytes(layer), x.device)
+    _check(_lib.moe_q4_ffn_forward_streamed(layer.ref, _p(x), T, _p(y), _p(workspace), workspace.numel(),
+                                            _p(staging), staging.numel(), _stream(stream)),
+           "moe_q4_ffn_forward_streamed")
     return y

@@ -455,6 +455,93 @@ int moe_q4_gemv(const uint8_t* W, int64_t N, int32_t H, const float* x, int64_t 
     return cuda_rc(launch_gemv_dp4a(W, N, H, qa, da, (int)T, y, status, dev, s));
 }
 
+// Staging copy of a layer's experts on the device: gate [E] | up [E] | down [E]
+// | shared gate | shared up | shared down, each region 256-byte aligned.
+static void staging_layout(const moe_q4_layer* L, size_t off[7]) {
+    const size_t gu = (size_t)L->ffn * (L->hidden / QK) * Q4_BYTES;
+    const size_t dn = (size_t)L->hidden * (L->ffn / QK) * Q4_BYTES;
+    const size_t E = (size_t)L->n_experts, S = L->has_shared ? 1 : 0;
+    const size_t sz[6] = {E * gu, E * gu, E * dn, S * gu, S * gu, S * dn};
+    off[0] = 0;
+    for (int i = 0; i < 6; ++i) off[i + 1] = off[i] + align256(sz[i]);
+}
+
+static bool pinned_host(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeHost;
+}
+
+static bool on_device(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+size_t moe_q4_staging_bytes(const moe_q4_layer* L) {
+    if (check_layer(L)) return 0;
+    size_t off[7];
+    staging_layout(L, off);
+    return off[6];
+}
+
+int moe_q4_ffn_forward_streamed(const moe_q4_layer* L, const float* x, int64_t T, float* y, void* workspace,
+                                size_t ws_bytes, void* staging, size_t staging_bytes, moe_q4_stream_t stream) {
+    int rc = check_layer(L);
+    if (rc) return rc;
+    if (T < 0 || T > T_LIMIT) return MOE_Q4_ERR_INVALID_ARG;
+    if (T == 0) return MOE_Q4_OK;
+    if (!x || !y || !workspace || !staging) return MOE_Q4_ERR_INVALID_ARG;
+    if (!aligned(staging, 256) || !aligned(workspace, 256)) return MOE_Q4_ERR_ALIGN;
+    size_t soff[7];
+    staging_layout(L, soff);
+    if (staging_bytes < soff[6]) return MOE_Q4_ERR_WORKSPACE;
+    // the experts must be page-locked host memory (read by the GPU through
+    // unified addressing); the router weights and x, y device memory
+    const void* host_mats[6] = {L->w_gate, L->w_up, L->w_down, L->sh_gate, L->sh_up, L->sh_down};
+    for (int i = 0; i < (L->has_shared ? 6 : 3); ++i)
+        if (!pinned_host(host_mats[i])) return MOE_Q4_ERR_INVALID_ARG;
+    if (!on_device(L->w_router) || (L->router_bias && !on_device(L->router_bias)) || !on_device(x) ||
+        !on_device(y) || !on_device(staging) || !on_device(workspace))
+        return MOE_Q4_ERR_INVALID_ARG;
+    const LayerView Lv = view(L);
+    size_t off[WS_COUNT];
+    layout(Lv, T, off);
+    if (ws_bytes < off[WS_TOTAL]) return MOE_Q4_ERR_WORKSPACE;
+    DeviceInfo dev;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Workspace w = carve(workspace, off);
+    // routing and its per-expert counts, on the device
+    MOE_TRY(launch_router_logits(Lv, x, T, w.logits, w.status, s));
+    MOE_TRY(launch_topk(w.logits, T, Lv.E, Lv.k, w.topk_idx, w.topk_w, s));
+    MOE_TRY(launch_permute(w.topk_idx, T, Lv.k, Lv.E, Lv.S, DP4A_TT, w, s));
+    uint8_t* st = static_cast<uint8_t*>(staging);
+    StageParams sp;
+    sp.E = Lv.E; sp.S = Lv.S;
+    sp.gu_bytes = (size_t)Lv.F * (Lv.H / QK) * Q4_BYTES;
+    sp.dn_bytes = (size_t)Lv.H * (Lv.F / QK) * Q4_BYTES;
+    sp.cnt = w.cnt;
+    sp.h_gate = L->w_gate; sp.h_up = L->w_up; sp.h_down = L->w_down;
+    sp.h_sh_gate = L->sh_gate; sp.h_sh_up = L->sh_up; sp.h_sh_down = L->sh_down;
+    sp.d_gate = st + soff[0]; sp.d_up = st + soff[1]; sp.d_down = st + soff[2];
+    sp.d_sh_gate = st + soff[3]; sp.d_sh_up = st + soff[4]; sp.d_sh_down = st + soff[5];
+    MOE_TRY(launch_stage_experts(sp, dev, s));
+    moe_q4_layer Ls = *L;
+    Ls.w_gate = sp.d_gate; Ls.w_up = sp.d_up; Ls.w_down = sp.d_down;
+    if (L->has_shared) {
+        Ls.sh_gate = sp.d_sh_gate; Ls.sh_up = sp.d_sh_up; Ls.sh_down = sp.d_sh_down;
+    }
+    return forward_impl(&Ls, x, T, y, workspace, ws_bytes, nullptr, s);
+}
+
 int moe_q4_block_dots(const uint8_t* w_blocks, const int8_t* qa, int64_t n, int32_t* out, moe_q4_stream_t stream) {
     if (n < 0 || n > (int64_t(1) << 31) || (n % 8)) return MOE_Q4_ERR_INVALID_ARG;
     if (n == 0) return MOE_Q4_OK;

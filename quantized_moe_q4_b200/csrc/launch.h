@@ -84,6 +84,27 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
 cudaError_t launch_block_dots(const uint8_t* w, const int8_t* qa, int64_t n, int32_t* out,
                               cudaStream_t s);
 
+// k_stage.cu: copy the experts with cnt[g] > 0 (and the shared expert) from
+// pinned host memory (h_*) into the device staging copy (d_*).
+struct StageParams {
+    int E, S;
+    size_t gu_bytes, dn_bytes;  // one expert's gate (or up) matrix, one down matrix
+    const int32_t* cnt;
+    const uint8_t* h_gate;
+    const uint8_t* h_up;
+    const uint8_t* h_down;
+    const uint8_t* h_sh_gate;
+    const uint8_t* h_sh_up;
+    const uint8_t* h_sh_down;
+    uint8_t* d_gate;
+    uint8_t* d_up;
+    uint8_t* d_down;
+    uint8_t* d_sh_gate;
+    uint8_t* d_sh_up;
+    uint8_t* d_sh_down;
+};
+cudaError_t launch_stage_experts(const StageParams& p, const DeviceInfo& dev, cudaStream_t s);
+
 // k_stack.cu: x += y (if y), then xn = RMSNorm(x) (if xn); H a multiple of 128.
 cudaError_t launch_residual_rmsnorm(float* x, const float* y, int64_t T, int H, float eps, float* xn,
                                     cudaStream_t s);

@@ -1,0 +1,75 @@
+"""Host-streamed experts: the expert matrices in page-locked host memory,
+the routing-selected experts copied to the device per call.  Results equal
+the resident layer's (bit for bit on the deterministic T = 1 path; within
+the fp32 atomic-combine order elsewhere), exactly the selected experts are
+staged, and pageable host memory is refused before anything runs."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import rule13, workload
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import quantized_moe_q4_b200 as m  # noqa: E402
+
+
+def _both(name, T=None):
+    x, lw = workload(name, T=T)
+    return x, lw, m.Layer.from_host(lw), m.Layer.from_host_pinned(lw)
+
+
+def test_streamed_decode_tokens_bit_identical():
+    x, lw, Ld, Lh = _both("decode_t1", T=1000)
+    for t in (0, 1, 2, 999):
+        xt = torch.from_numpy(x[t:t + 1].copy()).cuda()
+        y_res = m.moe_q4_ffn_forward(Ld, xt)
+        y_str = m.moe_q4_ffn_forward_streamed(Lh, xt)
+        torch.cuda.synchronize()
+        assert torch.equal(y_res, y_str)
+
+
+@pytest.mark.parametrize("name,T", [("prefill_t947", 16), ("prefill_t947", None), ("tiny_t16", None)])
+def test_streamed_matches_resident(name, T):
+    x, lw, Ld, Lh = _both(name)
+    x = x if T is None else x[:T]
+    xd = torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    y_res = m.moe_q4_ffn_forward(Ld, xd).cpu().numpy()
+    y_str = m.moe_q4_ffn_forward_streamed(Lh, xd).cpu().numpy()
+    ok, worst = rule13(y_str, y_res, 1e-5)
+    assert ok, worst
+
+
+def test_only_selected_experts_are_staged():
+    x, lw, Ld, Lh = _both("decode_t1", T=1000)
+    xt = torch.from_numpy(x[:3].copy()).cuda()
+    staging = m.alloc_workspace(m.moe_q4_staging_bytes(Lh))
+    staging.fill_(0xA5)
+    ws = m.alloc_workspace(m.moe_q4_ffn_workspace_bytes(Lh, 3))
+    m.moe_q4_ffn_forward_streamed(Lh, xt, workspace=ws, staging=staging)
+    torch.cuda.synchronize()
+    idx = m.workspace_views(Lh, 3, ws)["topk_idx"].cpu().numpy()
+    active = set(idx.ravel().tolist())
+    st = staging.cpu().numpy()
+    E, F, H = lw.n_experts, lw.ffn, lw.hidden
+    gu = F * (H // 32) * 18
+    for e in range(E):
+        seg = st[e * gu:(e + 1) * gu]
+        if e in active:
+            assert np.array_equal(seg, lw.w_gate[e].reshape(-1))
+        else:
+            assert np.all(seg == 0xA5), f"expert {e} was staged without being selected"
+
+
+def test_pageable_host_memory_is_refused():
+    x, lw = workload("tiny_t16")
+    d = lambda a: None if a is None else torch.from_numpy(a).cuda()  # noqa: E731
+    h = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a))  # noqa: E731  (not pinned)
+    L = m.Layer(lw.hidden, lw.ffn, lw.n_experts, lw.top_k, d(lw.w_router), d(lw.router_bias),
+                h(lw.w_gate), h(lw.w_up), h(lw.w_down))
+    with pytest.raises(m.MoeQ4Error) as e:
+        m.moe_q4_ffn_forward_streamed(L, torch.from_numpy(x).cuda())
+    assert e.value.code == -1

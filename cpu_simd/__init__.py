@@ -3,6 +3,7 @@ own decode method, integer multiply-adds over unpacked nibbles), built with
 gcc for the machine it runs on.  Independent of the CUDA library and of the
 oracle; the GPU library never loads it."""
 import ctypes
+import hashlib
 import os
 import subprocess
 from typing import Optional
@@ -11,8 +12,25 @@ import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "w4a8_simd.c")
-LIB = os.path.join(HERE, "libw4a8_simd.so")
 CFLAGS = ["-O3", "-march=native", "-fPIC", "-shared", "-fopenmp", "-std=c11"]
+
+
+def _cpu_tag() -> str:
+    """Short hash of this CPU's feature flags: the library is built with
+    -march=native, so a copy built on another machine is never reused."""
+    flags = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("flags"):
+                    flags = line
+                    break
+    except OSError:
+        pass
+    return hashlib.sha256(flags.encode()).hexdigest()[:12]
+
+
+LIB = os.path.join(HERE, f"libw4a8_simd_{_cpu_tag()}.so")
 
 _lib = None
 

@@ -318,6 +318,38 @@ def chunked_lines(m, torch, stream):
     return out
 
 
+def batch64_lines(m, torch, stream):
+    """One layer on a decode batch of 64 tokens (the streaming dp4a path):
+    tokens/s, and HBM GB/s over the experts the batch activates + Wr + x/y;
+    the layer rotates over 4 device copies (912 MB) so every rep is L2-cold."""
+    import synth
+    hbm, src = measured_peaks()
+    x_np, lw = synth.workload_inputs("prefill_t947", seed=0)
+    base = m.Layer.from_host(lw)
+    layers = [base] + [base.replica() for _ in range(3)]
+    T = 64
+    x = torch.from_numpy(x_np[:T].copy()).cuda()
+    y = torch.empty_like(x)
+    ws = m.alloc_workspace(m.moe_q4_ffn_workspace_bytes(base, T))
+    times = []
+    for rep in range(12):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        m.moe_q4_ffn_forward(layers[rep % 4], x, y, ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if rep >= 4:
+            times.append(e0.elapsed_time(e1))
+    us = float(np.median(times)) * 1000.0
+    cnt = m.workspace_views(base, T, ws)["cnt"][:lw.n_experts].cpu().numpy()
+    active = int(np.count_nonzero(cnt)) + 1
+    nbytes = active * 3 * lw.ffn * (lw.hidden // 32) * 18 + lw.n_experts * lw.hidden * 4 + 2 * T * lw.hidden * 4
+    del layers
+    return {"T": T, "us": us, "tokens_per_s": T / (us * 1e-6), "active_experts": active,
+            "algorithmic_bytes": nbytes, "hbm_gbs": nbytes / (us * 1e-6) / 1e9,
+            "hbm_frac": nbytes / (us * 1e-6) / 1e9 / hbm, "peak_source": src}
+
+
 def gemv_lines(m, torch, stream):
     """The W4A8 LM-head GEMV: one 131072 x 2048 Q4_0 matrix (151 MB, beyond
     the 126 MB L2; two copies alternate so every rep is L2-cold) against
@@ -588,6 +620,7 @@ def run_ours(args):
     stack = stack_lines(m, torch, stream) if rank == 0 and "stack" in extras else None
     chunked = chunked_lines(m, torch, stream) if rank == 0 and "chunked" in extras else None
     gemv = gemv_lines(m, torch, stream) if rank == 0 and "gemv" in extras else None
+    batch64 = batch64_lines(m, torch, stream) if rank == 0 and "batch64" in extras else None
     streamed = streamed_lines(m, torch, stream) if rank == 0 and "streamed" in extras else None
 
     cpu = None
@@ -624,6 +657,7 @@ def run_ours(args):
         "stack": stack,
         "chunked_prefill": chunked,
         "lm_head_gemv": gemv,
+        "decode_batch64": batch64,
         "host_streamed_experts": streamed,
     }
     if rank == 0:
@@ -643,8 +677,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--replicas", type=int, default=REPLICAS,
                     help="device copies of the decode layer the tokens rotate over (16: L2-cold)")
-    ap.add_argument("--extras", default="prefill,stack,chunked,gemv,streamed,cpu",
-                    help="comma list of the extra lines (prefill, stack, chunked, gemv, streamed, cpu) or 'none'")
+    ap.add_argument("--extras", default="prefill,stack,chunked,gemv,batch64,streamed,cpu",
+                    help="comma list of the extra lines (prefill, stack, chunked, gemv, batch64, streamed, cpu) "
+                         "or 'none'")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -97,6 +97,33 @@ def rank_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The slowest rank's value (every rank calls this in the same order); the
+    value itself on one rank or without a process group."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Units every rank processed, over the slowest rank's time (weak scaling)."""
+    return world * units_per_rank / (ms / 1000.0)
+
+
+def rank_tokens(x0: np.ndarray, rank: int) -> np.ndarray:
+    """The decode tokens of one replica: rank 0 the workload's own, rank r > 0
+    its own seeded draw of the same shape (the layer weights are the same on
+    every rank)."""
+    if rank == 0:
+        return x0
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([17, rank])))
+    return rng.standard_normal(x0.shape, dtype=np.float32)
+
+
 def run_reference(args):
     rank, world, _ = rank_env()
     if rank != 0:
@@ -491,7 +518,8 @@ def run_ours(args):
     import quantized_moe_q4_b200 as m
     import synth
 
-    x_np, lw = synth.workload_inputs(WORKLOAD, seed=0, T=N_TOKENS)
+    x0_np, lw = synth.workload_inputs(WORKLOAD, seed=0, T=N_TOKENS)
+    x_np = rank_tokens(x0_np, rank)          # each replica decodes its own tokens
     base = m.Layer.from_host(lw)
     replicas = args.replicas
     layers = [base] + [base.replica() for _ in range(replicas - 1)]
@@ -544,12 +572,9 @@ def run_ours(args):
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
     clk = clocks.stop()
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, "cuda")
     ms_per_step = ms / args.steps
-    value = world * N_TOKENS * args.steps / (ms / 1000.0)
+    value = whole_job_rate(N_TOKENS * args.steps, world, ms)
 
     # dominant kernel (the fused T=1 FFN kernel) timed live with events around each launch
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(N_TOKENS)]
@@ -608,11 +633,8 @@ def run_ours(args):
     ev1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * N_TOKENS * args.steps / (e2e_ms / 1000.0)
+    e2e_ms = max_over_ranks(e2e_ms, "cuda")
+    e2e_value = whole_job_rate(N_TOKENS * args.steps, world, e2e_ms)
     del g3
 
     extras = set(args.extras.split(",")) if args.extras != "none" else set()

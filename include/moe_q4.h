@@ -275,6 +275,10 @@ typedef struct {
     int32_t path;     /* MOE_Q4_PATH_* */
     void* ev_start;   /* cudaEvent_t recorded just before the dominant (gate/up) kernel, or NULL */
     void* ev_stop;    /* cudaEvent_t recorded just after it, or NULL */
+    int32_t force_spin_timeout;  /* nonzero: the fused T = 1 kernel's grid barrier waits for one more
+                                    CTA than exists, so its bounded wait runs out; the call completes
+                                    with correct results and MOE_Q4_STATUS_SPIN_TIMEOUT in the status
+                                    word (tests of the timeout report; about a second per call) */
 } moe_q4_debug;
 
 /* moe_q4_ffn_forward with inspection options (see moe_q4_debug). */

@@ -69,7 +69,7 @@ class _Layer(ctypes.Structure):
 
 class _Debug(ctypes.Structure):
     _fields_ = [("h_out", ctypes.c_void_p), ("path", ctypes.c_int32),
-                ("ev_start", ctypes.c_void_p), ("ev_stop", ctypes.c_void_p)]
+                ("ev_start", ctypes.c_void_p), ("ev_stop", ctypes.c_void_p), ("force_spin_timeout", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -234,11 +234,11 @@ def moe_q4_ffn_forward(layer: Layer, x: torch.Tensor, y=None, workspace=None, st
 
 
 def moe_q4_ffn_forward_debug(layer: Layer, x: torch.Tensor, y, workspace, h_out=None, path=PATH_AUTO,
-                             ev_start=None, ev_stop=None, stream=None):
+                             ev_start=None, ev_stop=None, stream=None, force_spin_timeout=False):
     T = x.shape[0]
     dbg = _Debug(None if h_out is None else h_out.data_ptr(), int(path),
                  None if ev_start is None else ev_start.cuda_event,
-                 None if ev_stop is None else ev_stop.cuda_event)
+                 None if ev_stop is None else ev_stop.cuda_event, int(bool(force_spin_timeout)))
     _check(_lib.moe_q4_ffn_forward_debug(layer.ref, _p(x), T, _p(y), _p(workspace), workspace.numel(),
                                          ctypes.byref(dbg), _stream(stream)), "moe_q4_ffn_forward_debug")
     return y

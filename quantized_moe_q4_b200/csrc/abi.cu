@@ -227,7 +227,8 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
     cudaEvent_t ev1 = dbg ? static_cast<cudaEvent_t>(dbg->ev_stop) : nullptr;
     const int path = dbg ? dbg->path : MOE_Q4_PATH_AUTO;
     if ((path == MOE_Q4_PATH_AUTO || path == MOE_Q4_PATH_DECODE) && decode_eligible(L, T, dev))
-        return cuda_rc(launch_decode(L, x, y, w, dbg ? dbg->h_out : nullptr, dev, ev0, ev1, s));
+        return cuda_rc(launch_decode(L, x, y, w, dbg ? dbg->h_out : nullptr, dev, ev0, ev1,
+                                     dbg && dbg->force_spin_timeout, s));
 
     // grouped paths: tensor cores once experts see tens of tokens, else dp4a
     const bool tc = (path == MOE_Q4_PATH_TENSOR_CORE) || (path == MOE_Q4_PATH_AUTO && T >= TC_MIN_TOKENS);

@@ -40,6 +40,7 @@ struct DecodeParams {
     int H, F, E, k, S;
     int rows_per_cta;  // down rows of H per FFN CTA
     int nctas;         // grid of decode_ffn_kernel
+    int barrier_target;  // arrivals the grid barrier waits for (nctas; nctas + 1 only in the timeout test)
     const float* x;
     const float* w_router;
     const float* bias;
@@ -449,7 +450,7 @@ __global__ void __maxnreg__(96) decode_ffn_kernel(DecodeParams p) {
 
     // ---- every CTA's requantised rows are written: grid barrier
     __threadfence();
-    grid_barrier_bounded(p.status + 1, (uint32_t)p.nctas, p.status, STATUS_SPIN_TIMEOUT);
+    grid_barrier_bounded(p.status + 1, (uint32_t)p.barrier_target, p.status, STATUS_SPIN_TIMEOUT);
 
     if (rows > 0) {
         // requantised SwiGLU rows of all k+1 slots (L2: written by other SMs)
@@ -502,10 +503,12 @@ bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev) {
 }
 
 cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Workspace& ws, float* h_dbg,
-                          const DeviceInfo& dev, cudaEvent_t ev_start, cudaEvent_t ev_stop, cudaStream_t s) {
+                          const DeviceInfo& dev, cudaEvent_t ev_start, cudaEvent_t ev_stop, bool force_timeout,
+                          cudaStream_t s) {
     DecodeParams p;
     p.H = L.H; p.F = L.F; p.E = L.E; p.k = L.k; p.S = L.S;
     p.nctas = dev.sm_count;
+    p.barrier_target = p.nctas + (force_timeout ? 1 : 0);
     p.rows_per_cta = decode_rows_per_cta(L.H, p.nctas);
     p.x = x; p.w_router = L.w_router; p.bias = L.router_bias;
     p.w_gate = L.w_gate; p.w_up = L.w_up; p.w_down = L.w_down;

@@ -78,8 +78,11 @@ cudaError_t launch_down_tc(const LayerView& L, int64_t T, const Workspace& ws, f
 // chained with programmatic dependent launch).  Events, if given, bracket the
 // FFN kernel.
 bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev);
+// force_timeout: the grid barrier waits for one CTA more than exist (the
+// bounded wait runs out; used only to test the timeout report).
 cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Workspace& ws, float* h_dbg,
-                          const DeviceInfo& dev, cudaEvent_t ev_start, cudaEvent_t ev_stop, cudaStream_t s);
+                          const DeviceInfo& dev, cudaEvent_t ev_start, cudaEvent_t ev_stop, bool force_timeout,
+                          cudaStream_t s);
 
 cudaError_t launch_block_dots(const uint8_t* w, const int8_t* qa, int64_t n, int32_t* out,
                               cudaStream_t s);

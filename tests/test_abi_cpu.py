@@ -142,8 +142,8 @@ def test_other_entry_points_reject_bad_args(lib):
 
     class _D(ctypes.Structure):
         _fields_ = [("h_out", ctypes.c_void_p), ("path", ctypes.c_int32), ("ev_start", ctypes.c_void_p),
-                    ("ev_stop", ctypes.c_void_p)]
-    dbg = _D(None, 9, None, None)
+                    ("ev_stop", ctypes.c_void_p), ("force_spin_timeout", ctypes.c_int32)]
+    dbg = _D(None, 9, None, None, 0)
     assert d(ctypes.byref(L), FAKE, 4, FAKE + 0x1000000, FAKE + 0x2000000, 1 << 40, ctypes.byref(dbg), None) == -1
 
 

@@ -110,9 +110,12 @@ __device__ __forceinline__ void tma_load_2d_(void* dst, const CUtensorMap* map, 
 // Bounded wait; once any wait of the CTA has run out, every later one
 // returns false soon after.
 __device__ __forceinline__ bool wait_phase_s(uint64_t* bar, uint32_t parity, volatile int* abort) {
-    for (uint32_t i = 0; i < LIMIT; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 255u && *abort) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;   // sleeps instead of spinning
+        if (*abort) return false;
+        if (global_ns() - t0 > 2000000000ull) break;                  // 2 s bound
     }
     *abort = 1;
     return false;

@@ -140,10 +140,15 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 
 // Bounded wait shared by all roles: once any wait of the CTA has run out,
 // `abort` is set and every later wait returns false soon after.
+// The waiting thread sleeps in try_wait (suspend hint) rather than spinning;
+// the bound is 2 s of wall time (globaltimer).
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort) {
-    for (uint32_t i = 0; i < LIMIT; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 255u && *abort) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+        if (*abort) return false;
+        if (global_ns() - t0 > 2000000000ull) break;
     }
     *abort = 1;
     return false;

@@ -40,12 +40,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for phase `parity` of `bar`, giving up after `limit` polls.  Returns
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about hint_ns nanoseconds pass, instead of returning at once
+// and spinning (a spinning warp takes issue slots from the warps doing work).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `parity` of `bar`: one immediate test, then try_wait with a
+// suspend hint (the thread sleeps instead of spinning), giving up after about
+// `limit` x 0.5 us of wall time (globaltimer; 2^22 -> about 2 s).  Returns
 // false on timeout (the caller records it; nothing hangs).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit = 1u << 24) {
-    for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns(), bound = (uint64_t)limit * 500u;
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (global_ns() - t0 > bound) return false;
+    }
 }
 
 // Order this thread's earlier generic-proxy accesses of shared memory before

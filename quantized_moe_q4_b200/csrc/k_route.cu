@@ -7,6 +7,8 @@
 // (equal logits: lower expert index first), weights = softmax over those k.
 #include <float.h>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -65,38 +67,72 @@ __global__ void __launch_bounds__(256) router_logits_split(const float* __restri
 }
 
 // ---------------------------------------------------------------------------
-// Logits, many tokens: 64x64 output tile per CTA, K step 16, 4x4 per thread.
+// Logits, many tokens: a 64-token x 64-expert output tile per cluster of RKS
+// CTAs.  CTA z of the cluster covers one contiguous slice of H (whole 32-wide
+// chunks), with the next chunk's loads in flight while the current one is
+// multiplied (4x4 outputs a thread); the RKS partial tiles are then added
+// through distributed shared memory in rank order, each CTA finishing a
+// quarter of the tile, so the sum order is fixed (deterministic).  Splitting
+// H spreads a 947-token batch over 120 SMs instead of 30, and the prefetch
+// hides the L2 latency that a load-then-sync loop pays once per chunk.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) router_logits_tiled(const float* __restrict__ x, int T, int H,
-                                                            const float* __restrict__ Wr,
-                                                            const float* __restrict__ bias, int E,
-                                                            float* __restrict__ logits,
-                                                            uint32_t* __restrict__ status_clear) {
-    if (status_clear && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status_clear = 0u;
-    __shared__ __align__(16) float As[16][68];
-    __shared__ __align__(16) float Bs[16][68];
+constexpr int RKS = 4;     // CTAs per cluster (slices of H)
+constexpr int RBK = 32;    // K chunk
+constexpr int RLD = 68;    // padded row length of the staged tiles
+
+__global__ void __cluster_dims__(1, 1, RKS) __launch_bounds__(256)
+    router_logits_tiled(const float* __restrict__ x, int T, int H, const float* __restrict__ Wr,
+                        const float* __restrict__ bias, int E, float* __restrict__ logits,
+                        uint32_t* __restrict__ status_clear) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    if (status_clear && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) *status_clear = 0u;
+    __shared__ __align__(16) float As[2][RBK][RLD];   // [buffer][k][token]
+    __shared__ __align__(16) float Bs[2][RBK][RLD];   // [buffer][k][expert]
     const int tid = threadIdx.x;
     const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+    const int rank = (int)cluster.block_rank();
     const int tm = tid >> 4, tn = tid & 15;
+    // loader: row lr of the tile, k offsets lc and lc + 16 of the chunk
     const int lr = tid >> 2, lc = (tid & 3) * 4;
+    const bool arow = (m0 + lr) < T, brow = (n0 + lr) < E;
+    const float* xa = x + (size_t)(arow ? m0 + lr : 0) * H + lc;
+    const float* wb = Wr + (size_t)(brow ? n0 + lr : 0) * H + lc;
+    const int nch = H / RBK;
+    const int c0 = rank * nch / RKS, c1 = (rank + 1) * nch / RKS;
+
     float acc[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-    const bool arow = (m0 + lr) < T, brow = (n0 + lr) < E;
-    const float* xa = x + (size_t)(arow ? m0 + lr : 0) * H + lc;
-    const float* wb = Wr + (size_t)(brow ? n0 + lr : 0) * H + lc;
-    for (int k0 = 0; k0 < H; k0 += 16) {
-        const float4 a = arow ? __ldg(reinterpret_cast<const float4*>(xa + k0)) : make_float4(0, 0, 0, 0);
-        const float4 b = brow ? __ldg(reinterpret_cast<const float4*>(wb + k0)) : make_float4(0, 0, 0, 0);
-        As[lc + 0][lr] = a.x; As[lc + 1][lr] = a.y; As[lc + 2][lr] = a.z; As[lc + 3][lr] = a.w;
-        Bs[lc + 0][lr] = b.x; Bs[lc + 1][lr] = b.y; Bs[lc + 2][lr] = b.z; Bs[lc + 3][lr] = b.w;
-        __syncthreads();
+
+    float4 a0 = make_float4(0, 0, 0, 0), a1 = a0, b0 = a0, b1 = a0;
+    auto load = [&](int c) {
+        const int k0 = c * RBK;
+        a0 = arow ? __ldg(reinterpret_cast<const float4*>(xa + k0)) : make_float4(0, 0, 0, 0);
+        a1 = arow ? __ldg(reinterpret_cast<const float4*>(xa + k0 + 16)) : make_float4(0, 0, 0, 0);
+        b0 = brow ? __ldg(reinterpret_cast<const float4*>(wb + k0)) : make_float4(0, 0, 0, 0);
+        b1 = brow ? __ldg(reinterpret_cast<const float4*>(wb + k0 + 16)) : make_float4(0, 0, 0, 0);
+    };
+    auto stage = [&](int buf) {
+        As[buf][lc + 0][lr] = a0.x; As[buf][lc + 1][lr] = a0.y; As[buf][lc + 2][lr] = a0.z; As[buf][lc + 3][lr] = a0.w;
+        As[buf][lc + 16][lr] = a1.x; As[buf][lc + 17][lr] = a1.y; As[buf][lc + 18][lr] = a1.z; As[buf][lc + 19][lr] = a1.w;
+        Bs[buf][lc + 0][lr] = b0.x; Bs[buf][lc + 1][lr] = b0.y; Bs[buf][lc + 2][lr] = b0.z; Bs[buf][lc + 3][lr] = b0.w;
+        Bs[buf][lc + 16][lr] = b1.x; Bs[buf][lc + 17][lr] = b1.y; Bs[buf][lc + 18][lr] = b1.z; Bs[buf][lc + 19][lr] = b1.w;
+    };
+    if (c0 < c1) {
+        load(c0);
+        stage(0);
+    }
+    __syncthreads();
+    for (int c = c0; c < c1; ++c) {
+        const int buf = (c - c0) & 1;
+        if (c + 1 < c1) load(c + 1);   // in flight while this chunk is multiplied
 #pragma unroll
-        for (int kk = 0; kk < 16; ++kk) {
-            const float4 av = *reinterpret_cast<const float4*>(&As[kk][tm * 4]);
-            const float4 bv = *reinterpret_cast<const float4*>(&Bs[kk][tn * 4]);
+        for (int kk = 0; kk < RBK; ++kk) {
+            const float4 av = *reinterpret_cast<const float4*>(&As[buf][kk][tm * 4]);
+            const float4 bv = *reinterpret_cast<const float4*>(&Bs[buf][kk][tn * 4]);
             const float ar[4] = {av.x, av.y, av.z, av.w};
             const float br[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
@@ -104,18 +140,35 @@ __global__ void __launch_bounds__(256) router_logits_tiled(const float* __restri
 #pragma unroll
                 for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(ar[i], br[j], acc[i][j]);
         }
+        // the other buffer was last read in the previous chunk, before the
+        // barrier that ended it
+        if (c + 1 < c1) stage(buf ^ 1);
         __syncthreads();
     }
+
+    // this CTA's partial tile [token][expert] (stride 65) in the A staging area
+    float* part = &As[0][0][0];
+    static_assert(sizeof(As) >= 64 * 65 * sizeof(float), "partial tile fits the A staging area");
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int t = m0 + tm * 4 + i;
-        if (t >= T) continue;
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int e = n0 + tn * 4 + j;
-            if (e < E) logits[(size_t)t * E + e] = acc[i][j] + (bias ? __ldg(bias + e) : 0.0f);
-        }
+        for (int j = 0; j < 4; ++j) part[(tm * 4 + i) * 65 + tn * 4 + j] = acc[i][j];
+    cluster.sync();
+    // CTA `rank` adds rows 16 rank .. 16 rank + 15 of the RKS partials in rank order
+    float* parts[RKS];
+#pragma unroll
+    for (int q = 0; q < RKS; ++q) parts[q] = cluster.map_shared_rank(part, q);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int idx = u * 256 + tid;            // 0 .. 1023 over 16 rows x 64 columns
+        const int r = rank * 16 + (idx >> 6), col = idx & 63;
+        float v = parts[0][r * 65 + col];
+#pragma unroll
+        for (int q = 1; q < RKS; ++q) v += parts[q][r * 65 + col];
+        const int t = m0 + r, e = n0 + col;
+        if (t < T && e < E) logits[(size_t)t * E + e] = v + (bias ? __ldg(bias + e) : 0.0f);
     }
+    cluster.sync();   // the partials stay alive until every CTA of the cluster has read them
 }
 
 // ---------------------------------------------------------------------------
@@ -177,13 +230,13 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
 
 cudaError_t launch_router_logits(const LayerView& L, const float* x, int64_t T, float* logits,
                                  uint32_t* status_clear, cudaStream_t s) {
-    if (T <= 512) {
-        // x rows are re-read once per expert from L2 (at most 512 x H x 4 x E bytes)
+    if (T <= 128) {
+        // x rows are re-read once per expert from L2 (at most 128 x H x 4 x E bytes)
         dim3 grid((unsigned)L.E, (unsigned)ceil_div(T, RT));
         router_logits_split<<<grid, 256, 0, s>>>(x, (int)T, L.H, L.w_router, L.router_bias, L.E, logits,
                                                  status_clear);
     } else {
-        dim3 grid((unsigned)ceil_div(L.E, 64), (unsigned)ceil_div(T, 64));
+        dim3 grid((unsigned)ceil_div(L.E, 64), (unsigned)ceil_div(T, 64), RKS);
         router_logits_tiled<<<grid, 256, 0, s>>>(x, (int)T, L.H, L.w_router, L.router_bias, L.E, logits,
                                                  status_clear);
     }

@@ -82,6 +82,24 @@ def test_route_standalone(name, T):
     assert np.allclose(v["topk_w"].sum(axis=1, dtype=np.float64), 1.0, atol=1e-6)
 
 
+@pytest.mark.parametrize("name,T", [("tiny_t16", 129), ("tiny_t16", 300), ("prefill_t947", 129),
+                                    ("prefill_t947", 1000), ("zipf_t16384", 2048)])
+def test_route_many_tokens_cluster_path(name, T):
+    """Above 128 tokens the logits come from the cluster kernel (H split over 4
+    CTAs, partials added in rank order): ragged token tiles, fewer experts than
+    a tile (E = 16), and the sum order fixed, so two calls agree bit for bit."""
+    x, lw = workload(name, T=T)
+    L = m.Layer.from_host(lw)
+    xd = torch.from_numpy(x).cuda()
+    idx, w, logits = m.moe_q4_route(L, xd)
+    idx2, w2, logits2 = m.moe_q4_route(L, xd)
+    torch.cuda.synchronize()
+    v = dict(logits=logits.cpu().numpy(), topk_idx=idx.cpu().numpy(), topk_w=w.cpu().numpy())
+    check_routing(lw, x, v)
+    assert np.array_equal(v["logits"], logits2.cpu().numpy())
+    assert np.array_equal(v["topk_idx"], idx2.cpu().numpy())
+
+
 # --------------------------------------------------------------- whole layer
 
 @pytest.mark.parametrize("path", PATHS)

@@ -25,30 +25,33 @@
 // Warp roles (14 warps):
 //   0      producer: 2D tensor copies (TMA) of the packed weight rows (a box
 //          of 64 or 128 rows x 144 B = 8 blocks) and 16-byte cp.async gathers
-//          of the slots' int8 activations and their scales, four input stages
-//          in flight (a stage takes about 2 us to land under load);
-//   1..4   converters: nibbles -> binary16 (nib - 8) written straight into
-//          TMEM (tcgen05.st; A is read by the MMA from there, so the weight
-//          operand never touches shared memory), int8 -> binary16 activations
-//          into the K-major shared-memory layout (8-row x 16-byte core
-//          matrices); two operand stages of 4 blocks; block scales into a ring
-//          shared with the epilogue;
-//   5      MMA issuer (one thread): two MMAs per block (A from TMEM, B from
-//          shared memory), one commit per pair of blocks,
-//          descriptors precomputed (the issue path is a handful of instructions);
-//   6..13  epilogue: 4 TMEM lane quarters x 2 column halves; per pair of
-//          blocks two TMEM loads of 32 columns, rescale-accumulate; after the
-//          last block of a tile gate/up -> SwiGLU + Q8_0 requantisation, down ->
-//          y += w_slot * o (fp32 atomics).
-// TMEM: six accumulators of 64 columns, then the A ring (2 stages x 4 blocks x
-// 16 columns); a 16-entry scale ring (so the converters
-// run up to four operand stages ahead of the epilogue); full/empty mbarriers between every pair of
-// roles; every wait bounded, and one that runs out makes every role leave its
-// loop and records STATUS_SPIN_TIMEOUT.
-// The MMA issuer and the epilogue hand accumulators over in pairs (one
-// mbarrier phase per two blocks in each direction): measured on B200, halving
-// the hand-offs took 10-12% off both projections, while deeper rings (eight
-// accumulators, two more input stages) changed nothing.
+//          of the slots' int8 activations and their scales, two input stages
+//          of 8 blocks in flight;
+//   1..4   converters: nibbles -> binary16 (nib - 8) for the A operand and
+//          int8 -> binary16 activations for the B operand, both written into
+//          the K-major shared-memory layout (8-row x 16-byte core matrices);
+//          two operand stages of 4 blocks; block scales into a ring shared
+//          with the epilogue;
+//   5      MMA issuer (one thread): two MMAs per block (A and B from shared
+//          memory), descriptors precomputed; one wait and one commit per
+//          operand stage for its quad of accumulators;
+//   6..13  epilogue: 4 TMEM lane quarters x 2 column halves; per quad of
+//          blocks one wait, then two passes of two TMEM loads of 32 columns
+//          and the rescale-accumulate; after the last block of a tile gate/up
+//          -> SwiGLU + Q8_0 requantisation, down -> y += w_slot * o (fp32
+//          atomics).
+// TMEM: eight accumulators of 64 columns (all 512 columns), handed between the
+// MMA issuer and the epilogue a quad (one operand stage) at a time; a 16-entry
+// scale ring (so the converters run up to four operand stages ahead of the
+// epilogue); full/empty mbarriers between every pair of roles; every wait
+// bounded, and one that runs out makes every role leave its loop and records
+// STATUS_SPIN_TIMEOUT.
+// Why quads: the kernel is bound by its hand-off skeleton rather than by any
+// role's arithmetic (measured on B200: with every role's work removed half of
+// the time remains).  One mbarrier phase per block in each direction became
+// one per pair (-10 to -12%) and then one per quad (-4 to -5% more, which
+// needs all of TMEM for the accumulators and so the A operand in shared
+// memory); deeper rings or more input stages changed nothing.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -69,15 +72,14 @@ constexpr int TM = 128;            // MMA M: weight rows per tile
 constexpr int TN = TC_TILE_TOKENS; // MMA N: slots per tile
 constexpr int IN_KB = 8;           // Q4_0 blocks per input stage (144-byte rows: a 16-byte multiple)
 constexpr int OP_KB = 4;           // blocks per operand stage
-constexpr int NIN = 4, NOP = 2, NTM = 6, NSC = 16;  // input, operand, accumulator and scale ring depths
+constexpr int NIN = 2, NOP = 2, NTM = 8, NSC = 16;  // input, operand, accumulator and scale ring depths
 constexpr int IN_ROW = IN_KB * Q4_BYTES;          // 144
 constexpr int THREADS = 14 * 32;  // 4 warps on some SM sub-partitions: at most 128 registers a thread
 constexpr int W_PROD = 0, W_CONV0 = 1, W_MMA = 5, W_EPI0 = 6;
 constexpr int N_CONV = 128, N_EPI = 256;
-constexpr uint32_t A_COL0 = NTM * TN;             // TMEM columns of the A ring (after the accumulators)
-constexpr uint32_t A_COLS_PER_BLOCK = QK / 2;      // 32 binary16 per row = 16 columns
 constexpr uint32_t TMEM_COLS = 512;
-static_assert(A_COL0 + NOP * OP_KB * A_COLS_PER_BLOCK <= TMEM_COLS, "TMEM budget");
+static_assert(NTM * TN <= TMEM_COLS, "TMEM budget");
+static_assert(NTM == 2 * OP_KB, "two quads of accumulators, one per operand stage");
 constexpr uint32_t LIMIT = 1u << 22;
 static_assert(TN == 64, "the epilogue maps two warps of 32 columns onto a tile");
 
@@ -92,7 +94,10 @@ constexpr size_t OFF_IN_W = 0;
 constexpr size_t OFF_IN_B = OFF_IN_W + NIN * SZ_IN_W;
 constexpr size_t OFF_IN_DA = OFF_IN_B + NIN * SZ_IN_B;
 constexpr size_t OFF_OP_B = (OFF_IN_DA + NIN * SZ_IN_DA + 1023) & ~size_t(1023);
-constexpr size_t OFF_DW = OFF_OP_B + NOP * SZ_OP_B;
+constexpr size_t SZ_KSTEP_A = (size_t)TM * 32;
+constexpr size_t SZ_OP_A = (size_t)OP_KB * 2 * SZ_KSTEP_A;
+constexpr size_t OFF_OP_A = OFF_OP_B + NOP * SZ_OP_B;
+constexpr size_t OFF_DW = OFF_OP_A + NOP * SZ_OP_A;
 constexpr size_t OFF_DA = OFF_DW + (size_t)NSC * TM * 4;
 constexpr size_t OFF_XCH = OFF_DA + (size_t)NSC * TN * 4;
 constexpr size_t SMEM_BYTES = OFF_XCH + (size_t)TM * XCH_LD * 4;
@@ -190,38 +195,17 @@ __device__ __forceinline__ void rescale_acc(float2 (&acc)[16], const uint32_t (&
     }
 }
 
-// D[tmem] (=|+=) A[tmem] x B[smem]^T, binary16 operands, fp32 accumulator;
-// A holds row m in TMEM lane m, K along the columns (two binary16 a column).
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+// D[tmem] (=|+=) A[smem] x B[smem]^T, binary16 operands, fp32 accumulator;
+// both operands K-major in 8-row x 16-byte core matrices.
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                            bool accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
         : "memory");
 }
-
-// 64 consecutive 32-bit columns of this warp's 32 TMEM lanes.
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&v)[64]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,"
-        "%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
-        "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
-        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
-        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31]), "r"(v[32]),
-        "r"(v[33]), "r"(v[34]), "r"(v[35]), "r"(v[36]), "r"(v[37]), "r"(v[38]), "r"(v[39]), "r"(v[40]),
-        "r"(v[41]), "r"(v[42]), "r"(v[43]), "r"(v[44]), "r"(v[45]), "r"(v[46]), "r"(v[47]), "r"(v[48]),
-        "r"(v[49]), "r"(v[50]), "r"(v[51]), "r"(v[52]), "r"(v[53]), "r"(v[54]), "r"(v[55]), "r"(v[56]),
-        "r"(v[57]), "r"(v[58]), "r"(v[59]), "r"(v[60]), "r"(v[61]), "r"(v[62]), "r"(v[63])
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // kind::f16 instruction descriptor: binary16 A and B, fp32 accumulator, both
 // operands K-major, M x N.
@@ -297,8 +281,8 @@ template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, const __grid_constant__ TcMaps maps) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t in_full[NIN], in_empty[NIN], op_full[NOP], op_empty[NOP], tm_full[NTM / 2],
-        tm_empty[NTM / 2], sc_full[NSC], sc_empty[NSC], epi_bar;
+    __shared__ __align__(8) uint64_t in_full[NIN], in_empty[NIN], op_full[NOP], op_empty[NOP], tm_full[2],
+        tm_empty[2], sc_full[NSC], sc_empty[NSC], epi_bar;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ int tile_off_s[258], off_s[258];
@@ -307,6 +291,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
     int8_t* in_b = reinterpret_cast<int8_t*>(smem + OFF_IN_B);
     uint16_t* in_da = reinterpret_cast<uint16_t*>(smem + OFF_IN_DA);
     uint8_t* op_b = smem + OFF_OP_B;
+    uint8_t* op_a = smem + OFF_OP_A;
     float* dw_ring = reinterpret_cast<float*>(smem + OFF_DW);
     float* da_ring = reinterpret_cast<float*>(smem + OFF_DA);
     float* xch = reinterpret_cast<float*>(smem + OFF_XCH);
@@ -334,7 +319,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
             mbar_init(&op_full[i], N_CONV);
             mbar_init(&op_empty[i], 1);
         }
-        for (int i = 0; i < NTM / 2; ++i) {  // one pair of accumulators each
+        for (int i = 0; i < 2; ++i) {  // one quad of accumulators each
             mbar_init(&tm_full[i], 1);
             mbar_init(&tm_empty[i], N_EPI / 32);
         }
@@ -419,7 +404,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
     } else if (warp >= W_CONV0 && warp < W_CONV0 + 4) {
         // ------------------------------------------------------------ converters
         const int ct = tid - W_CONV0 * 32;        // slot column ct & 63 of the activation work
-        const int crow = 32 * (warp & 3) + lane;  // weight row = the TMEM lane this warp may write
+        const int crow = 32 * (warp & 3) + lane;  // weight row this thread converts
         uint32_t i_op = 0, gb = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -431,7 +416,6 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                 const int o = i_op % NOP;
                 if (!wait_phase(&op_empty[o], ((i_op / NOP) & 1) ^ 1, abort)) { ok = false; break; }
                 tc_fence_after_sync();
-                const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + A_COL0 + o * OP_KB * A_COLS_PER_BLOCK;
                 uint8_t* ob = op_b + (size_t)o * SZ_OP_B;
 
                 // weights: this row's 4 blocks, 72 bytes at an 8-byte boundary
@@ -445,7 +429,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                     w[2 * i + 1] = v.y;
                 }
                 float dws[OP_KB];
-                uint32_t v[OP_KB * 16];  // the 4 blocks' binary16 pairs, 64 consecutive TMEM columns
+                uint32_t v[OP_KB * 16];  // the 4 blocks' binary16 pairs of this row, in K order
 #pragma unroll
                 for (int kb = 0; kb < OP_KB; ++kb) {
                     // block kb starts at byte 18 kb: scale, then 16 nibble bytes
@@ -472,9 +456,19 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                         v[16 * kb + 8 + 2 * i + 1] = hi.y;
                     }
                 }
-                // one asynchronous TMEM store of all four blocks; the activation
-                // work below overlaps it, tcgen05.wait::st before the hand-off
-                tmem_st64(ta, v);
+                // this row of the A operand: block kb, K-step ks, core matrix
+                // `core` holds binary16 pairs 16 kb + 8 ks + 4 core .. + 3
+                uint8_t* oa = op_a + (size_t)o * SZ_OP_A;
+#pragma unroll
+                for (int kb = 0; kb < OP_KB; ++kb)
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                        for (int core = 0; core < 2; ++core) {
+                            const int c0 = 16 * kb + 8 * ks + 4 * core;
+                            *reinterpret_cast<uint4*>(oa + op_off(kb, ks, TM, crow, core)) =
+                                make_uint4(v[c0], v[c0 + 1], v[c0 + 2], v[c0 + 3]);
+                        }
                 // activations: slot n = ct & 63, blocks (ct >> 6) and (ct >> 6) + 2
                 const int n = ct & 63;
                 const bool valid = n < T.nslots;
@@ -505,14 +499,12 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                 for (int kb = 0; kb < OP_KB; ++kb)
                     das[kb] = valid ? half_bits_to_float(in_da[(size_t)s * TN * IN_KB + n * IN_KB + sub * OP_KB + kb])
                                     : 0.0f;
-                tmem_wait_st();
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 mbar_arrive(&op_full[o]);
                 if (sub == 1) mbar_arrive(&in_empty[s]);
                 // scales of these 4 blocks into the ring read by the epilogue; the
-                // epilogue frees the odd entry of each pair, in order, so the last
-                // entry being free means all four are
+                // epilogue frees the last entry of each group of four, in order
                 const uint32_t glast = gb + OP_KB - 1, buf0 = gb % NSC;
                 if (!wait_phase(&sc_empty[glast % NSC], ((glast / NSC) & 1) ^ 1, abort)) { ok = false; break; }
 #pragma unroll
@@ -534,39 +526,34 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
             // descriptors of the first K-step of each operand stage; a later
             // K-step adds its byte offset / 16 to the start-address field
             const uint64_t b0 = smem_desc_kmajor(op_b, 128, 256), b1 = smem_desc_kmajor(op_b + SZ_OP_B, 128, 256);
+            const uint64_t a0 = smem_desc_kmajor(op_a, 128, 256), a1 = smem_desc_kmajor(op_a + SZ_OP_A, 128, 256);
             static_assert(NOP == 2, "two operand stages");
             uint32_t i_op = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 for (int c = 0; c < nbK / OP_KB; ++c, ++i_op) {
                     const int o = i_op & 1;
-                    const uint32_t g0 = i_op * OP_KB;
                     if (!wait_phase(&op_full[o], (i_op / NOP) & 1, abort)) {
                         ok = false;
                         break;
                     }
-                    const uint64_t bd = o ? b1 : b0;
-                    const uint32_t ta = tmem + A_COL0 + o * OP_KB * A_COLS_PER_BLOCK;
+                    // the quad of accumulators of this operand stage: buffers 4o .. 4o + 3,
+                    // freed by the epilogue two stages ago
+                    if (!wait_phase(&tm_empty[o], ((i_op / 2) & 1) ^ 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint64_t bd = o ? b1 : b0, ad = o ? a1 : a0;
 #pragma unroll
                     for (int kb = 0; kb < OP_KB; ++kb) {
-                        // accumulators go round in pairs: pair pg = g / 2 holds
-                        // buffers g and g + 1 and has one empty and one full
-                        // mbarrier (entry pg mod NTM/2)
-                        const uint32_t g = g0 + kb, buf = g % NTM, pg = g >> 1, pb = pg % (NTM / 2);
-                        if ((kb & 1) == 0) {
-                            if (!wait_phase(&tm_empty[pb], ((pg / (NTM / 2)) & 1) ^ 1, abort)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after_sync();
-                        }
-                        const uint32_t d = tmem + buf * TN;
-                        mma_f16_ts(d, ta + kb * A_COLS_PER_BLOCK, bd + (uint64_t)((kb * 2) * (SZ_KSTEP_B >> 4)), idesc,
-                                   false);
-                        mma_f16_ts(d, ta + kb * A_COLS_PER_BLOCK + A_COLS_PER_BLOCK / 2,
+                        const uint32_t d = tmem + (uint32_t)(OP_KB * o + kb) * TN;
+                        mma_f16_ss(d, ad + (uint64_t)((kb * 2) * (SZ_KSTEP_A >> 4)),
+                                   bd + (uint64_t)((kb * 2) * (SZ_KSTEP_B >> 4)), idesc, false);
+                        mma_f16_ss(d, ad + (uint64_t)((kb * 2 + 1) * (SZ_KSTEP_A >> 4)),
                                    bd + (uint64_t)((kb * 2 + 1) * (SZ_KSTEP_B >> 4)), idesc, true);
-                        if (kb & 1) mma_commit(&tm_full[pb]);  // covers both blocks' MMAs
                     }
+                    mma_commit(&tm_full[o]);  // covers the quad's eight MMAs
                     mma_commit(&op_empty[o]);
                     if (!ok) break;
                 }
@@ -587,31 +574,34 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
             float2 acc[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = make_float2(0.0f, 0.0f);
-            // two blocks per pass: both TMEM loads in flight before either is used
-            for (int b = 0; b < nbK; b += 2, gb += 2) {
-                static_assert(NTM % 2 == 0, "pairs of accumulators never wrap");
-                const uint32_t b0 = gb % NTM, b1 = b0 + 1, pg = gb >> 1, pb = pg % (NTM / 2);
-                const uint32_t s0 = gb % NSC, s1 = s0 + 1, spar = (gb / NSC) & 1;
-                // one commit covers the pair; the converters arrive on the scale
-                // entries in order, so entry s1 complete means s0 is too
-                if (!wait_phase(&tm_full[pb], (pg / (NTM / 2)) & 1, abort) || !wait_phase(&sc_full[s1], spar, abort)) {
+            // one wait per quad of blocks (one operand stage); two blocks per pass,
+            // both TMEM loads in flight before either is used
+            for (int b = 0; b < nbK; b += OP_KB, gb += OP_KB) {
+                const uint32_t qd = (gb / OP_KB) & 1, qpar = (gb / (2 * OP_KB)) & 1;
+                const uint32_t s0 = gb % NSC, spar = (gb / NSC) & 1;
+                // the converters arrive on the four scale entries in order, so the
+                // last one complete means all four are
+                if (!wait_phase(&tm_full[qd], qpar, abort) || !wait_phase(&sc_full[s0 + 3], spar, abort)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
-                uint32_t r0[32], r1[32];
-                tmem_ld32(taddr + b0 * TN, r0);
-                tmem_ld32(taddr + b1 * TN, r1);
-                tmem_wait_ld();
-                rescale_acc(acc, r0, dw_ring[s0 * TM + row], da_ring + s0 * TN + 32 * hcol);
-                rescale_acc(acc, r1, dw_ring[s1 * TM + row], da_ring + s1 * TN + 32 * hcol);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const uint32_t bb = OP_KB * qd + 2 * h2, sa = s0 + 2 * h2;
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(taddr + bb * TN, r0);
+                    tmem_ld32(taddr + (bb + 1) * TN, r1);
+                    tmem_wait_ld();
+                    rescale_acc(acc, r0, dw_ring[sa * TM + row], da_ring + sa * TN + 32 * hcol);
+                    rescale_acc(acc, r1, dw_ring[(sa + 1) * TM + row], da_ring + (sa + 1) * TN + 32 * hcol);
+                }
                 tc_fence_before_sync();
                 __syncwarp();
                 // the converters wait only on the last entry of each group of four
-                // (an odd entry), so the odd entry of the pair is the one freed
                 if (lane == 0) {
-                    mbar_arrive(&tm_empty[pb]);
-                    mbar_arrive(&sc_empty[s1]);
+                    mbar_arrive(&tm_empty[qd]);
+                    mbar_arrive(&sc_empty[s0 + 3]);
                 }
             }
             if (!ok) break;

@@ -236,9 +236,15 @@ cudaError_t launch_router_logits(const LayerView& L, const float* x, int64_t T, 
         router_logits_split<<<grid, 256, 0, s>>>(x, (int)T, L.H, L.w_router, L.router_bias, L.E, logits,
                                                  status_clear);
     } else {
-        dim3 grid((unsigned)ceil_div(L.E, 64), (unsigned)ceil_div(T, 64), RKS);
-        router_logits_tiled<<<grid, 256, 0, s>>>(x, (int)T, L.H, L.w_router, L.router_bias, L.E, logits,
-                                                 status_clear);
+        // grid.y holds the 64-token tiles, at most 65535 a launch: larger
+        // batches take several launches over consecutive token ranges
+        const int64_t max_tokens = (int64_t)65535 * 64;
+        for (int64_t t0 = 0; t0 < T; t0 += max_tokens) {
+            const int64_t Tc = (T - t0 < max_tokens) ? T - t0 : max_tokens;
+            dim3 grid((unsigned)ceil_div(L.E, 64), (unsigned)ceil_div(Tc, 64), RKS);
+            router_logits_tiled<<<grid, 256, 0, s>>>(x + t0 * L.H, (int)Tc, L.H, L.w_router, L.router_bias, L.E,
+                                                     logits + t0 * L.E, t0 == 0 ? status_clear : nullptr);
+        }
     }
     return cudaGetLastError();
 }

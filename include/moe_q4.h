@@ -66,9 +66,16 @@ enum {
 
 /* Bits of the device status word (first uint32 of a workspace, or the
  * optional `status` argument): set with atomicOr, never cleared by the
- * library except at the start of moe_q4_ffn_forward. */
+ * library except at the start of a forward call (moe_q4_ffn_forward and its
+ * variants clear it per call; moe_q4_stack_forward once per call, so it
+ * accumulates over the layers). */
 #define MOE_Q4_STATUS_SCALE_OVERFLOW 0x1u /* a binary16 Q8_0 scale overflowed */
 #define MOE_Q4_STATUS_SPIN_TIMEOUT 0x2u   /* a bounded device-side wait gave up */
+#define MOE_Q4_STATUS_NONFINITE_LOGIT 0x4u /* a router logit was NaN or infinite: NaN ranks below
+                                              every number, so the token still gets k distinct
+                                              experts in [0, E), but its weights are undefined */
+#define MOE_Q4_STATUS_BAD_EXPERT_INDEX 0x8u /* the permutation met an expert index outside [0, E)
+                                               (counted as expert 0; the top-k never produces one) */
 
 /* One MoE layer.  Expert e's matrices are consecutive Q4_0 blocks:
  *   w_gate, w_up : [n_experts][ffn][hidden/32] blocks (18 B each)
@@ -135,9 +142,13 @@ int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t 
  * synchronisation, and code that may not allocate while it records a CUDA
  * graph.
  * moe_q4_ffn_forward with the workspace replaced by a static device array of
- * MOE_Q4_NOALLOC_SCRATCH_BYTES held by the library on every GPU that loads
- * it, until the process exits.  Nothing is allocated or freed.
+ * MOE_Q4_NOALLOC_SCRATCH_BYTES owned by the library.  Nothing is allocated
+ * or freed by the call.  The array occupies device memory on each GPU where
+ * this entry is used, from its first call there (CUDA's default lazy module
+ * loading places it then; with lazy loading off, when the library's module is
+ * loaded into the device's context) until the process exits.
  *   - x, y: as for moe_q4_ffn_forward (caller-owned device buffers).
+ *   - The device is checked (MOE_Q4_ERR_ARCH) before the scratch is touched.
  *   - A problem whose workspace (moe_q4_ffn_workspace_bytes(L, T)) exceeds
  *     the scratch returns MOE_Q4_ERR_WORKSPACE and enqueues nothing; for a
  *     layer with hidden 2048, ffn 512, 128 experts, top-8 and a shared expert
@@ -185,7 +196,10 @@ size_t moe_q4_stack_workspace_bytes(const moe_q4_layer* L, int64_t T_max);
  * ffn, n_experts, top_k and has_shared) applied in order to x [T][H] fp32 in
  * place: for each layer, x <- x + MoE_l(RMSNorm(x)).  Same conventions and
  * errors as moe_q4_ffn_forward; MOE_Q4_ERR_SHAPE if the layers differ in
- * shape.  The device status word of the workspace accumulates over layers. */
+ * shape.  The device status word (the first uint32 of the layer workspace,
+ * which starts after the two [T_max][H] fp32 buffers, each rounded up to 256
+ * bytes) is cleared once at the start of the call and accumulates the
+ * conditions of every layer. */
 int moe_q4_stack_forward(const moe_q4_layer* layers, int32_t n_layers, float* x, int64_t T, float eps,
                          void* workspace, size_t ws_bytes, moe_q4_stream_t stream);
 
@@ -279,12 +293,36 @@ typedef struct {
                                     CTA than exists, so its bounded wait runs out; the call completes
                                     with correct results and MOE_Q4_STATUS_SPIN_TIMEOUT in the status
                                     word (tests of the timeout report; about a second per call) */
+    /* Per-block integer dot products I_b = sum_{i<32} (nibble_i - 8) * q_i of
+     * the grouped paths (tensor-core and streaming), exactly as the projection
+     * kernel computed them (the tensor-core path: the MMA's accumulator before
+     * the rescale), for one row block of one expert group:
+     *   block_dots_out[s][r][b], s = slot - off[g] over the group's slots in
+     *   slot order, r < R rows of the row block, b < K/32 blocks along K.
+     * Tensor-core path: R = 128; gate/up rows r < 64 are gate rows 64 rb + r,
+     * r >= 64 the up rows 64 rb + r - 64; down rows are 128 rb + r.
+     * Streaming path: R = 64; gate/up rows r < 32 are gate rows 32 rb + r,
+     * r >= 32 the up rows 32 rb + r - 32; down rows are 64 rb + r.
+     * The buffer must hold count(g) * R * K/32 int32 (K = hidden for gate/up,
+     * ffn for down); ignored by the T = 1 fused path.  NULL: no capture. */
+    int32_t* block_dots_out;
+    int32_t block_dots_down;   /* 0: the gate/up projection, 1: the down projection */
+    int32_t block_dots_group;  /* expert group g (n_experts: the shared expert) */
+    int32_t block_dots_rb;     /* row block */
 } moe_q4_debug;
 
 /* moe_q4_ffn_forward with inspection options (see moe_q4_debug). */
 int moe_q4_ffn_forward_debug(const moe_q4_layer* L, const float* x, int64_t T, float* y,
                              void* workspace, size_t ws_bytes, const moe_q4_debug* dbg,
                              moe_q4_stream_t stream);
+
+/* Test hook: with enable != 0 every entry point sees the current device as
+ * compute capability major.minor instead of asking the driver, so the
+ * MOE_Q4_ERR_ARCH rejection (anything but 10.0, checked before any CUDA call
+ * and before anything is enqueued) can be exercised on any host; enable == 0
+ * restores the real query.  Not thread-safe: for tests only.  Returns
+ * MOE_Q4_OK. */
+int moe_q4_test_override_device(int32_t enable, int32_t major, int32_t minor);
 
 /* Per-block W4A8 integer dot products through the device routine every
  * projection kernel uses: out[i] = sum_{j<32} (nibble_j(w[i]) - 8) * qa[32*i+j]

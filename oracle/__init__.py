@@ -51,6 +51,7 @@ def _load():
         lib.orc_q4_0_dequant.argtypes = [P, i64, P]
         lib.orc_block_dot.argtypes = [P, P]
         lib.orc_block_dot.restype = ctypes.c_int32
+        lib.orc_block_dots.argtypes = [P, i64, P, P]
         lib.orc_q4_matvec.argtypes = [P, i32, i32, P, P, P]
         lib.orc_router_logits.argtypes = [P, i64, i32, P, P, i32, P]
         lib.orc_topk_softmax.argtypes = [P, i64, i32, i32, P, P]
@@ -126,6 +127,17 @@ def block_dot(blk: np.ndarray, qa: np.ndarray) -> int:
     blk = np.ascontiguousarray(blk, dtype=np.uint8).reshape(Q4_BYTES)
     qa = np.ascontiguousarray(qa, dtype=np.int8).reshape(QK)
     return int(_load().orc_block_dot(_ptr(blk), _ptr(qa)))
+
+
+def block_dots(blocks: np.ndarray, qa: np.ndarray) -> np.ndarray:
+    """block_dot over many blocks: blocks [..., 18] uint8 and qa [..., 32]
+    int8 with the same leading shape -> int32 [...]."""
+    blocks = np.ascontiguousarray(blocks, dtype=np.uint8)
+    qa = np.ascontiguousarray(qa, dtype=np.int8)
+    assert blocks.shape[-1] == Q4_BYTES and qa.shape[-1] == QK and blocks.shape[:-1] == qa.shape[:-1]
+    out = np.empty(blocks.shape[:-1], dtype=np.int32)
+    _load().orc_block_dots(_ptr(blocks), out.size, _ptr(qa), _ptr(out))
+    return out
 
 
 def q4_matvec(W: np.ndarray, qa: np.ndarray, da: np.ndarray) -> np.ndarray:

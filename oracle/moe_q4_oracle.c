@@ -161,6 +161,12 @@ int32_t orc_block_dot(const uint8_t* blk, const int8_t* qa) {
     return s;
 }
 
+/* out[i] = orc_block_dot(blocks[i], qa[32 i .. 32 i + 31]) for n blocks (18
+ * bytes each, consecutive) against n * 32 int8 activations. */
+void orc_block_dots(const uint8_t* blocks, int64_t n, const int8_t* qa, int32_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_block_dot(blocks + i * Q4_BYTES, qa + i * QK);
+}
+
 /* out[n] = fp32( sum_b d_w[n,b] * d_a[b] * I[n,b] ) for a Q4_0 matrix of N
  * rows and K inputs (row n = K/32 consecutive blocks) against one Q8_0 row.
  * Each term is exact in binary64 (11+11+15 significant bits). */

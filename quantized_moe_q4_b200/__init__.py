@@ -33,6 +33,8 @@ ERRORS = {
 }
 STATUS_SCALE_OVERFLOW = 0x1
 STATUS_SPIN_TIMEOUT = 0x2
+STATUS_NONFINITE_LOGIT = 0x4
+STATUS_BAD_EXPERT_INDEX = 0x8
 
 PATH_AUTO, PATH_GROUPED_DP4A, PATH_DECODE, PATH_TENSOR_CORE = 0, 1, 2, 3
 
@@ -45,7 +47,7 @@ EXPORTS = ["moe_q4_quantize_act", "moe_q4_route", "moe_q4_ffn_workspace_bytes", 
            "moe_q4_workspace_layout", "moe_q4_ffn_forward_debug", "moe_q4_block_dots",
            "moe_q4_ffn_forward_noalloc", "moe_q4_last_cuda_error", "moe_q4_residual_rmsnorm",
            "moe_q4_stack_workspace_bytes", "moe_q4_stack_forward", "moe_q4_gemv_workspace_bytes", "moe_q4_gemv",
-           "moe_q4_staging_bytes", "moe_q4_ffn_forward_streamed"]
+           "moe_q4_staging_bytes", "moe_q4_ffn_forward_streamed", "moe_q4_test_override_device"]
 
 
 class MoeQ4Error(RuntimeError):
@@ -69,14 +71,16 @@ class _Layer(ctypes.Structure):
 
 class _Debug(ctypes.Structure):
     _fields_ = [("h_out", ctypes.c_void_p), ("path", ctypes.c_int32),
-                ("ev_start", ctypes.c_void_p), ("ev_stop", ctypes.c_void_p), ("force_spin_timeout", ctypes.c_int32)]
+                ("ev_start", ctypes.c_void_p), ("ev_stop", ctypes.c_void_p), ("force_spin_timeout", ctypes.c_int32),
+                ("block_dots_out", ctypes.c_void_p), ("block_dots_down", ctypes.c_int32),
+                ("block_dots_group", ctypes.c_int32), ("block_dots_rb", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing: build the CUDA library first "
-            "(python -m quantized_moe_q4_b200.build, or __graft_entry__.build()). There is no CPU fallback.")
+            "(python quantized_moe_q4_b200/build.py, or __graft_entry__.build()). There is no CPU fallback.")
     lib = ctypes.CDLL(LIB_PATH)
     P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
     sigs = {
@@ -99,6 +103,7 @@ def _load() -> ctypes.CDLL:
         "moe_q4_gemv": ([P, i64, i32, P, i64, P, P, sz, P], ctypes.c_int),
         "moe_q4_staging_bytes": ([P], sz),
         "moe_q4_ffn_forward_streamed": ([P, P, i64, P, P, sz, P, sz, P], ctypes.c_int),
+        "moe_q4_test_override_device": ([i32, i32, i32], ctypes.c_int),
     }
     for name, (args, res) in sigs.items():
         f = getattr(lib, name)
@@ -234,11 +239,17 @@ def moe_q4_ffn_forward(layer: Layer, x: torch.Tensor, y=None, workspace=None, st
 
 
 def moe_q4_ffn_forward_debug(layer: Layer, x: torch.Tensor, y, workspace, h_out=None, path=PATH_AUTO,
-                             ev_start=None, ev_stop=None, stream=None, force_spin_timeout=False):
+                             ev_start=None, ev_stop=None, stream=None, force_spin_timeout=False,
+                             block_dots=None):
+    """block_dots: None or (out int32 tensor, down (bool), group, row block):
+    capture the per-block integer dot products of that row block (see
+    moe_q4_debug in include/moe_q4.h for the layout)."""
     T = x.shape[0]
+    bd_out, bd_down, bd_group, bd_rb = (None, 0, 0, 0) if block_dots is None else block_dots
     dbg = _Debug(None if h_out is None else h_out.data_ptr(), int(path),
                  None if ev_start is None else ev_start.cuda_event,
-                 None if ev_stop is None else ev_stop.cuda_event, int(bool(force_spin_timeout)))
+                 None if ev_stop is None else ev_stop.cuda_event, int(bool(force_spin_timeout)),
+                 None if bd_out is None else bd_out.data_ptr(), int(bool(bd_down)), int(bd_group), int(bd_rb))
     _check(_lib.moe_q4_ffn_forward_debug(layer.ref, _p(x), T, _p(y), _p(workspace), workspace.numel(),
                                          ctypes.byref(dbg), _stream(stream)), "moe_q4_ffn_forward_debug")
     return y
@@ -366,3 +377,10 @@ def moe_q4_ffn_forward_streamed(layer: Layer, x: torch.Tensor, y=None, workspace
                                             _p(staging), staging.numel(), _stream(stream)),
            "moe_q4_ffn_forward_streamed")
     return y
+
+
+def moe_q4_test_override_device(enable: bool, major: int = 10, minor: int = 0) -> None:
+    """Test hook: make every entry point see the current device as compute
+    capability major.minor (enable=True) or query the driver again (False)."""
+    _check(_lib.moe_q4_test_override_device(int(bool(enable)), int(major), int(minor)),
+           "moe_q4_test_override_device")

@@ -1,6 +1,8 @@
 """Build the CUDA library libmoe_q4.so (sm_100a only) in-tree with nvcc.
 
-    python -m quantized_moe_q4_b200.build [--force]
+    python quantized_moe_q4_b200/build.py [--force]
+
+(run by path: importing the package itself needs the built library)
 """
 import concurrent.futures as cf
 import os

@@ -22,7 +22,11 @@ struct DeviceState {
 };
 static DeviceState g_dev[MAX_DEVICES];
 
+// Test override of the device's compute capability (moe_q4_test_override_device).
+static int g_cc_override[3] = {0, 0, 0};  // enabled, major, minor
+
 static int current_device(DeviceInfo* out) {
+    if (g_cc_override[0] && !(g_cc_override[1] == 10 && g_cc_override[2] == 0)) return MOE_Q4_ERR_ARCH;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return MOE_Q4_ERR_CUDA;
     DeviceState& st = g_dev[dev];
@@ -203,8 +207,10 @@ static int cuda_rc(cudaError_t e) {
         if (e_ != cudaSuccess) return cuda_rc(e_); \
     } while (0)
 
+// clear_status: zero the workspace's status word first (every public forward
+// does; the stack entry clears it once and lets it accumulate over layers).
 static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float* y, void* ws, size_t ws_bytes,
-                        const moe_q4_debug* dbg, cudaStream_t s) {
+                        const moe_q4_debug* dbg, cudaStream_t s, bool clear_status = true) {
     int rc = check_layer(Lp);
     if (rc) return rc;
     if (T < 0 || T > T_LIMIT) return MOE_Q4_ERR_INVALID_ARG;
@@ -218,6 +224,10 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
     const size_t xy_bytes = sizeof(float) * (size_t)(T * L.H);
     if (overlap(x, xy_bytes, y, xy_bytes) || overlap(y, xy_bytes, ws, off[WS_TOTAL])) return MOE_Q4_ERR_OVERLAP;
     if (dbg && dbg->h_out && !aligned(dbg->h_out, 4)) return MOE_Q4_ERR_ALIGN;
+    if (dbg && dbg->block_dots_out &&
+        (!aligned(dbg->block_dots_out, 4) || dbg->block_dots_group < 0 ||
+         dbg->block_dots_group > Lp->n_experts - (Lp->has_shared ? 0 : 1) || dbg->block_dots_rb < 0))
+        return MOE_Q4_ERR_INVALID_ARG;
     DeviceInfo dev;
     rc = current_device(&dev);
     if (rc) return rc;
@@ -228,25 +238,37 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
     const int path = dbg ? dbg->path : MOE_Q4_PATH_AUTO;
     if ((path == MOE_Q4_PATH_AUTO || path == MOE_Q4_PATH_DECODE) && decode_eligible(L, T, dev))
         return cuda_rc(launch_decode(L, x, y, w, dbg ? dbg->h_out : nullptr, dev, ev0, ev1,
-                                     dbg && dbg->force_spin_timeout, s));
+                                     dbg && dbg->force_spin_timeout, clear_status, s));
 
     // grouped paths: tensor cores once experts see tens of tokens, else dp4a
     const bool tc = (path == MOE_Q4_PATH_TENSOR_CORE) || (path == MOE_Q4_PATH_AUTO && T >= TC_MIN_TOKENS);
-    MOE_TRY(launch_router_logits(L, x, T, w.logits, w.status, s));
-    MOE_TRY(launch_topk(w.logits, T, L.E, L.k, w.topk_idx, w.topk_w, s));
+    MOE_TRY(launch_router_logits(L, x, T, w.logits, clear_status ? w.status : nullptr, s));
+    MOE_TRY(launch_topk(w.logits, T, L.E, L.k, w.topk_idx, w.topk_w, w.status, s));
     MOE_TRY(launch_quantize(x, T, L.H, w.qa, w.da, w.status, y, s));
     MOE_TRY(launch_permute(w.topk_idx, T, L.k, L.E, L.S, tc ? TC_TILE_TOKENS : DP4A_TT, w, s));
+    BlockDotCapture cap_store;
+    const BlockDotCapture* cap = nullptr;
+    if (dbg && dbg->block_dots_out) {
+        cap_store = BlockDotCapture{dbg->block_dots_out, dbg->block_dots_down ? 1 : 0, dbg->block_dots_group,
+                                    dbg->block_dots_rb};
+        cap = &cap_store;
+    }
     if (ev0) MOE_TRY(record_event(ev0, s));
     if (tc)
-        MOE_TRY(launch_gateup_tc(L, T, w, dbg ? dbg->h_out : nullptr, dev, s));
+        MOE_TRY(launch_gateup_tc(L, T, w, dbg ? dbg->h_out : nullptr, dev, cap, s));
     else
-        MOE_TRY(launch_gateup_dp4a(L, T, w, dbg ? dbg->h_out : nullptr, dev, s));
+        MOE_TRY(launch_gateup_dp4a(L, T, w, dbg ? dbg->h_out : nullptr, dev, cap, s));
     if (ev1) MOE_TRY(record_event(ev1, s));
     if (tc)
-        MOE_TRY(launch_down_tc(L, T, w, y, dev, s));
+        MOE_TRY(launch_down_tc(L, T, w, y, dev, cap, s));
     else
-        MOE_TRY(launch_down_dp4a(L, T, w, y, dev, s));
+        MOE_TRY(launch_down_dp4a(L, T, w, y, dev, cap, s));
     return MOE_Q4_OK;
+}
+
+int check_device() {
+    DeviceInfo dev;
+    return current_device(&dev);
 }
 
 }  // namespace moeq4
@@ -301,7 +323,7 @@ int moe_q4_route(const moe_q4_layer* L, const float* x, int64_t T, int32_t* topk
     const LayerView v = view(L);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     MOE_TRY(launch_router_logits(v, x, T, logits, nullptr, s));
-    MOE_TRY(launch_topk(logits, T, v.E, v.k, topk_idx, topk_w, s));
+    MOE_TRY(launch_topk(logits, T, v.E, v.k, topk_idx, topk_w, nullptr, s));
     return MOE_Q4_OK;
 }
 
@@ -418,10 +440,16 @@ int moe_q4_stack_forward(const moe_q4_layer* layers, int32_t n_layers, float* x,
     float* y = reinterpret_cast<float*>(base + xy);
     void* lws = base + 2 * xy;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    DeviceInfo dev;
+    int rc0 = current_device(&dev);
+    if (rc0) return rc0;
+    // one status word for the whole call: cleared here, then every layer's
+    // kernels OR their conditions into it
+    MOE_TRY(cudaMemsetAsync(static_cast<char*>(lws) + off[WS_STATUS], 0, 16, s));
     for (int32_t l = 0; l < n_layers; ++l) {
         int rc = moe_q4_residual_rmsnorm(x, l ? y : nullptr, T, H, eps, xn, stream);
         if (rc) return rc;
-        rc = forward_impl(&layers[l], xn, T, y, lws, off[WS_TOTAL], nullptr, s);
+        rc = forward_impl(&layers[l], xn, T, y, lws, off[WS_TOTAL], nullptr, s, /*clear_status=*/false);
         if (rc) return rc;
     }
     return moe_q4_residual_rmsnorm(x, y, T, H, eps, nullptr, stream);
@@ -503,6 +531,9 @@ int moe_q4_ffn_forward_streamed(const moe_q4_layer* L, const float* x, int64_t T
     size_t soff[7];
     staging_layout(L, soff);
     if (staging_bytes < soff[6]) return MOE_Q4_ERR_WORKSPACE;
+    DeviceInfo dev;
+    rc = current_device(&dev);
+    if (rc) return rc;
     // the experts must be page-locked host memory (read by the GPU through
     // unified addressing); the router weights and x, y device memory
     const void* host_mats[6] = {L->w_gate, L->w_up, L->w_down, L->sh_gate, L->sh_up, L->sh_down};
@@ -515,14 +546,11 @@ int moe_q4_ffn_forward_streamed(const moe_q4_layer* L, const float* x, int64_t T
     size_t off[WS_COUNT];
     layout(Lv, T, off);
     if (ws_bytes < off[WS_TOTAL]) return MOE_Q4_ERR_WORKSPACE;
-    DeviceInfo dev;
-    rc = current_device(&dev);
-    if (rc) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const Workspace w = carve(workspace, off);
     // routing and its per-expert counts, on the device
     MOE_TRY(launch_router_logits(Lv, x, T, w.logits, w.status, s));
-    MOE_TRY(launch_topk(w.logits, T, Lv.E, Lv.k, w.topk_idx, w.topk_w, s));
+    MOE_TRY(launch_topk(w.logits, T, Lv.E, Lv.k, w.topk_idx, w.topk_w, w.status, s));
     MOE_TRY(launch_permute(w.topk_idx, T, Lv.k, Lv.E, Lv.S, DP4A_TT, w, s));
     uint8_t* st = static_cast<uint8_t*>(staging);
     StageParams sp;
@@ -541,6 +569,13 @@ int moe_q4_ffn_forward_streamed(const moe_q4_layer* L, const float* x, int64_t T
         Ls.sh_gate = sp.d_sh_gate; Ls.sh_up = sp.d_sh_up; Ls.sh_down = sp.d_sh_down;
     }
     return forward_impl(&Ls, x, T, y, workspace, ws_bytes, nullptr, s);
+}
+
+int moe_q4_test_override_device(int32_t enable, int32_t major, int32_t minor) {
+    g_cc_override[1] = major;
+    g_cc_override[2] = minor;
+    g_cc_override[0] = enable ? 1 : 0;
+    return MOE_Q4_OK;
 }
 
 int moe_q4_block_dots(const uint8_t* w_blocks, const int8_t* qa, int64_t n, int32_t* out, moe_q4_stream_t stream) {

@@ -36,6 +36,8 @@ constexpr int DN_ROWS = 64;
 // Status word bits (the public header's MOE_Q4_STATUS_*).
 constexpr uint32_t STATUS_SCALE_OVERFLOW = 0x1u;
 constexpr uint32_t STATUS_SPIN_TIMEOUT = 0x2u;
+constexpr uint32_t STATUS_NONFINITE_LOGIT = 0x4u;
+constexpr uint32_t STATUS_BAD_EXPERT_INDEX = 0x8u;
 
 // ---------------------------------------------------------------------------
 // Scalar rules

@@ -41,6 +41,7 @@ struct DecodeParams {
     int rows_per_cta;  // down rows of H per FFN CTA
     int nctas;         // grid of decode_ffn_kernel
     int barrier_target;  // arrivals the grid barrier waits for (nctas; nctas + 1 only in the timeout test)
+    int clear_status;    // the router kernel zeroes the status word (else it accumulates)
     const float* x;
     const float* w_router;
     const float* bias;
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
     pdl_launch_dependents();
     pdl_wait();  // x and the workspace are now the previous kernels' results
     if (e == 0 && tid == 0) {
-        p.status[0] = 0u;  // status word
+        if (p.clear_status) p.status[0] = 0u;  // status word
         p.status[1] = 0u;  // grid-barrier counter of decode_ffn_kernel
     }
     const bool ok = mbar_wait_bounded(&bar, 0, MBAR_LIMIT);
@@ -321,7 +322,13 @@ __global__ void __maxnreg__(96) decode_ffn_kernel(DecodeParams p) {
     // summed with shuffles.  Ranks below k are the chosen experts, in order.
     const int E16 = (E + 15) & ~15;
     const int P = (E16 <= FFN_THREADS / 4) ? 4 : 2;
-    for (int e = tid; e < E16; e += blockDim.x) logit_s[e] = (e < E) ? __ldcg(p.logits + e) : -3.402823466e38f;
+    // a NaN logit (non-finite data, or the router kernel's timeout report)
+    // ranks as -infinity, so the ranks below stay a permutation of [0, E)
+    for (int e = tid; e < E16; e += blockDim.x) {
+        float l = (e < E) ? __ldcg(p.logits + e) : -INFINITY;
+        if (e < E && !isfinite(l)) atomicOr(&flags_s, (int)STATUS_NONFINITE_LOGIT);
+        logit_s[e] = (l != l) ? -INFINITY : l;
+    }
     for (int i = tid; i < H / 16; i += blockDim.x)
         reinterpret_cast<int4*>(qa_s)[i] = __ldcg(reinterpret_cast<const int4*>(p.qa) + i);
     for (int b = tid; b < nbH; b += blockDim.x) {
@@ -335,7 +342,6 @@ __global__ void __maxnreg__(96) decode_ffn_kernel(DecodeParams p) {
     int rank = 0;
     if (e_me < E) {
         my_l = logit_s[e_me];
-        if (part == 0 && my_l != my_l) atomicOr(&flags_s, (int)STATUS_SPIN_TIMEOUT);  // router timed out
         const float4* l4 = reinterpret_cast<const float4*>(logit_s);
         const int per4 = E16 / (4 * P);
 #pragma unroll 4
@@ -504,8 +510,9 @@ bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev) {
 
 cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Workspace& ws, float* h_dbg,
                           const DeviceInfo& dev, cudaEvent_t ev_start, cudaEvent_t ev_stop, bool force_timeout,
-                          cudaStream_t s) {
+                          bool clear_status, cudaStream_t s) {
     DecodeParams p;
+    p.clear_status = clear_status ? 1 : 0;
     p.H = L.H; p.F = L.F; p.E = L.E; p.k = L.k; p.S = L.S;
     p.nctas = dev.sm_count;
     p.barrier_target = p.nctas + (force_timeout ? 1 : 0);

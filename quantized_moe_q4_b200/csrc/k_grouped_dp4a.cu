@@ -83,6 +83,18 @@ struct StreamParams {
     float* h_dbg;
     float* y;
     uint32_t* status;
+    int32_t* cap_out;  // block-dot capture (the CAP instantiation only)
+    int cap_group, cap_rb;
+};
+
+// Where a capturing item writes its block dot products: cap + ((slot_rel + j)
+// * SR + row) * nb + block, for the lane's rows and blocks.
+struct CapPtr {
+    int32_t* out;  // NULL when this item is not captured
+    int slot_rel;  // first slot of the tile minus the group's first slot
+    int row0;      // this lane's first row within the item
+    int nb;        // blocks along K
+    int blk;       // block index along K of the current block
 };
 
 __device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
@@ -172,10 +184,10 @@ __device__ __forceinline__ float int_to_float_exact(int I) {
 
 // acc[r][s0 + j] += the W4A8 block term of block b for slots s0 .. s0 + SPW - 1
 // (activations of a slot: [half][block][16 B] at sa + slot * KC * 32).
-template <int SPW, int RPL_, int ST_>
+template <int SPW, int RPL_, int ST_, bool CAP>
 __device__ __forceinline__ void block_slots(float (&acc)[RPL_][ST_], int s0, const uint32_t (&qs)[RPL_][4],
                                             const float (&dW)[RPL_], const int8_t* sa, const uint16_t* sd, int KC,
-                                            int b) {
+                                            int b, const CapPtr& cap) {
     int qa[SPW][8];
     int base[SPW];
     float dA[SPW];
@@ -202,6 +214,7 @@ __device__ __forceinline__ void block_slots(float (&acc)[RPL_][ST_], int s0, con
                 I = dp4a_u8s8(qs[r][i] & 0x0f0f0f0fu, qa[j][i], I);
                 I = dp4a_u8s8((qs[r][i] >> 4) & 0x0f0f0f0fu, qa[j][4 + i], I);
             }
+            if (CAP && cap.out) cap.out[((size_t)(cap.slot_rel + s0 + j) * SR + cap.row0 + r) * cap.nb + cap.blk] = I;
             acc[r][s0 + j] = fmaf(int_to_float_exact(I), dW[r] * dA[j], acc[r][s0 + j]);
         }
     }
@@ -209,7 +222,9 @@ __device__ __forceinline__ void block_slots(float (&acc)[RPL_][ST_], int s0, con
 
 }  // namespace
 
-template <int MODE>
+// CAP: also write the per-block integer dot products of one row block of one
+// group to p.cap_out (test instantiation).
+template <int MODE, bool CAP>
 __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_constant__ StreamMaps maps) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
@@ -330,7 +345,13 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
                 const unsigned char* sw = smem + st * SZ_STAGE;
                 const int8_t* sa = reinterpret_cast<const int8_t*>(sw + SZ_W);
                 const uint16_t* sd = reinterpret_cast<const uint16_t*>(sw + SZ_W + SZ_A);
+                CapPtr cap{nullptr, 0, RPL * rg, nb, 0};
+                if (CAP && MODE != GEMV && it.g == p.cap_group && it.rb == p.cap_rb) {
+                    cap.out = p.cap_out;
+                    cap.slot_rel = it.slot0 - off_s[it.g];
+                }
                 for (int b = ks; b < KC; b += 16) {
+                    cap.blk = c * KC + b;
                     // this lane's weight blocks (its RPL rows, block b), loaded once
                     uint32_t qs[RPL][4];
                     float dW[RPL];
@@ -345,12 +366,12 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
                     for (int sp = 0; sp < ST; sp += 4) {
                         const int rem = it.nslots - sp;
                         if (rem >= 4) {
-                            block_slots<4>(acc, sp, qs, dW, sa, sd, KC, b);
+                            block_slots<4, RPL, ST, CAP>(acc, sp, qs, dW, sa, sd, KC, b, cap);
                         } else if (rem >= 2) {
-                            block_slots<2>(acc, sp, qs, dW, sa, sd, KC, b);
-                            if (rem == 3) block_slots<1>(acc, sp + 2, qs, dW, sa, sd, KC, b);
+                            block_slots<2, RPL, ST, CAP>(acc, sp, qs, dW, sa, sd, KC, b, cap);
+                            if (rem == 3) block_slots<1, RPL, ST, CAP>(acc, sp + 2, qs, dW, sa, sd, KC, b, cap);
                         } else if (rem == 1) {
-                            block_slots<1>(acc, sp, qs, dW, sa, sd, KC, b);
+                            block_slots<1, RPL, ST, CAP>(acc, sp, qs, dW, sa, sd, KC, b, cap);
                         }
                     }
                 }
@@ -450,6 +471,7 @@ StreamParams make_stream_params(const LayerView& L, int64_t T, const Workspace& 
     p.N = 0; p.T = 0;
     p.qa = ws.qa; p.da = ws.da; p.off = ws.off; p.tile_off = ws.tile_off; p.sorted = ws.sorted;
     p.topk_w = ws.topk_w; p.hq = ws.hq; p.dh = ws.dh; p.h_dbg = h_dbg; p.y = y; p.status = ws.status;
+    p.cap_out = nullptr; p.cap_group = -1; p.cap_rb = -1;
     return p;
 }
 
@@ -461,10 +483,12 @@ int64_t stream_max_tiles(const LayerView& L, int64_t T) {
 
 template <int MODE>
 cudaError_t launch_stream(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, float* y,
-                          const DeviceInfo& dev, cudaStream_t s) {
+                          const DeviceInfo& dev, const BlockDotCapture* cap, cudaStream_t s) {
+    const bool capture = cap && cap->down == (MODE == DOWN ? 1 : 0);
+    const void* kfn = capture ? reinterpret_cast<const void*>(stream_dp4a_kernel<MODE, true>)
+                              : reinterpret_cast<const void*>(stream_dp4a_kernel<MODE, false>);
     int per_sm = 0;
-    cudaError_t e =
-        kernel_occupancy(reinterpret_cast<const void*>(stream_dp4a_kernel<MODE>), THREADS, SMEM_ALLOC, &per_sm);
+    cudaError_t e = kernel_occupancy(kfn, THREADS, SMEM_ALLOC, &per_sm);
     if (e != cudaSuccess) return e;
     StreamMaps maps;
     std::memset(&maps, 0, sizeof(maps));
@@ -484,7 +508,15 @@ cudaError_t launch_stream(const LayerView& L, int64_t T, const Workspace& ws, fl
     const int n_rb = (MODE == GATEUP) ? L.F / 32 : L.H / SR;
     const int64_t items = stream_max_tiles(L, T) * n_rb;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, dev.sm_count));
-    stream_dp4a_kernel<MODE><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(make_stream_params(L, T, ws, h_dbg, y), maps);
+    StreamParams p = make_stream_params(L, T, ws, h_dbg, y);
+    if (capture) {
+        p.cap_out = cap->out;
+        p.cap_group = cap->group;
+        p.cap_rb = cap->rb;
+        stream_dp4a_kernel<MODE, true><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(p, maps);
+    } else {
+        stream_dp4a_kernel<MODE, false><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(p, maps);
+    }
     return cudaGetLastError();
 }
 
@@ -494,7 +526,7 @@ cudaError_t launch_gemv_dp4a(const uint8_t* W, int64_t N, int H, const int8_t* q
                              float* y, uint32_t* status, const DeviceInfo& dev, cudaStream_t s) {
     int per_sm = 0;
     cudaError_t e =
-        kernel_occupancy(reinterpret_cast<const void*>(stream_dp4a_kernel<GEMV>), THREADS, SMEM_ALLOC, &per_sm);
+        kernel_occupancy(reinterpret_cast<const void*>(stream_dp4a_kernel<GEMV, false>), THREADS, SMEM_ALLOC, &per_sm);
     if (e != cudaSuccess) return e;
     StreamMaps maps;
     std::memset(&maps, 0, sizeof(maps));
@@ -506,18 +538,19 @@ cudaError_t launch_gemv_dp4a(const uint8_t* W, int64_t N, int H, const int8_t* q
     p.H = H; p.N = (int)N; p.T = T; p.qa = qa; p.da = da; p.y = y; p.status = status;
     const int64_t items = ceil_div(N, SR);
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, dev.sm_count));
-    stream_dp4a_kernel<GEMV><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(p, maps);
+    p.cap_out = nullptr; p.cap_group = -1; p.cap_rb = -1;
+    stream_dp4a_kernel<GEMV, false><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(p, maps);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gateup_dp4a(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg,
-                               const DeviceInfo& dev, cudaStream_t s) {
-    return launch_stream<GATEUP>(L, T, ws, h_dbg, nullptr, dev, s);
+                               const DeviceInfo& dev, const BlockDotCapture* cap, cudaStream_t s) {
+    return launch_stream<GATEUP>(L, T, ws, h_dbg, nullptr, dev, cap, s);
 }
 
 cudaError_t launch_down_dp4a(const LayerView& L, int64_t T, const Workspace& ws, float* y,
-                             const DeviceInfo& dev, cudaStream_t s) {
-    return launch_stream<DOWN>(L, T, ws, nullptr, y, dev, s);
+                             const DeviceInfo& dev, const BlockDotCapture* cap, cudaStream_t s) {
+    return launch_stream<DOWN>(L, T, ws, nullptr, y, dev, cap, s);
 }
 
 // ---------------------------------------------------------------------------

@@ -48,14 +48,26 @@ cudaError_t launch_quantize(const float* x, int64_t T, int H, int8_t* q, uint16_
 // group E the shared expert (count S*T, slots P..P+S*T-1).
 // ---------------------------------------------------------------------------
 
+// Expert of pair p.  The top-k kernels only produce experts in [0, E); an
+// index outside it (which would address the counters out of bounds) is
+// counted as expert 0 by both the histogram and the scatter, so the
+// permutation stays a bijection, and reported as STATUS_BAD_EXPERT_INDEX.
+__device__ __forceinline__ int pair_expert(const int32_t* idx, int64_t p, int E, uint32_t* status) {
+    const int e = __ldg(idx + p);
+    if ((unsigned)e < (unsigned)E) return e;
+    if (status) atomicOr(status, STATUS_BAD_EXPERT_INDEX);
+    return 0;
+}
+
 // Per-chunk expert histogram.
 __global__ void __launch_bounds__(PERM_CHUNK) perm_hist_kernel(const int32_t* __restrict__ idx, int64_t P,
-                                                                int E, int32_t* __restrict__ chunk_cnt) {
+                                                                int E, int32_t* __restrict__ chunk_cnt,
+                                                                uint32_t* __restrict__ status) {
     __shared__ int cnt[256];
     for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
     __syncthreads();
     const int64_t p = (int64_t)blockIdx.x * PERM_CHUNK + threadIdx.x;
-    if (p < P) atomicAdd(&cnt[__ldg(idx + p)], 1);
+    if (p < P) atomicAdd(&cnt[pair_expert(idx, p, E, status)], 1);
     __syncthreads();
     for (int i = threadIdx.x; i < E; i += blockDim.x) chunk_cnt[(size_t)blockIdx.x * E + i] = cnt[i];
 }
@@ -132,13 +144,14 @@ __global__ void __launch_bounds__(PERM_CHUNK) perm_scatter_kernel(const int32_t*
                                                                    int E, const int32_t* __restrict__ chunk_base,
                                                                    int32_t* __restrict__ sorted,
                                                                    int32_t* __restrict__ pos) {
+    // (a bad index was reported by the histogram; the same mapping here)
     __shared__ int wcnt[PERM_CHUNK / 32][256];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int i = threadIdx.x; i < (PERM_CHUNK / 32) * 256; i += blockDim.x) (&wcnt[0][0])[i] = 0;
     __syncthreads();
     const int64_t p = (int64_t)blockIdx.x * PERM_CHUNK + threadIdx.x;
     const bool valid = p < P;
-    const int e = valid ? __ldg(idx + p) : -1;
+    const int e = valid ? pair_expert(idx, p, E, nullptr) : -1;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & ((1u << lane) - 1u));
     if (valid && rank == 0) wcnt[warp][e] = __popc(peers);
@@ -156,7 +169,7 @@ cudaError_t launch_permute(const int32_t* idx, int64_t T, int k, int E, int S, i
                            const Workspace& ws, cudaStream_t s) {
     const int64_t P = T * k;
     const int nchunks = (int)ceil_div(P, PERM_CHUNK);
-    perm_hist_kernel<<<nchunks, PERM_CHUNK, 0, s>>>(idx, P, E, ws.chunk_cnt);
+    perm_hist_kernel<<<nchunks, PERM_CHUNK, 0, s>>>(idx, P, E, ws.chunk_cnt, ws.status);
     perm_scan_kernel<<<1, 512, 0, s>>>(ws.chunk_cnt, nchunks, E, S, T, k, tile_tokens, ws.cnt, ws.off,
                                        ws.tile_off, ws.chunk_base);
     perm_scatter_kernel<<<nchunks, PERM_CHUNK, 0, s>>>(idx, P, E, ws.chunk_base, ws.sorted, ws.pos);

@@ -173,26 +173,36 @@ __global__ void __cluster_dims__(1, 1, RKS) __launch_bounds__(256)
 
 // ---------------------------------------------------------------------------
 // Top-k + softmax over the chosen logits: one warp per token, E <= 256.
+// A NaN logit ranks as -infinity (below every number; equal keys go to the
+// lower expert index), so every pick is an expert in [0, E) whatever the
+// logits hold; a NaN or infinite logit sets STATUS_NONFINITE_LOGIT in
+// *status (if given), and the weights of such a token are then undefined.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits, int T, int E,
                                                             int k, int32_t* __restrict__ idx,
-                                                            float* __restrict__ w) {
+                                                            float* __restrict__ w, uint32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31;
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
     float v[8];
+    bool nonfinite = false;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int e = i * 32 + lane;
-        v[i] = (e < E) ? logits[(size_t)t * E + e] : -FLT_MAX;
+        float l = (e < E) ? logits[(size_t)t * E + e] : -INFINITY;
+        if (e < E && !isfinite(l)) nonfinite = true;
+        v[i] = (l != l) ? -INFINITY : l;
     }
+    if (status && __any_sync(0xffffffffu, nonfinite) && lane == 0) atomicOr(status, STATUS_NONFINITE_LOGIT);
     uint32_t taken = 0;
     for (int i = 0; i < 8; ++i)
         if (i * 32 + lane >= E) taken |= 1u << i;
     float my_l = 0.0f;
     int my_e = 0;
     for (int j = 0; j < k; ++j) {
-        float bv = -FLT_MAX;
+        // every untaken expert beats the start value (-inf with an index
+        // above any expert's), and k <= E leaves at least one untaken
+        float bv = -INFINITY;
         int be = 0x7fffffff;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -250,9 +260,9 @@ cudaError_t launch_router_logits(const LayerView& L, const float* x, int64_t T, 
 }
 
 cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* idx, float* w,
-                        cudaStream_t s) {
+                        uint32_t* status, cudaStream_t s) {
     const unsigned blocks = (unsigned)ceil_div(T, 8);
-    topk_softmax_kernel<<<blocks, 256, 0, s>>>(logits, (int)T, E, k, idx, w);
+    topk_softmax_kernel<<<blocks, 256, 0, s>>>(logits, (int)T, E, k, idx, w, status);
     return cudaGetLastError();
 }
 

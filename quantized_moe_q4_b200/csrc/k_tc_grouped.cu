@@ -132,6 +132,8 @@ struct TcParams {
     float* h_dbg;
     float* y;
     uint32_t* status;
+    int32_t* cap_out;  // block-dot capture (the CAP instantiation only)
+    int cap_group, cap_rb;
 };
 
 // ---------------------------------------------------------------- helpers
@@ -277,7 +279,9 @@ __device__ __forceinline__ void slot_info(const TcParams& p, int g, int s, int& 
 
 }  // namespace
 
-template <int MODE>
+// CAP: also write the per-block integer sums (the MMA accumulators before the
+// rescale) of one row block of one group to p.cap_out (test instantiation).
+template <int MODE, bool CAP>
 __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, const __grid_constant__ TcMaps maps) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -593,6 +597,19 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                     tmem_ld32(taddr + bb * TN, r0);
                     tmem_ld32(taddr + (bb + 1) * TN, r1);
                     tmem_wait_ld();
+                    if (CAP && T.g == p.cap_group && T.rb == p.cap_rb) {
+                        // exact integers held in binary32: convert back without rounding
+                        const size_t s0 = (size_t)(T.slot0 - off_s[T.g]);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int n = 32 * hcol + j;
+                            if (n < T.nslots) {
+                                int32_t* o = p.cap_out + ((s0 + n) * TM + row) * nbK + b + 2 * h2;
+                                o[0] = __float2int_rn(__uint_as_float(r0[j]));
+                                o[1] = __float2int_rn(__uint_as_float(r1[j]));
+                            }
+                        }
+                    }
                     rescale_acc(acc, r0, dw_ring[sa * TM + row], da_ring + sa * TN + 32 * hcol);
                     rescale_acc(acc, r1, dw_ring[(sa + 1) * TM + row], da_ring + (sa + 1) * TN + 32 * hcol);
                 }
@@ -683,6 +700,7 @@ static TcParams make_tc_params(const LayerView& L, int64_t T, const Workspace& w
     p.sh_gate = L.sh_gate; p.sh_up = L.sh_up; p.sh_down = L.sh_down;
     p.qa = ws.qa; p.da = ws.da; p.off = ws.off; p.tile_off = ws.tile_off; p.sorted = ws.sorted;
     p.topk_w = ws.topk_w; p.hq = ws.hq; p.dh = ws.dh; p.h_dbg = h_dbg; p.y = y; p.status = ws.status;
+    p.cap_out = nullptr; p.cap_group = -1; p.cap_rb = -1;
     return p;
 }
 
@@ -744,10 +762,12 @@ static cudaError_t make_maps(const LayerView& L, TcMaps* maps) {
 
 template <int MODE>
 static cudaError_t launch_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, float* y,
-                             const DeviceInfo& dev, cudaStream_t s) {
+                             const DeviceInfo& dev, const BlockDotCapture* cap, cudaStream_t s) {
+    const bool capture = cap && cap->down == (MODE == DOWN ? 1 : 0);
+    const void* kfn = capture ? reinterpret_cast<const void*>(tc_grouped_kernel<MODE, true>)
+                              : reinterpret_cast<const void*>(tc_grouped_kernel<MODE, false>);
     int per_sm = 0;
-    cudaError_t e =
-        kernel_occupancy(reinterpret_cast<const void*>(tc_grouped_kernel<MODE>), THREADS, SMEM_ALLOC, &per_sm);
+    cudaError_t e = kernel_occupancy(kfn, THREADS, SMEM_ALLOC, &per_sm);
     if (e != cudaSuccess) return e;
     TcMaps maps;
     e = make_maps<MODE>(L, &maps);
@@ -755,18 +775,26 @@ static cudaError_t launch_tc(const LayerView& L, int64_t T, const Workspace& ws,
     const int n_rb = (MODE == GATEUP) ? L.F / 64 : L.H / TM;
     const int64_t items = tc_max_tiles(L, T) * n_rb;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, dev.sm_count));
-    tc_grouped_kernel<MODE><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(make_tc_params(L, T, ws, h_dbg, y), maps);
+    TcParams p = make_tc_params(L, T, ws, h_dbg, y);
+    if (capture) {
+        p.cap_out = cap->out;
+        p.cap_group = cap->group;
+        p.cap_rb = cap->rb;
+        tc_grouped_kernel<MODE, true><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(p, maps);
+    } else {
+        tc_grouped_kernel<MODE, false><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(p, maps);
+    }
     return cudaGetLastError();
 }
 
 cudaError_t launch_gateup_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, const DeviceInfo& dev,
-                             cudaStream_t s) {
-    return launch_tc<GATEUP>(L, T, ws, h_dbg, nullptr, dev, s);
+                             const BlockDotCapture* cap, cudaStream_t s) {
+    return launch_tc<GATEUP>(L, T, ws, h_dbg, nullptr, dev, cap, s);
 }
 
 cudaError_t launch_down_tc(const LayerView& L, int64_t T, const Workspace& ws, float* y, const DeviceInfo& dev,
-                           cudaStream_t s) {
-    return launch_tc<DOWN>(L, T, ws, nullptr, y, dev, s);
+                           const BlockDotCapture* cap, cudaStream_t s) {
+    return launch_tc<DOWN>(L, T, ws, nullptr, y, dev, cap, s);
 }
 
 }  // namespace moeq4

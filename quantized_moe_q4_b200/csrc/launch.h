@@ -39,6 +39,15 @@ struct Workspace {
     uint16_t* dh;
 };
 
+// Test capture of the per-block integer dot products I_b of one row block of
+// one expert group (moe_q4_debug.block_dots_*): out[slot - off[g]][row][block].
+struct BlockDotCapture {
+    int32_t* out;
+    int down;   // 0: gate/up projection, 1: down projection
+    int group;  // expert group (E: the shared expert)
+    int rb;     // row block of the kernel family
+};
+
 struct DeviceInfo {
     int sm_count;
     int max_smem_optin;
@@ -48,8 +57,9 @@ struct DeviceInfo {
 // status_clear (may be NULL): a status word the first thread zeroes.
 cudaError_t launch_router_logits(const LayerView& L, const float* x, int64_t T, float* logits,
                                  uint32_t* status_clear, cudaStream_t s);
+// status (may be NULL) receives STATUS_NONFINITE_LOGIT.
 cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* idx, float* w,
-                        cudaStream_t s);
+                        uint32_t* status, cudaStream_t s);
 
 // k_quant_perm.cu
 cudaError_t launch_quantize(const float* x, int64_t T, int H, int8_t* q, uint16_t* d,
@@ -58,10 +68,11 @@ cudaError_t launch_permute(const int32_t* idx, int64_t T, int k, int E, int S, i
                            const Workspace& ws, cudaStream_t s);
 
 // k_grouped_dp4a.cu
+// cap (may be NULL): capture the block dot products of one row block.
 cudaError_t launch_gateup_dp4a(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg,
-                               const DeviceInfo& dev, cudaStream_t s);
+                               const DeviceInfo& dev, const BlockDotCapture* cap, cudaStream_t s);
 cudaError_t launch_down_dp4a(const LayerView& L, int64_t T, const Workspace& ws, float* y,
-                             const DeviceInfo& dev, cudaStream_t s);
+                             const DeviceInfo& dev, const BlockDotCapture* cap, cudaStream_t s);
 // y[t][n] (t < T <= 8, n < N) = W4A8 product of Q4_0 rows W [N][H/32] with the
 // Q8_0 activations qa/da of T tokens (the streaming kernel's GEMV mode).
 cudaError_t launch_gemv_dp4a(const uint8_t* W, int64_t N, int H, const int8_t* qa, const uint16_t* da, int T,
@@ -70,9 +81,9 @@ cudaError_t launch_gemv_dp4a(const uint8_t* W, int64_t N, int H, const int8_t* q
 // permutation must have been built with TC_TILE_TOKENS slots per tile.
 constexpr int TC_TILE_TOKENS = 64;
 cudaError_t launch_gateup_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, const DeviceInfo& dev,
-                             cudaStream_t s);
+                             const BlockDotCapture* cap, cudaStream_t s);
 cudaError_t launch_down_tc(const LayerView& L, int64_t T, const Workspace& ws, float* y, const DeviceInfo& dev,
-                           cudaStream_t s);
+                           const BlockDotCapture* cap, cudaStream_t s);
 
 // k_decode.cu: the fused T=1 path (router kernel + cooperative FFN kernel,
 // chained with programmatic dependent launch).  Events, if given, bracket the
@@ -80,9 +91,10 @@ cudaError_t launch_down_tc(const LayerView& L, int64_t T, const Workspace& ws, f
 bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev);
 // force_timeout: the grid barrier waits for one CTA more than exist (the
 // bounded wait runs out; used only to test the timeout report).
+// clear_status: zero the status word (else the kernels only OR into it).
 cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Workspace& ws, float* h_dbg,
                           const DeviceInfo& dev, cudaEvent_t ev_start, cudaEvent_t ev_stop, bool force_timeout,
-                          cudaStream_t s);
+                          bool clear_status, cudaStream_t s);
 
 cudaError_t launch_block_dots(const uint8_t* w, const int8_t* qa, int64_t n, int32_t* out,
                               cudaStream_t s);
@@ -113,6 +125,10 @@ cudaError_t launch_residual_rmsnorm(float* x, const float* y, int64_t T, int H, 
                                     cudaStream_t s);
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// MOE_Q4_OK if the current device is compute capability 10.0, else
+// MOE_Q4_ERR_ARCH (or MOE_Q4_ERR_CUDA if it cannot be queried); abi.cu.
+int check_device();
 
 // Resident CTAs per SM of `kernel` at `threads` and `smem` dynamic bytes, with
 // the dynamic shared-memory limit raised to `smem` first.  Cached per device,

@@ -8,11 +8,15 @@
 // builds CUDA graphs and may not allocate while doing so.  Such a caller still
 // owns x and y; only the scratch moves into the library.
 //
-// Cost: every GPU that loads this library holds MOE_Q4_NOALLOC_SCRATCH_BYTES
-// of device memory until the process exits.
+// Cost: MOE_Q4_NOALLOC_SCRATCH_BYTES of device memory on each GPU where the
+// entry is used, until the process exits.  With CUDA's default lazy module
+// loading the array is placed on a device by the first call there (its
+// address lookup loads the module); with lazy loading off, when the
+// library's module is loaded into that device's context.
 #include <mutex>
 
 #include "moe_q4.h"
+#include "launch.h"
 
 namespace {
 
@@ -52,8 +56,11 @@ extern "C" int moe_q4_ffn_forward_noalloc(const moe_q4_layer* L, const float* x,
     if (need == 0) return moe_q4_ffn_forward(L, x, T, y, nullptr, 0, stream);
     if (need > kScratchBytes) return MOE_Q4_ERR_WORKSPACE;
     if (T == 0) return MOE_Q4_OK;
+    // the architecture first: on another device the lookup itself would fail
+    int rc = moeq4::check_device();
+    if (rc != MOE_Q4_OK) return rc;
     void* scratch = nullptr;
-    const int rc = scratch_address(&scratch);
+    rc = scratch_address(&scratch);
     if (rc != MOE_Q4_OK) return rc;
     return moe_q4_ffn_forward(L, x, T, y, scratch, kScratchBytes, stream);
 }

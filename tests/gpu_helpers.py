@@ -136,3 +136,81 @@ def near_tie_tokens(lw, x_np, v):
         gaps = np.abs(np.diff(srt[:lw.top_k + 1]))
         bad.append((int(t), bool(gaps.min() <= 2 * dl + 1e-12)))
     return bad
+
+
+def expected_block_dots(lw, T, v, down, g, rb, R):
+    """The oracle's per-block integer dot products of one row block of one
+    expert group, in the layout of moe_q4_debug.block_dots_out: [slot of the
+    group][row][block], from the device's own Q8_0 activations (bit-exact with
+    the oracle's, checked separately) and the layer's Q4_0 rows."""
+    k, E = lw.top_k, lw.n_experts
+    P = T * k
+    s0, s1 = int(v["off"][g]), int(v["off"][g + 1])
+    slots = np.arange(s0, s1)
+    if down:
+        acts = v["hq"][slots]
+        W = lw.sh_down if g == E else lw.w_down[g]
+        Wr = W[rb * R:(rb + 1) * R]
+    else:
+        tok = (v["sorted"][slots] // k) if g < E else (slots - P)
+        acts = v["qa"][tok]
+        Wg = lw.sh_gate if g == E else lw.w_gate[g]
+        Wu = lw.sh_up if g == E else lw.w_up[g]
+        half = R // 2
+        Wr = np.concatenate([Wg[rb * half:(rb + 1) * half], Wu[rb * half:(rb + 1) * half]])
+    c, nb = len(slots), Wr.shape[1]
+    blocks = np.broadcast_to(Wr[None], (c, R, nb, 18))
+    a = np.broadcast_to(acts.reshape(c, 1, nb, 32), (c, R, nb, 32))
+    return oracle.block_dots(blocks, a)
+
+
+def tile_boundary_tokens(lw, T, v, groups, tile):
+    """Tokens of the first and the last slot of every `tile`-slot tile of the
+    given expert groups (group E: the shared expert, slot P + t = token t)."""
+    k, E = lw.top_k, lw.n_experts
+    P = T * k
+    toks = []
+    for g in groups:
+        s0, s1 = int(v["off"][g]), int(v["off"][g + 1])
+        if s1 <= s0:
+            continue
+        firsts = np.arange(s0, s1, tile)
+        lasts = np.minimum(firsts + tile - 1, s1 - 1)
+        sl = np.unique(np.concatenate([firsts, lasts]))
+        toks.append((v["sorted"][sl] // k) if g < E else (sl - P))
+    return np.unique(np.concatenate(toks)) if toks else np.zeros(0, np.int64)
+
+
+def free_running_report(lw, x_np, v, tokens):
+    """The device's free-running output against the independent oracle (its
+    own routing and requantisation) on `tokens`:
+      identical   tokens whose top-k matches the oracle's (same order);
+      near_tie    tokens whose top-k differs, each at a near-tie (the
+                  oracle's logit gap at a changed position within twice the
+                  largest logit difference);
+      other       tokens whose top-k differs beyond a near-tie (must be 0);
+      row_err     the largest norm-wise row error |y - y_ref| / |y_ref| over
+                  the identical tokens;
+      flips       Q8_0 codes of h that differ by one step (identical tokens),
+      big_flips   codes that differ by more (must be 0), scale_diffs the
+                  binary16 scales of h that differ."""
+    tokens = np.asarray(tokens)
+    T = x_np.shape[0]
+    y_ref, dbg = oracle.moe_forward(lw, x_np[tokens], debug=True)
+    idx_dev = v["topk_idx"][tokens]
+    same = np.all(idx_dev == dbg["idx"], axis=1)
+    ties = dict(near_tie_tokens(lw, x_np, v))
+    diff_toks = tokens[~same]
+    near = sum(1 for t in diff_toks if ties.get(int(t), False))
+    y = v["y"][tokens].astype(np.float64)
+    r = y_ref.astype(np.float64)
+    row_err = np.linalg.norm(y - r, axis=1) / np.maximum(np.linalg.norm(r, axis=1), 1e-30)
+    hq_dev = pairs_from_slots(lw, T, v, v["hq"])[tokens]
+    dh_dev = pairs_from_slots(lw, T, v, v["dh"].view(np.uint16))[tokens]
+    dq = np.abs(hq_dev[same].astype(np.int32) - dbg["hq"][same].astype(np.int32))
+    return dict(tokens=int(len(tokens)), identical=int(same.sum()), near_tie=int(near),
+                other=int(len(diff_toks) - near),
+                row_err=float(row_err[same].max()) if same.any() else 0.0,
+                row_err_median=float(np.median(row_err[same])) if same.any() else 0.0,
+                flips=int(np.count_nonzero(dq == 1)), big_flips=int(np.count_nonzero(dq > 1)),
+                scale_diffs=int(np.count_nonzero(dh_dev[same] != dbg["dh"][same])))

@@ -142,8 +142,15 @@ def test_other_entry_points_reject_bad_args(lib):
 
     class _D(ctypes.Structure):
         _fields_ = [("h_out", ctypes.c_void_p), ("path", ctypes.c_int32), ("ev_start", ctypes.c_void_p),
-                    ("ev_stop", ctypes.c_void_p), ("force_spin_timeout", ctypes.c_int32)]
-    dbg = _D(None, 9, None, None, 0)
+                    ("ev_stop", ctypes.c_void_p), ("force_spin_timeout", ctypes.c_int32),
+                    ("block_dots_out", ctypes.c_void_p), ("block_dots_down", ctypes.c_int32),
+                    ("block_dots_group", ctypes.c_int32), ("block_dots_rb", ctypes.c_int32)]
+    dbg = _D(None, 9, None, None, 0, None, 0, 0, 0)
+    assert d(ctypes.byref(L), FAKE, 4, FAKE + 0x1000000, FAKE + 0x2000000, 1 << 40, ctypes.byref(dbg), None) == -1
+    # block-dot capture of a group that does not exist (E = 128 routed + the shared group 128)
+    dbg = _D(None, 0, None, None, 0, FAKE + 0x4000000, 0, 129, 0)
+    assert d(ctypes.byref(L), FAKE, 4, FAKE + 0x1000000, FAKE + 0x2000000, 1 << 40, ctypes.byref(dbg), None) == -1
+    dbg = _D(None, 0, None, None, 0, FAKE + 0x4000002, 0, 3, 0)     # misaligned capture buffer
     assert d(ctypes.byref(L), FAKE, 4, FAKE + 0x1000000, FAKE + 0x2000000, 1 << 40, ctypes.byref(dbg), None) == -1
 
 
@@ -210,3 +217,63 @@ def test_product_package_does_not_use_the_oracle():
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
                 assert "libmoe_q4_oracle" not in src and "moe_q4_oracle" not in src, f
+
+
+def test_arch_rejection_through_the_device_override(lib):
+    """Every entry point refuses a device that is not compute capability
+    10.0 with MOE_Q4_ERR_ARCH, before any CUDA call (this host has no GPU,
+    so a CUDA call would return MOE_Q4_ERR_CUDA instead) and before anything
+    is enqueued; the allocation-free entry checks the device before it looks
+    up its scratch."""
+    ov = lib.moe_q4_test_override_device
+    ov.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
+    L = make()
+    X, Y, WS, ST = FAKE, FAKE + 0x1000000, FAKE + 0x2000000, FAKE + 0x40000000
+    for major, minor in ((9, 0), (10, 3), (12, 0), (8, 9)):
+        assert ov(1, major, minor) == 0
+        try:
+            assert fwd(lib, L) == -5
+            q = lib.moe_q4_quantize_act
+            q.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32] + [ctypes.c_void_p] * 4
+            assert q(X, 4, 2048, Y, WS, None, None) == -5
+            r = lib.moe_q4_route
+            r.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64] + [ctypes.c_void_p] * 4
+            assert r(ctypes.byref(L), X, 4, Y, Y + 4096, WS, None) == -5
+            h = lib.moe_q4_ffn_forward_host
+            h.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                          ctypes.c_size_t, ctypes.c_void_p]
+            assert h(ctypes.byref(L), X, 4, Y, WS, 1 << 40, None) == -5
+            n = lib.moe_q4_ffn_forward_noalloc
+            n.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+            assert n(ctypes.byref(L), X, 4, Y, None) == -5
+            nr = lib.moe_q4_residual_rmsnorm
+            nr.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float,
+                           ctypes.c_void_p, ctypes.c_void_p]
+            assert nr(X, Y, 4, 2048, 1e-6, WS, None) == -5
+            sf = lib.moe_q4_stack_forward
+            sf.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64, ctypes.c_float,
+                           ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+            arr = (_L * 2)(make(), make())
+            assert sf(arr, 2, X, 4, 1e-6, WS, 1 << 40, None) == -5
+            g = lib.moe_q4_gemv
+            g.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64,
+                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+            assert g(ST, 1000, 2048, X, 1, Y, WS, 1 << 20, None) == -5
+            st = lib.moe_q4_ffn_forward_streamed
+            st.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                           ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+            assert st(ctypes.byref(L), X, 4, Y, WS, 1 << 40, ST, 1 << 40, None) == -5
+            b = lib.moe_q4_block_dots
+            b.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+            assert b(X, Y, 8, WS, None) == -5
+            # argument errors still come first
+            assert fwd(lib, make(top_k=0)) == -1
+        finally:
+            ov(0, 0, 0)
+    # an override to 10.0 itself is not a rejection: on this GPU-less host the
+    # call goes on to the (failing) driver query
+    assert ov(1, 10, 0) == 0
+    try:
+        assert fwd(lib, L) == -6
+    finally:
+        ov(0, 0, 0)

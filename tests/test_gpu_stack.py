@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import synth
-from gpu_helpers import check_routing, rule13, run_forward, teacher_forced_check
+from gpu_helpers import check_routing, rule13, run_forward, teacher_forced_check, tile_boundary_tokens
 
 pytestmark = pytest.mark.gpu
 
@@ -87,7 +87,11 @@ def _run_stack(T, n_check, seed=0):
         assert u.max() <= 1, f"layer {l}: RMSNorm off by {u.max()} ulp"
         v = run_forward(lw, xn_np, want_h=False, L=L)
         check_routing(lw, xn_np, v)
-        toks = np.unique(np.concatenate([[0, T - 1], rng.choice(T, n_check, replace=False)]))
+        # the first and last slot of every 64-slot tile of the layer's most
+        # loaded expert and of the shared expert, plus a random sample
+        heavy = int(np.argmax(v["cnt"][:E]))
+        toks = np.unique(np.concatenate([[0, T - 1], rng.choice(T, n_check, replace=False),
+                                         tile_boundary_tokens(lw, T, v, [heavy, E], 64)]))
         teacher_forced_check(lw, xn_np, v, toks)
         assert v["status"][0] == 0, f"layer {l}: status {v['status'][0]}"
         y = torch.from_numpy(v["y"]).cuda()

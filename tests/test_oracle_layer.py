@@ -41,6 +41,31 @@ def test_block_dot_extremes():
     assert oracle.block_dot(blk, np.full(32, -127, np.int8)) == -7 * 127 * 32
 
 
+def test_block_dots_vs_dense_integer_dot():
+    """The batched block dot (used to check the device's per-block sums in
+    bulk) against numpy's integer dot of the dequantised nibbles: with the
+    scale set to 1.0 a Q4_0 block dequantises to exactly nibble - 8."""
+    rng = np.random.default_rng(21)
+    n = 3000
+    blocks = rng.integers(0, 256, size=(n, 18), dtype=np.uint8)
+    blocks[:, 0:2] = [0x00, 0x3C]
+    qa = rng.integers(-127, 128, size=(n, 32), dtype=np.int8)
+    qa[0], blocks[0, 2:] = 127, 0x00                  # -8 * 127 * 32
+    qa[1], blocks[1, 2:] = -127, 0xFF                 # 7 * -127 * 32
+    w = dequant_q4_0(blocks.reshape(n, 1, 18)).reshape(n, 32)
+    assert np.array_equal(w, np.rint(w)) and w.min() >= -8 and w.max() <= 7
+    ref = np.einsum("ij,ij->i", w.astype(np.int64), qa.astype(np.int64))
+    got = oracle.block_dots(blocks, qa)
+    assert got.dtype == np.int32 and np.array_equal(got, ref)
+    assert got[0] == -8 * 127 * 32 and got[1] == -7 * 127 * 32
+    # the hand-worked block, inside a batch of shape [2, 1]
+    for hx, acts, I, *_ in rows("block_dot.txt"):
+        blk = np.frombuffer(hexbytes(hx), dtype=np.uint8)
+        q = np.array([int(v) for v in acts.split()], dtype=np.int8)
+        out = oracle.block_dots(np.stack([blk, blk])[:, None], np.stack([q, -q])[:, None])
+        assert out.shape == (2, 1) and out[0, 0] == int(I) and out[1, 0] == -int(I)
+
+
 @pytest.mark.parametrize("N,K", [(7, 64), (33, 256), (16, 512)])
 def test_q4_matvec_vs_dense_binary64(N, K):
     rng = np.random.default_rng(N * K)

@@ -32,16 +32,20 @@ def _reference(L, x):
 
 def test_noalloc_matches_forward_on_two_calls_in_a_row():
     x1, lw1 = synth.workload_inputs("tiny_t16", seed=0)
-    x2, lw2 = synth.workload_inputs("decode_t1", seed=0, T=3)
+    x2, lw2 = synth.workload_inputs("decode_t1", seed=0, T=300)
     L1, L2 = m.Layer.from_host(lw1), m.Layer.from_host(lw2)
     xd1, xd2 = torch.from_numpy(x1).cuda(), torch.from_numpy(x2[1:2].copy()).cuda()
-    ref1, ref2 = _reference(L1, xd1), _reference(L2, xd2)
-    # two calls in a row on the shared scratch: a 16-token layer, then a
-    # one-token call of a different layer that reuses the same array
+    xd3 = torch.from_numpy(x2[:256].copy()).cuda()
+    ref1, ref2, ref3 = _reference(L1, xd1), _reference(L2, xd2), _reference(L2, xd3)
+    # calls in a row on the shared scratch: a 16-token layer (streaming
+    # kernels), a one-token call of a different layer (fused decode kernels),
+    # then 256 tokens of that layer (tensor-core kernels, another layout of
+    # the same array)
     y1 = m.moe_q4_ffn_forward_noalloc(L1, xd1)
     y2 = m.moe_q4_ffn_forward_noalloc(L2, xd2)
+    y3 = m.moe_q4_ffn_forward_noalloc(L2, xd3)
     torch.cuda.synchronize()
-    for y, ref in ((y1, ref1), (y2, ref2)):
+    for y, ref in ((y1, ref1), (y2, ref2), (y3, ref3)):
         ok, worst = rule13(y.cpu().numpy(), ref, 1e-3)
         assert ok, f"no-alloc output differs from moe_q4_ffn_forward: worst {worst:.3e}"
     # and once more with the first layer, after the scratch held the second call

@@ -131,7 +131,10 @@ size_t moe_q4_ffn_host_workspace_bytes(const moe_q4_layer* L, int64_t T_max);
 /* moe_q4_ffn_forward with x and y in HOST memory (pinned for asynchronous
  * copies): enqueues the host-to-device copy of x, the forward, and the
  * device-to-host copy of y on `stream`.  y is valid after the caller
- * synchronises the stream. */
+ * synchronises the stream.  For one token with both x and y page-locked (and
+ * 16-byte aligned) the copies are made by the kernels themselves: the router
+ * kernel reads x and a last kernel writes y over the bus, with no copy node
+ * between the kernels. */
 int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t T, float* y_host,
                             void* workspace, size_t ws_bytes, moe_q4_stream_t stream);
 
@@ -289,10 +292,11 @@ typedef struct {
     int32_t path;     /* MOE_Q4_PATH_* */
     void* ev_start;   /* cudaEvent_t recorded just before the dominant (gate/up) kernel, or NULL */
     void* ev_stop;    /* cudaEvent_t recorded just after it, or NULL */
-    int32_t force_spin_timeout;  /* nonzero: the fused T = 1 kernel's grid barrier waits for one more
-                                    CTA than exists, so its bounded wait runs out; the call completes
-                                    with correct results and MOE_Q4_STATUS_SPIN_TIMEOUT in the status
-                                    word (tests of the timeout report; about a second per call) */
+    int32_t force_spin_timeout;  /* nonzero: one CTA of the fused T = 1 FFN kernel waits for 16 bytes
+                                    more than its weight copies deliver, so its bounded wait runs out;
+                                    the call completes with correct results and
+                                    MOE_Q4_STATUS_SPIN_TIMEOUT in the status word (tests of the timeout
+                                    report; about half a second per call) */
     /* Per-block integer dot products I_b = sum_{i<32} (nibble_i - 8) * q_i of
      * the grouped paths (tensor-core and streaming), exactly as the projection
      * kernel computed them (the tensor-core path: the MMA's accumulator before
@@ -309,6 +313,11 @@ typedef struct {
     int32_t block_dots_down;   /* 0: the gate/up projection, 1: the down projection */
     int32_t block_dots_group;  /* expert group g (n_experts: the shared expert) */
     int32_t block_dots_rb;     /* row block */
+    /* Fused T = 1 path only: device uint64[2], 8-byte aligned; per call
+     * [0] += the FFN kernel's span in its first CTA (%globaltimer ns, from
+     * its start to its end, inside the programmatic-launch chain, with no
+     * event between the kernels), [1] += 1.  NULL: not timed. */
+    unsigned long long* decode_kernel_ns;
 } moe_q4_debug;
 
 /* moe_q4_ffn_forward with inspection options (see moe_q4_debug). */

@@ -73,7 +73,8 @@ class _Debug(ctypes.Structure):
     _fields_ = [("h_out", ctypes.c_void_p), ("path", ctypes.c_int32),
                 ("ev_start", ctypes.c_void_p), ("ev_stop", ctypes.c_void_p), ("force_spin_timeout", ctypes.c_int32),
                 ("block_dots_out", ctypes.c_void_p), ("block_dots_down", ctypes.c_int32),
-                ("block_dots_group", ctypes.c_int32), ("block_dots_rb", ctypes.c_int32)]
+                ("block_dots_group", ctypes.c_int32), ("block_dots_rb", ctypes.c_int32),
+                ("decode_kernel_ns", ctypes.c_void_p)]
 
 
 def _load() -> ctypes.CDLL:
@@ -240,7 +241,7 @@ def moe_q4_ffn_forward(layer: Layer, x: torch.Tensor, y=None, workspace=None, st
 
 def moe_q4_ffn_forward_debug(layer: Layer, x: torch.Tensor, y, workspace, h_out=None, path=PATH_AUTO,
                              ev_start=None, ev_stop=None, stream=None, force_spin_timeout=False,
-                             block_dots=None):
+                             block_dots=None, decode_kernel_ns=None):
     """block_dots: None or (out int32 tensor, down (bool), group, row block):
     capture the per-block integer dot products of that row block (see
     moe_q4_debug in include/moe_q4.h for the layout)."""
@@ -249,7 +250,8 @@ def moe_q4_ffn_forward_debug(layer: Layer, x: torch.Tensor, y, workspace, h_out=
     dbg = _Debug(None if h_out is None else h_out.data_ptr(), int(path),
                  None if ev_start is None else ev_start.cuda_event,
                  None if ev_stop is None else ev_stop.cuda_event, int(bool(force_spin_timeout)),
-                 None if bd_out is None else bd_out.data_ptr(), int(bool(bd_down)), int(bd_group), int(bd_rb))
+                 None if bd_out is None else bd_out.data_ptr(), int(bool(bd_down)), int(bd_group), int(bd_rb),
+                 None if decode_kernel_ns is None else decode_kernel_ns.data_ptr())
     _check(_lib.moe_q4_ffn_forward_debug(layer.ref, _p(x), T, _p(y), _p(workspace), workspace.numel(),
                                          ctypes.byref(dbg), _stream(stream)), "moe_q4_ffn_forward_debug")
     return y

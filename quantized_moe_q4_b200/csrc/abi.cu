@@ -195,6 +195,26 @@ static Workspace carve(void* base, const size_t off[WS_COUNT]) {
     return w;
 }
 
+// Page-locked host memory the GPU can address (unified addressing), or device
+// memory, by the runtime's pointer attributes.
+static bool pinned_host(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeHost;
+}
+
+static bool on_device(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
 static int cuda_rc(cudaError_t e) {
     if (e == cudaSuccess) return MOE_Q4_OK;
     g_last_cuda_error = e;
@@ -224,6 +244,7 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
     const size_t xy_bytes = sizeof(float) * (size_t)(T * L.H);
     if (overlap(x, xy_bytes, y, xy_bytes) || overlap(y, xy_bytes, ws, off[WS_TOTAL])) return MOE_Q4_ERR_OVERLAP;
     if (dbg && dbg->h_out && !aligned(dbg->h_out, 4)) return MOE_Q4_ERR_ALIGN;
+    if (dbg && dbg->decode_kernel_ns && !aligned(dbg->decode_kernel_ns, 8)) return MOE_Q4_ERR_ALIGN;
     if (dbg && dbg->block_dots_out &&
         (!aligned(dbg->block_dots_out, 4) || dbg->block_dots_group < 0 ||
          dbg->block_dots_group > Lp->n_experts - (Lp->has_shared ? 0 : 1) || dbg->block_dots_rb < 0))
@@ -238,7 +259,8 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
     const int path = dbg ? dbg->path : MOE_Q4_PATH_AUTO;
     if ((path == MOE_Q4_PATH_AUTO || path == MOE_Q4_PATH_DECODE) && decode_eligible(L, T, dev))
         return cuda_rc(launch_decode(L, x, y, w, dbg ? dbg->h_out : nullptr, dev, ev0, ev1,
-                                     dbg && dbg->force_spin_timeout, clear_status, s));
+                                     dbg && dbg->force_spin_timeout, clear_status,
+                                     dbg ? dbg->decode_kernel_ns : nullptr, nullptr, s));
 
     // grouped paths: tensor cores once experts see tens of tokens, else dp4a
     const bool tc = (path == MOE_Q4_PATH_TENSOR_CORE) || (path == MOE_Q4_PATH_AUTO && T >= TC_MIN_TOKENS);
@@ -382,6 +404,16 @@ int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t 
     DeviceInfo dev;
     rc = current_device(&dev);
     if (rc) return rc;
+    // one token with page-locked x and y: the decode kernels read x and write
+    // y over the bus themselves, so the call stays one programmatic-launch
+    // chain (a copy node would end it)
+    const LayerView Lv = view(L);
+    if (T == 1 && decode_eligible(Lv, T, dev) && aligned(x_host, 16) && aligned(y_host, 16) && pinned_host(x_host) &&
+        pinned_host(y_host)) {
+        const Workspace w = carve(workspace, off);
+        return cuda_rc(launch_decode(Lv, x_host, y_dev, w, nullptr, dev, nullptr, nullptr, false, true, nullptr,
+                                     y_host, s));
+    }
     MOE_TRY(cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s));
     rc = forward_impl(L, x_dev, T, y_dev, workspace, off[WS_TOTAL], nullptr, s);
     if (rc) return rc;
@@ -493,24 +525,6 @@ static void staging_layout(const moe_q4_layer* L, size_t off[7]) {
     const size_t sz[6] = {E * gu, E * gu, E * dn, S * gu, S * gu, S * dn};
     off[0] = 0;
     for (int i = 0; i < 6; ++i) off[i + 1] = off[i] + align256(sz[i]);
-}
-
-static bool pinned_host(const void* p) {
-    cudaPointerAttributes a;
-    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
-        cudaGetLastError();
-        return false;
-    }
-    return a.type == cudaMemoryTypeHost;
-}
-
-static bool on_device(const void* p) {
-    cudaPointerAttributes a;
-    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
-        cudaGetLastError();
-        return false;
-    }
-    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
 }
 
 size_t moe_q4_staging_bytes(const moe_q4_layer* L) {

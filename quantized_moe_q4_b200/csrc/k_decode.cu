@@ -10,23 +10,35 @@
 //
 //   decode_router_kernel: one CTA per expert.  Before waiting on the previous
 //     kernel it bulk-copies its router row into shared memory; then the logit
-//     (four independent FMA chains), and the first H/32 CTAs quantise one
-//     Q8_0 block of x each.  CTA 0 zeroes the status word and the grid-barrier
-//     counter of the next kernel.
-//   decode_ffn_kernel: cooperative, one CTA of 16 warps per SM.  Before
-//     waiting on the router, bulk-copies the shared expert's weights
-//     (routing-independent); then the top-k (every thread ranks one logit),
-//     bulk copies of its gate/up row block (32 rows of F = one Q8_0 block of
-//     h) and of its slice of down rows for all k+1 experts; gate/up dot
-//     products (the activation block loaded once for four rows, four
-//     independent chains per lane), SwiGLU, requantisation; one bounded grid
-//     barrier; down dot products (eight rows per lane group) and the
-//     router-weighted combine into y in a fixed order (no atomics).
+//     (four independent FMA chains); the first H/32 CTAs quantise one Q8_0
+//     block of x each; y is zeroed (the FFN kernel accumulates into it).
+//   decode_ffn_kernel: clusters of 8 CTAs, one cluster per (expert of the
+//     token, 256-wide part of F).  CTA r of a cluster owns one 32-row block
+//     of h (32 gate rows and the same 32 up rows) and, for the down
+//     projection, H/8 rows restricted to the cluster's 8 blocks of F.  The
+//     shared expert's weights are copied before the wait on the router (they
+//     do not depend on the routing); routed CTAs rank the logits (every CTA
+//     the same way), then copy their gate/up rows (bulk copies) and their
+//     down slice (a 2D tensor copy: 144 bytes of each of H/8 rows) at once.
+//     Gate/up dot products, SwiGLU and the Q8_0 requantisation give the
+//     CTA's h block, which it writes into the shared memory of all 8 CTAs of
+//     its cluster (distributed shared memory); one cluster barrier, then the
+//     down partial sums over the cluster's 8 h blocks, and the router-weighted
+//     partial rows are added into y with vector reductions (red.v4.f32).
 //
-// Every phase runs once per launch on every SM, so each is written as short,
-// independent dependency chains: measured on B200, the same arithmetic with
-// one row at a time and a reduction per row took 3.7x longer.
+// No grid-wide barrier: the only exchange between CTAs is inside a cluster,
+// and the clusters are independent of one another (y collects their partial
+// sums), so the grid needs no co-residency.  The order of the (k+S) x F/256
+// partial sums added into an element of y is not fixed: results agree across
+// runs to binary32 rounding, not bit for bit.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include <cooperative_groups.h>
 
 #include "common.cuh"
 #include "launch.h"
@@ -34,23 +46,31 @@
 
 namespace moeq4 {
 
-constexpr uint32_t MBAR_LIMIT = 1u << 20;
+namespace {
+
+constexpr uint32_t MBAR_LIMIT = 1u << 20;   // bounded waits: about 0.5 s
+constexpr int CL = 8;                       // CTAs per cluster = h blocks per F part
+constexpr int FFN_THREADS = 512;            // 16 warps
+constexpr int FFN_WARPS = FFN_THREADS / 32;
+constexpr int DN_KB = 8;                    // down blocks per F part (144 bytes of a row)
+constexpr int DN_BOX_ROWS = 256;            // rows per 2D tensor copy of the down slice
+// The router kernel's timeout report: a NaN logit with this payload (arithmetic
+// on data never produces it).
+constexpr uint32_t TIMEOUT_NAN = 0x7fc0deadu;
 
 struct DecodeParams {
     int H, F, E, k, S;
-    int rows_per_cta;  // down rows of H per FFN CTA
-    int nctas;         // grid of decode_ffn_kernel
-    int barrier_target;  // arrivals the grid barrier waits for (nctas; nctas + 1 only in the timeout test)
+    int nF;              // F parts of 256 per expert (clusters per expert)
+    int box_rows;        // rows per tensor copy of the down slice (divides H/8)
     int clear_status;    // the router kernel zeroes the status word (else it accumulates)
+    int force_timeout;   // CTA 0's first gate/up barrier expects 16 bytes that never come
     const float* x;
     const float* w_router;
     const float* bias;
     const uint8_t* w_gate;
     const uint8_t* w_up;
-    const uint8_t* w_down;
     const uint8_t* sh_gate;
     const uint8_t* sh_up;
-    const uint8_t* sh_down;
     float* logits;
     int32_t* topk_idx;
     float* topk_w;
@@ -64,7 +84,14 @@ struct DecodeParams {
     uint16_t* dh;
     float* h_dbg;
     float* y;
-    uint32_t* status;  // status[0] = status word, status[1] = grid-barrier counter
+    uint32_t* status;
+    unsigned long long* kernel_ns;  // optional: [0] += CTA 0's span of the FFN kernel, [1] += 1
+};
+
+// 2D views of the down matrices for the tensor copies: rows of F/32 blocks of
+// 18 bytes, a box is 144 bytes (8 blocks) x up to 256 rows.
+struct DecodeMaps {
+    CUtensorMap down, sh_down;
 };
 
 // ---------------------------------------------------------------------------
@@ -107,12 +134,45 @@ __device__ __forceinline__ bool bf_owner(int lane) {
     return (lane & (W / V - 1)) == 0;
 }
 
+// acc[r] += W4A8 term of one block in NR rows (stride row_bytes) against one
+// staged Q8_0 block, the activation loaded once for all rows: NR independent
+// dependency chains per lane.
+template <int NR>
+__device__ __forceinline__ void block_rows(const uint8_t* rows, size_t row_bytes, const int8_t* q_blk, int qsum,
+                                           float da, float (&acc)[NR]) {
+    const int4* qv = reinterpret_cast<const int4*>(q_blk);
+    const int4 a0 = qv[0], a1 = qv[1];
+    const int qa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        uint32_t qs[4], dbits;
+        load_q4_block_smem(rows + (size_t)r * row_bytes, qs, dbits);
+        acc[r] = fmaf((float)q4_q8_dot(qs, qa, qsum), half_bits_to_float(dbits) * da, acc[r]);
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// y[0..3] += v (one vector reduction at L2; y 16-byte aligned)
+__device__ __forceinline__ void red_add_v4(float* y, float4 v) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(y), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
+}  // namespace
+
 // ---------------------------------------------------------------------------
-// K1: router logits (one CTA per expert) + Q8_0 of x.
+// K1: router logits (one CTA per expert), Q8_0 of x, y zeroed.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
-    extern __shared__ __align__(16) unsigned char dsm[];
-    float* wr_s = reinterpret_cast<float*>(dsm);
+    extern __shared__ __align__(16) unsigned char dsm_router[];
+    float* wr_s = reinterpret_cast<float*>(dsm_router);
     __shared__ __align__(8) uint64_t bar;
     __shared__ float red[4];
     const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -128,10 +188,8 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
     }
     pdl_launch_dependents();
     pdl_wait();  // x and the workspace are now the previous kernels' results
-    if (e == 0 && tid == 0) {
-        if (p.clear_status) p.status[0] = 0u;  // status word
-        p.status[1] = 0u;  // grid-barrier counter of decode_ffn_kernel
-    }
+    if (e == 0 && tid == 0 && p.clear_status) p.status[0] = 0u;
+    for (int i = e * 128 + tid; i < H; i += (int)gridDim.x * 128) p.y[i] = 0.0f;
     const bool ok = mbar_wait_bounded(&bar, 0, MBAR_LIMIT);
     const float4* x4 = reinterpret_cast<const float4*>(p.x);
     const float4* w4 = reinterpret_cast<const float4*>(wr_s);
@@ -150,7 +208,7 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
     __syncthreads();
     if (tid == 0) {
         const float l = (red[0] + red[1]) + (red[2] + red[3]) + (p.bias ? __ldg(p.bias + e) : 0.0f);
-        p.logits[e] = ok ? l : __int_as_float(0x7fc00000);  // a NaN logit reports the timeout
+        p.logits[e] = ok ? l : __uint_as_float(TIMEOUT_NAN);
     }
     // Q8_0 of x: block b by warp 0 of CTA b (and CTA b + E, ... when H/32 > E).
     // A binary16 scale overflow is visible to the next kernel as an infinite scale.
@@ -166,177 +224,136 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// K2: top-k, gate/up + SwiGLU + requant, grid barrier, down + combine.
+// K2: gate/up + SwiGLU + requant, cluster exchange, down + combine.
 // ---------------------------------------------------------------------------
 struct DecodeSmem {
-    size_t gu, dn, qa, da, qsum, hq, dhs, hsum, o, total;  // byte offsets
+    size_t gu, dn, qa, da, qsum, o, total;  // byte offsets
 };
 
-__host__ __device__ inline size_t al16(size_t v) { return (v + 15) & ~size_t(15); }
+__host__ __device__ inline size_t al128(size_t v) { return (v + 127) & ~size_t(127); }
 
-__host__ __device__ inline DecodeSmem decode_smem_layout(int H, int F, int J, int R) {
-    const int nbH = H / QK, nbF = F / QK;
+__host__ __device__ inline DecodeSmem decode_smem_layout(int H) {
+    const int nbH = H / QK;
     DecodeSmem L;
     size_t o = 0;
-    L.gu = o;   o += al16((size_t)64 * nbH * Q4_BYTES);
-    L.dn = o;   o += al16((size_t)J * R * nbF * Q4_BYTES);
-    L.qa = o;   o += al16((size_t)H);
-    L.da = o;   o += al16((size_t)nbH * 4);
-    L.qsum = o; o += al16((size_t)nbH * 4);
-    L.hq = o;   o += al16((size_t)J * F);
-    L.dhs = o;  o += al16((size_t)J * nbF * 4);
-    L.hsum = o; o += al16((size_t)J * nbF * 4);
-    L.o = o;    o += al16((size_t)J * R * 4);
-    L.total = o;
+    L.gu = o;   o += al128((size_t)64 * nbH * Q4_BYTES);       // 32 gate + 32 up rows
+    L.dn = o;   o += al128((size_t)(H / CL) * DN_KB * Q4_BYTES); // H/8 rows x 8 blocks
+    L.qa = o;   o += al128((size_t)H);
+    L.da = o;   o += al128((size_t)nbH * 4);
+    L.qsum = o; o += al128((size_t)nbH * 4);
+    L.o = o;    o += al128((size_t)(H / CL) * 4);
+    L.total = o + 128;   // slack to align the map to 128 bytes
     return L;
 }
 
-// acc[r] += W4A8 term of block b of NR rows (stride row_bytes) against one
-// staged Q8_0 block, the activation loaded once for all rows: NR independent
-// dependency chains per lane.
-template <int NR>
-__device__ __forceinline__ void block_rows(const uint8_t* rows, size_t row_bytes, int nrows, int b, const int8_t* q_s,
-                                           int qsum, float da, float (&acc)[NR]) {
-    const int4* qv = reinterpret_cast<const int4*>(q_s + b * QK);
-    const int4 a0 = qv[0], a1 = qv[1];
-    const int qa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-        if (r < nrows) {
-            uint32_t qs[4], dbits;
-            load_q4_block_smem(rows + (size_t)r * row_bytes + (size_t)b * Q4_BYTES, qs, dbits);
-            acc[r] = fmaf((float)q4_q8_dot(qs, qa, qsum), half_bits_to_float(dbits) * da, acc[r]);
-        }
-    }
-}
-
-// Down projection for the CTA's rows: tasks (pair jj, chunk of 8 rows), one per
-// lane group of W lanes; lanes split the F/32 blocks.
-template <int W>
-__device__ __forceinline__ void down_tasks(const uint8_t* dn_s, size_t row_dn, int R, int rows, int J, int nbF, int F,
-                                           const int8_t* hq_s, const float* dh_s, const int* hsum_s, const int* slot_s,
-                                           float* o_s, int warp, int n_warps) {
-    constexpr int G = 32 / W;  // lane groups per warp
-    const int lane = threadIdx.x & 31, grp = lane / W, sub = lane % W;
-    const int chunks = (rows + 7) / 8;
-    const int n_tasks = J * chunks;
-#pragma unroll 1
-    for (int t0 = warp * G; t0 < n_tasks; t0 += n_warps * G) {  // warp-uniform trip count
-        const int task = min(t0 + grp, n_tasks - 1);
-        const int jj = task / chunks, r0 = (task % chunks) * 8;
-        const int nr = min(8, rows - r0);
-        const int slot = slot_s[jj];
-        const int8_t* q = hq_s + (size_t)slot * F;
-        const uint8_t* base = dn_s + ((size_t)jj * R + r0) * row_dn;
-        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll 1
-        for (int b = sub; b < nbF; b += W)
-            block_rows<8>(base, row_dn, nr, b, q, hsum_s[slot * nbF + b], dh_s[slot * nbF + b], acc);
-        const float s = butterfly<8, W>(acc);
-        const int r = bf_index<8, W>(sub);
-        if (bf_owner<8, W>(sub) && t0 + grp < n_tasks && r < nr) o_s[jj * R + r0 + r] = s;
-    }
-}
-
-constexpr int FFN_THREADS = 512;  // 16 warps
-constexpr int FFN_WARPS = FFN_THREADS / 32;
-
-// At most 96 registers per thread: 512 x 96 plus the router kernel's CTAs fit
-// one SM's register file, so the next router kernel can become resident
-// beside this one under programmatic dependent launch.
-__global__ void __maxnreg__(96) decode_ffn_kernel(DecodeParams p) {
-    extern __shared__ __align__(16) unsigned char dsm[];
+__global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams p,
+                                                                    const __grid_constant__ DecodeMaps maps) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    extern __shared__ __align__(16) unsigned char dsm_raw[];
+    // tensor-copy destinations 128-byte aligned (the allocation has 128 bytes of slack)
+    unsigned char* dsm = dsm_raw + ((128u - (smem_u32(dsm_raw) & 127u)) & 127u);
     __shared__ __align__(8) uint64_t bar_gu[4];
     __shared__ __align__(8) uint64_t bar_dn;
-    __shared__ __align__(16) float logit_s[256];  // E rounded up to 16
+    __shared__ __align__(16) float logit_s[256];
     __shared__ int idx_s[16];
-    __shared__ float w_s[16];
     __shared__ float ex_s[16];
+    __shared__ float w_s[16];
     __shared__ int slot_s[17];
     __shared__ int warp_chosen[FFN_WARPS];
     __shared__ float gs[32], us[32];
+    __shared__ __align__(16) int8_t hx_q[CL][QK];   // the cluster's 8 requantised h blocks
+    __shared__ float hx_d[CL];
+    __shared__ int hx_sum[CL];
     __shared__ int flags_s;
 
+    unsigned long long t_entry = 0;
+    if (p.kernel_ns && blockIdx.x == 0 && threadIdx.x == 0) t_entry = global_ns();
+
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int H = p.H, F = p.F, E = p.E, k = p.k, S = p.S;
-    const int J = k + S, nbH = H / QK, nbF = F / QK, nrb = F / GU_ROWS;
-    const int R = p.rows_per_cta;
-    const size_t row_gu = (size_t)nbH * Q4_BYTES, row_dn = (size_t)nbF * Q4_BYTES;
-    const size_t gu_stride = (size_t)F * row_gu, dn_stride = (size_t)H * row_dn;
-    const DecodeSmem SL = decode_smem_layout(H, F, J, R);
+    const int H = p.H, F = p.F, E = p.E, k = p.k;
+    const int nbH = H / QK, nbF = F / QK;
+    const int c = blockIdx.x / CL;                  // cluster
+    const int r = (int)cluster.block_rank();        // CTA within the cluster
+    const int j = c / p.nF;                         // expert of the token: rank j < k, or k = shared
+    const int fp = c % p.nF;                        // F part: h blocks 8 fp .. 8 fp + 7
+    const int hb = fp * CL + r;                     // this CTA's h block
+    const bool is_shared = (j == k);
+    const int Hs = H / CL;                          // down rows of this CTA
+    const int n0 = r * Hs;
+    const size_t row_gu = (size_t)nbH * Q4_BYTES;
+    const size_t gu_stride = (size_t)F * row_gu;    // bytes of one expert's gate (or up) matrix
+    const DecodeSmem SL = decode_smem_layout(H);
     uint8_t* gu_s = dsm + SL.gu;
     uint8_t* dn_s = dsm + SL.dn;
     int8_t* qa_s = reinterpret_cast<int8_t*>(dsm + SL.qa);
     float* da_s = reinterpret_cast<float*>(dsm + SL.da);
     int* qsum_s = reinterpret_cast<int*>(dsm + SL.qsum);
-    int8_t* hq_s = reinterpret_cast<int8_t*>(dsm + SL.hq);
-    float* dh_s = reinterpret_cast<float*>(dsm + SL.dhs);
-    int* hsum_s = reinterpret_cast<int*>(dsm + SL.hsum);
     float* o_s = reinterpret_cast<float*>(dsm + SL.o);
-
-    const int n_items = J * nrb;
-    const int n0 = blockIdx.x * R;
-    const int rows = max(0, min(R, H - n0));
     bool timed_out = false;
 
     if (tid == 0) {
-        for (int c = 0; c < 4; ++c) mbar_init(&bar_gu[c], 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&bar_gu[i], 1);
         mbar_init(&bar_dn, 1);
         mbar_fence_init();
         flags_s = 0;
     }
+    // first phase of the cluster barrier: its wait (before the first write into
+    // another CTA's shared memory) guarantees every CTA of the cluster runs
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     __syncthreads();
 
-    // gate/up copies of one item, issued by warp 0: chunk c = 8 gate rows + 8
-    // up rows on bar_gu[c]; lane 2c + mat issues one copy
+    // copies of this CTA's weights, issued by warp 0: gate/up chunk i = 8 gate
+    // rows + the same 8 up rows on bar_gu[i] (lane 2i + m issues matrix m);
+    // the down slice = rows n0 .. n0 + Hs, blocks 8 fp .. 8 fp + 7
     const uint32_t chunk_bytes = (uint32_t)(8 * row_gu);
-    auto issue_gateup = [&](const uint8_t* Wg, const uint8_t* Wu, int rb) {
-        if (lane < 4) mbar_arrive_expect_tx(&bar_gu[lane], 2u * chunk_bytes);
+    auto issue_copies = [&](const uint8_t* Wg, const uint8_t* Wu, const CUtensorMap* dmap, int drow0) {
+        if (lane < 4) {
+            const uint32_t extra = (p.force_timeout && blockIdx.x == 0 && lane == 0) ? 16u : 0u;
+            mbar_arrive_expect_tx(&bar_gu[lane], 2u * chunk_bytes + extra);
+        }
+        if (lane == 4) mbar_arrive_expect_tx(&bar_dn, (uint32_t)(Hs * DN_KB * Q4_BYTES));
         __syncwarp();
         if (lane < 8) {
-            const int c = lane >> 1, mat = lane & 1;
-            bulk_g2s(gu_s + (size_t)(mat * 32 + 8 * c) * row_gu, (mat ? Wu : Wg) + (size_t)(rb * GU_ROWS + 8 * c) * row_gu,
-                     chunk_bytes, &bar_gu[c]);
+            const int ch = lane >> 1, m = lane & 1;
+            bulk_g2s(gu_s + (size_t)(m * 32 + 8 * ch) * row_gu, (m ? Wu : Wg) + (size_t)(hb * 32 + 8 * ch) * row_gu,
+                     chunk_bytes, &bar_gu[ch]);
+        } else if (lane == 8) {
+            for (int r0 = 0; r0 < Hs; r0 += p.box_rows)
+                tma_load_2d(dn_s + (size_t)r0 * DN_KB * Q4_BYTES, dmap, fp * DN_KB * Q4_BYTES, drow0 + r0, &bar_dn);
         }
     };
 
-    // ---- prologue: routing-independent copies (the shared expert), before the wait
-    const int item0 = blockIdx.x;
-    const bool item0_shared = S && item0 < n_items && (item0 / nrb) == k;
-    if (warp == 0) {
-        if (rows > 0 && lane == 0) {
-            mbar_arrive_expect_tx(&bar_dn, (uint32_t)(J * rows * row_dn));
-            if (S)
-                bulk_g2s(dn_s + (size_t)k * R * row_dn, p.sh_down + (size_t)n0 * row_dn, (uint32_t)(rows * row_dn),
-                         &bar_dn);
-        }
-        if (item0_shared) issue_gateup(p.sh_gate, p.sh_up, item0 % nrb);
-    }
+    // ---- prologue: the shared expert's copies do not depend on the routing
+    if (is_shared && warp == 0) issue_copies(p.sh_gate, p.sh_up, &maps.sh_down, n0);
 
-    pdl_wait();  // logits, Q8_0 of x and the zeroed status words are visible
+    pdl_wait();  // logits, Q8_0 of x and the zeroed y are visible
     pdl_launch_dependents();
 
-    // ---- top-k: expert e is ranked by P consecutive threads (P = 4 for
-    // E <= 128, else 2), each comparing logit e with a 1/P share of the logits
-    // (descending, equal logits by expert index); the P partial ranks are
-    // summed with shuffles.  Ranks below k are the chosen experts, in order.
+    // ---- routing inputs: logits (a NaN ranks as -infinity), Q8_0 of x
     const int E16 = (E + 15) & ~15;
-    const int P = (E16 <= FFN_THREADS / 4) ? 4 : 2;
-    // a NaN logit (non-finite data, or the router kernel's timeout report)
-    // ranks as -infinity, so the ranks below stay a permutation of [0, E)
-    for (int e = tid; e < E16; e += blockDim.x) {
-        float l = (e < E) ? __ldcg(p.logits + e) : -INFINITY;
-        if (e < E && !isfinite(l)) atomicOr(&flags_s, (int)STATUS_NONFINITE_LOGIT);
+    for (int e = tid; e < E16; e += FFN_THREADS) {
+        const float l = (e < E) ? __ldcg(p.logits + e) : -INFINITY;
+        if (e < E && !isfinite(l))
+            atomicOr(&flags_s,
+                     (int)((__float_as_uint(l) == TIMEOUT_NAN) ? STATUS_SPIN_TIMEOUT : STATUS_NONFINITE_LOGIT));
         logit_s[e] = (l != l) ? -INFINITY : l;
     }
-    for (int i = tid; i < H / 16; i += blockDim.x)
+    for (int i = tid; i < H / 16; i += FFN_THREADS)
         reinterpret_cast<int4*>(qa_s)[i] = __ldcg(reinterpret_cast<const int4*>(p.qa) + i);
-    for (int b = tid; b < nbH; b += blockDim.x) {
+    for (int b = tid; b < nbH; b += FFN_THREADS) {
         const uint32_t bits = __ldcg(p.da + b);
         if ((bits & 0x7fffu) == 0x7c00u) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
         da_s[b] = half_bits_to_float(bits);
     }
     __syncthreads();
+
+    // ---- top-k: expert e is ranked by P consecutive threads (P = 4 for
+    // E <= 128, else 2), each comparing logit e with a 1/P share of the logits
+    // (descending, equal logits by expert index); the partial ranks are summed
+    // with shuffles.  Ranks below k are the chosen experts, in order.  The
+    // keys are a total order, so the ranks are a permutation of [0, E).
+    const int P = (E16 <= FFN_THREADS / 4) ? 4 : 2;
     const int e_me = tid / P, part = tid % P;
     float my_l = 0.0f;
     int rank = 0;
@@ -357,20 +374,27 @@ __global__ void __maxnreg__(96) decode_ffn_kernel(DecodeParams p) {
     rank += __shfl_xor_sync(0xffffffffu, rank, 1);
     if (P == 4) rank += __shfl_xor_sync(0xffffffffu, rank, 2);
     const int my_rank = (e_me < E) ? rank : k;
-    if (part == 0 && my_rank < k) idx_s[my_rank] = e_me;
+    const bool chosen = part == 0 && my_rank < k;
+    if (chosen) idx_s[my_rank] = e_me;
     // slot of a chosen expert = number of chosen experts with a lower index
     // (slots are grouped by ascending expert, as in the grouped path)
-    const bool chosen = part == 0 && my_rank < k;
     const unsigned chosen_mask = __ballot_sync(0xffffffffu, chosen);
     if (lane == 0) warp_chosen[warp] = __popc(chosen_mask);
-    for (int b = tid; b < nbH; b += blockDim.x) {
+    // block sums of the activation codes (the -8 offset of the nibbles)
+    for (int b = tid; b < nbH; b += FFN_THREADS) {
         const int* qw = reinterpret_cast<const int*>(qa_s + b * QK);
         int s = 0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) s = __dp4a(qw[j], 0x01010101, s);
+        for (int q = 0; q < 8; ++q) s = __dp4a(qw[q], 0x01010101, s);
         qsum_s[b] = s;
     }
     __syncthreads();
+
+    // ---- routed copies (warp 0); slots and softmax terms
+    if (!is_shared && warp == 0) {
+        const size_t eo = (size_t)idx_s[j] * gu_stride;
+        issue_copies(p.w_gate + eo, p.w_up + eo, &maps.down, idx_s[j] * H + n0);
+    }
     if (chosen) {
         int before = __popc(chosen_mask & ((1u << lane) - 1u));
         for (int w2 = 0; w2 < warp; ++w2) before += warp_chosen[w2];
@@ -379,32 +403,20 @@ __global__ void __maxnreg__(96) decode_ffn_kernel(DecodeParams p) {
     }
     if (tid == 0) slot_s[k] = k;  // the shared expert's slot: P + t
     __syncthreads();
-
-    // ---- routed copies (warp 0), softmax weights (warp 1), inspection arrays (CTA 0)
-    if (warp == 0) {
-        // gate/up first: the grid barrier waits for the last CTA's gate/up
-        // data, while the down rows are needed only after it
-        if (item0 < n_items && !item0_shared) {
-            const size_t eo = (size_t)idx_s[item0 / nrb] * gu_stride;
-            issue_gateup(p.w_gate + eo, p.w_up + eo, item0 % nrb);
-        }
-        __syncwarp();
-        if (rows > 0 && lane < k)
-            bulk_g2s(dn_s + (size_t)lane * R * row_dn, p.w_down + (size_t)idx_s[lane] * dn_stride + (size_t)n0 * row_dn,
-                     (uint32_t)(rows * row_dn), &bar_dn);
-    } else if (warp == 1 && lane < k) {
+    if (warp == 1 && lane < k) {
         float z = 0.0f;
-        for (int j = 0; j < k; ++j) z += ex_s[j];
+        for (int i = 0; i < k; ++i) z += ex_s[i];
         w_s[lane] = __fdiv_rn(ex_s[lane], z);
     }
+    // inspection arrays of the workspace (the same as the grouped path's)
     if (blockIdx.x == 0) {
         if (part == 0 && e_me < E) p.cnt[e_me] = chosen ? 1 : 0;
-        if (tid == 0) p.cnt[E] = S;
-        for (int e = tid; e <= E + 1; e += blockDim.x) {
+        if (tid == 0) p.cnt[E] = p.S;
+        for (int e = tid; e <= E + 1; e += FFN_THREADS) {
             int o = 0;
             if (e <= E)
-                for (int j = 0; j < k; ++j) o += (idx_s[j] < e) ? 1 : 0;
-            p.off[e] = (e <= E) ? o : k + S;
+                for (int i = 0; i < k; ++i) o += (idx_s[i] < e) ? 1 : 0;
+            p.off[e] = (e <= E) ? o : k + p.S;
         }
     }
     __syncthreads();
@@ -415,120 +427,179 @@ __global__ void __maxnreg__(96) decode_ffn_kernel(DecodeParams p) {
         p.sorted[slot_s[tid]] = tid;
     }
 
-    // ---- gate/up + SwiGLU + requant, one item per pass.  Warp w computes the
-    // rows 4w..4w+3 of the 64 (0..31 gate, 32..63 up): chunk (w mod 8) / 2.
-    uint32_t gu_phase = 0;
-    for (int item = item0; item < n_items; item += gridDim.x) {
-        const int j = item / nrb, rb = item % nrb;
-        if (item != item0 && warp == 0) {
-            if (lane == 0) fence_proxy_async_smem();
-            __syncwarp();
-            const size_t eo = (j < k) ? (size_t)idx_s[j] * gu_stride : 0;
-            issue_gateup((j < k) ? p.w_gate + eo : p.sh_gate, (j < k) ? p.w_up + eo : p.sh_up, rb);
-        }
-        if (!mbar_wait_bounded(&bar_gu[(warp & 7) >> 1], gu_phase, MBAR_LIMIT)) timed_out = true;
+    // ---- gate/up: warp w computes rows 4w .. 4w + 3 of the 64 (0..31 gate,
+    // 32..63 up), from chunk (w mod 8) / 2; lanes split the blocks along H
+    {
+        if (!mbar_wait_bounded(&bar_gu[(warp & 7) >> 1], 0, MBAR_LIMIT)) timed_out = true;
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         const uint8_t* rows4 = gu_s + (size_t)(warp * 4) * row_gu;
 #pragma unroll 1
-        for (int b = lane; b < nbH; b += 32) block_rows<4>(rows4, row_gu, 4, b, qa_s, qsum_s[b], da_s[b], acc);
+        for (int b = lane; b < nbH; b += 32)
+            block_rows<4>(rows4 + (size_t)b * Q4_BYTES, row_gu, qa_s + b * QK, qsum_s[b], da_s[b], acc);
         const float s = butterfly<4, 32>(acc);
         if (bf_owner<4, 32>(lane)) {
             const int row64 = warp * 4 + bf_index<4, 32>(lane);
             (row64 < 32 ? gs : us)[row64 & 31] = s;
         }
-        __syncthreads();
-        if (warp == 0) {
-            const int slot = slot_s[j];
-            const float h = swiglu(gs[lane], us[lane]);
-            if (p.h_dbg) p.h_dbg[(size_t)slot * F + rb * GU_ROWS + lane] = h;
-            uint16_t db;
-            bool ov;
-            const int q = q8_0_lane(h, db, ov);
-            p.hq[(size_t)slot * F + rb * GU_ROWS + lane] = (int8_t)q;
+    }
+    __syncthreads();
+
+    // ---- SwiGLU + Q8_0 of this CTA's h block; into every CTA of the cluster
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    if (warp == 0) {
+        const int slot = slot_s[j];
+        const float h = swiglu(gs[lane], us[lane]);
+        if (p.h_dbg) p.h_dbg[(size_t)slot * F + hb * QK + lane] = h;
+        uint16_t db;
+        bool ov;
+        const int q = q8_0_lane(h, db, ov);
+        p.hq[(size_t)slot * F + hb * QK + lane] = (int8_t)q;
+        int qs = q;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+        const float dv = half_bits_to_float(db);
+        if (lane == 0) {
+            p.dh[(size_t)slot * nbF + hb] = db;
+            if (ov) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
+        }
+#pragma unroll
+        for (int peer = 0; peer < CL; ++peer) {
+            int8_t* dq = cluster.map_shared_rank(&hx_q[r][0], peer);
+            dq[lane] = (int8_t)q;
             if (lane == 0) {
-                p.dh[(size_t)slot * nbF + rb] = db;
-                if (ov) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
+                *cluster.map_shared_rank(&hx_d[r], peer) = dv;
+                *cluster.map_shared_rank(&hx_sum[r], peer) = qs;
             }
         }
-        gu_phase ^= 1u;
-        __syncthreads();
     }
+    cluster.sync();  // release/acquire: every CTA's h block is in every CTA
 
-    // ---- every CTA's requantised rows are written: grid barrier
-    __threadfence();
-    grid_barrier_bounded(p.status + 1, (uint32_t)p.barrier_target, p.status, STATUS_SPIN_TIMEOUT);
-
-    if (rows > 0) {
-        // requantised SwiGLU rows of all k+1 slots (L2: written by other SMs)
-        for (int i = tid; i < J * F / 16; i += blockDim.x)
-            reinterpret_cast<int4*>(hq_s)[i] = __ldcg(reinterpret_cast<const int4*>(p.hq) + i);
-        for (int i = tid; i < J * nbF; i += blockDim.x) dh_s[i] = half_bits_to_float(__ldcg(p.dh + i));
-        __syncthreads();
-        for (int i = tid; i < J * nbF; i += blockDim.x) {
-            const int* qw = reinterpret_cast<const int*>(hq_s + i * QK);
-            int s = 0;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) s = __dp4a(qw[q], 0x01010101, s);
-            hsum_s[i] = s;
+    // ---- down: o[n] = sum over the cluster's 8 blocks, n < Hs.  A task is 4
+    // rows; 8 lanes share a task, one block each, and add with a butterfly.
+    if (!mbar_wait_bounded(&bar_dn, 0, MBAR_LIMIT)) timed_out = true;
+    {
+        const int kb = lane & 7, grp = lane >> 3;
+        const size_t row_dn = (size_t)DN_KB * Q4_BYTES;
+        const int qsum = hx_sum[kb];
+        const float dv = hx_d[kb];
+        for (int t0 = 0; t0 < Hs; t0 += FFN_WARPS * 16) {
+            const int row0 = t0 + warp * 16 + grp * 4;
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            if (row0 < Hs)
+                block_rows<4>(dn_s + (size_t)row0 * row_dn + (size_t)kb * Q4_BYTES, row_dn, &hx_q[kb][0], qsum, dv,
+                              acc);
+            const float s = butterfly<4, 8>(acc);
+            if (bf_owner<4, 8>(kb) && row0 < Hs) o_s[row0 + bf_index<4, 8>(kb)] = s;
         }
-        __syncthreads();
-        if (!mbar_wait_bounded(&bar_dn, 0, MBAR_LIMIT)) timed_out = true;
-        if (nbF >= 32)
-            down_tasks<32>(dn_s, row_dn, R, rows, J, nbF, F, hq_s, dh_s, hsum_s, slot_s, o_s, warp, FFN_WARPS);
-        else if (nbF >= 16)
-            down_tasks<16>(dn_s, row_dn, R, rows, J, nbF, F, hq_s, dh_s, hsum_s, slot_s, o_s, warp, FFN_WARPS);
-        else
-            down_tasks<8>(dn_s, row_dn, R, rows, J, nbF, F, hq_s, dh_s, hsum_s, slot_s, o_s, warp, FFN_WARPS);
-        __syncthreads();
-        for (int r = tid; r < rows; r += blockDim.x) {
-            float acc = 0.0f;
-            for (int j = 0; j < k; ++j) acc = fmaf(w_s[j], o_s[j * R + r], acc);
-            if (S) acc += o_s[k * R + r];
-            p.y[n0 + r] = acc;
+    }
+    __syncthreads();
+    // ---- combine: y[n0 + n] += w_j * o[n] (weight 1 for the shared expert)
+    {
+        const float wj = is_shared ? 1.0f : w_s[j];
+        for (int t = tid; t < Hs / 4; t += FFN_THREADS) {
+            const float4 o = reinterpret_cast<const float4*>(o_s)[t];
+            red_add_v4(p.y + n0 + 4 * t, make_float4(wj * o.x, wj * o.y, wj * o.z, wj * o.w));
         }
     }
     if (timed_out) atomicOr(&flags_s, (int)STATUS_SPIN_TIMEOUT);
     __syncthreads();
     if (tid == 0 && flags_s) atomicOr(p.status, (uint32_t)flags_s);
+    if (p.kernel_ns && blockIdx.x == 0 && tid == 0) {
+        atomicAdd(p.kernel_ns, global_ns() - t_entry);
+        atomicAdd(p.kernel_ns + 1, 1ull);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// K3 (host entry only): y copied to page-locked host memory by the GPU, so the
+// call stays one programmatic-launch chain with no copy node in it.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) decode_copy_out_kernel(const float* __restrict__ y, float* __restrict__ y_host,
+                                                              int H) {
+    pdl_launch_dependents();
+    pdl_wait();  // the FFN kernel's partial sums are all in y
+    for (int i = threadIdx.x; i < H / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(y_host)[i] = __ldcg(reinterpret_cast<const float4*>(y) + i);
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-static int decode_rows_per_cta(int H, int G) { return (int)ceil_div(H, G); }
+namespace {
 
-static size_t router_smem(const LayerView& L) { return (size_t)L.H * 4; }
+PFN_cuTensorMapEncodeTiled_v12000 decode_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// `rows` rows of F/32 blocks at `base` as bytes, copied as boxes of 144 bytes
+// (8 blocks) x `box_rows` rows.
+cudaError_t encode_down(CUtensorMap* map, const uint8_t* base, uint64_t rows, int F, uint32_t box_rows) {
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = decode_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t row_bytes = (cuuint64_t)(F / QK) * Q4_BYTES;
+    const cuuint64_t dims[2] = {row_bytes, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)(DN_KB * Q4_BYTES), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+size_t router_smem(const LayerView& L) { return (size_t)L.H * 4; }
+
+}  // namespace
 
 bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev) {
     if (T != 1 || L.E > 256 || L.k > 16) return false;
-    const int G = dev.sm_count;
-    const int R = decode_rows_per_cta(L.H, G);
-    const DecodeSmem SL = decode_smem_layout(L.H, L.F, L.k + L.S, R);
+    const DecodeSmem SL = decode_smem_layout(L.H);
     // the FFN kernel must fit with room for the router kernel's CTA beside it
     return SL.total <= (size_t)std::min(dev.max_smem_optin - 4096, 200 * 1024) && router_smem(L) <= 96 * 1024;
 }
 
 cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Workspace& ws, float* h_dbg,
                           const DeviceInfo& dev, cudaEvent_t ev_start, cudaEvent_t ev_stop, bool force_timeout,
-                          bool clear_status, cudaStream_t s) {
+                          bool clear_status, unsigned long long* kernel_ns, float* y_host, cudaStream_t s) {
     DecodeParams p;
-    p.clear_status = clear_status ? 1 : 0;
     p.H = L.H; p.F = L.F; p.E = L.E; p.k = L.k; p.S = L.S;
-    p.nctas = dev.sm_count;
-    p.barrier_target = p.nctas + (force_timeout ? 1 : 0);
-    p.rows_per_cta = decode_rows_per_cta(L.H, p.nctas);
+    p.nF = L.F / (CL * QK);
+    p.clear_status = clear_status ? 1 : 0;
+    p.force_timeout = force_timeout ? 1 : 0;
     p.x = x; p.w_router = L.w_router; p.bias = L.router_bias;
-    p.w_gate = L.w_gate; p.w_up = L.w_up; p.w_down = L.w_down;
-    p.sh_gate = L.sh_gate; p.sh_up = L.sh_up; p.sh_down = L.sh_down;
+    p.w_gate = L.w_gate; p.w_up = L.w_up; p.sh_gate = L.sh_gate; p.sh_up = L.sh_up;
     p.logits = ws.logits; p.topk_idx = ws.topk_idx; p.topk_w = ws.topk_w; p.qa = ws.qa; p.da = ws.da;
     p.cnt = ws.cnt; p.off = ws.off; p.sorted = ws.sorted; p.pos = ws.pos; p.hq = ws.hq; p.dh = ws.dh;
-    p.h_dbg = h_dbg; p.y = y; p.status = ws.status;
+    p.h_dbg = h_dbg; p.y = y; p.status = ws.status; p.kernel_ns = kernel_ns;
+
+    // rows per tensor copy: a multiple of 32 that divides H/8 (a multiple of
+    // 32), so the copies tile the CTA's rows exactly
+    const int Hs = L.H / CL;
+    int box = DN_BOX_ROWS;
+    while (Hs % box) box -= 32;
+    const uint32_t box_rows = (uint32_t)box;
+    DecodeMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    p.box_rows = box;
+    cudaError_t e = encode_down(&maps.down, L.w_down, (uint64_t)L.E * L.H, L.F, box_rows);
+    if (e == cudaSuccess && L.S) e = encode_down(&maps.sh_down, L.sh_down, (uint64_t)L.H, L.F, box_rows);
+    if (e != cudaSuccess) return e;
 
     int per_sm = 0;
     const size_t smem1 = router_smem(L);
-    cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(decode_router_kernel), 128, smem1, &per_sm);
+    e = kernel_occupancy(reinterpret_cast<const void*>(decode_router_kernel), 128, smem1, &per_sm);
     if (e != cudaSuccess) return e;
-    const DecodeSmem SL = decode_smem_layout(L.H, L.F, L.k + L.S, p.rows_per_cta);
+    const DecodeSmem SL = decode_smem_layout(L.H);
     e = kernel_occupancy(reinterpret_cast<const void*>(decode_ffn_kernel), FFN_THREADS, SL.total, &per_sm);
     if (e != cudaSuccess) return e;
 
@@ -546,15 +617,25 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
     if (e != cudaSuccess) return e;
 
     if (ev_start && (e = record_event(ev_start, s)) != cudaSuccess) return e;
-    attrs[1].id = cudaLaunchAttributeCooperative;
-    attrs[1].val.cooperative = 1;
-    cfg.gridDim = dim3((unsigned)p.nctas);
+    attrs[1].id = cudaLaunchAttributeClusterDimension;
+    attrs[1].val.clusterDim.x = CL;
+    attrs[1].val.clusterDim.y = 1;
+    attrs[1].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)((L.k + L.S) * p.nF * CL));
     cfg.blockDim = dim3(FFN_THREADS);
     cfg.dynamicSmemBytes = SL.total;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, decode_ffn_kernel, p);
+    e = cudaLaunchKernelEx(&cfg, decode_ffn_kernel, p, maps);
     if (e != cudaSuccess) return e;
     if (ev_stop && (e = record_event(ev_stop, s)) != cudaSuccess) return e;
+    if (y_host) {
+        cfg.gridDim = dim3(1);
+        cfg.blockDim = dim3(256);
+        cfg.dynamicSmemBytes = 0;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, decode_copy_out_kernel, (const float*)y, y_host, L.H);
+        if (e != cudaSuccess) return e;
+    }
     return cudaSuccess;
 }
 

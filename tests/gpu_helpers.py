@@ -189,8 +189,14 @@ def free_running_report(lw, x_np, v, tokens):
                   oracle's logit gap at a changed position within twice the
                   largest logit difference);
       other       tokens whose top-k differs beyond a near-tie (must be 0);
+      requant     identical tokens whose requantised SwiGLU output (a code
+                  or a binary16 scale of h) differs from the oracle's: the
+                  binary32 h of the device and the binary64-then-binary32 h
+                  of the oracle straddle a rounding boundary;
       row_err     the largest norm-wise row error |y - y_ref| / |y_ref| over
-                  the identical tokens;
+                  the identical tokens without a requantisation difference;
+      requant_row_err  the same over the tokens with one;
+      within_1e3  the fraction of identical tokens with row error <= 1e-3;
       flips       Q8_0 codes of h that differ by one step (identical tokens),
       big_flips   codes that differ by more (must be 0), scale_diffs the
                   binary16 scales of h that differ."""
@@ -207,10 +213,16 @@ def free_running_report(lw, x_np, v, tokens):
     row_err = np.linalg.norm(y - r, axis=1) / np.maximum(np.linalg.norm(r, axis=1), 1e-30)
     hq_dev = pairs_from_slots(lw, T, v, v["hq"])[tokens]
     dh_dev = pairs_from_slots(lw, T, v, v["dh"].view(np.uint16))[tokens]
-    dq = np.abs(hq_dev[same].astype(np.int32) - dbg["hq"][same].astype(np.int32))
+    dq = np.abs(hq_dev.astype(np.int32) - dbg["hq"].astype(np.int32))
+    req = same & ((dq.reshape(len(tokens), -1).max(axis=1) > 0) |
+                  np.any((dh_dev != dbg["dh"]).reshape(len(tokens), -1), axis=1))
+    exact = same & ~req
+    dqs = dq[same]
     return dict(tokens=int(len(tokens)), identical=int(same.sum()), near_tie=int(near),
-                other=int(len(diff_toks) - near),
-                row_err=float(row_err[same].max()) if same.any() else 0.0,
-                row_err_median=float(np.median(row_err[same])) if same.any() else 0.0,
-                flips=int(np.count_nonzero(dq == 1)), big_flips=int(np.count_nonzero(dq > 1)),
+                other=int(len(diff_toks) - near), requant=int(req.sum()),
+                row_err=float(row_err[exact].max()) if exact.any() else 0.0,
+                row_err_median=float(np.median(row_err[exact])) if exact.any() else 0.0,
+                requant_row_err=float(row_err[req].max()) if req.any() else 0.0,
+                within_1e3=float(np.mean(row_err[same] <= 1e-3)) if same.any() else 1.0,
+                flips=int(np.count_nonzero(dqs == 1)), big_flips=int(np.count_nonzero(dqs > 1)),
                 scale_diffs=int(np.count_nonzero(dh_dev[same] != dbg["dh"][same])))

@@ -144,13 +144,14 @@ def test_other_entry_points_reject_bad_args(lib):
         _fields_ = [("h_out", ctypes.c_void_p), ("path", ctypes.c_int32), ("ev_start", ctypes.c_void_p),
                     ("ev_stop", ctypes.c_void_p), ("force_spin_timeout", ctypes.c_int32),
                     ("block_dots_out", ctypes.c_void_p), ("block_dots_down", ctypes.c_int32),
-                    ("block_dots_group", ctypes.c_int32), ("block_dots_rb", ctypes.c_int32)]
-    dbg = _D(None, 9, None, None, 0, None, 0, 0, 0)
+                    ("block_dots_group", ctypes.c_int32), ("block_dots_rb", ctypes.c_int32),
+                    ("decode_kernel_ns", ctypes.c_void_p)]
+    dbg = _D(None, 9, None, None, 0, None, 0, 0, 0, None)
     assert d(ctypes.byref(L), FAKE, 4, FAKE + 0x1000000, FAKE + 0x2000000, 1 << 40, ctypes.byref(dbg), None) == -1
     # block-dot capture of a group that does not exist (E = 128 routed + the shared group 128)
-    dbg = _D(None, 0, None, None, 0, FAKE + 0x4000000, 0, 129, 0)
+    dbg = _D(None, 0, None, None, 0, FAKE + 0x4000000, 0, 129, 0, None)
     assert d(ctypes.byref(L), FAKE, 4, FAKE + 0x1000000, FAKE + 0x2000000, 1 << 40, ctypes.byref(dbg), None) == -1
-    dbg = _D(None, 0, None, None, 0, FAKE + 0x4000002, 0, 3, 0)     # misaligned capture buffer
+    dbg = _D(None, 0, None, None, 0, FAKE + 0x4000002, 0, 3, 0, None)     # misaligned capture buffer
     assert d(ctypes.byref(L), FAKE, 4, FAKE + 0x1000000, FAKE + 0x2000000, 1 << 40, ctypes.byref(dbg), None) == -1
 
 

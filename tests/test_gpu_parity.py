@@ -103,15 +103,19 @@ def test_route_many_tokens_cluster_path(name, T):
 # --------------------------------------------------------------- whole layer
 
 def check_free_running(name, path, lw, x, v, tokens):
-    """The free-running report against the independent oracle: routing may
-    differ only at near-ties, the norm-wise row error of every token with
-    identical routing is within 1e-3, and a requantised SwiGLU code moves by
-    at most one step (printed with the counts)."""
+    """The free-running report against the independent oracle (printed):
+    routing may differ only at near-ties; a token with identical routing and
+    identical requantised SwiGLU output is within 1e-3 norm-wise (in practice
+    binary32 rounding); a requantised code moves by at most one step, which
+    moves its token by less than 1e-2 norm-wise; and at least 99% of the
+    tokens with identical routing are within 1e-3."""
     rep = free_running_report(lw, x, v, tokens)
     print(f"free-running {name} path {path}: {rep}")
     assert rep["other"] == 0, rep
     assert rep["row_err"] <= 1e-3, rep
     assert rep["big_flips"] == 0, rep
+    assert rep["requant_row_err"] <= 1e-2, rep
+    assert rep["within_1e3"] >= 0.99, rep
     return rep
 
 
@@ -308,6 +312,27 @@ def test_forward_host_matches_device():
     torch.cuda.synchronize()
     ok, worst = rule13(yh.numpy(), y_dev, 1e-5)
     assert ok, worst
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+def test_forward_host_single_token(pinned):
+    """One token through the host entry: with page-locked x and y the decode
+    kernels read x and write y over the bus (no copy node); with pageable
+    memory the entry falls back to stream copies.  Either way the result is
+    the device forward's, call after call."""
+    x, lw = workload("decode_t1", T=1000)
+    L = m.Layer.from_host(lw)
+    ws = m.alloc_workspace(m.moe_q4_ffn_host_workspace_bytes(L, 1))
+    for t in (0, 5, 999):
+        xt = torch.from_numpy(x[t:t + 1].copy())
+        y_dev = m.moe_q4_ffn_forward(L, xt.cuda()).cpu().numpy()
+        xh = xt.pin_memory() if pinned else xt
+        yh = torch.full_like(xh, float("nan"))
+        yh = yh.pin_memory() if pinned else yh
+        m.moe_q4_ffn_forward_host(L, xh, yh, ws)
+        torch.cuda.synchronize()
+        ok, worst = rule13(yh.numpy(), y_dev, 1e-6)
+        assert ok, worst
 
 
 def test_scale_overflow_reported_in_status():

@@ -1,8 +1,8 @@
 """Host-streamed experts: the expert matrices in page-locked host memory,
 the routing-selected experts copied to the device per call.  Results equal
-the resident layer's (bit for bit on the deterministic T = 1 path; within
-the fp32 atomic-combine order elsewhere), exactly the selected experts are
-staged, and pageable host memory is refused before anything runs."""
+the resident layer's (within the order of the binary32 partial sums added
+into y), exactly the selected experts are staged, and pageable host memory
+is refused before anything runs."""
 import numpy as np
 import pytest
 import torch
@@ -22,14 +22,15 @@ def _both(name, T=None):
     return x, lw, m.Layer.from_host(lw), m.Layer.from_host_pinned(lw)
 
 
-def test_streamed_decode_tokens_bit_identical():
+def test_streamed_decode_tokens_match_resident():
     x, lw, Ld, Lh = _both("decode_t1", T=1000)
     for t in (0, 1, 2, 999):
         xt = torch.from_numpy(x[t:t + 1].copy()).cuda()
         y_res = m.moe_q4_ffn_forward(Ld, xt)
         y_str = m.moe_q4_ffn_forward_streamed(Lh, xt)
         torch.cuda.synchronize()
-        assert torch.equal(y_res, y_str)
+        ok, worst = rule13(y_str.cpu().numpy(), y_res.cpu().numpy(), 1e-6)
+        assert ok, worst
 
 
 @pytest.mark.parametrize("name,T", [("prefill_t947", 16), ("prefill_t947", None), ("tiny_t16", None)])

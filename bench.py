@@ -280,6 +280,7 @@ def prefill_lines(m, torch, stream):
     out = {}
     peak, peak_src = int8_peak_tops()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    variants = (("auto", m.PATH_AUTO), ("tc_n32", m.PATH_TENSOR_CORE_N32), ("tc_n128", m.PATH_TENSOR_CORE_N128))
     for name in ("prefill_t947", "zipf_t16384"):
         x_np, lw = synth.workload_inputs(name, seed=0)
         L = m.Layer.from_host(lw)
@@ -287,26 +288,34 @@ def prefill_lines(m, torch, stream):
         T = x.shape[0]
         y = torch.empty_like(x)
         ws = m.alloc_workspace(m.moe_q4_ffn_workspace_bytes(L, T))
-        tot, gu = [], []
-        for rep in range(8):
-            flush.zero_()
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-            for e in evs[2:]:
-                e.record(stream)  # torch creates the CUDA event on first record
-            evs[0].record(stream)
-            m.moe_q4_ffn_forward_debug(L, x, y, ws, ev_start=evs[2], ev_stop=evs[3], stream=stream)
-            evs[1].record(stream)
-            torch.cuda.synchronize()
-            if rep >= 3:
-                tot.append(evs[0].elapsed_time(evs[1]))
-                gu.append(evs[2].elapsed_time(evs[3]))
-        ms, gu_ms = float(np.median(tot)), float(np.median(gu))
         pairs = T * (lw.top_k + 1)
         gu_ops = 2.0 * pairs * 2 * lw.ffn * lw.hidden
-        out[name] = {"tokens_per_s": T / (ms * 1e-3), "ms": ms, "gateup_ms": gu_ms,
-                     "gateup_int8_tops": gu_ops / (gu_ms * 1e-3) / 1e12, "int8_peak_tops": peak,
-                     "gateup_frac_of_int8_peak": gu_ops / (gu_ms * 1e-3) / 1e12 / peak, "peak_source": peak_src,
-                     "l2": "256 MB flush before each rep"}
+        all_ops = 2.0 * pairs * 3 * lw.ffn * lw.hidden
+        for vname, path in variants:
+            tot, gu = [], []
+            for rep in range(8):
+                flush.zero_()
+                evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                for e in evs[2:]:
+                    e.record(stream)  # torch creates the CUDA event on first record
+                evs[0].record(stream)
+                m.moe_q4_ffn_forward_debug(L, x, y, ws, path=path, ev_start=evs[2], ev_stop=evs[3], stream=stream)
+                evs[1].record(stream)
+                torch.cuda.synchronize()
+                if rep >= 3:
+                    tot.append(evs[0].elapsed_time(evs[1]))
+                    gu.append(evs[2].elapsed_time(evs[3]))
+            ms, gu_ms = float(np.median(tot)), float(np.median(gu))
+            rec = {"tokens_per_s": T / (ms * 1e-3), "ms": ms, "gateup_ms": gu_ms,
+                   "gateup_int8_tops": gu_ops / (gu_ms * 1e-3) / 1e12,
+                   "gateup_frac_of_int8_peak": gu_ops / (gu_ms * 1e-3) / 1e12 / peak,
+                   "layer_int8_tops": all_ops / (ms * 1e-3) / 1e12,
+                   "layer_frac_of_int8_peak": all_ops / (ms * 1e-3) / 1e12 / peak}
+            if vname == "auto":
+                rec.update({"int8_peak_tops": peak, "peak_source": peak_src, "l2": "256 MB flush before each rep"})
+                out[name] = rec
+            else:
+                out[name][vname] = rec
         del L, x, y, ws
     del flush
     return out
@@ -351,35 +360,43 @@ def chunked_lines(m, torch, stream):
 
 
 def batch64_lines(m, torch, stream):
-    """One layer on a decode batch of 64 tokens (the streaming dp4a path):
-    tokens/s, and HBM GB/s over the experts the batch activates + Wr + x/y;
-    the layer rotates over 4 device copies (912 MB) so every rep is L2-cold."""
+    """One layer on decode batches of 8 to 128 tokens, on the automatic path,
+    the streaming dp4a kernels and the 32-slot tensor-core kernels: tokens/s,
+    and HBM GB/s over the experts the batch activates + Wr + x/y; the layer
+    rotates over 4 device copies (912 MB) so every rep is L2-cold."""
     import synth
     hbm, src = measured_peaks()
     x_np, lw = synth.workload_inputs("prefill_t947", seed=0)
     base = m.Layer.from_host(lw)
     layers = [base] + [base.replica() for _ in range(3)]
-    T = 64
-    x = torch.from_numpy(x_np[:T].copy()).cuda()
-    y = torch.empty_like(x)
-    ws = m.alloc_workspace(m.moe_q4_ffn_workspace_bytes(base, T))
-    times = []
-    for rep in range(12):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        m.moe_q4_ffn_forward(layers[rep % 4], x, y, ws, stream=stream)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        if rep >= 4:
-            times.append(e0.elapsed_time(e1))
-    us = float(np.median(times)) * 1000.0
-    cnt = m.workspace_views(base, T, ws)["cnt"][:lw.n_experts].cpu().numpy()
-    active = int(np.count_nonzero(cnt)) + 1
-    nbytes = active * 3 * lw.ffn * (lw.hidden // 32) * 18 + lw.n_experts * lw.hidden * 4 + 2 * T * lw.hidden * 4
+    out = {"peak_source": src}
+    for T in (8, 16, 32, 64, 96, 128):
+        x = torch.from_numpy(x_np[:T].copy()).cuda()
+        y = torch.empty_like(x)
+        ws = m.alloc_workspace(m.moe_q4_ffn_workspace_bytes(base, T))
+        rec = {}
+        for vname, path in (("auto", m.PATH_AUTO), ("dp4a", m.PATH_GROUPED_DP4A), ("tc_n32", m.PATH_TENSOR_CORE_N32)):
+            times = []
+            for rep in range(12):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                m.moe_q4_ffn_forward_debug(layers[rep % 4], x, y, ws, path=path, stream=stream)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if rep >= 4:
+                    times.append(e0.elapsed_time(e1))
+            us = float(np.median(times)) * 1000.0
+            cnt = m.workspace_views(base, T, ws)["cnt"][:lw.n_experts].cpu().numpy()
+            active = int(np.count_nonzero(cnt)) + 1
+            nbytes = (active * 3 * lw.ffn * (lw.hidden // 32) * 18 + lw.n_experts * lw.hidden * 4 +
+                      2 * T * lw.hidden * 4)
+            rec[vname] = {"us": us, "tokens_per_s": T / (us * 1e-6), "active_experts": active,
+                          "algorithmic_bytes": nbytes, "hbm_gbs": nbytes / (us * 1e-6) / 1e9,
+                          "hbm_frac": nbytes / (us * 1e-6) / 1e9 / hbm}
+        out[f"T{T}"] = rec
+        del ws
     del layers
-    return {"T": T, "us": us, "tokens_per_s": T / (us * 1e-6), "active_experts": active,
-            "algorithmic_bytes": nbytes, "hbm_gbs": nbytes / (us * 1e-6) / 1e9,
-            "hbm_frac": nbytes / (us * 1e-6) / 1e9 / hbm, "peak_source": src}
+    return out
 
 
 def gemv_lines(m, torch, stream):
@@ -696,7 +713,7 @@ def run_ours(args):
         "stack": stack,
         "chunked_prefill": chunked,
         "lm_head_gemv": gemv,
-        "decode_batch64": batch64,
+        "decode_batches": batch64,
         "host_streamed_experts": streamed,
     }
     if rank == 0:

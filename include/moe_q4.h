@@ -264,7 +264,7 @@ const char* moe_q4_last_cuda_error(void);
  *   | qa i8[T][H] | da u16[T][H/32] | cnt i32[E+1] | off i32[E+2]
  *   | tile_off i32[E+2] | chunk_cnt i32[C][E] | chunk_base i32[C][E]
  *   | sorted i32[P] | pos i32[P] | hq i8[P+S*T][F] | dh u16[P+S*T][F/32]
- *   | total
+ *   | sync u32[(k+S)*F/256] | total
  * with P = T*k routed pairs and S = has_shared.  Slots (rows of hq/dh) are
  * grouped by expert: routed expert e owns slots off[e]..off[e+1]-1 holding
  * pairs sorted[...] = t*k+j in increasing (t, j) order; the shared expert
@@ -274,7 +274,7 @@ const char* moe_q4_last_cuda_error(void);
 enum {
     MOE_Q4_WS_STATUS = 0, MOE_Q4_WS_LOGITS, MOE_Q4_WS_TOPK_IDX, MOE_Q4_WS_TOPK_W, MOE_Q4_WS_QA,
     MOE_Q4_WS_DA, MOE_Q4_WS_CNT, MOE_Q4_WS_OFF, MOE_Q4_WS_TILE_OFF, MOE_Q4_WS_CHUNK_CNT,
-    MOE_Q4_WS_CHUNK_BASE, MOE_Q4_WS_SORTED, MOE_Q4_WS_POS, MOE_Q4_WS_HQ, MOE_Q4_WS_DH,
+    MOE_Q4_WS_CHUNK_BASE, MOE_Q4_WS_SORTED, MOE_Q4_WS_POS, MOE_Q4_WS_HQ, MOE_Q4_WS_DH, MOE_Q4_WS_SYNC,
     MOE_Q4_WS_TOTAL, MOE_Q4_WS_COUNT
 };
 int moe_q4_workspace_layout(const moe_q4_layer* L, int64_t T, size_t* offsets, int n);
@@ -284,7 +284,9 @@ enum {
     MOE_Q4_PATH_AUTO = 0,     /* what moe_q4_ffn_forward does */
     MOE_Q4_PATH_GROUPED_DP4A = 1,
     MOE_Q4_PATH_DECODE = 2,
-    MOE_Q4_PATH_TENSOR_CORE = 3
+    MOE_Q4_PATH_TENSOR_CORE = 3,     /* tensor cores, tile width chosen by T */
+    MOE_Q4_PATH_TENSOR_CORE_N32 = 4, /* tensor cores, tiles of 32 slots */
+    MOE_Q4_PATH_TENSOR_CORE_N128 = 5 /* tensor cores, tiles of 128 slots */
 };
 
 typedef struct {
@@ -303,7 +305,7 @@ typedef struct {
      * the rescale), for one row block of one expert group:
      *   block_dots_out[s][r][b], s = slot - off[g] over the group's slots in
      *   slot order, r < R rows of the row block, b < K/32 blocks along K.
-     * Tensor-core path: R = 128; gate/up rows r < 64 are gate rows 64 rb + r,
+     * Tensor-core paths: R = 128; gate/up rows r < 64 are gate rows 64 rb + r,
      * r >= 64 the up rows 64 rb + r - 64; down rows are 128 rb + r.
      * Streaming path: R = 64; gate/up rows r < 32 are gate rows 32 rb + r,
      * r >= 32 the up rows 32 rb + r - 32; down rows are 64 rb + r.

@@ -165,6 +165,7 @@ static void layout(const LayerView& L, int64_t T, size_t off[WS_COUNT]) {
         sizeof(int32_t) * (size_t)P,                   // pos
         (size_t)(slots * L.F),                         // hq
         sizeof(uint16_t) * (size_t)(slots * (L.F / QK)),  // dh
+        sizeof(uint32_t) * (size_t)((L.k + L.S) * ((L.F + 255) / 256)),  // sync
     };
     size_t o = 0;
     for (int i = 0; i < WS_COUNT - 1; ++i) {
@@ -192,6 +193,7 @@ static Workspace carve(void* base, const size_t off[WS_COUNT]) {
     w.pos = reinterpret_cast<int32_t*>(b + off[WS_POS]);
     w.hq = reinterpret_cast<int8_t*>(b + off[WS_HQ]);
     w.dh = reinterpret_cast<uint16_t*>(b + off[WS_DH]);
+    w.sync = reinterpret_cast<uint32_t*>(b + off[WS_SYNC]);
     return w;
 }
 
@@ -263,11 +265,16 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
                                      dbg ? dbg->decode_kernel_ns : nullptr, nullptr, s));
 
     // grouped paths: tensor cores once experts see tens of tokens, else dp4a
-    const bool tc = (path == MOE_Q4_PATH_TENSOR_CORE) || (path == MOE_Q4_PATH_AUTO && T >= TC_MIN_TOKENS);
+    const bool tc = (path == MOE_Q4_PATH_TENSOR_CORE) || (path == MOE_Q4_PATH_TENSOR_CORE_N32) ||
+                    (path == MOE_Q4_PATH_TENSOR_CORE_N128) || (path == MOE_Q4_PATH_AUTO && T >= TC_MIN_TOKENS);
+    const int tile = tc ? tc_tile_tokens(L, T, path == MOE_Q4_PATH_TENSOR_CORE_N32    ? 32
+                                               : path == MOE_Q4_PATH_TENSOR_CORE_N128 ? 128
+                                                                                      : 0)
+                        : DP4A_TT;
     MOE_TRY(launch_router_logits(L, x, T, w.logits, clear_status ? w.status : nullptr, s));
     MOE_TRY(launch_topk(w.logits, T, L.E, L.k, w.topk_idx, w.topk_w, w.status, s));
     MOE_TRY(launch_quantize(x, T, L.H, w.qa, w.da, w.status, y, s));
-    MOE_TRY(launch_permute(w.topk_idx, T, L.k, L.E, L.S, tc ? TC_TILE_TOKENS : DP4A_TT, w, s));
+    MOE_TRY(launch_permute(w.topk_idx, T, L.k, L.E, L.S, tile, w, s));
     BlockDotCapture cap_store;
     const BlockDotCapture* cap = nullptr;
     if (dbg && dbg->block_dots_out) {
@@ -277,12 +284,12 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
     }
     if (ev0) MOE_TRY(record_event(ev0, s));
     if (tc)
-        MOE_TRY(launch_gateup_tc(L, T, w, dbg ? dbg->h_out : nullptr, dev, cap, s));
+        MOE_TRY(launch_gateup_tc(L, T, w, dbg ? dbg->h_out : nullptr, dev, tile, cap, s));
     else
         MOE_TRY(launch_gateup_dp4a(L, T, w, dbg ? dbg->h_out : nullptr, dev, cap, s));
     if (ev1) MOE_TRY(record_event(ev1, s));
     if (tc)
-        MOE_TRY(launch_down_tc(L, T, w, y, dev, cap, s));
+        MOE_TRY(launch_down_tc(L, T, w, y, dev, tile, cap, s));
     else
         MOE_TRY(launch_down_dp4a(L, T, w, y, dev, cap, s));
     return MOE_Q4_OK;
@@ -373,7 +380,7 @@ int moe_q4_ffn_forward(const moe_q4_layer* L, const float* x, int64_t T, float* 
 
 int moe_q4_ffn_forward_debug(const moe_q4_layer* L, const float* x, int64_t T, float* y, void* workspace,
                              size_t ws_bytes, const moe_q4_debug* dbg, moe_q4_stream_t stream) {
-    if (dbg && (dbg->path < MOE_Q4_PATH_AUTO || dbg->path > MOE_Q4_PATH_TENSOR_CORE)) return MOE_Q4_ERR_INVALID_ARG;
+    if (dbg && (dbg->path < MOE_Q4_PATH_AUTO || dbg->path > MOE_Q4_PATH_TENSOR_CORE_N128)) return MOE_Q4_ERR_INVALID_ARG;
     return forward_impl(L, x, T, y, workspace, ws_bytes, dbg, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -12,33 +12,36 @@
 //     kernel it bulk-copies its router row into shared memory; then the logit
 //     (four independent FMA chains); the first H/32 CTAs quantise one Q8_0
 //     block of x each; y is zeroed (the FFN kernel accumulates into it).
-//   decode_ffn_kernel: clusters of 8 CTAs, one cluster per (expert of the
-//     token, 256-wide part of F).  CTA r of a cluster owns one 32-row block
-//     of h (32 gate rows and the same 32 up rows) and, for the down
-//     projection, H/8 rows restricted to the cluster's 8 blocks of F.  The
-//     shared expert's weights are copied before the wait on the router (they
-//     do not depend on the routing); routed CTAs rank the logits (every CTA
-//     the same way), then copy their gate/up rows (bulk copies) and their
-//     down slice (a 2D tensor copy: 144 bytes of each of H/8 rows) at once.
-//     Gate/up dot products, SwiGLU and the Q8_0 requantisation give the
-//     CTA's h block, which it writes into the shared memory of all 8 CTAs of
-//     its cluster (distributed shared memory); one cluster barrier, then the
-//     down partial sums over the cluster's 8 h blocks, and the router-weighted
-//     partial rows are added into y with vector reductions (red.v4.f32).
+//   decode_ffn_kernel: a cooperative grid of (k+S) x F/256 groups of 8 CTAs,
+//     one group per (expert of the token, 256-wide part of F).  CTA r of a
+//     group owns one 32-row block of h (32 gate rows and the same 32 up
+//     rows) and, for the down projection, H/8 rows restricted to the group's
+//     8 blocks of F.  The shared expert's weights are copied before the wait
+//     on the router (they do not depend on the routing); routed CTAs rank the
+//     logits (every CTA the same way), then copy their gate/up rows (bulk
+//     copies) and their down slice (a 2D tensor copy: 144 bytes of each of
+//     H/8 rows) at once.  Gate/up dot products, SwiGLU and the Q8_0
+//     requantisation give the CTA's h block, which it writes to the
+//     workspace and announces on its group's counter; once the group's 8
+//     blocks are in (a bounded wait on that counter only), the down partial
+//     sums over the group's 8 h blocks, and the router-weighted partial rows
+//     are added into y with vector reductions (red.v4.f32).
 //
-// No grid-wide barrier: the only exchange between CTAs is inside a cluster,
-// and the clusters are independent of one another (y collects their partial
-// sums), so the grid needs no co-residency.  The order of the (k+S) x F/256
-// partial sums added into an element of y is not fixed: results agree across
-// runs to binary32 rounding, not bit for bit.
+// No grid-wide barrier: a CTA waits only for the 7 others of its group (the
+// cooperative launch makes every CTA resident, so such a wait always ends),
+// and the groups are independent of one another (y collects their partial
+// sums).  Groups of 8 as thread-block clusters would exchange through
+// distributed shared memory instead, but with one such CTA per SM only 15
+// clusters of 8 fit on a B200 at once (GPC granularity; measured with
+// cudaOccupancyMaxActiveClusters) against the 18 a token needs.  The order of
+// the (k+S) x F/256 partial sums added into an element of y is not fixed:
+// results agree across runs to binary32 rounding, not bit for bit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <cstring>
 #include <mutex>
-
-#include <cooperative_groups.h>
 
 #include "common.cuh"
 #include "launch.h"
@@ -49,7 +52,7 @@ namespace moeq4 {
 namespace {
 
 constexpr uint32_t MBAR_LIMIT = 1u << 20;   // bounded waits: about 0.5 s
-constexpr int CL = 8;                       // CTAs per cluster = h blocks per F part
+constexpr int CL = 8;                       // CTAs per group = h blocks per F part
 constexpr int FFN_THREADS = 512;            // 16 warps
 constexpr int FFN_WARPS = FFN_THREADS / 32;
 constexpr int DN_KB = 8;                    // down blocks per F part (144 bytes of a row)
@@ -60,7 +63,7 @@ constexpr uint32_t TIMEOUT_NAN = 0x7fc0deadu;
 
 struct DecodeParams {
     int H, F, E, k, S;
-    int nF;              // F parts of 256 per expert (clusters per expert)
+    int nF;              // F parts of 256 per expert (groups per expert)
     int box_rows;        // rows per tensor copy of the down slice (divides H/8)
     int clear_status;    // the router kernel zeroes the status word (else it accumulates)
     int force_timeout;   // CTA 0's first gate/up barrier expects 16 bytes that never come
@@ -85,6 +88,7 @@ struct DecodeParams {
     float* h_dbg;
     float* y;
     uint32_t* status;
+    uint32_t* group_cnt;  // [(k+S) x nF] h blocks written per group (zeroed by the router kernel)
     unsigned long long* kernel_ns;  // optional: [0] += CTA 0's span of the FFN kernel, [1] += 1
 };
 
@@ -190,6 +194,7 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
     pdl_wait();  // x and the workspace are now the previous kernels' results
     if (e == 0 && tid == 0 && p.clear_status) p.status[0] = 0u;
     for (int i = e * 128 + tid; i < H; i += (int)gridDim.x * 128) p.y[i] = 0.0f;
+    for (int i = e * 128 + tid; i < (p.k + p.S) * p.nF; i += (int)gridDim.x * 128) p.group_cnt[i] = 0u;
     const bool ok = mbar_wait_bounded(&bar, 0, MBAR_LIMIT);
     const float4* x4 = reinterpret_cast<const float4*>(p.x);
     const float4* w4 = reinterpret_cast<const float4*>(wr_s);
@@ -224,7 +229,7 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// K2: gate/up + SwiGLU + requant, cluster exchange, down + combine.
+// K2: gate/up + SwiGLU + requant, exchange within a group, down + combine.
 // ---------------------------------------------------------------------------
 struct DecodeSmem {
     size_t gu, dn, qa, da, qsum, o, total;  // byte offsets
@@ -248,8 +253,6 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int H) {
 
 __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams p,
                                                                     const __grid_constant__ DecodeMaps maps) {
-    namespace cg = cooperative_groups;
-    cg::cluster_group cluster = cg::this_cluster();
     extern __shared__ __align__(16) unsigned char dsm_raw[];
     // tensor-copy destinations 128-byte aligned (the allocation has 128 bytes of slack)
     unsigned char* dsm = dsm_raw + ((128u - (smem_u32(dsm_raw) & 127u)) & 127u);
@@ -262,7 +265,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     __shared__ int slot_s[17];
     __shared__ int warp_chosen[FFN_WARPS];
     __shared__ float gs[32], us[32];
-    __shared__ __align__(16) int8_t hx_q[CL][QK];   // the cluster's 8 requantised h blocks
+    __shared__ __align__(16) int8_t hx_q[CL][QK];   // the group's 8 requantised h blocks
     __shared__ float hx_d[CL];
     __shared__ int hx_sum[CL];
     __shared__ int flags_s;
@@ -273,8 +276,8 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = p.H, F = p.F, E = p.E, k = p.k;
     const int nbH = H / QK, nbF = F / QK;
-    const int c = blockIdx.x / CL;                  // cluster
-    const int r = (int)cluster.block_rank();        // CTA within the cluster
+    const int c = blockIdx.x / CL;                  // group
+    const int r = blockIdx.x % CL;                  // CTA within the group
     const int j = c / p.nF;                         // expert of the token: rank j < k, or k = shared
     const int fp = c % p.nF;                        // F part: h blocks 8 fp .. 8 fp + 7
     const int hb = fp * CL + r;                     // this CTA's h block
@@ -298,9 +301,6 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
         mbar_fence_init();
         flags_s = 0;
     }
-    // first phase of the cluster barrier: its wait (before the first write into
-    // another CTA's shared memory) guarantees every CTA of the cluster runs
-    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     __syncthreads();
 
     // copies of this CTA's weights, issued by warp 0: gate/up chunk i = 8 gate
@@ -444,37 +444,55 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     }
     __syncthreads();
 
-    // ---- SwiGLU + Q8_0 of this CTA's h block; into every CTA of the cluster
-    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    // ---- SwiGLU + Q8_0 of this CTA's h block into the workspace (hq, dh),
+    // announced on the group's counter
+    const int slot = slot_s[j];
     if (warp == 0) {
-        const int slot = slot_s[j];
         const float h = swiglu(gs[lane], us[lane]);
         if (p.h_dbg) p.h_dbg[(size_t)slot * F + hb * QK + lane] = h;
         uint16_t db;
         bool ov;
         const int q = q8_0_lane(h, db, ov);
         p.hq[(size_t)slot * F + hb * QK + lane] = (int8_t)q;
-        int qs = q;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
-        const float dv = half_bits_to_float(db);
         if (lane == 0) {
             p.dh[(size_t)slot * nbF + hb] = db;
             if (ov) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
         }
-#pragma unroll
-        for (int peer = 0; peer < CL; ++peer) {
-            int8_t* dq = cluster.map_shared_rank(&hx_q[r][0], peer);
-            dq[lane] = (int8_t)q;
-            if (lane == 0) {
-                *cluster.map_shared_rank(&hx_d[r], peer) = dv;
-                *cluster.map_shared_rank(&hx_sum[r], peer) = qs;
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) red_release_add_gpu(p.group_cnt + c, 1u);
+    }
+    // ---- the group's 8 blocks: a bounded wait on its counter (every CTA of
+    // the cooperative grid is resident, so the 7 others get there)
+    if (tid == 0) {
+        const uint64_t t0 = global_ns();
+        while (ld_acquire_gpu(p.group_cnt + c) < (uint32_t)CL) {
+            if (global_ns() - t0 > 1000000000ull) {   // 1 s
+                timed_out = true;
+                break;
             }
+            __nanosleep(32);
         }
     }
-    cluster.sync();  // release/acquire: every CTA's h block is in every CTA
+    __syncthreads();
+    if (tid < CL * QK / 16) {
+        const int b = tid >> 1;
+        reinterpret_cast<int4*>(&hx_q[b][0])[tid & 1] =
+            __ldcg(reinterpret_cast<const int4*>(p.hq + (size_t)slot * F + (fp * CL + b) * QK) + (tid & 1));
+    } else if (tid >= 32 && tid < 32 + CL) {
+        hx_d[tid - 32] = half_bits_to_float(__ldcg(p.dh + (size_t)slot * nbF + fp * CL + (tid - 32)));
+    }
+    __syncthreads();
+    if (tid < CL) {
+        const int* qw = reinterpret_cast<const int*>(&hx_q[tid][0]);
+        int sq = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sq = __dp4a(qw[i], 0x01010101, sq);
+        hx_sum[tid] = sq;
+    }
+    __syncthreads();
 
-    // ---- down: o[n] = sum over the cluster's 8 blocks, n < Hs.  A task is 4
+    // ---- down: o[n] = sum over the group's 8 blocks, n < Hs.  A task is 4
     // rows; 8 lanes share a task, one block each, and add with a butterfly.
     if (!mbar_wait_bounded(&bar_dn, 0, MBAR_LIMIT)) timed_out = true;
     {
@@ -563,6 +581,8 @@ size_t router_smem(const LayerView& L) { return (size_t)L.H * 4; }
 
 bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev) {
     if (T != 1 || L.E > 256 || L.k > 16) return false;
+    // one CTA per SM, all resident (the cooperative launch)
+    if ((int64_t)(L.k + L.S) * (L.F / (CL * QK)) * CL > dev.sm_count) return false;
     const DecodeSmem SL = decode_smem_layout(L.H);
     // the FFN kernel must fit with room for the router kernel's CTA beside it
     return SL.total <= (size_t)std::min(dev.max_smem_optin - 4096, 200 * 1024) && router_smem(L) <= 96 * 1024;
@@ -580,7 +600,7 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
     p.w_gate = L.w_gate; p.w_up = L.w_up; p.sh_gate = L.sh_gate; p.sh_up = L.sh_up;
     p.logits = ws.logits; p.topk_idx = ws.topk_idx; p.topk_w = ws.topk_w; p.qa = ws.qa; p.da = ws.da;
     p.cnt = ws.cnt; p.off = ws.off; p.sorted = ws.sorted; p.pos = ws.pos; p.hq = ws.hq; p.dh = ws.dh;
-    p.h_dbg = h_dbg; p.y = y; p.status = ws.status; p.kernel_ns = kernel_ns;
+    p.h_dbg = h_dbg; p.y = y; p.status = ws.status; p.group_cnt = ws.sync; p.kernel_ns = kernel_ns;
 
     // rows per tensor copy: a multiple of 32 that divides H/8 (a multiple of
     // 32), so the copies tile the CTA's rows exactly
@@ -617,10 +637,8 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
     if (e != cudaSuccess) return e;
 
     if (ev_start && (e = record_event(ev_start, s)) != cudaSuccess) return e;
-    attrs[1].id = cudaLaunchAttributeClusterDimension;
-    attrs[1].val.clusterDim.x = CL;
-    attrs[1].val.clusterDim.y = 1;
-    attrs[1].val.clusterDim.z = 1;
+    attrs[1].id = cudaLaunchAttributeCooperative;
+    attrs[1].val.cooperative = 1;
     cfg.gridDim = dim3((unsigned)((L.k + L.S) * p.nF * CL));
     cfg.blockDim = dim3(FFN_THREADS);
     cfg.dynamicSmemBytes = SL.total;

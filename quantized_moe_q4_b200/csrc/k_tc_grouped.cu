@@ -20,38 +20,32 @@
 // bound the kernel.
 //
 // Tile: 128 weight rows (gate/up: 64 gate rows + the same 64 up rows; down:
-// 128 rows of H) x 64 slots of one expert (MMA M = 128, N = 64).
+// 128 rows of H) x 128 slots of one expert (MMA M = 128, N = 128), so one MMA
+// pair covers 128 x 128 x 32 and a weight block converted once serves 128
+// slots.
 //
-// Warp roles (14 warps):
+// Warp roles (22 warps):
 //   0      producer: 2D tensor copies (TMA) of the packed weight rows (a box
-//          of 64 or 128 rows x 144 B = 8 blocks) and 16-byte cp.async gathers
-//          of the slots' int8 activations and their scales, two input stages
-//          of 8 blocks in flight;
-//   1..4   converters: nibbles -> binary16 (nib - 8) for the A operand and
-//          int8 -> binary16 activations for the B operand, both written into
-//          the K-major shared-memory layout (8-row x 16-byte core matrices);
-//          two operand stages of 4 blocks; block scales into a ring shared
-//          with the epilogue;
+//          of 64 or 128 rows x 144 B = 8 blocks), two input stages in flight;
+//   1..4   converters: nibbles -> binary16 (nib - 8) for the A operand, and
+//          the slots' int8 activations, read from L2 with 16-byte loads
+//          issued before the wait for a free operand stage, -> binary16 for
+//          the B operand; both into the K-major shared-memory layout (8-row x
+//          16-byte core matrices); two operand stages of 2 blocks; block
+//          scales into a ring read by the epilogue;
 //   5      MMA issuer (one thread): two MMAs per block (A and B from shared
-//          memory), descriptors precomputed; one wait and one commit per
-//          operand stage for its quad of accumulators;
-//   6..13  epilogue: 4 TMEM lane quarters x 2 column halves; per quad of
-//          blocks one wait, then two passes of two TMEM loads of 32 columns
-//          and the rescale-accumulate; after the last block of a tile gate/up
-//          -> SwiGLU + Q8_0 requantisation, down -> y += w_slot * o (fp32
-//          atomics).
-// TMEM: eight accumulators of 64 columns (all 512 columns), handed between the
-// MMA issuer and the epilogue a quad (one operand stage) at a time; a 16-entry
-// scale ring (so the converters run up to four operand stages ahead of the
-// epilogue); full/empty mbarriers between every pair of roles; every wait
-// bounded, and one that runs out makes every role leave its loop and records
+//          memory); one wait and one commit per operand stage, for its pair
+//          of accumulators;
+//   6..21  epilogue: 4 TMEM lane quarters x 4 column quarters; per operand
+//          stage one wait, two TMEM loads of 32 columns and the
+//          rescale-accumulate; after the last block of a tile gate/up ->
+//          SwiGLU + Q8_0 requantisation, down -> y += w_slot * o with vector
+//          reductions (red.v4.f32) of 4 consecutive rows of H of one token.
+// TMEM: four accumulators of 128 columns (all 512 columns), handed between
+// the MMA issuer and the epilogue a pair (one operand stage) at a time;
+// full/empty mbarriers between every pair of roles; every wait bounded, and
+// one that runs out makes every role leave its loop and records
 // STATUS_SPIN_TIMEOUT.
-// Why quads: the kernel is bound by its hand-off skeleton rather than by any
-// role's arithmetic (measured on B200: with every role's work removed half of
-// the time remains).  One mbarrier phase per block in each direction became
-// one per pair (-10 to -12%) and then one per quad (-4 to -5% more, which
-// needs all of TMEM for the accumulators and so the A operand in shared
-// memory); deeper rings or more input stages changed nothing.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -69,40 +63,37 @@ namespace moeq4 {
 namespace {
 
 constexpr int TM = 128;            // MMA M: weight rows per tile
-constexpr int TN = TC_TILE_TOKENS; // MMA N: slots per tile
 constexpr int IN_KB = 8;           // Q4_0 blocks per input stage (144-byte rows: a 16-byte multiple)
-constexpr int OP_KB = 4;           // blocks per operand stage
-constexpr int NIN = 2, NOP = 2, NTM = 8, NSC = 16;  // input, operand, accumulator and scale ring depths
+constexpr int OP_KB = 2;           // blocks per operand stage
+constexpr int NIN = 2, NOP = 2, NSC = 4;  // input, operand and scale-ring stages
+constexpr int NACC = 2 * OP_KB;    // accumulators: two pairs
 constexpr int IN_ROW = IN_KB * Q4_BYTES;          // 144
-constexpr int THREADS = 14 * 32;  // 4 warps on some SM sub-partitions: at most 128 registers a thread
+constexpr int N_CONV = 128;        // converter threads: one weight row (and one slot) each
 constexpr int W_PROD = 0, W_CONV0 = 1, W_MMA = 5, W_EPI0 = 6;
-constexpr int N_CONV = 128, N_EPI = 256;
-constexpr uint32_t TMEM_COLS = 512;
-static_assert(NTM * TN <= TMEM_COLS, "TMEM budget");
-static_assert(NTM == 2 * OP_KB, "two quads of accumulators, one per operand stage");
 constexpr uint32_t LIMIT = 1u << 22;
-static_assert(TN == 64, "the epilogue maps two warps of 32 columns onto a tile");
-
-// dynamic shared memory map (bytes)
 constexpr size_t SZ_IN_W = (size_t)TM * IN_ROW;           // one input stage of packed weight rows
-constexpr size_t SZ_IN_B = (size_t)TN * IN_KB * QK;       // int8 activations, [16-byte chunk][slot]
-constexpr size_t SZ_IN_DA = (size_t)TN * IN_KB * 2;       // activation scale bits, [slot][block]
-constexpr size_t SZ_KSTEP_B = (size_t)TN * 32;
-constexpr size_t SZ_OP_B = (size_t)OP_KB * 2 * SZ_KSTEP_B;
-constexpr int XCH_LD = TN + 1;
-constexpr size_t OFF_IN_W = 0;
-constexpr size_t OFF_IN_B = OFF_IN_W + NIN * SZ_IN_W;
-constexpr size_t OFF_IN_DA = OFF_IN_B + NIN * SZ_IN_B;
-constexpr size_t OFF_OP_B = (OFF_IN_DA + NIN * SZ_IN_DA + 1023) & ~size_t(1023);
-constexpr size_t SZ_KSTEP_A = (size_t)TM * 32;
-constexpr size_t SZ_OP_A = (size_t)OP_KB * 2 * SZ_KSTEP_A;
-constexpr size_t OFF_OP_A = OFF_OP_B + NOP * SZ_OP_B;
-constexpr size_t OFF_DW = OFF_OP_A + NOP * SZ_OP_A;
-constexpr size_t OFF_DA = OFF_DW + (size_t)NSC * TM * 4;
-constexpr size_t OFF_XCH = OFF_DA + (size_t)NSC * TN * 4;
-constexpr size_t SMEM_BYTES = OFF_XCH + (size_t)TM * XCH_LD * 4;
-constexpr size_t SMEM_ALLOC = SMEM_BYTES + 1024;          // slack to align the map to 1024 B
-static_assert(SMEM_ALLOC <= 220 * 1024, "shared memory map too large");
+constexpr size_t SZ_OP_A = (size_t)OP_KB * 2 * TM * 32;   // one operand stage of A (K-steps of 16 x binary16)
+
+// Per tile width TN (slots, the MMA N): the epilogue has TN/32 column groups
+// of 4 warps (one per TMEM lane quarter), and the shared-memory map.
+template <int TN>
+struct TcCfg {
+    static_assert(TN == 32 || TN == 128, "tile widths");
+    static constexpr int N_EPI = 4 * TN;
+    static constexpr int THREADS = 6 * 32 + N_EPI;        // TN = 128: 704, at most 80 registers a thread
+    static constexpr uint32_t TMEM_COLS = NACC * TN;      // 512 or 128 columns
+    static constexpr size_t SZ_OP_B = (size_t)OP_KB * 2 * TN * 32;
+    static constexpr int XCH_LD = TN + 1;
+    static constexpr size_t OFF_IN_W = 0;
+    static constexpr size_t OFF_OP_A = (OFF_IN_W + NIN * SZ_IN_W + 1023) & ~size_t(1023);
+    static constexpr size_t OFF_OP_B = OFF_OP_A + NOP * SZ_OP_A;
+    static constexpr size_t OFF_DW = OFF_OP_B + NOP * SZ_OP_B;
+    static constexpr size_t OFF_DA = OFF_DW + (size_t)NSC * OP_KB * TM * 4;
+    static constexpr size_t OFF_XCH = OFF_DA + (size_t)NSC * OP_KB * TN * 4;
+    static constexpr size_t SMEM_BYTES = OFF_XCH + (size_t)TM * XCH_LD * 4;
+    static constexpr size_t SMEM_ALLOC = SMEM_BYTES + 1024;   // slack to align the map to 1024 B
+    static_assert(SMEM_ALLOC <= 200 * 1024, "shared memory map too large");
+};
 
 enum { GATEUP = 0, DOWN = 1 };
 
@@ -142,13 +133,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Arrive on `bar` once this thread's earlier cp.async copies complete; the
-// arrival counts towards the barrier's expected count.
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-
 // Bounded wait shared by all roles: once any wait of the CTA has run out,
 // `abort` is set and every later wait returns false soon after.
 // The waiting thread sleeps in try_wait (suspend hint) rather than spinning;
@@ -180,6 +164,12 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
             "r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
+}
+
+// y[0..3] += v (one vector reduction at L2; y 16-byte aligned)
+__device__ __forceinline__ void red_add_v4(float* y, float4 v) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(y), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
 }
 
 // acc[slot pair j] += I (32 columns of one block) * dW * dA[slot].
@@ -233,11 +223,46 @@ constexpr uint32_t BIAS_NIB = 0x64086408u;   // binary16 1032, twice: 1024 + n -
 constexpr uint32_t BIAS_ACT = 0x64806480u;   // binary16 1152, twice: 1024 + (q ^ 0x80) - 1152 = q
 
 // Byte offset of the 16-byte core-matrix piece `core` (0/1) of row r in K-step
-// `ks` of block `kb` of an operand stage with `rows` rows: K-steps are 32-byte
+// `ks` of block `kb` of an operand stage of `rows` rows: K-steps are 32-byte
 // (16 x binary16) slabs; inside one, 8-row groups are 256 B apart and the two
 // pieces of a row 128 B apart (the descriptor's SBO and LBO).
-__device__ __forceinline__ uint32_t op_off(int kb, int ks, int rows, int r, int core) {
+__device__ __forceinline__ uint32_t op_off(int rows, int kb, int ks, int r, int core) {
     return (uint32_t)((kb * 2 + ks) * rows * 32 + (r >> 3) * 256 + core * 128 + (r & 7) * 16);
+}
+
+// 16 activation codes (one 16-byte load) -> the two core-matrix pieces of one
+// K-step of slot n.
+__device__ __forceinline__ void store_act16(uint8_t* ob, int rows, int kb, int ks, int n, uint4 a) {
+    const uint2 a0 = bytes_to_f16(a.x ^ 0x80808080u, BIAS_ACT);
+    const uint2 a1 = bytes_to_f16(a.y ^ 0x80808080u, BIAS_ACT);
+    const uint2 a2 = bytes_to_f16(a.z ^ 0x80808080u, BIAS_ACT);
+    const uint2 a3 = bytes_to_f16(a.w ^ 0x80808080u, BIAS_ACT);
+    *reinterpret_cast<uint4*>(ob + op_off(rows, kb, ks, n, 0)) = make_uint4(a0.x, a0.y, a1.x, a1.y);
+    *reinterpret_cast<uint4*>(ob + op_off(rows, kb, ks, n, 1)) = make_uint4(a2.x, a2.y, a3.x, a3.y);
+}
+
+// One Q4_0 block (qs as four words) -> the four core-matrix pieces of weight
+// row r: columns 0..7 of a K-step pair are the low nibbles (weights 0..15),
+// 8..15 the high nibbles (16..31).
+__device__ __forceinline__ void store_weights(uint8_t* oa, int kb, int r, const uint32_t (&qs)[4]) {
+    uint32_t v[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint2 lo = bytes_to_f16(qs[i] & 0x0f0f0f0fu, BIAS_NIB);
+        const uint2 hi = bytes_to_f16((qs[i] >> 4) & 0x0f0f0f0fu, BIAS_NIB);
+        v[2 * i] = lo.x;
+        v[2 * i + 1] = lo.y;
+        v[8 + 2 * i] = hi.x;
+        v[8 + 2 * i + 1] = hi.y;
+    }
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+        for (int core = 0; core < 2; ++core) {
+            const int c0 = 8 * ks + 4 * core;
+            *reinterpret_cast<uint4*>(oa + op_off(TM, kb, ks, r, core)) =
+                make_uint4(v[c0], v[c0 + 1], v[c0 + 2], v[c0 + 3]);
+        }
 }
 
 __device__ __forceinline__ int find_group(const int* tile_off, int ngroups, int tile) {
@@ -254,6 +279,7 @@ struct Tile {
 };
 
 // Work item -> (group, first slot, slots in the tile, row block).
+template <int TN>
 __device__ __forceinline__ Tile tile_of(int item, int n_rb, const int* tile_off_s, const int* off_s, int ngroups) {
     Tile t;
     const int tile = item / n_rb;
@@ -281,8 +307,12 @@ __device__ __forceinline__ void slot_info(const TcParams& p, int g, int s, int& 
 
 // CAP: also write the per-block integer sums (the MMA accumulators before the
 // rescale) of one row block of one group to p.cap_out (test instantiation).
-template <int MODE, bool CAP>
-__global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, const __grid_constant__ TcMaps maps) {
+template <int MODE, int TN, bool CAP>
+__global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
+    tc_grouped_kernel(TcParams p, const __grid_constant__ TcMaps maps) {
+    using C = TcCfg<TN>;
+    constexpr int N_EPI = C::N_EPI, THREADS = C::THREADS, XCH_LD = C::XCH_LD;
+    constexpr uint32_t TMEM_COLS = C::TMEM_COLS;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __shared__ __align__(8) uint64_t in_full[NIN], in_empty[NIN], op_full[NOP], op_empty[NOP], tm_full[2],
@@ -290,15 +320,15 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ int tile_off_s[258], off_s[258];
+    __shared__ int tok_s[TN];
+    __shared__ float wt_s[TN];
 
-    uint8_t* in_w = smem + OFF_IN_W;
-    int8_t* in_b = reinterpret_cast<int8_t*>(smem + OFF_IN_B);
-    uint16_t* in_da = reinterpret_cast<uint16_t*>(smem + OFF_IN_DA);
-    uint8_t* op_b = smem + OFF_OP_B;
-    uint8_t* op_a = smem + OFF_OP_A;
-    float* dw_ring = reinterpret_cast<float*>(smem + OFF_DW);
-    float* da_ring = reinterpret_cast<float*>(smem + OFF_DA);
-    float* xch = reinterpret_cast<float*>(smem + OFF_XCH);
+    uint8_t* in_w = smem + C::OFF_IN_W;
+    uint8_t* op_a = smem + C::OFF_OP_A;
+    uint8_t* op_b = smem + C::OFF_OP_B;
+    float* dw_ring = reinterpret_cast<float*>(smem + C::OFF_DW);
+    float* da_ring = reinterpret_cast<float*>(smem + C::OFF_DA);
+    float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);
     volatile int* abort = &abort_s;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -316,14 +346,14 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
     if (tid == 32) {
         abort_s = 0;
         for (int i = 0; i < NIN; ++i) {
-            mbar_init(&in_full[i], 64);   // 32 producer-lane arrivals + 32 cp.async arrivals
+            mbar_init(&in_full[i], 1);
             mbar_init(&in_empty[i], N_CONV);
         }
         for (int i = 0; i < NOP; ++i) {
             mbar_init(&op_full[i], N_CONV);
             mbar_init(&op_empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {  // one quad of accumulators each
+        for (int i = 0; i < 2; ++i) {  // one pair of accumulators each
             mbar_init(&tm_full[i], 1);
             mbar_init(&tm_empty[i], N_EPI / 32);
         }
@@ -349,178 +379,112 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
         uint32_t i_in = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-            const Tile T = tile_of(item, n_rb, tile_off_s, off_s, ngroups);
+            const Tile T = tile_of<TN>(item, n_rb, tile_off_s, off_s, ngroups);
             // weight rows of this item: one box of 64 gate + one of 64 up rows, or 128 down rows
             const bool shared_g = T.g >= E;
             const CUtensorMap* map0 = &maps.m[shared_g ? 2 : 0];
             const CUtensorMap* map1 = &maps.m[shared_g ? 3 : 1];
             const int wy = (shared_g ? 0 : T.g * ((MODE == GATEUP) ? F : H)) + T.rb * ((MODE == GATEUP) ? 64 : TM);
-            const int8_t* arow[2];
-            const uint16_t* ascale[2];
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int n = lane + 32 * j;
-                arow[j] = nullptr;
-                ascale[j] = nullptr;
-                if (n < T.nslots) {
-                    const int s = T.slot0 + n;
-                    int tok;
-                    float w;
-                    slot_info(p, T.g, s, tok, w);
-                    if (MODE == GATEUP) {
-                        arow[j] = p.qa + (size_t)tok * H;
-                        ascale[j] = p.da + (size_t)tok * (H / QK);
-                    } else {
-                        arow[j] = p.hq + (size_t)s * F;
-                        ascale[j] = p.dh + (size_t)s * nbF;
-                    }
-                }
-            }
             for (int c = 0; c < nbK / IN_KB; ++c, ++i_in) {
                 const int s = i_in % NIN;
                 if (!wait_phase(&in_empty[s], ((i_in / NIN) & 1) ^ 1, abort)) { ok = false; break; }
                 uint8_t* dw = in_w + (size_t)s * SZ_IN_W;
-                int8_t* db = in_b + (size_t)s * SZ_IN_B;
-                uint16_t* dda = in_da + (size_t)s * TN * IN_KB;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&in_full[s], (uint32_t)(TM * IN_ROW));
                     tma_load_2d(dw, map0, c * IN_ROW, wy, &in_full[s]);
                     if (MODE == GATEUP) tma_load_2d(dw + 64 * IN_ROW, map1, c * IN_ROW, wy, &in_full[s]);
-                } else {
-                    mbar_arrive(&in_full[s]);
                 }
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    if (arow[j]) {
-                        const int n = lane + 32 * j;
-                        const int8_t* src = arow[j] + (size_t)c * IN_KB * QK;
-#pragma unroll
-                        for (int q = 0; q < IN_KB * 2; ++q) cp_async16(db + ((size_t)q * TN + n) * 16, src + q * 16);
-                        cp_async16(dda + n * IN_KB, ascale[j] + c * IN_KB);   // 8 binary16 scales
-                    }
-                }
-                cp_async_arrive_noinc(&in_full[s]);
+                __syncwarp();
             }
         }
         // let the copies in flight land before the CTA can exit
-        cp_async_wait_all();
         if (i_in > 0) mbar_wait_bounded(&in_full[(i_in - 1) % NIN], ((i_in - 1) / NIN) & 1, LIMIT);
     } else if (warp >= W_CONV0 && warp < W_CONV0 + 4) {
         // ------------------------------------------------------------ converters
-        const int ct = tid - W_CONV0 * 32;        // slot column ct & 63 of the activation work
-        const int crow = 32 * (warp & 3) + lane;  // weight row this thread converts
-        uint32_t i_op = 0, gb = 0;
+        // thread ct converts weight row ct and (ct < TN) the activations of slot ct
+        const int ct = tid - W_CONV0 * 32;
+        uint32_t i_op = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-            const Tile T = tile_of(item, n_rb, tile_off_s, off_s, ngroups);
-            for (int c = 0; c < nbK / OP_KB && ok; ++c, ++i_op, gb += OP_KB) {
-                const uint32_t i_in = i_op >> 1;
-                const int s = i_in % NIN, sub = i_op & 1;
+            const Tile T = tile_of<TN>(item, n_rb, tile_off_s, off_s, ngroups);
+            const bool valid = ct < T.nslots;
+            const int8_t* arow = nullptr;
+            const uint16_t* ascale = nullptr;
+            if (valid) {
+                const int sl = T.slot0 + ct;
+                int tok;
+                float w;
+                slot_info(p, T.g, sl, tok, w);
+                if (MODE == GATEUP) {
+                    arow = p.qa + (size_t)tok * H;
+                    ascale = p.da + (size_t)tok * (H / QK);
+                } else {
+                    arow = p.hq + (size_t)sl * F;
+                    ascale = p.dh + (size_t)sl * nbF;
+                }
+            }
+            for (int c = 0; c < nbK / OP_KB && ok; ++c, ++i_op) {
+                // this slot's 2 blocks of activations and their scales: the
+                // loads are in flight while the stages below are awaited
+                uint4 a[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                              make_uint4(0, 0, 0, 0)};
+                uint32_t dab = 0;
+                if (valid) {
+                    const uint4* src = reinterpret_cast<const uint4*>(arow + (size_t)c * OP_KB * QK);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) a[i] = __ldcg(src + i);
+                    dab = __ldcg(reinterpret_cast<const uint32_t*>(ascale + c * OP_KB));
+                }
+                const uint32_t i_in = i_op / (IN_KB / OP_KB);
+                const int s = i_in % NIN, sub = i_op % (IN_KB / OP_KB);
                 if (sub == 0 && !wait_phase(&in_full[s], (i_in / NIN) & 1, abort)) { ok = false; break; }
                 const int o = i_op % NOP;
                 if (!wait_phase(&op_empty[o], ((i_op / NOP) & 1) ^ 1, abort)) { ok = false; break; }
                 tc_fence_after_sync();
-                uint8_t* ob = op_b + (size_t)o * SZ_OP_B;
 
-                // weights: this row's 4 blocks, 72 bytes at an 8-byte boundary
-                uint32_t w[18];
-                const uint2* wsrc = reinterpret_cast<const uint2*>(in_w + (size_t)s * SZ_IN_W + (size_t)crow * IN_ROW +
-                                                                   sub * OP_KB * Q4_BYTES);
+                // weights: this row's 2 blocks, 36 bytes at a 4-byte boundary
+                uint32_t w[9];
+                const uint32_t* wsrc = reinterpret_cast<const uint32_t*>(in_w + (size_t)s * SZ_IN_W + (size_t)ct * IN_ROW +
+                                                                         sub * OP_KB * Q4_BYTES);
 #pragma unroll
-                for (int i = 0; i < 9; ++i) {
-                    const uint2 v = wsrc[i];
-                    w[2 * i] = v.x;
-                    w[2 * i + 1] = v.y;
-                }
-                float dws[OP_KB];
-                uint32_t v[OP_KB * 16];  // the 4 blocks' binary16 pairs of this row, in K order
-#pragma unroll
-                for (int kb = 0; kb < OP_KB; ++kb) {
-                    // block kb starts at byte 18 kb: scale, then 16 nibble bytes
-                    const int bw = (18 * kb) / 4;
-                    uint32_t qs[4], dbits;
-                    if ((kb & 1) == 0) {
-                        dbits = w[bw] & 0xffffu;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) qs[i] = __funnelshift_r(w[bw + i], w[bw + i + 1], 16);
-                    } else {
-                        dbits = w[bw] >> 16;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) qs[i] = w[bw + 1 + i];
-                    }
-                    dws[kb] = half_bits_to_float(dbits);
-                    // columns 0..7 of a block: low nibbles (weights 0..15), 8..15: high nibbles (16..31)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint2 lo = bytes_to_f16(qs[i] & 0x0f0f0f0fu, BIAS_NIB);
-                        const uint2 hi = bytes_to_f16((qs[i] >> 4) & 0x0f0f0f0fu, BIAS_NIB);
-                        v[16 * kb + 2 * i] = lo.x;
-                        v[16 * kb + 2 * i + 1] = lo.y;
-                        v[16 * kb + 8 + 2 * i] = hi.x;
-                        v[16 * kb + 8 + 2 * i + 1] = hi.y;
-                    }
-                }
-                // this row of the A operand: block kb, K-step ks, core matrix
-                // `core` holds binary16 pairs 16 kb + 8 ks + 4 core .. + 3
+                for (int i = 0; i < 9; ++i) w[i] = wsrc[i];
                 uint8_t* oa = op_a + (size_t)o * SZ_OP_A;
+                uint8_t* ob = op_b + (size_t)o * C::SZ_OP_B;
+                float dws[OP_KB];
+                {
+                    // block 0 starts at byte 0 (scale, then 16 nibble bytes), block 1 at byte 18
+                    uint32_t qs[4];
+                    dws[0] = half_bits_to_float(w[0] & 0xffffu);
 #pragma unroll
-                for (int kb = 0; kb < OP_KB; ++kb)
+                    for (int i = 0; i < 4; ++i) qs[i] = __funnelshift_r(w[i], w[i + 1], 16);
+                    store_weights(oa, 0, ct, qs);
+                    dws[1] = half_bits_to_float(w[4] >> 16);
 #pragma unroll
-                    for (int ks = 0; ks < 2; ++ks)
-#pragma unroll
-                        for (int core = 0; core < 2; ++core) {
-                            const int c0 = 16 * kb + 8 * ks + 4 * core;
-                            *reinterpret_cast<uint4*>(oa + op_off(kb, ks, TM, crow, core)) =
-                                make_uint4(v[c0], v[c0 + 1], v[c0 + 2], v[c0 + 3]);
-                        }
-                // activations: slot n = ct & 63, blocks (ct >> 6) and (ct >> 6) + 2
-                const int n = ct & 63;
-                const bool valid = n < T.nslots;
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int kb = (ct >> 6) + 2 * j;
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
-                        uint4 v = make_uint4(0, 0, 0, 0), u = make_uint4(0, 0, 0, 0);
-                        if (valid) {
-                            const int q = (sub * OP_KB + kb) * 2 + ks;
-                            const uint4 a = *reinterpret_cast<const uint4*>(in_b + (size_t)s * SZ_IN_B +
-                                                                            ((size_t)q * TN + n) * 16);
-                            const uint2 a0 = bytes_to_f16(a.x ^ 0x80808080u, BIAS_ACT);
-                            const uint2 a1 = bytes_to_f16(a.y ^ 0x80808080u, BIAS_ACT);
-                            const uint2 a2 = bytes_to_f16(a.z ^ 0x80808080u, BIAS_ACT);
-                            const uint2 a3 = bytes_to_f16(a.w ^ 0x80808080u, BIAS_ACT);
-                            v = make_uint4(a0.x, a0.y, a1.x, a1.y);
-                            u = make_uint4(a2.x, a2.y, a3.x, a3.y);
-                        }
-                        *reinterpret_cast<uint4*>(ob + op_off(kb, ks, TN, n, 0)) = v;
-                        *reinterpret_cast<uint4*>(ob + op_off(kb, ks, TN, n, 1)) = u;
-                    }
+                    for (int i = 0; i < 4; ++i) qs[i] = w[5 + i];
+                    store_weights(oa, 1, ct, qs);
                 }
-                // this slot's activation scales, read before the input stage is released
-                float das[OP_KB];
+                // activations of slot ct (zeros past the tile's slots)
+                if (ct < TN) {
 #pragma unroll
-                for (int kb = 0; kb < OP_KB; ++kb)
-                    das[kb] = valid ? half_bits_to_float(in_da[(size_t)s * TN * IN_KB + n * IN_KB + sub * OP_KB + kb])
-                                    : 0.0f;
+                    for (int kb = 0; kb < OP_KB; ++kb)
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks) store_act16(ob, TN, kb, ks, ct, a[2 * kb + ks]);
+                }
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 mbar_arrive(&op_full[o]);
-                if (sub == 1) mbar_arrive(&in_empty[s]);
-                // scales of these 4 blocks into the ring read by the epilogue; the
-                // epilogue frees the last entry of each group of four, in order
-                const uint32_t glast = gb + OP_KB - 1, buf0 = gb % NSC;
-                if (!wait_phase(&sc_empty[glast % NSC], ((glast / NSC) & 1) ^ 1, abort)) { ok = false; break; }
+                if (sub == IN_KB / OP_KB - 1) mbar_arrive(&in_empty[s]);
+                // block scales into the ring read by the epilogue
+                const int sc = i_op % NSC;
+                if (!wait_phase(&sc_empty[sc], ((i_op / NSC) & 1) ^ 1, abort)) { ok = false; break; }
 #pragma unroll
                 for (int kb = 0; kb < OP_KB; ++kb) {
-                    dw_ring[(buf0 + kb) * TM + crow] = dws[kb];
-                    if (ct < TN) da_ring[(buf0 + kb) * TN + ct] = das[kb];
+                    dw_ring[(sc * OP_KB + kb) * TM + ct] = dws[kb];
+                    if (ct < TN)
+                        da_ring[(sc * OP_KB + kb) * TN + ct] = valid ? half_bits_to_float(kb ? (dab >> 16) : dab) : 0.0f;
                 }
                 __syncwarp();
-                if (lane == 0) {
-#pragma unroll
-                    for (int kb = 0; kb < OP_KB; ++kb) mbar_arrive(&sc_full[buf0 + kb]);
-                }
+                if (lane == 0) mbar_arrive(&sc_full[sc]);
             }
         }
     } else if (warp == W_MMA) {
@@ -529,7 +493,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
             constexpr uint32_t idesc = idesc_f16(TM, TN);
             // descriptors of the first K-step of each operand stage; a later
             // K-step adds its byte offset / 16 to the start-address field
-            const uint64_t b0 = smem_desc_kmajor(op_b, 128, 256), b1 = smem_desc_kmajor(op_b + SZ_OP_B, 128, 256);
+            const uint64_t b0 = smem_desc_kmajor(op_b, 128, 256), b1 = smem_desc_kmajor(op_b + C::SZ_OP_B, 128, 256);
             const uint64_t a0 = smem_desc_kmajor(op_a, 128, 256), a1 = smem_desc_kmajor(op_a + SZ_OP_A, 128, 256);
             static_assert(NOP == 2, "two operand stages");
             uint32_t i_op = 0;
@@ -541,8 +505,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                         ok = false;
                         break;
                     }
-                    // the quad of accumulators of this operand stage: buffers 4o .. 4o + 3,
-                    // freed by the epilogue two stages ago
+                    // the pair of accumulators of this operand stage: buffers
+                    // 2o, 2o + 1, freed by the epilogue two stages ago
                     if (!wait_phase(&tm_empty[o], ((i_op / 2) & 1) ^ 1, abort)) {
                         ok = false;
                         break;
@@ -552,14 +516,12 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
 #pragma unroll
                     for (int kb = 0; kb < OP_KB; ++kb) {
                         const uint32_t d = tmem + (uint32_t)(OP_KB * o + kb) * TN;
-                        mma_f16_ss(d, ad + (uint64_t)((kb * 2) * (SZ_KSTEP_A >> 4)),
-                                   bd + (uint64_t)((kb * 2) * (SZ_KSTEP_B >> 4)), idesc, false);
-                        mma_f16_ss(d, ad + (uint64_t)((kb * 2 + 1) * (SZ_KSTEP_A >> 4)),
-                                   bd + (uint64_t)((kb * 2 + 1) * (SZ_KSTEP_B >> 4)), idesc, true);
+                        constexpr uint64_t KA = (uint64_t)TM * 32 >> 4, KB = (uint64_t)TN * 32 >> 4;  // K-step / 16
+                        mma_f16_ss(d, ad + (uint64_t)(kb * 2) * KA, bd + (uint64_t)(kb * 2) * KB, idesc, false);
+                        mma_f16_ss(d, ad + (uint64_t)(kb * 2 + 1) * KA, bd + (uint64_t)(kb * 2 + 1) * KB, idesc, true);
                     }
-                    mma_commit(&tm_full[o]);  // covers the quad's eight MMAs
+                    mma_commit(&tm_full[o]);  // covers the pair's four MMAs
                     mma_commit(&op_empty[o]);
-                    if (!ok) break;
                 }
             }
             // the last commit's arrival must land before the CTA can exit
@@ -567,76 +529,76 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        const int et = tid - W_EPI0 * 32;         // 0 .. N_EPI - 1
         const int q = warp & 3;                   // TMEM lane quarter this warp may access
-        const int hcol = (warp - W_EPI0) >> 2;    // column half: slots 32 hcol .. 32 hcol + 31
+        const int cq = (warp - W_EPI0) >> 2;      // column quarter: slots 32 cq .. 32 cq + 31
         const int row = 32 * q + lane;            // weight row (TMEM lane) of this thread
-        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + 32 * hcol;
-        uint32_t gb = 0, epi_phase = 0;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + 32 * cq;
+        uint32_t i_op = 0, epi_phase = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-            const Tile T = tile_of(item, n_rb, tile_off_s, off_s, ngroups);
+            const Tile T = tile_of<TN>(item, n_rb, tile_off_s, off_s, ngroups);
+            if (MODE == DOWN && et < TN) {
+                // token and weight of each slot, for the combine at the tile's end
+                // (the previous tile's readers passed the barrier that ended it)
+                int tok = 0;
+                float w = 0.0f;
+                if (et < T.nslots) slot_info(p, T.g, T.slot0 + et, tok, w);
+                tok_s[et] = tok;
+                wt_s[et] = w;
+            }
             float2 acc[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = make_float2(0.0f, 0.0f);
-            // one wait per quad of blocks (one operand stage); two blocks per pass,
-            // both TMEM loads in flight before either is used
-            for (int b = 0; b < nbK; b += OP_KB, gb += OP_KB) {
-                const uint32_t qd = (gb / OP_KB) & 1, qpar = (gb / (2 * OP_KB)) & 1;
-                const uint32_t s0 = gb % NSC, spar = (gb / NSC) & 1;
-                // the converters arrive on the four scale entries in order, so the
-                // last one complete means all four are
-                if (!wait_phase(&tm_full[qd], qpar, abort) || !wait_phase(&sc_full[s0 + 3], spar, abort)) {
+            for (int b = 0; b < nbK; b += OP_KB, ++i_op) {
+                const uint32_t pr = i_op & 1, ppar = (i_op >> 1) & 1;
+                const uint32_t sc = i_op % NSC, spar = (i_op / NSC) & 1;
+                if (!wait_phase(&tm_full[pr], ppar, abort) || !wait_phase(&sc_full[sc], spar, abort)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const uint32_t bb = OP_KB * qd + 2 * h2, sa = s0 + 2 * h2;
-                    uint32_t r0[32], r1[32];
-                    tmem_ld32(taddr + bb * TN, r0);
-                    tmem_ld32(taddr + (bb + 1) * TN, r1);
+                for (int kb = 0; kb < OP_KB; ++kb) {
+                    uint32_t r[32];
+                    tmem_ld32(taddr + (OP_KB * pr + kb) * TN, r);
                     tmem_wait_ld();
                     if (CAP && T.g == p.cap_group && T.rb == p.cap_rb) {
                         // exact integers held in binary32: convert back without rounding
                         const size_t s0 = (size_t)(T.slot0 - off_s[T.g]);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
-                            const int n = 32 * hcol + j;
-                            if (n < T.nslots) {
-                                int32_t* o = p.cap_out + ((s0 + n) * TM + row) * nbK + b + 2 * h2;
-                                o[0] = __float2int_rn(__uint_as_float(r0[j]));
-                                o[1] = __float2int_rn(__uint_as_float(r1[j]));
-                            }
+                            const int n = 32 * cq + j;
+                            if (n < T.nslots)
+                                p.cap_out[((s0 + n) * TM + row) * nbK + b + kb] = __float2int_rn(__uint_as_float(r[j]));
                         }
                     }
-                    rescale_acc(acc, r0, dw_ring[sa * TM + row], da_ring + sa * TN + 32 * hcol);
-                    rescale_acc(acc, r1, dw_ring[(sa + 1) * TM + row], da_ring + (sa + 1) * TN + 32 * hcol);
+                    rescale_acc(acc, r, dw_ring[(sc * OP_KB + kb) * TM + row], da_ring + (sc * OP_KB + kb) * TN + 32 * cq);
                 }
                 tc_fence_before_sync();
                 __syncwarp();
-                // the converters wait only on the last entry of each group of four
                 if (lane == 0) {
-                    mbar_arrive(&tm_empty[qd]);
-                    mbar_arrive(&sc_empty[s0 + 3]);
+                    mbar_arrive(&tm_empty[pr]);
+                    mbar_arrive(&sc_empty[sc]);
                 }
             }
             if (!ok) break;
-            if (MODE == GATEUP) {
-                float* xr = xch + (size_t)row * XCH_LD + 32 * hcol;
+            // this thread's row x 32 slots into the exchange tile
+            float* xr = xch + (size_t)row * XCH_LD + 32 * cq;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    xr[2 * j] = acc[j].x;
-                    xr[2 * j + 1] = acc[j].y;
-                }
-                if (!epi_sync(&epi_bar, epi_phase++, abort)) break;
+            for (int j = 0; j < 16; ++j) {
+                xr[2 * j] = acc[j].x;
+                xr[2 * j + 1] = acc[j].y;
+            }
+            if (!epi_sync(&epi_bar, epi_phase++, abort)) break;
+            if (MODE == GATEUP) {
                 // SwiGLU + Q8_0 of h.  A unit is one 32-row block of h (gate rows
                 // 32 fb .. 32 fb + 31) of one slot n; two lanes share a unit, 16
                 // rows each, so every value is independent of the others and a
                 // single shuffle gives the block's absolute maximum.  Both
                 // divisions of the Q8_0 rule stay IEEE (div.rn).
-                const int u = ((warp - W_EPI0) * 32 + lane) >> 1;   // 0..127
-                const int n = u & 63, fb = u >> 6, half = lane & 1;
+                const int u = et >> 1;                    // 0 .. 2 TN - 1
+                const int n = u % TN, fb = u / TN, half = lane & 1;
                 const int r0 = 32 * fb + 16 * half;
                 const int f0 = T.rb * 64;
                 float h[16];
@@ -669,21 +631,23 @@ __global__ void __launch_bounds__(THREADS, 1) tc_grouped_kernel(TcParams p, cons
                         if ((dbits & 0x7fffu) == 0x7c00u) atomicOr(p.status, STATUS_SCALE_OVERFLOW);
                     }
                 }
-                if (!epi_sync(&epi_bar, epi_phase++, abort)) break;  // xch is free for the next tile
             } else {
-                int tok = 0;
-                float w = 0.0f;
-                const int n_me = 32 * hcol + lane;
-                if (n_me < T.nslots) slot_info(p, T.g, T.slot0 + n_me, tok, w);
+                // y[token][h0 + 4 i .. + 3] += w * o: one vector reduction per
+                // (slot, 4 consecutive rows of H)
                 const int h0 = T.rb * TM;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int tj = __shfl_sync(0xffffffffu, tok, j);
-                    const float wj = __shfl_sync(0xffffffffu, w, j);
-                    const float v = (j & 1) ? acc[j >> 1].y : acc[j >> 1].x;
-                    if (32 * hcol + j < T.nslots) atomicAdd(p.y + (size_t)tj * H + h0 + row, wj * v);
+                for (int i = 0; i < TM * TN / 4 / N_EPI; ++i) {
+                    const int u = et + N_EPI * i;
+                    const int n = u % TN, rq = u / TN;
+                    if (n < T.nslots) {
+                        const float w = wt_s[n];
+                        const float* xc = xch + (size_t)(4 * rq) * XCH_LD + n;
+                        red_add_v4(p.y + (size_t)tok_s[n] * H + h0 + 4 * rq,
+                                   make_float4(w * xc[0], w * xc[XCH_LD], w * xc[2 * XCH_LD], w * xc[3 * XCH_LD]));
+                    }
                 }
             }
+            if (!epi_sync(&epi_bar, epi_phase++, abort)) break;  // xch is free for the next tile
         }
     }
 
@@ -704,7 +668,7 @@ static TcParams make_tc_params(const LayerView& L, int64_t T, const Workspace& w
     return p;
 }
 
-static int64_t tc_max_tiles(const LayerView& L, int64_t T) {
+static int64_t tc_max_tiles(const LayerView& L, int64_t T, int TN) {
     const int64_t P = T * L.k;
     return ceil_div(P, TN) + std::min<int64_t>(L.E, P) + (L.S ? ceil_div(T, TN) : 0);
 }
@@ -760,41 +724,57 @@ static cudaError_t make_maps(const LayerView& L, TcMaps* maps) {
     return e;
 }
 
-template <int MODE>
-static cudaError_t launch_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, float* y,
-                             const DeviceInfo& dev, const BlockDotCapture* cap, cudaStream_t s) {
-    const bool capture = cap && cap->down == (MODE == DOWN ? 1 : 0);
-    const void* kfn = capture ? reinterpret_cast<const void*>(tc_grouped_kernel<MODE, true>)
-                              : reinterpret_cast<const void*>(tc_grouped_kernel<MODE, false>);
+template <int MODE, int TN, bool CAP>
+static cudaError_t launch_tc_inst(const LayerView& L, int64_t T, const TcParams& p, const TcMaps& maps,
+                                  const DeviceInfo& dev, cudaStream_t s) {
+    using C = TcCfg<TN>;
     int per_sm = 0;
-    cudaError_t e = kernel_occupancy(kfn, THREADS, SMEM_ALLOC, &per_sm);
-    if (e != cudaSuccess) return e;
-    TcMaps maps;
-    e = make_maps<MODE>(L, &maps);
+    cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(tc_grouped_kernel<MODE, TN, CAP>), C::THREADS,
+                                     C::SMEM_ALLOC, &per_sm);
     if (e != cudaSuccess) return e;
     const int n_rb = (MODE == GATEUP) ? L.F / 64 : L.H / TM;
-    const int64_t items = tc_max_tiles(L, T) * n_rb;
+    const int64_t items = tc_max_tiles(L, T, TN) * n_rb;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, dev.sm_count));
+    tc_grouped_kernel<MODE, TN, CAP><<<(unsigned)grid, C::THREADS, C::SMEM_ALLOC, s>>>(p, maps);
+    return cudaGetLastError();
+}
+
+template <int MODE>
+static cudaError_t launch_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, float* y,
+                             const DeviceInfo& dev, int tile, const BlockDotCapture* cap, cudaStream_t s) {
+    if (tile != 32 && tile != 128) return cudaErrorInvalidValue;
+    const bool capture = cap && cap->down == (MODE == DOWN ? 1 : 0);
+    TcMaps maps;
+    cudaError_t e = make_maps<MODE>(L, &maps);
+    if (e != cudaSuccess) return e;
     TcParams p = make_tc_params(L, T, ws, h_dbg, y);
     if (capture) {
         p.cap_out = cap->out;
         p.cap_group = cap->group;
         p.cap_rb = cap->rb;
-        tc_grouped_kernel<MODE, true><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(p, maps);
-    } else {
-        tc_grouped_kernel<MODE, false><<<(unsigned)grid, THREADS, SMEM_ALLOC, s>>>(p, maps);
+        return tile == 128 ? launch_tc_inst<MODE, 128, true>(L, T, p, maps, dev, s)
+                           : launch_tc_inst<MODE, 32, true>(L, T, p, maps, dev, s);
     }
-    return cudaGetLastError();
+    return tile == 128 ? launch_tc_inst<MODE, 128, false>(L, T, p, maps, dev, s)
+                       : launch_tc_inst<MODE, 32, false>(L, T, p, maps, dev, s);
+}
+
+int tc_tile_tokens(const LayerView& L, int64_t T, int force) {
+    if (force == 32 || force == 128) return force;
+    // routed slots per expert on average: narrow tiles while most experts
+    // hold only a few tokens (decode batches), wide ones for prompts
+    const int64_t per_expert = T * L.k / L.E;
+    return per_expert >= 64 ? 128 : 32;
 }
 
 cudaError_t launch_gateup_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, const DeviceInfo& dev,
-                             const BlockDotCapture* cap, cudaStream_t s) {
-    return launch_tc<GATEUP>(L, T, ws, h_dbg, nullptr, dev, cap, s);
+                             int tile, const BlockDotCapture* cap, cudaStream_t s) {
+    return launch_tc<GATEUP>(L, T, ws, h_dbg, nullptr, dev, tile, cap, s);
 }
 
 cudaError_t launch_down_tc(const LayerView& L, int64_t T, const Workspace& ws, float* y, const DeviceInfo& dev,
-                           const BlockDotCapture* cap, cudaStream_t s) {
-    return launch_tc<DOWN>(L, T, ws, nullptr, y, dev, cap, s);
+                           int tile, const BlockDotCapture* cap, cudaStream_t s) {
+    return launch_tc<DOWN>(L, T, ws, nullptr, y, dev, tile, cap, s);
 }
 
 }  // namespace moeq4

@@ -37,6 +37,7 @@ struct Workspace {
     int32_t* pos;
     int8_t* hq;
     uint16_t* dh;
+    uint32_t* sync;   // per-group counters of the fused T = 1 kernels
 };
 
 // Test capture of the per-block integer dot products I_b of one row block of
@@ -77,13 +78,15 @@ cudaError_t launch_down_dp4a(const LayerView& L, int64_t T, const Workspace& ws,
 // Q8_0 activations qa/da of T tokens (the streaming kernel's GEMV mode).
 cudaError_t launch_gemv_dp4a(const uint8_t* W, int64_t N, int H, const int8_t* qa, const uint16_t* da, int T,
                              float* y, uint32_t* status, const DeviceInfo& dev, cudaStream_t s);
-// k_tc_grouped.cu: grouped projections on tcgen05 (kind::f16, TMEM); the
-// permutation must have been built with TC_TILE_TOKENS slots per tile.
-constexpr int TC_TILE_TOKENS = 64;
+// k_tc_grouped.cu: grouped projections on tcgen05 (kind::f16, TMEM) with
+// tiles of `tile` slots (32 or 128); the permutation must have been built with
+// the same tile width.  tc_tile_tokens: the width for T tokens (force = 32 or
+// 128 picks one, else automatic).
+int tc_tile_tokens(const LayerView& L, int64_t T, int force);
 cudaError_t launch_gateup_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, const DeviceInfo& dev,
-                             const BlockDotCapture* cap, cudaStream_t s);
+                             int tile, const BlockDotCapture* cap, cudaStream_t s);
 cudaError_t launch_down_tc(const LayerView& L, int64_t T, const Workspace& ws, float* y, const DeviceInfo& dev,
-                           const BlockDotCapture* cap, cudaStream_t s);
+                           int tile, const BlockDotCapture* cap, cudaStream_t s);
 
 // k_decode.cu: the fused T=1 path (router kernel + cooperative FFN kernel,
 // chained with programmatic dependent launch).  Events, if given, bracket the

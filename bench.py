@@ -272,7 +272,7 @@ def int8_peak_tops():
     return 1590.0 * 2.0, "fallback bf16 x nominal int8/bf16 ratio 2"
 
 
-def prefill_lines(m, torch, stream):
+def prefill_lines(m, torch, stream, names=("prefill_t947", "zipf_t16384")):
     """Single-pass prefill of the two prefill workloads on the automatic path
     (tensor cores at these sizes): tokens/s over whole forwards and the int8
     ops/s of the gate/up kernel, L2 flushed (256 MB written) before each rep."""
@@ -281,7 +281,7 @@ def prefill_lines(m, torch, stream):
     peak, peak_src = int8_peak_tops()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     variants = (("auto", m.PATH_AUTO), ("tc_n32", m.PATH_TENSOR_CORE_N32), ("tc_n128", m.PATH_TENSOR_CORE_N128))
-    for name in ("prefill_t947", "zipf_t16384"):
+    for name in names:
         x_np, lw = synth.workload_inputs(name, seed=0)
         L = m.Layer.from_host(lw)
         x = torch.from_numpy(x_np).cuda()
@@ -316,7 +316,26 @@ def prefill_lines(m, torch, stream):
                 out[name] = rec
             else:
                 out[name][vname] = rec
-        del L, x, y, ws
+        # the router (logits + top-k: the same kernels the forward launches)
+        # alone, and its share of the automatic forward
+        idx = torch.empty((T, lw.top_k), dtype=torch.int32, device="cuda")
+        wts = torch.empty((T, lw.top_k), dtype=torch.float32, device="cuda")
+        lg = torch.empty((T, lw.n_experts), dtype=torch.float32, device="cuda")
+        rt = []
+        for rep in range(8):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            m.moe_q4_route(L, x, idx, wts, lg, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 3:
+                rt.append(e0.elapsed_time(e1))
+        r_ms = float(np.median(rt))
+        out[name]["router_ms"] = r_ms
+        out[name]["router_share"] = r_ms / out[name]["ms"]
+        out[name]["router_fp32_tflops"] = 2.0 * T * lw.hidden * lw.n_experts / (r_ms * 1e-3) / 1e12
+        del L, x, y, ws, idx, wts, lg
     del flush
     return out
 
@@ -672,7 +691,11 @@ def run_ours(args):
     del g3
 
     extras = set(args.extras.split(",")) if args.extras != "none" else set()
-    prefill = prefill_lines(m, torch, stream) if rank == 0 and "prefill" in extras else None
+    prefill = None
+    if rank == 0 and "prefill" in extras:
+        prefill = prefill_lines(m, torch, stream)
+    elif rank == 0 and "prefill947" in extras:   # the 947-token line alone (small profiling runs)
+        prefill = prefill_lines(m, torch, stream, names=("prefill_t947",))
     stack = stack_lines(m, torch, stream) if rank == 0 and "stack" in extras else None
     chunked = chunked_lines(m, torch, stream) if rank == 0 and "chunked" in extras else None
     gemv = gemv_lines(m, torch, stream) if rank == 0 and "gemv" in extras else None
@@ -734,8 +757,8 @@ def main():
     ap.add_argument("--replicas", type=int, default=REPLICAS,
                     help="device copies of the decode layer the tokens rotate over (16: L2-cold)")
     ap.add_argument("--extras", default="prefill,stack,chunked,gemv,batch64,streamed,cpu",
-                    help="comma list of the extra lines (prefill, stack, chunked, gemv, batch64, streamed, cpu) "
-                         "or 'none'")
+                    help="comma list of the extra lines (prefill, prefill947, stack, chunked, gemv, batch64, "
+                         "streamed, cpu) or 'none'")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

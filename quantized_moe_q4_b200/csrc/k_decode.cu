@@ -303,29 +303,25 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     }
     __syncthreads();
 
-    // copies of this CTA's weights, issued by warp 0: gate/up chunk i = 8 gate
-    // rows + the same 8 up rows on bar_gu[i] (lane 2i + m issues matrix m);
-    // the down slice = rows n0 .. n0 + Hs, blocks 8 fp .. 8 fp + 7
+    // copies of this CTA's weights, issued by one thread: gate/up chunk i = 8
+    // gate rows + the same 8 up rows on bar_gu[i]; the down slice = rows
+    // n0 .. n0 + Hs, blocks 8 fp .. 8 fp + 7, on bar_dn
     const uint32_t chunk_bytes = (uint32_t)(8 * row_gu);
     auto issue_copies = [&](const uint8_t* Wg, const uint8_t* Wu, const CUtensorMap* dmap, int drow0) {
-        if (lane < 4) {
-            const uint32_t extra = (p.force_timeout && blockIdx.x == 0 && lane == 0) ? 16u : 0u;
-            mbar_arrive_expect_tx(&bar_gu[lane], 2u * chunk_bytes + extra);
+        for (int ch = 0; ch < 4; ++ch) {
+            const uint32_t extra = (p.force_timeout && blockIdx.x == 0 && ch == 0) ? 16u : 0u;
+            mbar_arrive_expect_tx(&bar_gu[ch], 2u * chunk_bytes + extra);
+            const size_t src = (size_t)(hb * 32 + 8 * ch) * row_gu;
+            bulk_g2s(gu_s + (size_t)(8 * ch) * row_gu, Wg + src, chunk_bytes, &bar_gu[ch]);
+            bulk_g2s(gu_s + (size_t)(32 + 8 * ch) * row_gu, Wu + src, chunk_bytes, &bar_gu[ch]);
         }
-        if (lane == 4) mbar_arrive_expect_tx(&bar_dn, (uint32_t)(Hs * DN_KB * Q4_BYTES));
-        __syncwarp();
-        if (lane < 8) {
-            const int ch = lane >> 1, m = lane & 1;
-            bulk_g2s(gu_s + (size_t)(m * 32 + 8 * ch) * row_gu, (m ? Wu : Wg) + (size_t)(hb * 32 + 8 * ch) * row_gu,
-                     chunk_bytes, &bar_gu[ch]);
-        } else if (lane == 8) {
-            for (int r0 = 0; r0 < Hs; r0 += p.box_rows)
-                tma_load_2d(dn_s + (size_t)r0 * DN_KB * Q4_BYTES, dmap, fp * DN_KB * Q4_BYTES, drow0 + r0, &bar_dn);
-        }
+        mbar_arrive_expect_tx(&bar_dn, (uint32_t)(Hs * DN_KB * Q4_BYTES));
+        for (int r0 = 0; r0 < Hs; r0 += p.box_rows)
+            tma_load_2d(dn_s + (size_t)r0 * DN_KB * Q4_BYTES, dmap, fp * DN_KB * Q4_BYTES, drow0 + r0, &bar_dn);
     };
 
     // ---- prologue: the shared expert's copies do not depend on the routing
-    if (is_shared && warp == 0) issue_copies(p.sh_gate, p.sh_up, &maps.sh_down, n0);
+    if (is_shared && tid == 0) issue_copies(p.sh_gate, p.sh_up, &maps.sh_down, n0);
 
     pdl_wait();  // logits, Q8_0 of x and the zeroed y are visible
     pdl_launch_dependents();
@@ -376,6 +372,11 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     const int my_rank = (e_me < E) ? rank : k;
     const bool chosen = part == 0 && my_rank < k;
     if (chosen) idx_s[my_rank] = e_me;
+    // the thread that found this CTA's expert issues its copies at once
+    if (!is_shared && chosen && my_rank == j) {
+        const size_t eo = (size_t)e_me * gu_stride;
+        issue_copies(p.w_gate + eo, p.w_up + eo, &maps.down, e_me * H + n0);
+    }
     // slot of a chosen expert = number of chosen experts with a lower index
     // (slots are grouped by ascending expert, as in the grouped path)
     const unsigned chosen_mask = __ballot_sync(0xffffffffu, chosen);
@@ -390,11 +391,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     }
     __syncthreads();
 
-    // ---- routed copies (warp 0); slots and softmax terms
-    if (!is_shared && warp == 0) {
-        const size_t eo = (size_t)idx_s[j] * gu_stride;
-        issue_copies(p.w_gate + eo, p.w_up + eo, &maps.down, idx_s[j] * H + n0);
-    }
+    // ---- slots and softmax terms
     if (chosen) {
         int before = __popc(chosen_mask & ((1u << lane) - 1u));
         for (int w2 = 0; w2 < warp; ++w2) before += warp_chosen[w2];

@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import rule13, workload
+from gpu_helpers import check_permutation, check_routing, rule13, teacher_forced_check, workload
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +42,28 @@ def test_streamed_matches_resident(name, T):
     y_str = m.moe_q4_ffn_forward_streamed(Lh, xd).cpu().numpy()
     ok, worst = rule13(y_str, y_res, 1e-5)
     assert ok, worst
+
+
+@pytest.mark.parametrize("name,T", [("decode_t1", 1), ("prefill_t947", 16), ("prefill_t947", None)])
+def test_streamed_against_the_oracle(name, T):
+    """The streamed layer teacher-forced against the oracle on every token:
+    its own routing (bit-exact given its logits), permutation, requantised
+    SwiGLU output (the oracle's Q8_0 of the device's h) and output."""
+    x, lw = workload(name, T=1000 if name == "decode_t1" else None)
+    x = np.ascontiguousarray(x if T is None else x[:T])
+    T = x.shape[0]
+    Lh = m.Layer.from_host_pinned(lw)
+    xd = torch.from_numpy(x).cuda()
+    y = torch.empty_like(xd)
+    ws = m.alloc_workspace(m.moe_q4_ffn_workspace_bytes(Lh, T))
+    m.moe_q4_ffn_forward_streamed(Lh, xd, y, workspace=ws)
+    torch.cuda.synchronize()
+    v = {k: t.cpu().numpy() for k, t in m.workspace_views(Lh, T, ws).items()}
+    v["y"] = y.cpu().numpy()
+    check_routing(lw, x, v)
+    check_permutation(lw, v)
+    teacher_forced_check(lw, x, v, np.arange(T))
+    assert v["status"][0] == 0
 
 
 def test_only_selected_experts_are_staged():

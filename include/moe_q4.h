@@ -132,8 +132,8 @@ size_t moe_q4_ffn_host_workspace_bytes(const moe_q4_layer* L, int64_t T_max);
  * copies): enqueues the host-to-device copy of x, the forward, and the
  * device-to-host copy of y on `stream`.  y is valid after the caller
  * synchronises the stream.  For one token with both x and y page-locked (and
- * 16-byte aligned) the copies are made by the kernels themselves: the router
- * kernel reads x and a last kernel writes y over the bus, with no copy node
+ * 16-byte aligned) the copies are made by kernels of the decode chain (a
+ * first one reads x, a last one writes y over the bus), with no copy node
  * between the kernels. */
 int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t T, float* y_host,
                             void* workspace, size_t ws_bytes, moe_q4_stream_t stream);

@@ -262,7 +262,7 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
     if ((path == MOE_Q4_PATH_AUTO || path == MOE_Q4_PATH_DECODE) && decode_eligible(L, T, dev))
         return cuda_rc(launch_decode(L, x, y, w, dbg ? dbg->h_out : nullptr, dev, ev0, ev1,
                                      dbg && dbg->force_spin_timeout, clear_status,
-                                     dbg ? dbg->decode_kernel_ns : nullptr, nullptr, s));
+                                     dbg ? dbg->decode_kernel_ns : nullptr, nullptr, nullptr, s));
 
     // grouped paths: tensor cores once experts see tens of tokens, else dp4a
     const bool tc = (path == MOE_Q4_PATH_TENSOR_CORE) || (path == MOE_Q4_PATH_TENSOR_CORE_N32) ||
@@ -411,15 +411,15 @@ int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t 
     DeviceInfo dev;
     rc = current_device(&dev);
     if (rc) return rc;
-    // one token with page-locked x and y: the decode kernels read x and write
-    // y over the bus themselves, so the call stays one programmatic-launch
+    // one token with page-locked x and y: kernels of the decode chain copy x
+    // in and y out over the bus, so the call stays one programmatic-launch
     // chain (a copy node would end it)
     const LayerView Lv = view(L);
     if (T == 1 && decode_eligible(Lv, T, dev) && aligned(x_host, 16) && aligned(y_host, 16) && pinned_host(x_host) &&
         pinned_host(y_host)) {
         const Workspace w = carve(workspace, off);
-        return cuda_rc(launch_decode(Lv, x_host, y_dev, w, nullptr, dev, nullptr, nullptr, false, true, nullptr,
-                                     y_host, s));
+        return cuda_rc(launch_decode(Lv, x_dev, y_dev, w, nullptr, dev, nullptr, nullptr, false, true, nullptr,
+                                     x_host, y_host, s));
     }
     MOE_TRY(cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s));
     rc = forward_impl(L, x_dev, T, y_dev, workspace, off[WS_TOTAL], nullptr, s);

@@ -526,9 +526,19 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
 }
 
 // ---------------------------------------------------------------------------
-// K3 (host entry only): y copied to page-locked host memory by the GPU, so the
-// call stays one programmatic-launch chain with no copy node in it.
+// K0 / K3 (host entry only): x copied from and y copied to page-locked host
+// memory by the GPU, so the call stays one programmatic-launch chain with no
+// copy node in it (one CTA reads x over the bus once; the router's CTAs then
+// read the device copy).
 // ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) decode_copy_in_kernel(const float* __restrict__ x_host, float* __restrict__ x,
+                                                             int H) {
+    pdl_launch_dependents();
+    pdl_wait();  // the previous call's kernels no longer read x
+    for (int i = threadIdx.x; i < H / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(x)[i] = reinterpret_cast<const float4*>(x_host)[i];
+}
+
 __global__ void __launch_bounds__(256) decode_copy_out_kernel(const float* __restrict__ y, float* __restrict__ y_host,
                                                               int H) {
     pdl_launch_dependents();
@@ -587,7 +597,8 @@ bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev) {
 
 cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Workspace& ws, float* h_dbg,
                           const DeviceInfo& dev, cudaEvent_t ev_start, cudaEvent_t ev_stop, bool force_timeout,
-                          bool clear_status, unsigned long long* kernel_ns, float* y_host, cudaStream_t s) {
+                          bool clear_status, unsigned long long* kernel_ns, const float* x_host, float* y_host,
+                          cudaStream_t s) {
     DecodeParams p;
     p.H = L.H; p.F = L.F; p.E = L.E; p.k = L.k; p.S = L.S;
     p.nF = L.F / (CL * QK);
@@ -624,6 +635,16 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
     attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attrs[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
+    cfg.stream = s;
+    cfg.attrs = attrs;
+    if (x_host) {
+        cfg.gridDim = dim3(1);
+        cfg.blockDim = dim3(256);
+        cfg.dynamicSmemBytes = 0;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, decode_copy_in_kernel, x_host, const_cast<float*>(x), L.H);
+        if (e != cudaSuccess) return e;
+    }
     cfg.gridDim = dim3((unsigned)L.E);
     cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = smem1;

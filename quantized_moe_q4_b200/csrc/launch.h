@@ -96,12 +96,13 @@ bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev);
 // never arrive (the bounded wait runs out; used only to test the timeout report).
 // clear_status: zero the status word (else the kernels only OR into it).
 // kernel_ns (may be NULL): [0] += the FFN kernel's span in CTA 0 (globaltimer
-// ns, entry to exit), [1] += 1, per launch.  y_host (may be NULL): page-locked
-// host memory that a third kernel of the chain copies y into (x may then be
-// page-locked host memory too: the router kernel reads it in place).
+// ns, entry to exit), [1] += 1, per launch.  x_host / y_host (may be NULL):
+// page-locked host memory that a first kernel of the chain copies into x (a
+// device buffer then) / a last kernel copies y into.
 cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Workspace& ws, float* h_dbg,
                           const DeviceInfo& dev, cudaEvent_t ev_start, cudaEvent_t ev_stop, bool force_timeout,
-                          bool clear_status, unsigned long long* kernel_ns, float* y_host, cudaStream_t s);
+                          bool clear_status, unsigned long long* kernel_ns, const float* x_host, float* y_host,
+                          cudaStream_t s);
 
 cudaError_t launch_block_dots(const uint8_t* w, const int8_t* qa, int64_t n, int32_t* out,
                               cudaStream_t s);

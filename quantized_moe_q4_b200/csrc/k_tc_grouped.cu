@@ -73,6 +73,11 @@ constexpr int W_PROD = 0, W_CONV0 = 1, W_MMA = 5, W_EPI0 = 6;
 constexpr uint32_t LIMIT = 1u << 22;
 constexpr size_t SZ_IN_W = (size_t)TM * IN_ROW;           // one input stage of packed weight rows
 constexpr size_t SZ_OP_A = (size_t)OP_KB * 2 * TM * 32;   // one operand stage of A (K-steps of 16 x binary16)
+// Activation prefetch ring of the converters: NPF operand stages, a slot's 2
+// blocks of int8 codes (64 B) and their 2 binary16 scales (4 B) per entry,
+// copied by the thread that converts them (cp.async), PF stages ahead.
+constexpr int NPF = 4, PF = 3;
+constexpr size_t BPF_SLOT = 80;
 
 // Per tile width TN (slots, the MMA N): the epilogue has TN/32 column groups
 // of 4 warps (one per TMEM lane quarter), and the shared-memory map.
@@ -90,9 +95,10 @@ struct TcCfg {
     static constexpr size_t OFF_DW = OFF_OP_B + NOP * SZ_OP_B;
     static constexpr size_t OFF_DA = OFF_DW + (size_t)NSC * OP_KB * TM * 4;
     static constexpr size_t OFF_XCH = OFF_DA + (size_t)NSC * OP_KB * TN * 4;
-    static constexpr size_t SMEM_BYTES = OFF_XCH + (size_t)TM * XCH_LD * 4;
+    static constexpr size_t OFF_BPF = OFF_XCH + (size_t)TM * XCH_LD * 4;
+    static constexpr size_t SMEM_BYTES = OFF_BPF + (size_t)NPF * TN * BPF_SLOT;
     static constexpr size_t SMEM_ALLOC = SMEM_BYTES + 1024;   // slack to align the map to 1024 B
-    static_assert(SMEM_ALLOC <= 200 * 1024, "shared memory map too large");
+    static_assert(SMEM_ALLOC <= 220 * 1024, "shared memory map too large");
 };
 
 enum { GATEUP = 0, DOWN = 1 };
@@ -166,10 +172,46 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// this thread's copies of all but the newest N committed groups have landed
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // y[0..3] += v (one vector reduction at L2; y 16-byte aligned)
 __device__ __forceinline__ void red_add_v4(float* y, float4 v) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(y), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
                  : "memory");
+}
+
+// 16 consecutive 32-bit columns of this warp's 32 TMEM lanes (lane = row).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+// acc[slot pair h8 + j] += I (16 columns of one block) * dW * dA[slot].
+__device__ __forceinline__ void rescale_acc16(float2 (&acc)[16], int h8, const uint32_t (&r)[16], float dwv,
+                                              const float* da) {
+    const float4* da4 = reinterpret_cast<const float4*>(da);
+    const float2 dw2 = make_float2(dwv, dwv);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float4 d = da4[j];
+        const float2 s0 = __fmul2_rn(dw2, make_float2(d.x, d.y));
+        const float2 s1 = __fmul2_rn(dw2, make_float2(d.z, d.w));
+        acc[h8 + 2 * j] =
+            __ffma2_rn(make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), s0, acc[h8 + 2 * j]);
+        acc[h8 + 2 * j + 1] = __ffma2_rn(make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), s1,
+                                         acc[h8 + 2 * j + 1]);
+    }
 }
 
 // acc[slot pair j] += I (32 columns of one block) * dW * dA[slot].
@@ -401,40 +443,63 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
         if (i_in > 0) mbar_wait_bounded(&in_full[(i_in - 1) % NIN], ((i_in - 1) / NIN) & 1, LIMIT);
     } else if (warp >= W_CONV0 && warp < W_CONV0 + 4) {
         // ------------------------------------------------------------ converters
-        // thread ct converts weight row ct and (ct < TN) the activations of slot ct
+        // thread ct converts weight row ct and (ct < TN) the activations of
+        // slot ct; it copies those activations PF operand stages ahead into
+        // its own entries of the prefetch ring (cp.async: no registers held,
+        // no wait on L2 in the loop)
         const int ct = tid - W_CONV0 * 32;
+        uint8_t* bpf = smem + C::OFF_BPF;
+        const int nst = nbK / OP_KB;                      // operand stages per item
+        // the prefetch cursor: item, stage, and this slot's rows (NULL: no slot)
+        int pf_item = blockIdx.x, pf_c = 0;
+        const int8_t* pf_arow = nullptr;
+        const uint16_t* pf_ascale = nullptr;
+        auto pf_rows = [&](int item) {
+            pf_arow = nullptr;
+            pf_ascale = nullptr;
+            if (item >= n_items || ct >= TN) return;
+            const Tile Tn = tile_of<TN>(item, n_rb, tile_off_s, off_s, ngroups);
+            if (ct >= Tn.nslots) return;
+            const int sl = Tn.slot0 + ct;
+            int tok;
+            float w;
+            slot_info(p, Tn.g, sl, tok, w);
+            if (MODE == GATEUP) {
+                pf_arow = p.qa + (size_t)tok * H;
+                pf_ascale = p.da + (size_t)tok * (H / QK);
+            } else {
+                pf_arow = p.hq + (size_t)sl * F;
+                pf_ascale = p.dh + (size_t)sl * nbF;
+            }
+        };
+        uint32_t i_pf = 0;
+        auto pf_issue = [&]() {   // one operand stage ahead, always one commit group
+            if (pf_item < n_items && pf_arow) {
+                uint8_t* dst = bpf + ((size_t)(i_pf % NPF) * TN + ct) * BPF_SLOT;
+                const int8_t* src = pf_arow + (size_t)pf_c * OP_KB * QK;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) cp_async16(dst + 16 * i, src + 16 * i);
+                cp_async4(dst + 64, pf_ascale + pf_c * OP_KB);
+            }
+            cp_async_commit();
+            ++i_pf;
+            if (++pf_c == nst) {
+                pf_c = 0;
+                pf_item += gridDim.x;
+                pf_rows(pf_item);
+            }
+        };
+        pf_rows(pf_item);
+#pragma unroll 1
+        for (int i = 0; i < PF; ++i) pf_issue();
+
         uint32_t i_op = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const Tile T = tile_of<TN>(item, n_rb, tile_off_s, off_s, ngroups);
             const bool valid = ct < T.nslots;
-            const int8_t* arow = nullptr;
-            const uint16_t* ascale = nullptr;
-            if (valid) {
-                const int sl = T.slot0 + ct;
-                int tok;
-                float w;
-                slot_info(p, T.g, sl, tok, w);
-                if (MODE == GATEUP) {
-                    arow = p.qa + (size_t)tok * H;
-                    ascale = p.da + (size_t)tok * (H / QK);
-                } else {
-                    arow = p.hq + (size_t)sl * F;
-                    ascale = p.dh + (size_t)sl * nbF;
-                }
-            }
-            for (int c = 0; c < nbK / OP_KB && ok; ++c, ++i_op) {
-                // this slot's 2 blocks of activations and their scales: the
-                // loads are in flight while the stages below are awaited
-                uint4 a[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
-                              make_uint4(0, 0, 0, 0)};
-                uint32_t dab = 0;
-                if (valid) {
-                    const uint4* src = reinterpret_cast<const uint4*>(arow + (size_t)c * OP_KB * QK);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) a[i] = __ldcg(src + i);
-                    dab = __ldcg(reinterpret_cast<const uint32_t*>(ascale + c * OP_KB));
-                }
+            for (int c = 0; c < nst && ok; ++c, ++i_op) {
+                pf_issue();                                   // stage i_op + PF
                 const uint32_t i_in = i_op / (IN_KB / OP_KB);
                 const int s = i_in % NIN, sub = i_op % (IN_KB / OP_KB);
                 if (sub == 0 && !wait_phase(&in_full[s], (i_in / NIN) & 1, abort)) { ok = false; break; }
@@ -463,12 +528,20 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     for (int i = 0; i < 4; ++i) qs[i] = w[5 + i];
                     store_weights(oa, 1, ct, qs);
                 }
-                // activations of slot ct (zeros past the tile's slots)
+                // activations of slot ct from the ring (zeros past the tile's slots)
+                uint32_t dab = 0;
+                cp_async_wait_group<PF>();                    // this thread's stage i_op has landed
                 if (ct < TN) {
+                    const uint8_t* src = bpf + ((size_t)(i_op % NPF) * TN + ct) * BPF_SLOT;
 #pragma unroll
                     for (int kb = 0; kb < OP_KB; ++kb)
 #pragma unroll
-                        for (int ks = 0; ks < 2; ++ks) store_act16(ob, TN, kb, ks, ct, a[2 * kb + ks]);
+                        for (int ks = 0; ks < 2; ++ks) {
+                            const uint4 a = valid ? *reinterpret_cast<const uint4*>(src + 16 * (2 * kb + ks))
+                                                  : make_uint4(0, 0, 0, 0);
+                            store_act16(ob, TN, kb, ks, ct, a);
+                        }
+                    if (valid) dab = *reinterpret_cast<const uint32_t*>(src + 64);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
@@ -487,6 +560,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 if (lane == 0) mbar_arrive(&sc_full[sc]);
             }
         }
+        cp_async_wait_all();   // the prefetches past the last stage land before the CTA exits
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -558,29 +632,43 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     break;
                 }
                 tc_fence_after_sync();
+                // four chunks of 16 columns (2 blocks x 2 halves), software
+                // pipelined: the TMEM load of chunk q + 1 is in flight while
+                // chunk q is rescaled; the accumulator pair is released as soon
+                // as its last chunk is in registers
+                uint32_t rA[16], rB[16];
+                tmem_ld16(taddr + (OP_KB * pr) * TN, rA);
+                tmem_wait_ld();
 #pragma unroll
-                for (int kb = 0; kb < OP_KB; ++kb) {
-                    uint32_t r[32];
-                    tmem_ld32(taddr + (OP_KB * pr + kb) * TN, r);
-                    tmem_wait_ld();
+                for (int qc = 0; qc < 2 * OP_KB; ++qc) {
+                    const int kb = qc >> 1, hf = qc & 1;
+                    if (qc + 1 < 2 * OP_KB) {
+                        const int kb1 = (qc + 1) >> 1, hf1 = (qc + 1) & 1;
+                        tmem_ld16(taddr + (OP_KB * pr + kb1) * TN + 16 * hf1, (qc & 1) ? rA : rB);
+                    }
+                    const uint32_t(&r)[16] = (qc & 1) ? rB : rA;
                     if (CAP && T.g == p.cap_group && T.rb == p.cap_rb) {
                         // exact integers held in binary32: convert back without rounding
                         const size_t s0 = (size_t)(T.slot0 - off_s[T.g]);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int n = 32 * cq + j;
+                        for (int j = 0; j < 16; ++j) {
+                            const int n = 32 * cq + 16 * hf + j;
                             if (n < T.nslots)
                                 p.cap_out[((s0 + n) * TM + row) * nbK + b + kb] = __float2int_rn(__uint_as_float(r[j]));
                         }
                     }
-                    rescale_acc(acc, r, dw_ring[(sc * OP_KB + kb) * TM + row], da_ring + (sc * OP_KB + kb) * TN + 32 * cq);
+                    rescale_acc16(acc, 8 * hf, r, dw_ring[(sc * OP_KB + kb) * TM + row],
+                                  da_ring + (sc * OP_KB + kb) * TN + 32 * cq + 16 * hf);
+                    if (qc + 1 < 2 * OP_KB) tmem_wait_ld();
+                    if (qc + 2 == 2 * OP_KB) {
+                        // every chunk of the pair is loaded: the accumulators are free
+                        tc_fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tm_empty[pr]);
+                    }
                 }
-                tc_fence_before_sync();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&tm_empty[pr]);
-                    mbar_arrive(&sc_empty[sc]);
-                }
+                if (lane == 0) mbar_arrive(&sc_empty[sc]);
             }
             if (!ok) break;
             // this thread's row x 32 slots into the exchange tile
@@ -761,10 +849,12 @@ static cudaError_t launch_tc(const LayerView& L, int64_t T, const Workspace& ws,
 
 int tc_tile_tokens(const LayerView& L, int64_t T, int force) {
     if (force == 32 || force == 128) return force;
-    // routed slots per expert on average: narrow tiles while most experts
-    // hold only a few tokens (decode batches), wide ones for prompts
-    const int64_t per_expert = T * L.k / L.E;
-    return per_expert >= 64 ? 128 : 32;
+    // measured on B200 (2048/512, 128 experts top-8 + shared): 128-slot tiles
+    // are faster from 947 tokens (59 routed slots per expert) up; below 128
+    // tokens the automatic choice does not use the tensor cores at all
+    (void)L;
+    (void)T;
+    return 128;
 }
 
 cudaError_t launch_gateup_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, const DeviceInfo& dev,

@@ -280,7 +280,8 @@ def prefill_lines(m, torch, stream, names=("prefill_t947", "zipf_t16384")):
     out = {}
     peak, peak_src = int8_peak_tops()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    variants = (("auto", m.PATH_AUTO), ("tc_n32", m.PATH_TENSOR_CORE_N32), ("tc_n128", m.PATH_TENSOR_CORE_N128))
+    variants = (("auto", m.PATH_AUTO), ("tc_n32", m.PATH_TENSOR_CORE_N32), ("tc_n64", m.PATH_TENSOR_CORE_N64),
+                ("tc_n128", m.PATH_TENSOR_CORE_N128))
     for name in names:
         x_np, lw = synth.workload_inputs(name, seed=0)
         L = m.Layer.from_host(lw)

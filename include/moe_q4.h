@@ -286,7 +286,8 @@ enum {
     MOE_Q4_PATH_DECODE = 2,
     MOE_Q4_PATH_TENSOR_CORE = 3,     /* tensor cores, tile width chosen by T */
     MOE_Q4_PATH_TENSOR_CORE_N32 = 4, /* tensor cores, tiles of 32 slots */
-    MOE_Q4_PATH_TENSOR_CORE_N128 = 5 /* tensor cores, tiles of 128 slots */
+    MOE_Q4_PATH_TENSOR_CORE_N128 = 5, /* tensor cores, tiles of 128 slots */
+    MOE_Q4_PATH_TENSOR_CORE_N64 = 6   /* tensor cores, tiles of 64 slots */
 };
 
 typedef struct {

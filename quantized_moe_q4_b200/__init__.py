@@ -37,7 +37,7 @@ STATUS_NONFINITE_LOGIT = 0x4
 STATUS_BAD_EXPERT_INDEX = 0x8
 
 PATH_AUTO, PATH_GROUPED_DP4A, PATH_DECODE, PATH_TENSOR_CORE = 0, 1, 2, 3
-PATH_TENSOR_CORE_N32, PATH_TENSOR_CORE_N128 = 4, 5
+PATH_TENSOR_CORE_N32, PATH_TENSOR_CORE_N128, PATH_TENSOR_CORE_N64 = 4, 5, 6
 
 WS_NAMES = ["status", "logits", "topk_idx", "topk_w", "qa", "da", "cnt", "off", "tile_off",
             "chunk_cnt", "chunk_base", "sorted", "pos", "hq", "dh", "sync", "total"]

@@ -266,8 +266,10 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
 
     // grouped paths: tensor cores once experts see tens of tokens, else dp4a
     const bool tc = (path == MOE_Q4_PATH_TENSOR_CORE) || (path == MOE_Q4_PATH_TENSOR_CORE_N32) ||
-                    (path == MOE_Q4_PATH_TENSOR_CORE_N128) || (path == MOE_Q4_PATH_AUTO && T >= TC_MIN_TOKENS);
+                    (path == MOE_Q4_PATH_TENSOR_CORE_N64) || (path == MOE_Q4_PATH_TENSOR_CORE_N128) ||
+                    (path == MOE_Q4_PATH_AUTO && T >= TC_MIN_TOKENS);
     const int tile = tc ? tc_tile_tokens(L, T, path == MOE_Q4_PATH_TENSOR_CORE_N32    ? 32
+                                               : path == MOE_Q4_PATH_TENSOR_CORE_N64  ? 64
                                                : path == MOE_Q4_PATH_TENSOR_CORE_N128 ? 128
                                                                                       : 0)
                         : DP4A_TT;
@@ -380,7 +382,7 @@ int moe_q4_ffn_forward(const moe_q4_layer* L, const float* x, int64_t T, float* 
 
 int moe_q4_ffn_forward_debug(const moe_q4_layer* L, const float* x, int64_t T, float* y, void* workspace,
                              size_t ws_bytes, const moe_q4_debug* dbg, moe_q4_stream_t stream) {
-    if (dbg && (dbg->path < MOE_Q4_PATH_AUTO || dbg->path > MOE_Q4_PATH_TENSOR_CORE_N128)) return MOE_Q4_ERR_INVALID_ARG;
+    if (dbg && (dbg->path < MOE_Q4_PATH_AUTO || dbg->path > MOE_Q4_PATH_TENSOR_CORE_N64)) return MOE_Q4_ERR_INVALID_ARG;
     return forward_impl(L, x, T, y, workspace, ws_bytes, dbg, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -155,6 +155,18 @@ __device__ __forceinline__ void block_rows(const uint8_t* rows, size_t row_bytes
     }
 }
 
+// block_rows with the activation block already in registers.
+template <int NR>
+__device__ __forceinline__ void block_rows_reg(const uint8_t* rows, size_t row_bytes, const int (&qa)[8], int qsum,
+                                               float da, float (&acc)[NR]) {
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        uint32_t qs[4], dbits;
+        load_q4_block_smem(rows + (size_t)r * row_bytes, qs, dbits);
+        acc[r] = fmaf((float)q4_q8_dot(qs, qa, qsum), half_bits_to_float(dbits) * da, acc[r]);
+    }
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
@@ -265,9 +277,6 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     __shared__ int slot_s[17];
     __shared__ int warp_chosen[FFN_WARPS];
     __shared__ float gs[32], us[32];
-    __shared__ __align__(16) int8_t hx_q[CL][QK];   // the group's 8 requantised h blocks
-    __shared__ float hx_d[CL];
-    __shared__ int hx_sum[CL];
     __shared__ int flags_s;
 
     unsigned long long t_entry = 0;
@@ -455,7 +464,8 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
             p.dh[(size_t)slot * nbF + hb] = db;
             if (ov) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
         }
-        __threadfence();
+        // the warp barrier orders every lane's stores before lane 0's release
+        // (cumulative, device scope), which the readers acquire
         __syncwarp();
         if (lane == 0) red_release_add_gpu(p.group_cnt + c, 1u);
     }
@@ -472,37 +482,24 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
         }
     }
     __syncthreads();
-    if (tid < CL * QK / 16) {
-        const int b = tid >> 1;
-        reinterpret_cast<int4*>(&hx_q[b][0])[tid & 1] =
-            __ldcg(reinterpret_cast<const int4*>(p.hq + (size_t)slot * F + (fp * CL + b) * QK) + (tid & 1));
-    } else if (tid >= 32 && tid < 32 + CL) {
-        hx_d[tid - 32] = half_bits_to_float(__ldcg(p.dh + (size_t)slot * nbF + fp * CL + (tid - 32)));
-    }
-    __syncthreads();
-    if (tid < CL) {
-        const int* qw = reinterpret_cast<const int*>(&hx_q[tid][0]);
-        int sq = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sq = __dp4a(qw[i], 0x01010101, sq);
-        hx_sum[tid] = sq;
-    }
-    __syncthreads();
 
     // ---- down: o[n] = sum over the group's 8 blocks, n < Hs.  A task is 4
     // rows; 8 lanes share a task, one block each, and add with a butterfly.
-    if (!mbar_wait_bounded(&bar_dn, 0, MBAR_LIMIT)) timed_out = true;
+    // Lane block kb: its 32 codes and scale straight from L2 into registers.
     {
         const int kb = lane & 7, grp = lane >> 3;
+        const int4* hsrc = reinterpret_cast<const int4*>(p.hq + (size_t)slot * F + (fp * CL + kb) * QK);
+        const int4 h0 = __ldcg(hsrc), h1 = __ldcg(hsrc + 1);
+        const float dv = half_bits_to_float(__ldcg(p.dh + (size_t)slot * nbF + fp * CL + kb));
+        const int hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+        const int qsum = q8_block_sum(hv);
+        if (!mbar_wait_bounded(&bar_dn, 0, MBAR_LIMIT)) timed_out = true;
         const size_t row_dn = (size_t)DN_KB * Q4_BYTES;
-        const int qsum = hx_sum[kb];
-        const float dv = hx_d[kb];
         for (int t0 = 0; t0 < Hs; t0 += FFN_WARPS * 16) {
             const int row0 = t0 + warp * 16 + grp * 4;
             float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             if (row0 < Hs)
-                block_rows<4>(dn_s + (size_t)row0 * row_dn + (size_t)kb * Q4_BYTES, row_dn, &hx_q[kb][0], qsum, dv,
-                              acc);
+                block_rows_reg<4>(dn_s + (size_t)row0 * row_dn + (size_t)kb * Q4_BYTES, row_dn, hv, qsum, dv, acc);
             const float s = butterfly<4, 8>(acc);
             if (bf_owner<4, 8>(kb) && row0 < Hs) o_s[row0 + bf_index<4, 8>(kb)] = s;
         }

@@ -83,9 +83,12 @@ constexpr size_t BPF_SLOT = 80;
 // of 4 warps (one per TMEM lane quarter), and the shared-memory map.
 template <int TN>
 struct TcCfg {
-    static_assert(TN == 32 || TN == 128, "tile widths");
-    static constexpr int N_EPI = 4 * TN;
-    static constexpr int THREADS = 6 * 32 + N_EPI;        // TN = 128: 704, at most 80 registers a thread
+    static_assert(TN == 32 || TN == 64 || TN == 128, "tile widths");
+    // epilogue: a thread owns one accumulator row x CW columns; 4 warps (the
+    // TMEM lane quarters) per CW-wide column group
+    static constexpr int CW = (TN == 128) ? 64 : 32;
+    static constexpr int N_EPI = 4 * (TN / CW) * 32;
+    static constexpr int THREADS = 6 * 32 + N_EPI;        // at most 14 warps: up to 128 registers a thread
     static constexpr uint32_t TMEM_COLS = NACC * TN;      // 512 or 128 columns
     static constexpr size_t SZ_OP_B = (size_t)OP_KB * 2 * TN * 32;
     static constexpr int XCH_LD = TN + 1;
@@ -198,7 +201,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 
 // acc[slot pair h8 + j] += I (16 columns of one block) * dW * dA[slot].
-__device__ __forceinline__ void rescale_acc16(float2 (&acc)[16], int h8, const uint32_t (&r)[16], float dwv,
+template <int NA>
+__device__ __forceinline__ void rescale_acc16(float2 (&acc)[NA], int h8, const uint32_t (&r)[16], float dwv,
                                               const float* da) {
     const float4* da4 = reinterpret_cast<const float4*>(da);
     const float2 dw2 = make_float2(dwv, dwv);
@@ -211,21 +215,6 @@ __device__ __forceinline__ void rescale_acc16(float2 (&acc)[16], int h8, const u
             __ffma2_rn(make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), s0, acc[h8 + 2 * j]);
         acc[h8 + 2 * j + 1] = __ffma2_rn(make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), s1,
                                          acc[h8 + 2 * j + 1]);
-    }
-}
-
-// acc[slot pair j] += I (32 columns of one block) * dW * dA[slot].
-__device__ __forceinline__ void rescale_acc(float2 (&acc)[16], const uint32_t (&r)[32], float dwv, const float* da) {
-    const float4* da4 = reinterpret_cast<const float4*>(da);
-    const float2 dw2 = make_float2(dwv, dwv);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const float4 d = da4[j];
-        const float2 s0 = __fmul2_rn(dw2, make_float2(d.x, d.y));
-        const float2 s1 = __fmul2_rn(dw2, make_float2(d.z, d.w));
-        acc[2 * j] = __ffma2_rn(make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), s0, acc[2 * j]);
-        acc[2 * j + 1] =
-            __ffma2_rn(make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), s1, acc[2 * j + 1]);
     }
 }
 
@@ -353,7 +342,7 @@ template <int MODE, int TN, bool CAP>
 __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
     tc_grouped_kernel(TcParams p, const __grid_constant__ TcMaps maps) {
     using C = TcCfg<TN>;
-    constexpr int N_EPI = C::N_EPI, THREADS = C::THREADS, XCH_LD = C::XCH_LD;
+    constexpr int N_EPI = C::N_EPI, THREADS = C::THREADS, XCH_LD = C::XCH_LD, CW = C::CW, NCH = CW / 16;
     constexpr uint32_t TMEM_COLS = C::TMEM_COLS;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -605,9 +594,9 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
         // ------------------------------------------------------------ epilogue
         const int et = tid - W_EPI0 * 32;         // 0 .. N_EPI - 1
         const int q = warp & 3;                   // TMEM lane quarter this warp may access
-        const int cq = (warp - W_EPI0) >> 2;      // column quarter: slots 32 cq .. 32 cq + 31
+        const int cq = (warp - W_EPI0) >> 2;      // column group: slots CW cq .. CW cq + CW - 1
         const int row = 32 * q + lane;            // weight row (TMEM lane) of this thread
-        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + 32 * cq;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + CW * cq;
         uint32_t i_op = 0, epi_phase = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -621,9 +610,9 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 tok_s[et] = tok;
                 wt_s[et] = w;
             }
-            float2 acc[16];
+            float2 acc[CW / 2];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) acc[j] = make_float2(0.0f, 0.0f);
+            for (int j = 0; j < CW / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
             for (int b = 0; b < nbK; b += OP_KB, ++i_op) {
                 const uint32_t pr = i_op & 1, ppar = (i_op >> 1) & 1;
                 const uint32_t sc = i_op % NSC, spar = (i_op / NSC) & 1;
@@ -632,18 +621,18 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     break;
                 }
                 tc_fence_after_sync();
-                // four chunks of 16 columns (2 blocks x 2 halves), software
-                // pipelined: the TMEM load of chunk q + 1 is in flight while
-                // chunk q is rescaled; the accumulator pair is released as soon
-                // as its last chunk is in registers
+                // chunks of 16 columns (2 blocks x CW / 16), software pipelined:
+                // the TMEM load of chunk qc + 1 is in flight while chunk qc is
+                // rescaled; the accumulator pair is released as soon as its
+                // last chunk is in registers
                 uint32_t rA[16], rB[16];
                 tmem_ld16(taddr + (OP_KB * pr) * TN, rA);
                 tmem_wait_ld();
 #pragma unroll
-                for (int qc = 0; qc < 2 * OP_KB; ++qc) {
-                    const int kb = qc >> 1, hf = qc & 1;
-                    if (qc + 1 < 2 * OP_KB) {
-                        const int kb1 = (qc + 1) >> 1, hf1 = (qc + 1) & 1;
+                for (int qc = 0; qc < NCH * OP_KB; ++qc) {
+                    const int kb = qc / NCH, hf = qc % NCH;
+                    if (qc + 1 < NCH * OP_KB) {
+                        const int kb1 = (qc + 1) / NCH, hf1 = (qc + 1) % NCH;
                         tmem_ld16(taddr + (OP_KB * pr + kb1) * TN + 16 * hf1, (qc & 1) ? rA : rB);
                     }
                     const uint32_t(&r)[16] = (qc & 1) ? rB : rA;
@@ -652,15 +641,15 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                         const size_t s0 = (size_t)(T.slot0 - off_s[T.g]);
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const int n = 32 * cq + 16 * hf + j;
+                            const int n = CW * cq + 16 * hf + j;
                             if (n < T.nslots)
                                 p.cap_out[((s0 + n) * TM + row) * nbK + b + kb] = __float2int_rn(__uint_as_float(r[j]));
                         }
                     }
                     rescale_acc16(acc, 8 * hf, r, dw_ring[(sc * OP_KB + kb) * TM + row],
-                                  da_ring + (sc * OP_KB + kb) * TN + 32 * cq + 16 * hf);
-                    if (qc + 1 < 2 * OP_KB) tmem_wait_ld();
-                    if (qc + 2 == 2 * OP_KB) {
+                                  da_ring + (sc * OP_KB + kb) * TN + CW * cq + 16 * hf);
+                    if (qc + 1 < NCH * OP_KB) tmem_wait_ld();
+                    if (qc + 2 == NCH * OP_KB) {
                         // every chunk of the pair is loaded: the accumulators are free
                         tc_fence_before_sync();
                         __syncwarp();
@@ -671,10 +660,10 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 if (lane == 0) mbar_arrive(&sc_empty[sc]);
             }
             if (!ok) break;
-            // this thread's row x 32 slots into the exchange tile
-            float* xr = xch + (size_t)row * XCH_LD + 32 * cq;
+            // this thread's row x CW slots into the exchange tile
+            float* xr = xch + (size_t)row * XCH_LD + CW * cq;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < CW / 2; ++j) {
                 xr[2 * j] = acc[j].x;
                 xr[2 * j + 1] = acc[j].y;
             }
@@ -685,7 +674,8 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 // rows each, so every value is independent of the others and a
                 // single shuffle gives the block's absolute maximum.  Both
                 // divisions of the Q8_0 rule stay IEEE (div.rn).
-                const int u = et >> 1;                    // 0 .. 2 TN - 1
+#pragma unroll 1
+                for (int u = et >> 1; u < 2 * TN; u += N_EPI / 2) {   // 2 TN units
                 const int n = u % TN, fb = u / TN, half = lane & 1;
                 const int r0 = 32 * fb + 16 * half;
                 const int f0 = T.rb * 64;
@@ -718,6 +708,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                         p.dh[(size_t)sl * nbF + (f0 >> 5) + fb] = dbits;
                         if ((dbits & 0x7fffu) == 0x7c00u) atomicOr(p.status, STATUS_SCALE_OVERFLOW);
                     }
+                }
                 }
             } else {
                 // y[token][h0 + 4 i .. + 3] += w * o: one vector reduction per
@@ -830,7 +821,7 @@ static cudaError_t launch_tc_inst(const LayerView& L, int64_t T, const TcParams&
 template <int MODE>
 static cudaError_t launch_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, float* y,
                              const DeviceInfo& dev, int tile, const BlockDotCapture* cap, cudaStream_t s) {
-    if (tile != 32 && tile != 128) return cudaErrorInvalidValue;
+    if (tile != 32 && tile != 64 && tile != 128) return cudaErrorInvalidValue;
     const bool capture = cap && cap->down == (MODE == DOWN ? 1 : 0);
     TcMaps maps;
     cudaError_t e = make_maps<MODE>(L, &maps);
@@ -841,20 +832,20 @@ static cudaError_t launch_tc(const LayerView& L, int64_t T, const Workspace& ws,
         p.cap_group = cap->group;
         p.cap_rb = cap->rb;
         return tile == 128 ? launch_tc_inst<MODE, 128, true>(L, T, p, maps, dev, s)
-                           : launch_tc_inst<MODE, 32, true>(L, T, p, maps, dev, s);
+               : tile == 64 ? launch_tc_inst<MODE, 64, true>(L, T, p, maps, dev, s)
+                            : launch_tc_inst<MODE, 32, true>(L, T, p, maps, dev, s);
     }
     return tile == 128 ? launch_tc_inst<MODE, 128, false>(L, T, p, maps, dev, s)
-                       : launch_tc_inst<MODE, 32, false>(L, T, p, maps, dev, s);
+           : tile == 64 ? launch_tc_inst<MODE, 64, false>(L, T, p, maps, dev, s)
+                        : launch_tc_inst<MODE, 32, false>(L, T, p, maps, dev, s);
 }
 
 int tc_tile_tokens(const LayerView& L, int64_t T, int force) {
-    if (force == 32 || force == 128) return force;
-    // measured on B200 (2048/512, 128 experts top-8 + shared): 128-slot tiles
-    // are faster from 947 tokens (59 routed slots per expert) up; below 128
-    // tokens the automatic choice does not use the tensor cores at all
-    (void)L;
-    (void)T;
-    return 128;
+    if (force == 32 || force == 64 || force == 128) return force;
+    // routed slots per expert on average: the tile the average expert fills
+    // (64 slots for a 947-token prompt's 59 per expert, 128 from 96 up)
+    const int64_t per_expert = T * L.k / L.E;
+    return per_expert >= 96 ? 128 : 64;
 }
 
 cudaError_t launch_gateup_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, const DeviceInfo& dev,

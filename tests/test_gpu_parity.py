@@ -25,8 +25,9 @@ if not torch.cuda.is_available():  # collected on CPU hosts only with -m gpu
 import quantized_moe_q4_b200 as m  # noqa: E402  (loads the CUDA library; fails loudly if missing)
 
 # every kernel family: automatic choice, streaming dp4a, fused decode (T = 1;
-# other T take the grouped paths), tensor cores with 32- and 128-slot tiles
-PATHS = [m.PATH_AUTO, m.PATH_GROUPED_DP4A, m.PATH_DECODE, m.PATH_TENSOR_CORE_N32, m.PATH_TENSOR_CORE_N128]
+# other T take the grouped paths), tensor cores with 32-, 64- and 128-slot tiles
+PATHS = [m.PATH_AUTO, m.PATH_GROUPED_DP4A, m.PATH_DECODE, m.PATH_TENSOR_CORE_N32, m.PATH_TENSOR_CORE_N64,
+         m.PATH_TENSOR_CORE_N128]
 
 
 # --------------------------------------------------------------- building blocks
@@ -209,8 +210,8 @@ def _groups_to_capture(v, E, tile):
     return sorted({ragged[0], int(np.argmax(cnt)), E})
 
 
-@pytest.mark.parametrize("path,R,tile", [(m.PATH_TENSOR_CORE_N32, 128, 32), (m.PATH_TENSOR_CORE_N128, 128, 128),
-                                         (m.PATH_GROUPED_DP4A, 64, 8)])
+@pytest.mark.parametrize("path,R,tile", [(m.PATH_TENSOR_CORE_N32, 128, 32), (m.PATH_TENSOR_CORE_N64, 128, 64),
+                                         (m.PATH_TENSOR_CORE_N128, 128, 128), (m.PATH_GROUPED_DP4A, 64, 8)])
 @pytest.mark.parametrize("down", [False, True])
 def test_block_dots_of_the_projection_kernels_bit_exact(path, R, tile, down):
     """The per-block integer sums I_b inside the grouped projection kernels
@@ -233,8 +234,8 @@ def test_block_dots_of_the_projection_kernels_bit_exact(path, R, tile, down):
             assert bad.size == 0, f"group {g} row block {rb}: {len(bad)} block sums differ, first {bad[:3]}"
 
 
-@pytest.mark.parametrize("path,R", [(m.PATH_TENSOR_CORE_N32, 128), (m.PATH_TENSOR_CORE_N128, 128),
-                                    (m.PATH_GROUPED_DP4A, 64)])
+@pytest.mark.parametrize("path,R", [(m.PATH_TENSOR_CORE_N32, 128), (m.PATH_TENSOR_CORE_N64, 128),
+                                    (m.PATH_TENSOR_CORE_N128, 128), (m.PATH_GROUPED_DP4A, 64)])
 def test_block_dots_extreme_values(path, R):
     """All nibbles 0 or 15 against activations at +-127 (Q8_0 of rows whose
     blocks hold one large value of either sign and equal smaller ones): the
@@ -346,7 +347,8 @@ def test_scale_overflow_reported_in_status():
     assert v["status"][0] & m.STATUS_SCALE_OVERFLOW
 
 
-@pytest.mark.parametrize("path", [m.PATH_GROUPED_DP4A, m.PATH_TENSOR_CORE_N32, m.PATH_TENSOR_CORE_N128])
+@pytest.mark.parametrize("path", [m.PATH_GROUPED_DP4A, m.PATH_TENSOR_CORE_N32, m.PATH_TENSOR_CORE_N64,
+                                  m.PATH_TENSOR_CORE_N128])
 def test_workspace_reuse_across_sizes(path):
     # one workspace sized for the largest T serves smaller calls; both calls
     # take the same kernel family (different families may round g or u

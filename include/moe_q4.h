@@ -155,7 +155,7 @@ int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t 
  *   - A problem whose workspace (moe_q4_ffn_workspace_bytes(L, T)) exceeds
  *     the scratch returns MOE_Q4_ERR_WORKSPACE and enqueues nothing; for a
  *     layer with hidden 2048, ffn 512, 128 experts, top-8 and a shared expert
- *     that allows T up to 199 tokens.
+ *     that allows T up to 542 tokens.
  *   - The first call on a device looks up the scratch's device address (once
  *     per device, with that device current); make that first call before any
  *     stream capture.
@@ -264,9 +264,7 @@ const char* moe_q4_last_cuda_error(void);
  *   | qa i8[T][H] | da u16[T][H/32] | cnt i32[E+1] | off i32[E+2]
  *   | tile_off i32[E+2] | chunk_cnt i32[C][E] | chunk_base i32[C][E]
  *   | sorted i32[P] | pos i32[P] | hq i8[P+S*T][F] | dh u16[P+S*T][F/32]
- *   | sync u32[(k+S)*F/256] | qa16 u16[T][H] | hq16 u16[P+S*T][F] | total
- * (qa16 and hq16: the codes of qa and hq as binary16, written and read by the
- * tensor-core path only)
+ *   | sync u32[(k+S)*F/256] | total
  * with P = T*k routed pairs and S = has_shared.  Slots (rows of hq/dh) are
  * grouped by expert: routed expert e owns slots off[e]..off[e+1]-1 holding
  * pairs sorted[...] = t*k+j in increasing (t, j) order; the shared expert
@@ -277,7 +275,7 @@ enum {
     MOE_Q4_WS_STATUS = 0, MOE_Q4_WS_LOGITS, MOE_Q4_WS_TOPK_IDX, MOE_Q4_WS_TOPK_W, MOE_Q4_WS_QA,
     MOE_Q4_WS_DA, MOE_Q4_WS_CNT, MOE_Q4_WS_OFF, MOE_Q4_WS_TILE_OFF, MOE_Q4_WS_CHUNK_CNT,
     MOE_Q4_WS_CHUNK_BASE, MOE_Q4_WS_SORTED, MOE_Q4_WS_POS, MOE_Q4_WS_HQ, MOE_Q4_WS_DH, MOE_Q4_WS_SYNC,
-    MOE_Q4_WS_QA16, MOE_Q4_WS_HQ16, MOE_Q4_WS_TOTAL, MOE_Q4_WS_COUNT
+    MOE_Q4_WS_TOTAL, MOE_Q4_WS_COUNT
 };
 int moe_q4_workspace_layout(const moe_q4_layer* L, int64_t T, size_t* offsets, int n);
 

@@ -166,8 +166,6 @@ static void layout(const LayerView& L, int64_t T, size_t off[WS_COUNT]) {
         (size_t)(slots * L.F),                         // hq
         sizeof(uint16_t) * (size_t)(slots * (L.F / QK)),  // dh
         sizeof(uint32_t) * (size_t)((L.k + L.S) * ((L.F + 255) / 256)),  // sync
-        sizeof(uint16_t) * (size_t)(T * L.H),          // qa16
-        sizeof(uint16_t) * (size_t)(slots * L.F),      // hq16
     };
     size_t o = 0;
     for (int i = 0; i < WS_COUNT - 1; ++i) {
@@ -196,8 +194,6 @@ static Workspace carve(void* base, const size_t off[WS_COUNT]) {
     w.hq = reinterpret_cast<int8_t*>(b + off[WS_HQ]);
     w.dh = reinterpret_cast<uint16_t*>(b + off[WS_DH]);
     w.sync = reinterpret_cast<uint32_t*>(b + off[WS_SYNC]);
-    w.qa16 = reinterpret_cast<uint16_t*>(b + off[WS_QA16]);
-    w.hq16 = reinterpret_cast<uint16_t*>(b + off[WS_HQ16]);
     return w;
 }
 
@@ -279,7 +275,7 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
                         : DP4A_TT;
     MOE_TRY(launch_router_logits(L, x, T, w.logits, clear_status ? w.status : nullptr, s));
     MOE_TRY(launch_topk(w.logits, T, L.E, L.k, w.topk_idx, w.topk_w, w.status, s));
-    MOE_TRY(launch_quantize(x, T, L.H, w.qa, w.da, w.status, y, s, tc ? w.qa16 : nullptr));
+    MOE_TRY(launch_quantize(x, T, L.H, w.qa, w.da, w.status, y, s));
     MOE_TRY(launch_permute(w.topk_idx, T, L.k, L.E, L.S, tile, w, s));
     BlockDotCapture cap_store;
     const BlockDotCapture* cap = nullptr;

@@ -329,18 +329,13 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
             tma_load_2d(dn_s + (size_t)r0 * DN_KB * Q4_BYTES, dmap, fp * DN_KB * Q4_BYTES, drow0 + r0, &bar_dn);
     };
 
-    // ---- prologue: the shared expert's copies do not depend on the routing;
-    // the down matrices' tensor-map descriptors are fetched ahead of their use
-    if (tid == 0) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.down)) : "memory");
-        if (p.S) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.sh_down)) : "memory");
-    }
+    // ---- prologue: the shared expert's copies do not depend on the routing
     if (is_shared && tid == 0) issue_copies(p.sh_gate, p.sh_up, &maps.sh_down, n0);
 
     pdl_wait();  // logits, Q8_0 of x and the zeroed y are visible
     pdl_launch_dependents();
 
-    // ---- the logits (a NaN ranks as -infinity): all the routing needs
+    // ---- routing inputs: logits (a NaN ranks as -infinity), Q8_0 of x
     const int E16 = (E + 15) & ~15;
     for (int e = tid; e < E16; e += FFN_THREADS) {
         const float l = (e < E) ? __ldcg(p.logits + e) : -INFINITY;
@@ -348,6 +343,13 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
             atomicOr(&flags_s,
                      (int)((__float_as_uint(l) == TIMEOUT_NAN) ? STATUS_SPIN_TIMEOUT : STATUS_NONFINITE_LOGIT));
         logit_s[e] = (l != l) ? -INFINITY : l;
+    }
+    for (int i = tid; i < H / 16; i += FFN_THREADS)
+        reinterpret_cast<int4*>(qa_s)[i] = __ldcg(reinterpret_cast<const int4*>(p.qa) + i);
+    for (int b = tid; b < nbH; b += FFN_THREADS) {
+        const uint32_t bits = __ldcg(p.da + b);
+        if ((bits & 0x7fffu) == 0x7c00u) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
+        da_s[b] = half_bits_to_float(bits);
     }
     __syncthreads();
 
@@ -388,16 +390,6 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     // (slots are grouped by ascending expert, as in the grouped path)
     const unsigned chosen_mask = __ballot_sync(0xffffffffu, chosen);
     if (lane == 0) warp_chosen[warp] = __popc(chosen_mask);
-    // ---- everything below until the gate/up dot products overlaps the weight
-    // copies in flight: the Q8_0 of x, its block sums, slots, softmax terms
-    for (int i = tid; i < H / 16; i += FFN_THREADS)
-        reinterpret_cast<int4*>(qa_s)[i] = __ldcg(reinterpret_cast<const int4*>(p.qa) + i);
-    for (int b = tid; b < nbH; b += FFN_THREADS) {
-        const uint32_t bits = __ldcg(p.da + b);
-        if ((bits & 0x7fffu) == 0x7c00u) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
-        da_s[b] = half_bits_to_float(bits);
-    }
-    __syncthreads();
     // block sums of the activation codes (the -8 offset of the nibbles)
     for (int b = tid; b < nbH; b += FFN_THREADS) {
         const int* qw = reinterpret_cast<const int*>(qa_s + b * QK);
@@ -406,6 +398,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
         for (int q = 0; q < 8; ++q) s = __dp4a(qw[q], 0x01010101, s);
         qsum_s[b] = s;
     }
+    __syncthreads();
 
     // ---- slots and softmax terms
     if (chosen) {

@@ -12,15 +12,12 @@
 namespace moeq4 {
 
 // One warp per 32-value block, lane = element.  Optionally zeroes y (same
-// [T][H] shape as x) so the down projection can accumulate into it, and
-// writes the codes as binary16 too (q16: exact small integers, the tensor-core
-// projections' operand format).
+// [T][H] shape as x) so the down projection can accumulate into it.
 __global__ void __launch_bounds__(256) quantize_q8_0_kernel(const float* __restrict__ x, int64_t nblocks,
                                                              int8_t* __restrict__ q,
                                                              uint16_t* __restrict__ d,
                                                              uint32_t* __restrict__ status,
-                                                             float* __restrict__ y_zero,
-                                                             uint16_t* __restrict__ q16) {
+                                                             float* __restrict__ y_zero) {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
     for (int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); b < nblocks; b += nwarps) {
@@ -34,16 +31,15 @@ __global__ void __launch_bounds__(256) quantize_q8_0_kernel(const float* __restr
             if (ov && status) atomicOr(status, STATUS_SCALE_OVERFLOW);
         }
         if (y_zero) y_zero[b * QK + lane] = 0.0f;
-        if (q16) q16[b * QK + lane] = __half_as_ushort(__int2half_rn(qi));
     }
 }
 
 cudaError_t launch_quantize(const float* x, int64_t T, int H, int8_t* q, uint16_t* d, uint32_t* status,
-                            float* y_zero, cudaStream_t s, uint16_t* q16) {
+                            float* y_zero, cudaStream_t s) {
     const int64_t nblocks = T * (H / QK);
     int64_t ctas = ceil_div(nblocks, 8);
     if (ctas > 148 * 16) ctas = 148 * 16;
-    quantize_q8_0_kernel<<<(unsigned)ctas, 256, 0, s>>>(x, nblocks, q, d, status, y_zero, q16);
+    quantize_q8_0_kernel<<<(unsigned)ctas, 256, 0, s>>>(x, nblocks, q, d, status, y_zero);
     return cudaGetLastError();
 }
 

@@ -27,14 +27,12 @@
 // Warp roles (22 warps):
 //   0      producer: 2D tensor copies (TMA) of the packed weight rows (a box
 //          of 64 or 128 rows x 144 B = 8 blocks), two input stages in flight;
-//   1..4   converters: nibbles -> binary16 (nib - 8) for the A operand, into
-//          the K-major shared-memory layout (8-row x 16-byte core matrices);
-//          two operand stages of 2 blocks; and the B operand: each thread
-//          copies its slot's activations, already binary16 in global memory
-//          (written by the quantisation kernel, and by this kernel's gate/up
-//          epilogue for h), straight into the core-matrix layout of a 4-stage
-//          B ring with cp.async, two operand stages ahead; block scales into
-//          a ring read by the epilogue;
+//   1..4   converters: nibbles -> binary16 (nib - 8) for the A operand, and
+//          the slots' int8 activations, read from L2 with 16-byte loads
+//          issued before the wait for a free operand stage, -> binary16 for
+//          the B operand; both into the K-major shared-memory layout (8-row x
+//          16-byte core matrices); two operand stages of 2 blocks; block
+//          scales into a ring read by the epilogue;
 //   5      MMA issuer (one thread): two MMAs per block (A and B from shared
 //          memory); one wait and one commit per operand stage, for its pair
 //          of accumulators;
@@ -75,11 +73,11 @@ constexpr int W_PROD = 0, W_CONV0 = 1, W_MMA = 5, W_EPI0 = 6;
 constexpr uint32_t LIMIT = 1u << 22;
 constexpr size_t SZ_IN_W = (size_t)TM * IN_ROW;           // one input stage of packed weight rows
 constexpr size_t SZ_OP_A = (size_t)OP_KB * 2 * TM * 32;   // one operand stage of A (K-steps of 16 x binary16)
-// The B operand ring: NBO operand stages of binary16 activations, filled by
-// cp.async PF stages ahead of their use; beside it a ring of the slots' 2
-// binary16 block scales per stage (4 bytes an entry).
-constexpr int NBO = 4, PF = 2;
-static_assert(PF < NBO, "a prefetched stage never overwrites one the MMAs may still read");
+// Activation prefetch ring of the converters: NPF operand stages, a slot's 2
+// blocks of int8 codes (64 B) and their 2 binary16 scales (4 B) per entry,
+// copied by the thread that converts them (cp.async), PF stages ahead.
+constexpr int NPF = 4, PF = 3;
+constexpr size_t BPF_SLOT = 80;
 
 // Per tile width TN (slots, the MMA N): the epilogue has TN/32 column groups
 // of 4 warps (one per TMEM lane quarter), and the shared-memory map.
@@ -97,11 +95,11 @@ struct TcCfg {
     static constexpr size_t OFF_IN_W = 0;
     static constexpr size_t OFF_OP_A = (OFF_IN_W + NIN * SZ_IN_W + 1023) & ~size_t(1023);
     static constexpr size_t OFF_OP_B = OFF_OP_A + NOP * SZ_OP_A;
-    static constexpr size_t OFF_DW = OFF_OP_B + NBO * SZ_OP_B;
+    static constexpr size_t OFF_DW = OFF_OP_B + NOP * SZ_OP_B;
     static constexpr size_t OFF_DA = OFF_DW + (size_t)NSC * OP_KB * TM * 4;
     static constexpr size_t OFF_XCH = OFF_DA + (size_t)NSC * OP_KB * TN * 4;
-    static constexpr size_t OFF_BSC = OFF_XCH + (size_t)TM * XCH_LD * 4;
-    static constexpr size_t SMEM_BYTES = OFF_BSC + (size_t)NBO * TN * 4;
+    static constexpr size_t OFF_BPF = OFF_XCH + (size_t)TM * XCH_LD * 4;
+    static constexpr size_t SMEM_BYTES = OFF_BPF + (size_t)NPF * TN * BPF_SLOT;
     static constexpr size_t SMEM_ALLOC = SMEM_BYTES + 1024;   // slack to align the map to 1024 B
     static_assert(SMEM_ALLOC <= 220 * 1024, "shared memory map too large");
 };
@@ -124,14 +122,12 @@ struct TcParams {
     const uint8_t* sh_up;
     const uint8_t* sh_down;
     const int8_t* qa;
-    const uint16_t* qa16;
     const uint16_t* da;
     const int32_t* off;
     const int32_t* tile_off;
     const int32_t* sorted;
     const float* topk_w;
     int8_t* hq;
-    uint16_t* hq16;
     uint16_t* dh;
     float* h_dbg;
     float* y;
@@ -255,6 +251,7 @@ __device__ __forceinline__ uint2 bytes_to_f16(uint32_t w, uint32_t bias2) {
 }
 
 constexpr uint32_t BIAS_NIB = 0x64086408u;   // binary16 1032, twice: 1024 + n - 1032 = n - 8
+constexpr uint32_t BIAS_ACT = 0x64806480u;   // binary16 1152, twice: 1024 + (q ^ 0x80) - 1152 = q
 
 // Byte offset of the 16-byte core-matrix piece `core` (0/1) of row r in K-step
 // `ks` of block `kb` of an operand stage of `rows` rows: K-steps are 32-byte
@@ -262,6 +259,17 @@ constexpr uint32_t BIAS_NIB = 0x64086408u;   // binary16 1032, twice: 1024 + n -
 // pieces of a row 128 B apart (the descriptor's SBO and LBO).
 __device__ __forceinline__ uint32_t op_off(int rows, int kb, int ks, int r, int core) {
     return (uint32_t)((kb * 2 + ks) * rows * 32 + (r >> 3) * 256 + core * 128 + (r & 7) * 16);
+}
+
+// 16 activation codes (one 16-byte load) -> the two core-matrix pieces of one
+// K-step of slot n.
+__device__ __forceinline__ void store_act16(uint8_t* ob, int rows, int kb, int ks, int n, uint4 a) {
+    const uint2 a0 = bytes_to_f16(a.x ^ 0x80808080u, BIAS_ACT);
+    const uint2 a1 = bytes_to_f16(a.y ^ 0x80808080u, BIAS_ACT);
+    const uint2 a2 = bytes_to_f16(a.z ^ 0x80808080u, BIAS_ACT);
+    const uint2 a3 = bytes_to_f16(a.w ^ 0x80808080u, BIAS_ACT);
+    *reinterpret_cast<uint4*>(ob + op_off(rows, kb, ks, n, 0)) = make_uint4(a0.x, a0.y, a1.x, a1.y);
+    *reinterpret_cast<uint4*>(ob + op_off(rows, kb, ks, n, 1)) = make_uint4(a2.x, a2.y, a3.x, a3.y);
 }
 
 // One Q4_0 block (qs as four words) -> the four core-matrix pieces of weight
@@ -338,8 +346,8 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
     constexpr uint32_t TMEM_COLS = C::TMEM_COLS;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t in_full[NIN], in_empty[NIN], op_full[NOP], op_empty[NOP], b_empty[NBO],
-        tm_full[2], tm_empty[2], sc_full[NSC], sc_empty[NSC], epi_bar;
+    __shared__ __align__(8) uint64_t in_full[NIN], in_empty[NIN], op_full[NOP], op_empty[NOP], tm_full[2],
+        tm_empty[2], sc_full[NSC], sc_empty[NSC], epi_bar;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ int tile_off_s[258], off_s[258];
@@ -376,7 +384,6 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
             mbar_init(&op_full[i], N_CONV);
             mbar_init(&op_empty[i], 1);
         }
-        for (int i = 0; i < NBO; ++i) mbar_init(&b_empty[i], 1);
         for (int i = 0; i < 2; ++i) {  // one pair of accumulators each
             mbar_init(&tm_full[i], 1);
             mbar_init(&tm_empty[i], N_EPI / 32);
@@ -425,17 +432,16 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
         if (i_in > 0) mbar_wait_bounded(&in_full[(i_in - 1) % NIN], ((i_in - 1) / NIN) & 1, LIMIT);
     } else if (warp >= W_CONV0 && warp < W_CONV0 + 4) {
         // ------------------------------------------------------------ converters
-        // thread ct converts weight row ct, and (ct < TN) copies the binary16
-        // activations and the block scales of slot ct PF operand stages ahead
-        // (cp.async into the B ring and the scale ring: no registers held, no
-        // wait on L2 in the loop; a slot past the tile's end is not copied,
-        // its columns are never stored)
+        // thread ct converts weight row ct and (ct < TN) the activations of
+        // slot ct; it copies those activations PF operand stages ahead into
+        // its own entries of the prefetch ring (cp.async: no registers held,
+        // no wait on L2 in the loop)
         const int ct = tid - W_CONV0 * 32;
-        uint8_t* op_b_ring = op_b;
-        uint32_t* bsc = reinterpret_cast<uint32_t*>(smem + C::OFF_BSC);
+        uint8_t* bpf = smem + C::OFF_BPF;
         const int nst = nbK / OP_KB;                      // operand stages per item
+        // the prefetch cursor: item, stage, and this slot's rows (NULL: no slot)
         int pf_item = blockIdx.x, pf_c = 0;
-        const uint16_t* pf_arow = nullptr;
+        const int8_t* pf_arow = nullptr;
         const uint16_t* pf_ascale = nullptr;
         auto pf_rows = [&](int item) {
             pf_arow = nullptr;
@@ -448,31 +454,21 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
             float w;
             slot_info(p, Tn.g, sl, tok, w);
             if (MODE == GATEUP) {
-                pf_arow = p.qa16 + (size_t)tok * H;
+                pf_arow = p.qa + (size_t)tok * H;
                 pf_ascale = p.da + (size_t)tok * (H / QK);
             } else {
-                pf_arow = p.hq16 + (size_t)sl * F;
+                pf_arow = p.hq + (size_t)sl * F;
                 pf_ascale = p.dh + (size_t)sl * nbF;
             }
         };
         uint32_t i_pf = 0;
-        bool ok = true;
-        // one operand stage ahead; always one commit group, so that the group
-        // count tells which stage has landed
-        auto pf_issue = [&]() -> bool {
-            const int slot = i_pf % NBO;
-            if (i_pf >= (uint32_t)NBO && !wait_phase(&b_empty[slot], ((i_pf / NBO) & 1) ^ 1, abort)) return false;
+        auto pf_issue = [&]() {   // one operand stage ahead, always one commit group
             if (pf_item < n_items && pf_arow) {
-                uint8_t* ob = op_b_ring + (size_t)slot * C::SZ_OP_B;
-                const uint16_t* src = pf_arow + (size_t)pf_c * OP_KB * QK;
+                uint8_t* dst = bpf + ((size_t)(i_pf % NPF) * TN + ct) * BPF_SLOT;
+                const int8_t* src = pf_arow + (size_t)pf_c * OP_KB * QK;
 #pragma unroll
-                for (int kb = 0; kb < OP_KB; ++kb)
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks)
-#pragma unroll
-                        for (int core = 0; core < 2; ++core)
-                            cp_async16(ob + op_off(TN, kb, ks, ct, core), src + kb * QK + ks * 16 + core * 8);
-                cp_async4(bsc + slot * TN + ct, pf_ascale + pf_c * OP_KB);
+                for (int i = 0; i < 4; ++i) cp_async16(dst + 16 * i, src + 16 * i);
+                cp_async4(dst + 64, pf_ascale + pf_c * OP_KB);
             }
             cp_async_commit();
             ++i_pf;
@@ -481,18 +477,18 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 pf_item += gridDim.x;
                 pf_rows(pf_item);
             }
-            return true;
         };
         pf_rows(pf_item);
 #pragma unroll 1
-        for (int i = 0; i < PF && ok; ++i) ok = pf_issue();
+        for (int i = 0; i < PF; ++i) pf_issue();
 
         uint32_t i_op = 0;
+        bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const Tile T = tile_of<TN>(item, n_rb, tile_off_s, off_s, ngroups);
             const bool valid = ct < T.nslots;
             for (int c = 0; c < nst && ok; ++c, ++i_op) {
-                if (!pf_issue()) { ok = false; break; }      // stage i_op + PF
+                pf_issue();                                   // stage i_op + PF
                 const uint32_t i_in = i_op / (IN_KB / OP_KB);
                 const int s = i_in % NIN, sub = i_op % (IN_KB / OP_KB);
                 if (sub == 0 && !wait_phase(&in_full[s], (i_in / NIN) & 1, abort)) { ok = false; break; }
@@ -507,6 +503,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
 #pragma unroll
                 for (int i = 0; i < 9; ++i) w[i] = wsrc[i];
                 uint8_t* oa = op_a + (size_t)o * SZ_OP_A;
+                uint8_t* ob = op_b + (size_t)o * C::SZ_OP_B;
                 float dws[OP_KB];
                 {
                     // block 0 starts at byte 0 (scale, then 16 nibble bytes), block 1 at byte 18
@@ -520,10 +517,22 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     for (int i = 0; i < 4; ++i) qs[i] = w[5 + i];
                     store_weights(oa, 1, ct, qs);
                 }
-                cp_async_wait_group<PF>();                    // this thread's stage i_op (B, scales) has landed
+                // activations of slot ct from the ring (zeros past the tile's slots)
                 uint32_t dab = 0;
-                if (valid) dab = bsc[(i_op % NBO) * TN + ct];
-                fence_proxy_async_smem();                     // A stores and B copies -> the tensor core
+                cp_async_wait_group<PF>();                    // this thread's stage i_op has landed
+                if (ct < TN) {
+                    const uint8_t* src = bpf + ((size_t)(i_op % NPF) * TN + ct) * BPF_SLOT;
+#pragma unroll
+                    for (int kb = 0; kb < OP_KB; ++kb)
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks) {
+                            const uint4 a = valid ? *reinterpret_cast<const uint4*>(src + 16 * (2 * kb + ks))
+                                                  : make_uint4(0, 0, 0, 0);
+                            store_act16(ob, TN, kb, ks, ct, a);
+                        }
+                    if (valid) dab = *reinterpret_cast<const uint32_t*>(src + 64);
+                }
+                fence_proxy_async_smem();
                 tc_fence_before_sync();
                 mbar_arrive(&op_full[o]);
                 if (sub == IN_KB / OP_KB - 1) mbar_arrive(&in_empty[s]);
@@ -547,7 +556,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
             constexpr uint32_t idesc = idesc_f16(TM, TN);
             // descriptors of the first K-step of each operand stage; a later
             // K-step adds its byte offset / 16 to the start-address field
-            const uint64_t bdesc0 = smem_desc_kmajor(op_b, 128, 256);   // + ring slot x (SZ_OP_B / 16)
+            const uint64_t b0 = smem_desc_kmajor(op_b, 128, 256), b1 = smem_desc_kmajor(op_b + C::SZ_OP_B, 128, 256);
             const uint64_t a0 = smem_desc_kmajor(op_a, 128, 256), a1 = smem_desc_kmajor(op_a + SZ_OP_A, 128, 256);
             static_assert(NOP == 2, "two operand stages");
             uint32_t i_op = 0;
@@ -566,7 +575,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint64_t bd = bdesc0 + (uint64_t)(i_op % NBO) * (C::SZ_OP_B >> 4), ad = o ? a1 : a0;
+                    const uint64_t bd = o ? b1 : b0, ad = o ? a1 : a0;
 #pragma unroll
                     for (int kb = 0; kb < OP_KB; ++kb) {
                         const uint32_t d = tmem + (uint32_t)(OP_KB * o + kb) * TN;
@@ -576,14 +585,10 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     }
                     mma_commit(&tm_full[o]);  // covers the pair's four MMAs
                     mma_commit(&op_empty[o]);
-                    mma_commit(&b_empty[i_op % NBO]);
                 }
             }
-            // the last commits' arrivals must land before the CTA can exit
-            if (i_op > 0) {
-                mbar_wait_bounded(&op_empty[(i_op - 1) % NOP], ((i_op - 1) / NOP) & 1, LIMIT);
-                mbar_wait_bounded(&b_empty[(i_op - 1) % NBO], ((i_op - 1) / NBO) & 1, LIMIT);
-            }
+            // the last commit's arrival must land before the CTA can exit
+            if (i_op > 0) mbar_wait_bounded(&op_empty[(i_op - 1) % NOP], ((i_op - 1) / NOP) & 1, LIMIT);
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -695,18 +700,6 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     const int sl = T.slot0 + n;
                     *reinterpret_cast<uint4*>(p.hq + (size_t)sl * F + f0 + r0) =
                         make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                    // the same codes as binary16: the down projection's B operand
-                    uint32_t hw[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int q0 = (int)(int8_t)(packed[(2 * j) >> 2] >> (8 * ((2 * j) & 3)));
-                        const int q1 = (int)(int8_t)(packed[(2 * j + 1) >> 2] >> (8 * ((2 * j + 1) & 3)));
-                        hw[j] = (uint32_t)__half_as_ushort(__int2half_rn(q0)) |
-                                ((uint32_t)__half_as_ushort(__int2half_rn(q1)) << 16);
-                    }
-                    uint4* h16 = reinterpret_cast<uint4*>(p.hq16 + (size_t)sl * F + f0 + r0);
-                    h16[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    h16[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
                     if (p.h_dbg) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) p.h_dbg[(size_t)sl * F + f0 + r0 + j] = h[j];
@@ -748,9 +741,8 @@ static TcParams make_tc_params(const LayerView& L, int64_t T, const Workspace& w
     p.H = L.H; p.F = L.F; p.E = L.E; p.k = L.k; p.P = (int)(T * L.k);
     p.w_gate = L.w_gate; p.w_up = L.w_up; p.w_down = L.w_down;
     p.sh_gate = L.sh_gate; p.sh_up = L.sh_up; p.sh_down = L.sh_down;
-    p.qa = ws.qa; p.qa16 = ws.qa16; p.da = ws.da; p.off = ws.off; p.tile_off = ws.tile_off; p.sorted = ws.sorted;
-    p.topk_w = ws.topk_w; p.hq = ws.hq; p.hq16 = ws.hq16; p.dh = ws.dh; p.h_dbg = h_dbg; p.y = y;
-    p.status = ws.status;
+    p.qa = ws.qa; p.da = ws.da; p.off = ws.off; p.tile_off = ws.tile_off; p.sorted = ws.sorted;
+    p.topk_w = ws.topk_w; p.hq = ws.hq; p.dh = ws.dh; p.h_dbg = h_dbg; p.y = y; p.status = ws.status;
     p.cap_out = nullptr; p.cap_group = -1; p.cap_rb = -1;
     return p;
 }

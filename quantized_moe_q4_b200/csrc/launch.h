@@ -38,8 +38,6 @@ struct Workspace {
     int8_t* hq;
     uint16_t* dh;
     uint32_t* sync;   // per-group counters of the fused T = 1 kernels
-    uint16_t* qa16;   // [T][H] the Q8_0 codes of x as binary16 (tensor-core path)
-    uint16_t* hq16;   // [P+S*T][F] the requantised h codes as binary16 (tensor-core path)
 };
 
 // Test capture of the per-block integer dot products I_b of one row block of
@@ -65,9 +63,8 @@ cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* i
                         uint32_t* status, cudaStream_t s);
 
 // k_quant_perm.cu
-// q16 (may be NULL): the codes as binary16 as well.
 cudaError_t launch_quantize(const float* x, int64_t T, int H, int8_t* q, uint16_t* d,
-                            uint32_t* status, float* y_zero, cudaStream_t s, uint16_t* q16 = nullptr);
+                            uint32_t* status, float* y_zero, cudaStream_t s);
 cudaError_t launch_permute(const int32_t* idx, int64_t T, int k, int E, int S, int tile_tokens,
                            const Workspace& ws, cudaStream_t s);
 

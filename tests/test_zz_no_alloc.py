@@ -35,11 +35,11 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row():
     x2, lw2 = synth.workload_inputs("decode_t1", seed=0, T=300)
     L1, L2 = m.Layer.from_host(lw1), m.Layer.from_host(lw2)
     xd1, xd2 = torch.from_numpy(x1).cuda(), torch.from_numpy(x2[1:2].copy()).cuda()
-    xd3 = torch.from_numpy(x2[:160].copy()).cuda()
+    xd3 = torch.from_numpy(x2[:256].copy()).cuda()
     ref1, ref2, ref3 = _reference(L1, xd1), _reference(L2, xd2), _reference(L2, xd3)
     # calls in a row on the shared scratch: a 16-token layer (streaming
     # kernels), a one-token call of a different layer (fused decode kernels),
-    # then 160 tokens of that layer (tensor-core kernels, another layout of
+    # then 256 tokens of that layer (tensor-core kernels, another layout of
     # the same array)
     y1 = m.moe_q4_ffn_forward_noalloc(L1, xd1)
     y2 = m.moe_q4_ffn_forward_noalloc(L2, xd2)
@@ -58,9 +58,9 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row():
 def test_noalloc_rejects_problems_beyond_the_scratch():
     _, lw = synth.workload_inputs("decode_t1", seed=0, T=1)
     L = m.Layer.from_host(lw)
-    limit = m.moe_q4_ffn_workspace_bytes(L, 199)
-    assert limit <= (4 << 20) < m.moe_q4_ffn_workspace_bytes(L, 200)
-    x = torch.zeros((200, lw.hidden), device="cuda")
+    limit = m.moe_q4_ffn_workspace_bytes(L, 542)
+    assert limit <= (4 << 20) < m.moe_q4_ffn_workspace_bytes(L, 543)
+    x = torch.zeros((543, lw.hidden), device="cuda")
     y = torch.full_like(x, 7.0)
     with pytest.raises(m.MoeQ4Error) as e:
         m.moe_q4_ffn_forward_noalloc(L, x, y)

@@ -46,6 +46,7 @@
 #include "common.cuh"
 #include "launch.h"
 #include "ptx.cuh"
+#include "tc.cuh"
 
 namespace moeq4 {
 
@@ -244,7 +245,7 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
 // K2: gate/up + SwiGLU + requant, exchange within a group, down + combine.
 // ---------------------------------------------------------------------------
 struct DecodeSmem {
-    size_t gu, dn, qa, da, qsum, o, total;  // byte offsets
+    size_t gu, dn, qa, da, dab, qsum, o, total;  // byte offsets
 };
 
 __host__ __device__ inline size_t al128(size_t v) { return (v + 127) & ~size_t(127); }
@@ -257,6 +258,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int H) {
     L.dn = o;   o += al128((size_t)(H / CL) * DN_KB * Q4_BYTES); // H/8 rows x 8 blocks
     L.qa = o;   o += al128((size_t)H);
     L.da = o;   o += al128((size_t)nbH * 4);
+    L.dab = o;  o += al128((size_t)nbH * 2);
     L.qsum = o; o += al128((size_t)nbH * 4);
     L.o = o;    o += al128((size_t)(H / CL) * 4);
     L.total = o + 128;   // slack to align the map to 128 bytes
@@ -300,6 +302,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     uint8_t* dn_s = dsm + SL.dn;
     int8_t* qa_s = reinterpret_cast<int8_t*>(dsm + SL.qa);
     float* da_s = reinterpret_cast<float*>(dsm + SL.da);
+    uint16_t* dab_s = reinterpret_cast<uint16_t*>(dsm + SL.dab);
     int* qsum_s = reinterpret_cast<int*>(dsm + SL.qsum);
     float* o_s = reinterpret_cast<float*>(dsm + SL.o);
     bool timed_out = false;
@@ -329,13 +332,22 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
             tma_load_2d(dn_s + (size_t)r0 * DN_KB * Q4_BYTES, dmap, fp * DN_KB * Q4_BYTES, drow0 + r0, &bar_dn);
     };
 
-    // ---- prologue: the shared expert's copies do not depend on the routing
+    // ---- prologue: the shared expert's copies do not depend on the routing;
+    // the down matrices' tensor-map descriptors are fetched ahead of their use
+    if (tid == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.down)) : "memory");
+        if (p.S) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.sh_down)) : "memory");
+    }
     if (is_shared && tid == 0) issue_copies(p.sh_gate, p.sh_up, &maps.sh_down, n0);
 
     pdl_wait();  // logits, Q8_0 of x and the zeroed y are visible
     pdl_launch_dependents();
 
-    // ---- routing inputs: logits (a NaN ranks as -infinity), Q8_0 of x
+    // ---- routing inputs.  The Q8_0 of x goes to shared memory by cp.async,
+    // issued first so that it is not queued behind this CTA's weight copies;
+    // only the logits (a NaN ranks as -infinity) are awaited before ranking
+    for (int i = tid; i < H / 16; i += FFN_THREADS) cp_async16(qa_s + 16 * i, p.qa + 16 * i);
+    for (int i = tid; i < nbH / 8; i += FFN_THREADS) cp_async16(dab_s + 8 * i, p.da + 8 * i);
     const int E16 = (E + 15) & ~15;
     for (int e = tid; e < E16; e += FFN_THREADS) {
         const float l = (e < E) ? __ldcg(p.logits + e) : -INFINITY;
@@ -343,13 +355,6 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
             atomicOr(&flags_s,
                      (int)((__float_as_uint(l) == TIMEOUT_NAN) ? STATUS_SPIN_TIMEOUT : STATUS_NONFINITE_LOGIT));
         logit_s[e] = (l != l) ? -INFINITY : l;
-    }
-    for (int i = tid; i < H / 16; i += FFN_THREADS)
-        reinterpret_cast<int4*>(qa_s)[i] = __ldcg(reinterpret_cast<const int4*>(p.qa) + i);
-    for (int b = tid; b < nbH; b += FFN_THREADS) {
-        const uint32_t bits = __ldcg(p.da + b);
-        if ((bits & 0x7fffu) == 0x7c00u) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
-        da_s[b] = half_bits_to_float(bits);
     }
     __syncthreads();
 
@@ -390,6 +395,13 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     // (slots are grouped by ascending expert, as in the grouped path)
     const unsigned chosen_mask = __ballot_sync(0xffffffffu, chosen);
     if (lane == 0) warp_chosen[warp] = __popc(chosen_mask);
+    cp_async_wait_all();
+    __syncthreads();
+    for (int b = tid; b < nbH; b += FFN_THREADS) {
+        const uint32_t bits = dab_s[b];
+        if ((bits & 0x7fffu) == 0x7c00u) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
+        da_s[b] = half_bits_to_float(bits);
+    }
     // block sums of the activation codes (the -8 offset of the nibbles)
     for (int b = tid; b < nbH; b += FFN_THREADS) {
         const int* qw = reinterpret_cast<const int*>(qa_s + b * QK);

@@ -380,8 +380,8 @@ def chunked_lines(m, torch, stream):
 
 
 def batch64_lines(m, torch, stream):
-    """One layer on decode batches of 8 to 128 tokens, on the automatic path,
-    the streaming dp4a kernels and the 32-slot tensor-core kernels: tokens/s,
+    """One layer on batches of 8 to 512 tokens, on the automatic path, the
+    streaming dp4a kernels and the 32- and 64-slot tensor-core kernels: tokens/s,
     and HBM GB/s over the experts the batch activates + Wr + x/y; the layer
     rotates over 4 device copies (912 MB) so every rep is L2-cold."""
     import synth
@@ -390,12 +390,13 @@ def batch64_lines(m, torch, stream):
     base = m.Layer.from_host(lw)
     layers = [base] + [base.replica() for _ in range(3)]
     out = {"peak_source": src}
-    for T in (8, 16, 32, 64, 96, 128):
+    for T in (8, 16, 32, 64, 96, 128, 192, 256, 384, 512):
         x = torch.from_numpy(x_np[:T].copy()).cuda()
         y = torch.empty_like(x)
         ws = m.alloc_workspace(m.moe_q4_ffn_workspace_bytes(base, T))
         rec = {}
-        for vname, path in (("auto", m.PATH_AUTO), ("dp4a", m.PATH_GROUPED_DP4A), ("tc_n32", m.PATH_TENSOR_CORE_N32)):
+        for vname, path in (("auto", m.PATH_AUTO), ("dp4a", m.PATH_GROUPED_DP4A), ("tc_n32", m.PATH_TENSOR_CORE_N32),
+                            ("tc_n64", m.PATH_TENSOR_CORE_N64)):
             times = []
             for rep in range(12):
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

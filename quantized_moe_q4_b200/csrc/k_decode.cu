@@ -265,6 +265,58 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int H) {
     return L;
 }
 
+// Order key of a logit: unsigned integers in the order of the values, with
+// -0 folded into +0 (equal logits compare equal).  Key 0 lies below every
+// logit's key (-infinity's is 0x007fffff) and marks an expert that is out of
+// range or already chosen.
+__device__ __forceinline__ uint32_t logit_key(float l) {
+    const uint32_t u = __float_as_uint(l == 0.0f ? 0.0f : l);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_logit(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+// Top-k of E <= 32 NK logits by one warp (a NaN ranks as -infinity): lane l
+// holds the keys of experts l, l + 32, ...; each of the k rounds takes the
+// largest key (warp max), the lowest expert index among equal keys (warp
+// min) and retires it, so round r names the expert of rank r (descending
+// logits, equal logits by the lower index).  on_round(r, e, logit) runs in
+// every lane after round r.  Returns the status bits of non-finite logits.
+template <int NK, class OnRound>
+__device__ __forceinline__ int topk_rounds(const float* __restrict__ logits, int E, int k, int lane,
+                                           OnRound&& on_round) {
+    uint32_t key[NK];
+    unsigned fl = 0;
+#pragma unroll
+    for (int i = 0; i < NK; ++i) {
+        const int e = lane + 32 * i;
+        key[i] = 0u;
+        if (e < E) {
+            const float l = __ldcg(logits + e);
+            if (!isfinite(l))
+                fl |= (__float_as_uint(l) == TIMEOUT_NAN) ? STATUS_SPIN_TIMEOUT : STATUS_NONFINITE_LOGIT;
+            key[i] = logit_key(l != l ? -INFINITY : l);
+        }
+    }
+    for (int r = 0; r < k; ++r) {
+        uint32_t lm = key[0];
+#pragma unroll
+        for (int i = 1; i < NK; ++i) lm = max(lm, key[i]);
+        const uint32_t m = __reduce_max_sync(0xffffffffu, lm);
+        uint32_t cand = 0xffffffffu;
+#pragma unroll
+        for (int i = NK - 1; i >= 0; --i)
+            if (key[i] == m) cand = (uint32_t)(lane + 32 * i);
+        const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+#pragma unroll
+        for (int i = 0; i < NK; ++i)
+            if ((uint32_t)(lane + 32 * i) == win) key[i] = 0u;
+        on_round(r, (int)win, key_logit(m));
+    }
+    return (int)__reduce_or_sync(0xffffffffu, fl);
+}
+
 __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams p,
                                                                     const __grid_constant__ DecodeMaps maps) {
     extern __shared__ __align__(16) unsigned char dsm_raw[];
@@ -272,12 +324,10 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     unsigned char* dsm = dsm_raw + ((128u - (smem_u32(dsm_raw) & 127u)) & 127u);
     __shared__ __align__(8) uint64_t bar_gu[4];
     __shared__ __align__(8) uint64_t bar_dn;
-    __shared__ __align__(16) float logit_s[256];
     __shared__ int idx_s[16];
     __shared__ float ex_s[16];
     __shared__ float w_s[16];
     __shared__ int slot_s[17];
-    __shared__ int warp_chosen[FFN_WARPS];
     __shared__ float gs[32], us[32];
     __shared__ int flags_s;
 
@@ -315,21 +365,24 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     }
     __syncthreads();
 
-    // copies of this CTA's weights, issued by one thread: gate/up chunk i = 8
-    // gate rows + the same 8 up rows on bar_gu[i]; the down slice = rows
-    // n0 .. n0 + Hs, blocks 8 fp .. 8 fp + 7, on bar_dn
+    // copies of this CTA's weights, issued by lanes 0..4 of warp 0 at once:
+    // lane i < 4 gate/up chunk i = 8 gate rows + the same 8 up rows on
+    // bar_gu[i]; lane 4 the down slice = rows n0 .. n0 + Hs, blocks 8 fp ..
+    // 8 fp + 7, on bar_dn
     const uint32_t chunk_bytes = (uint32_t)(8 * row_gu);
     auto issue_copies = [&](const uint8_t* Wg, const uint8_t* Wu, const CUtensorMap* dmap, int drow0) {
-        for (int ch = 0; ch < 4; ++ch) {
+        if (lane < 4) {
+            const int ch = lane;
             const uint32_t extra = (p.force_timeout && blockIdx.x == 0 && ch == 0) ? 16u : 0u;
             mbar_arrive_expect_tx(&bar_gu[ch], 2u * chunk_bytes + extra);
             const size_t src = (size_t)(hb * 32 + 8 * ch) * row_gu;
             bulk_g2s(gu_s + (size_t)(8 * ch) * row_gu, Wg + src, chunk_bytes, &bar_gu[ch]);
             bulk_g2s(gu_s + (size_t)(32 + 8 * ch) * row_gu, Wu + src, chunk_bytes, &bar_gu[ch]);
+        } else if (lane == 4) {
+            mbar_arrive_expect_tx(&bar_dn, (uint32_t)(Hs * DN_KB * Q4_BYTES));
+            for (int r0 = 0; r0 < Hs; r0 += p.box_rows)
+                tma_load_2d(dn_s + (size_t)r0 * DN_KB * Q4_BYTES, dmap, fp * DN_KB * Q4_BYTES, drow0 + r0, &bar_dn);
         }
-        mbar_arrive_expect_tx(&bar_dn, (uint32_t)(Hs * DN_KB * Q4_BYTES));
-        for (int r0 = 0; r0 < Hs; r0 += p.box_rows)
-            tma_load_2d(dn_s + (size_t)r0 * DN_KB * Q4_BYTES, dmap, fp * DN_KB * Q4_BYTES, drow0 + r0, &bar_dn);
     };
 
     // ---- prologue: the shared expert's copies do not depend on the routing;
@@ -338,111 +391,90 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.down)) : "memory");
         if (p.S) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.sh_down)) : "memory");
     }
-    if (is_shared && tid == 0) issue_copies(p.sh_gate, p.sh_up, &maps.sh_down, n0);
+    if (is_shared && warp == 0) issue_copies(p.sh_gate, p.sh_up, &maps.sh_down, n0);
 
     pdl_wait();  // logits, Q8_0 of x and the zeroed y are visible
     pdl_launch_dependents();
 
-    // ---- routing inputs.  The Q8_0 of x goes to shared memory by cp.async,
-    // issued first so that it is not queued behind this CTA's weight copies;
-    // only the logits (a NaN ranks as -infinity) are awaited before ranking
-    for (int i = tid; i < H / 16; i += FFN_THREADS) cp_async16(qa_s + 16 * i, p.qa + 16 * i);
-    for (int i = tid; i < nbH / 8; i += FFN_THREADS) cp_async16(dab_s + 8 * i, p.da + 8 * i);
-    const int E16 = (E + 15) & ~15;
-    for (int e = tid; e < E16; e += FFN_THREADS) {
-        const float l = (e < E) ? __ldcg(p.logits + e) : -INFINITY;
-        if (e < E && !isfinite(l))
-            atomicOr(&flags_s,
-                     (int)((__float_as_uint(l) == TIMEOUT_NAN) ? STATUS_SPIN_TIMEOUT : STATUS_NONFINITE_LOGIT));
-        logit_s[e] = (l != l) ? -INFINITY : l;
-    }
-    __syncthreads();
-
-    // ---- top-k: expert e is ranked by P consecutive threads (P = 4 for
-    // E <= 128, else 2), each comparing logit e with a 1/P share of the logits
-    // (descending, equal logits by expert index); the partial ranks are summed
-    // with shuffles.  Ranks below k are the chosen experts, in order.  The
-    // keys are a total order, so the ranks are a permutation of [0, E).
-    const int P = (E16 <= FFN_THREADS / 4) ? 4 : 2;
-    const int e_me = tid / P, part = tid % P;
-    float my_l = 0.0f;
-    int rank = 0;
-    if (e_me < E) {
-        my_l = logit_s[e_me];
-        const float4* l4 = reinterpret_cast<const float4*>(logit_s);
-        const int per4 = E16 / (4 * P);
-#pragma unroll 4
-        for (int e4 = part * per4; e4 < (part + 1) * per4; ++e4) {
-            const float4 v = l4[e4];
-            const int e = 4 * e4;
-            rank += (v.x > my_l || (v.x == my_l && e < e_me)) ? 1 : 0;
-            rank += (v.y > my_l || (v.y == my_l && e + 1 < e_me)) ? 1 : 0;
-            rank += (v.z > my_l || (v.z == my_l && e + 2 < e_me)) ? 1 : 0;
-            rank += (v.w > my_l || (v.w == my_l && e + 3 < e_me)) ? 1 : 0;
+    if (warp == 0) {
+        // ---- top-k by warp 0, straight from the logits in L2 (a NaN ranks as
+        // -infinity).  The CTA of routed rank j issues its copies as soon as
+        // round j has named its expert; lane r < k keeps round r's expert.
+        int e_r = 0;
+        float l_r = 0.0f, l_0 = 0.0f;
+        auto on_round = [&](int rr, int e, float l) {
+            if (rr == 0) l_0 = l;
+            if (lane == rr) {
+                e_r = e;
+                l_r = l;
+            }
+            if (!is_shared && rr == j) {
+                const size_t eo = (size_t)e * gu_stride;
+                issue_copies(p.w_gate + eo, p.w_up + eo, &maps.down, e * H + n0);
+            }
+        };
+        const int fl = (E <= 128) ? topk_rounds<4>(p.logits, E, k, lane, on_round)
+                                  : topk_rounds<8>(p.logits, E, k, lane, on_round);
+        if (fl && lane == 0) atomicOr(&flags_s, fl);
+        // softmax over the k chosen logits (terms relative to the largest,
+        // summed in rank order) and the slots: slot of a chosen expert = the
+        // number of chosen experts with a lower index (slots are grouped by
+        // ascending expert, as in the grouped path)
+        if (lane < k) {
+            idx_s[lane] = e_r;
+            ex_s[lane] = expf(l_r - l_0);
+        }
+        __syncwarp();
+        if (lane < k) {
+            float z = 0.0f;
+            int before = 0;
+            for (int i = 0; i < k; ++i) {
+                z += ex_s[i];
+                before += (idx_s[i] < e_r) ? 1 : 0;
+            }
+            w_s[lane] = __fdiv_rn(ex_s[lane], z);
+            slot_s[lane] = before;
+        }
+        if (lane == 0) slot_s[k] = k;  // the shared expert's slot: P + t
+    } else {
+        // ---- warps 1..: the Q8_0 of x into shared memory by cp.async, then
+        // its block scales and block sums (the -8 offset of the nibbles)
+        const int t = tid - 32, nt = FFN_THREADS - 32;
+        for (int i = t; i < H / 16; i += nt) cp_async16(qa_s + 16 * i, p.qa + 16 * i);
+        for (int i = t; i < nbH / 8; i += nt) cp_async16(dab_s + 8 * i, p.da + 8 * i);
+        cp_async_wait_all();
+        asm volatile("bar.sync 1, %0;" ::"n"(FFN_THREADS - 32) : "memory");
+        for (int b = t; b < nbH; b += nt) {
+            const uint32_t bits = dab_s[b];
+            if ((bits & 0x7fffu) == 0x7c00u) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
+            da_s[b] = half_bits_to_float(bits);
+            const int* qw = reinterpret_cast<const int*>(qa_s + b * QK);
+            int s = 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) s = __dp4a(qw[q], 0x01010101, s);
+            qsum_s[b] = s;
         }
     }
-    rank += __shfl_xor_sync(0xffffffffu, rank, 1);
-    if (P == 4) rank += __shfl_xor_sync(0xffffffffu, rank, 2);
-    const int my_rank = (e_me < E) ? rank : k;
-    const bool chosen = part == 0 && my_rank < k;
-    if (chosen) idx_s[my_rank] = e_me;
-    // the thread that found this CTA's expert issues its copies at once
-    if (!is_shared && chosen && my_rank == j) {
-        const size_t eo = (size_t)e_me * gu_stride;
-        issue_copies(p.w_gate + eo, p.w_up + eo, &maps.down, e_me * H + n0);
-    }
-    // slot of a chosen expert = number of chosen experts with a lower index
-    // (slots are grouped by ascending expert, as in the grouped path)
-    const unsigned chosen_mask = __ballot_sync(0xffffffffu, chosen);
-    if (lane == 0) warp_chosen[warp] = __popc(chosen_mask);
-    cp_async_wait_all();
-    __syncthreads();
-    for (int b = tid; b < nbH; b += FFN_THREADS) {
-        const uint32_t bits = dab_s[b];
-        if ((bits & 0x7fffu) == 0x7c00u) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
-        da_s[b] = half_bits_to_float(bits);
-    }
-    // block sums of the activation codes (the -8 offset of the nibbles)
-    for (int b = tid; b < nbH; b += FFN_THREADS) {
-        const int* qw = reinterpret_cast<const int*>(qa_s + b * QK);
-        int s = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) s = __dp4a(qw[q], 0x01010101, s);
-        qsum_s[b] = s;
-    }
     __syncthreads();
 
-    // ---- slots and softmax terms
-    if (chosen) {
-        int before = __popc(chosen_mask & ((1u << lane) - 1u));
-        for (int w2 = 0; w2 < warp; ++w2) before += warp_chosen[w2];
-        slot_s[my_rank] = before;
-        ex_s[my_rank] = expf(my_l - logit_s[idx_s[0]]);
-    }
-    if (tid == 0) slot_s[k] = k;  // the shared expert's slot: P + t
-    __syncthreads();
-    if (warp == 1 && lane < k) {
-        float z = 0.0f;
-        for (int i = 0; i < k; ++i) z += ex_s[i];
-        w_s[lane] = __fdiv_rn(ex_s[lane], z);
-    }
     // inspection arrays of the workspace (the same as the grouped path's)
     if (blockIdx.x == 0) {
-        if (part == 0 && e_me < E) p.cnt[e_me] = chosen ? 1 : 0;
-        if (tid == 0) p.cnt[E] = p.S;
         for (int e = tid; e <= E + 1; e += FFN_THREADS) {
-            int o = 0;
-            if (e <= E)
-                for (int i = 0; i < k; ++i) o += (idx_s[i] < e) ? 1 : 0;
+            int o = 0, chosen = 0;
+            for (int i = 0; i < k; ++i) {
+                o += (idx_s[i] < e) ? 1 : 0;
+                chosen |= (idx_s[i] == e) ? 1 : 0;
+            }
+            if (e < E) p.cnt[e] = chosen;
+            if (e == E) p.cnt[E] = p.S;
             p.off[e] = (e <= E) ? o : k + p.S;
         }
-    }
-    __syncthreads();
-    if (blockIdx.x == 0 && tid < k) {
-        p.topk_idx[tid] = idx_s[tid];
-        p.topk_w[tid] = w_s[tid];
-        p.pos[tid] = slot_s[tid];
-        p.sorted[slot_s[tid]] = tid;
+        if (tid < k) {
+            p.topk_idx[tid] = idx_s[tid];
+            p.topk_w[tid] = w_s[tid];
+            p.pos[tid] = slot_s[tid];
+            p.sorted[slot_s[tid]] = tid;
+        }
     }
 
     // ---- gate/up: warp w computes rows 4w .. 4w + 3 of the 64 (0..31 gate,

@@ -842,10 +842,12 @@ static cudaError_t launch_tc(const LayerView& L, int64_t T, const Workspace& ws,
 
 int tc_tile_tokens(const LayerView& L, int64_t T, int force) {
     if (force == 32 || force == 64 || force == 128) return force;
-    // routed slots per expert on average: the tile the average expert fills
-    // (64 slots for a 947-token prompt's 59 per expert, 128 from 96 up)
+    // routed slots per expert on average, against the measured crossovers of
+    // the three widths (one 2048/512 layer, 128 experts top-8): 32 slots up to
+    // 27 per expert (T <= 384), 64 from 28 (T = 512; a 947-token prompt's 59),
+    // 128 from 96
     const int64_t per_expert = T * L.k / L.E;
-    return per_expert >= 96 ? 128 : 64;
+    return per_expert >= 96 ? 128 : per_expert >= 28 ? 64 : 32;
 }
 
 cudaError_t launch_gateup_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, const DeviceInfo& dev,

@@ -264,7 +264,7 @@ const char* moe_q4_last_cuda_error(void);
  *   | qa i8[T][H] | da u16[T][H/32] | cnt i32[E+1] | off i32[E+2]
  *   | tile_off i32[E+2] | chunk_cnt i32[C][E] | chunk_base i32[C][E]
  *   | sorted i32[P] | pos i32[P] | hq i8[P+S*T][F] | dh u16[P+S*T][F/32]
- *   | sync u32[(k+S)*F/256] | total
+ *   | total
  * with P = T*k routed pairs and S = has_shared.  Slots (rows of hq/dh) are
  * grouped by expert: routed expert e owns slots off[e]..off[e+1]-1 holding
  * pairs sorted[...] = t*k+j in increasing (t, j) order; the shared expert
@@ -274,7 +274,7 @@ const char* moe_q4_last_cuda_error(void);
 enum {
     MOE_Q4_WS_STATUS = 0, MOE_Q4_WS_LOGITS, MOE_Q4_WS_TOPK_IDX, MOE_Q4_WS_TOPK_W, MOE_Q4_WS_QA,
     MOE_Q4_WS_DA, MOE_Q4_WS_CNT, MOE_Q4_WS_OFF, MOE_Q4_WS_TILE_OFF, MOE_Q4_WS_CHUNK_CNT,
-    MOE_Q4_WS_CHUNK_BASE, MOE_Q4_WS_SORTED, MOE_Q4_WS_POS, MOE_Q4_WS_HQ, MOE_Q4_WS_DH, MOE_Q4_WS_SYNC,
+    MOE_Q4_WS_CHUNK_BASE, MOE_Q4_WS_SORTED, MOE_Q4_WS_POS, MOE_Q4_WS_HQ, MOE_Q4_WS_DH,
     MOE_Q4_WS_TOTAL, MOE_Q4_WS_COUNT
 };
 int moe_q4_workspace_layout(const moe_q4_layer* L, int64_t T, size_t* offsets, int n);
@@ -316,10 +316,12 @@ typedef struct {
     int32_t block_dots_down;   /* 0: the gate/up projection, 1: the down projection */
     int32_t block_dots_group;  /* expert group g (n_experts: the shared expert) */
     int32_t block_dots_rb;     /* row block */
-    /* Fused T = 1 path only: device uint64[2], 8-byte aligned; per call
-     * [0] += the FFN kernel's span in its first CTA (%globaltimer ns, from
-     * its start to its end, inside the programmatic-launch chain, with no
-     * event between the kernels), [1] += 1.  NULL: not timed. */
+    /* Fused T = 1 path only: device uint64[3], 8-byte aligned; per call, in
+     * the FFN kernel's first CTA (%globaltimer ns, inside the programmatic-
+     * launch chain, with no event between the kernels): [0] += the span from
+     * its wait on the router kernel returning to its end, [1] += 1, [2] +=
+     * the span from its start (the launch overlaps the router kernel, so
+     * this includes the wait) to its end.  NULL: not timed. */
     unsigned long long* decode_kernel_ns;
 } moe_q4_debug;
 

@@ -40,7 +40,7 @@ PATH_AUTO, PATH_GROUPED_DP4A, PATH_DECODE, PATH_TENSOR_CORE = 0, 1, 2, 3
 PATH_TENSOR_CORE_N32, PATH_TENSOR_CORE_N128, PATH_TENSOR_CORE_N64 = 4, 5, 6
 
 WS_NAMES = ["status", "logits", "topk_idx", "topk_w", "qa", "da", "cnt", "off", "tile_off",
-            "chunk_cnt", "chunk_base", "sorted", "pos", "hq", "dh", "sync", "total"]
+            "chunk_cnt", "chunk_base", "sorted", "pos", "hq", "dh", "total"]
 
 # Every extern "C" symbol of include/moe_q4.h.
 EXPORTS = ["moe_q4_quantize_act", "moe_q4_route", "moe_q4_ffn_workspace_bytes", "moe_q4_ffn_forward",

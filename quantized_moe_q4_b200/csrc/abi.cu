@@ -165,7 +165,6 @@ static void layout(const LayerView& L, int64_t T, size_t off[WS_COUNT]) {
         sizeof(int32_t) * (size_t)P,                   // pos
         (size_t)(slots * L.F),                         // hq
         sizeof(uint16_t) * (size_t)(slots * (L.F / QK)),  // dh
-        sizeof(uint32_t) * (size_t)((L.k + L.S) * ((L.F + 255) / 256)),  // sync
     };
     size_t o = 0;
     for (int i = 0; i < WS_COUNT - 1; ++i) {
@@ -193,7 +192,6 @@ static Workspace carve(void* base, const size_t off[WS_COUNT]) {
     w.pos = reinterpret_cast<int32_t*>(b + off[WS_POS]);
     w.hq = reinterpret_cast<int8_t*>(b + off[WS_HQ]);
     w.dh = reinterpret_cast<uint16_t*>(b + off[WS_DH]);
-    w.sync = reinterpret_cast<uint32_t*>(b + off[WS_SYNC]);
     return w;
 }
 

@@ -19,7 +19,7 @@ constexpr int Q4_BYTES = 18;    // binary16 scale + 16 nibble bytes
 // Workspace layout (indices match MOE_Q4_WS_* of the public header).
 enum WsIndex {
     WS_STATUS = 0, WS_LOGITS, WS_TOPK_IDX, WS_TOPK_W, WS_QA, WS_DA, WS_CNT, WS_OFF, WS_TILE_OFF,
-    WS_CHUNK_CNT, WS_CHUNK_BASE, WS_SORTED, WS_POS, WS_HQ, WS_DH, WS_SYNC, WS_TOTAL, WS_COUNT
+    WS_CHUNK_CNT, WS_CHUNK_BASE, WS_SORTED, WS_POS, WS_HQ, WS_DH, WS_TOTAL, WS_COUNT
 };
 
 // Token-to-expert permutation chunk: pairs handled by one CTA of the

@@ -12,30 +12,26 @@
 //     kernel it bulk-copies its router row into shared memory; then the logit
 //     (four independent FMA chains); the first H/32 CTAs quantise one Q8_0
 //     block of x each; y is zeroed (the FFN kernel accumulates into it).
-//   decode_ffn_kernel: a cooperative grid of (k+S) x F/256 groups of 8 CTAs,
-//     one group per (expert of the token, 256-wide part of F).  CTA r of a
-//     group owns one 32-row block of h (32 gate rows and the same 32 up
-//     rows) and, for the down projection, H/8 rows restricted to the group's
-//     8 blocks of F.  The shared expert's weights are copied before the wait
-//     on the router (they do not depend on the routing); routed CTAs rank the
-//     logits (every CTA the same way), then copy their gate/up rows (bulk
-//     copies) and their down slice (a 2D tensor copy: 144 bytes of each of
-//     H/8 rows) at once.  Gate/up dot products, SwiGLU and the Q8_0
-//     requantisation give the CTA's h block, which it writes to the
-//     workspace and announces on its group's counter; once the group's 8
-//     blocks are in (a bounded wait on that counter only), the down partial
-//     sums over the group's 8 h blocks, and the router-weighted partial rows
-//     are added into y with vector reductions (red.v4.f32).
+//   decode_ffn_kernel: a grid of (k+S) x F/32 CTAs (one wave), one per (expert
+//     of the token, 32-row block of h).  The shared expert's weights are
+//     copied before the wait on the router (they do not depend on the
+//     routing).  Warp 0 selects the top-k straight from the logits (one warp
+//     max and one warp min per round); the CTA of rank j issues its copies as
+//     soon as round j names its expert: the block's 32 gate rows and 32 up
+//     rows (bulk copies) and its column of the down matrix (block hb of all H
+//     rows, 2D tensor copies of 32 bytes x 256 rows) at once, while the other
+//     warps stage the Q8_0 of x.  Gate/up dot products, SwiGLU and the Q8_0
+//     requantisation give the CTA's h block; the down column against that
+//     block gives its share of every output row, added into y with vector
+//     reductions (red.v4.f32).
 //
-// No grid-wide barrier: a CTA waits only for the 7 others of its group (the
-// cooperative launch makes every CTA resident, so such a wait always ends),
-// and the groups are independent of one another (y collects their partial
-// sums).  Groups of 8 as thread-block clusters would exchange through
-// distributed shared memory instead, but with one such CTA per SM only 15
-// clusters of 8 fit on a B200 at once (GPC granularity; measured with
-// cudaOccupancyMaxActiveClusters) against the 18 a token needs.  The order of
-// the (k+S) x F/256 partial sums added into an element of y is not fixed:
-// results agree across runs to binary32 rounding, not bit for bit.
+// No CTA waits for another: a CTA's h block is all its down column needs, so
+// nothing is exchanged between CTAs and y collects (k+S) x F/32 partial sums
+// per element.  (An earlier design split the down rows over groups of 8 CTAs,
+// which exchanged their h blocks through L2 behind a release/acquire counter:
+// about 2 us more per token.)  The order of the partial sums added into an
+// element of y is not fixed: results agree across runs to binary32 rounding,
+// not bit for bit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -53,19 +49,17 @@ namespace moeq4 {
 namespace {
 
 constexpr uint32_t MBAR_LIMIT = 1u << 20;   // bounded waits: about 0.5 s
-constexpr int CL = 8;                       // CTAs per group = h blocks per F part
 constexpr int FFN_THREADS = 512;            // 16 warps
 constexpr int FFN_WARPS = FFN_THREADS / 32;
-constexpr int DN_KB = 8;                    // down blocks per F part (144 bytes of a row)
-constexpr int DN_BOX_ROWS = 256;            // rows per 2D tensor copy of the down slice
+constexpr int DN_BOX_BYTES = 32;            // bytes of each down row per tensor copy (holds the 18-byte block)
+constexpr int DN_BOX_ROWS = 256;            // rows per 2D tensor copy of the down column
 // The router kernel's timeout report: a NaN logit with this payload (arithmetic
 // on data never produces it).
 constexpr uint32_t TIMEOUT_NAN = 0x7fc0deadu;
 
 struct DecodeParams {
     int H, F, E, k, S;
-    int nF;              // F parts of 256 per expert (groups per expert)
-    int box_rows;        // rows per tensor copy of the down slice (divides H/8)
+    int nbF;             // h blocks per expert (F / 32) = CTAs per expert
     int clear_status;    // the router kernel zeroes the status word (else it accumulates)
     int force_timeout;   // CTA 0's first gate/up barrier expects 16 bytes that never come
     const float* x;
@@ -89,12 +83,12 @@ struct DecodeParams {
     float* h_dbg;
     float* y;
     uint32_t* status;
-    uint32_t* group_cnt;  // [(k+S) x nF] h blocks written per group (zeroed by the router kernel)
-    unsigned long long* kernel_ns;  // optional: [0] += CTA 0's span of the FFN kernel, [1] += 1
+    unsigned long long* kernel_ns;  // optional: CTA 0's spans, [0] from the wait, [2] from the start; [1] += 1
 };
 
 // 2D views of the down matrices for the tensor copies: rows of F/32 blocks of
-// 18 bytes, a box is 144 bytes (8 blocks) x up to 256 rows.
+// 18 bytes; a box is 32 bytes (from a 16-byte boundary, so it holds one whole
+// block) x 256 rows, written to shared memory with the 32-byte swizzle.
 struct DecodeMaps {
     CUtensorMap down, sh_down;
 };
@@ -203,17 +197,25 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
         mbar_arrive_expect_tx(&bar, (uint32_t)H * 4u);
         bulk_g2s(wr_s, p.w_router + (size_t)e * H, (uint32_t)H * 4u, &bar);
     }
+    // x into L2 ahead of the wait: a prefetch returns no data, and L2 is where
+    // the previous kernel's stores land, so the loads after the wait still see
+    // them (each CTA fetches its share of the 128-byte lines)
+    for (int i = e * 128 + tid; i < H / 32; i += (int)gridDim.x * 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p.x + 32 * i));
     pdl_launch_dependents();
     pdl_wait();  // x and the workspace are now the previous kernels' results
     if (e == 0 && tid == 0 && p.clear_status) p.status[0] = 0u;
     for (int i = e * 128 + tid; i < H; i += (int)gridDim.x * 128) p.y[i] = 0.0f;
-    for (int i = e * 128 + tid; i < (p.k + p.S) * p.nF; i += (int)gridDim.x * 128) p.group_cnt[i] = 0u;
     const bool ok = mbar_wait_bounded(&bar, 0, MBAR_LIMIT);
     const float4* x4 = reinterpret_cast<const float4*>(p.x);
     const float4* w4 = reinterpret_cast<const float4*>(wr_s);
+    float* xq_s = wr_s + H;   // the Q8_0 blocks b = e, e + E, ... of x, kept for the quantisation below
     float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;  // four independent chains
     for (int h4 = tid; h4 < H / 4; h4 += 128) {
         const float4 a = __ldcg(x4 + h4), b = w4[h4];
+        const int blk = h4 / (QK / 4);
+        if (blk % (int)gridDim.x == e)
+            reinterpret_cast<float4*>(xq_s)[(blk / (int)gridDim.x) * (QK / 4) + h4 % (QK / 4)] = a;
         a0 = fmaf(a.x, b.x, a0);
         a1 = fmaf(a.y, b.y, a1);
         a2 = fmaf(a.z, b.z, a2);
@@ -228,13 +230,14 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
         const float l = (red[0] + red[1]) + (red[2] + red[3]) + (p.bias ? __ldg(p.bias + e) : 0.0f);
         p.logits[e] = ok ? l : __uint_as_float(TIMEOUT_NAN);
     }
-    // Q8_0 of x: block b by warp 0 of CTA b (and CTA b + E, ... when H/32 > E).
+    // Q8_0 of x: block b by warp 0 of CTA b (and CTA b + E, ... when H/32 > E),
+    // from the copy in shared memory (the barrier above orders its stores).
     // A binary16 scale overflow is visible to the next kernel as an infinite scale.
     if (warp == 0) {
         for (int b = e; b < H / QK; b += gridDim.x) {
             uint16_t db;
             bool ov;
-            const int q = q8_0_lane(__ldcg(p.x + b * QK + lane), db, ov);
+            const int q = q8_0_lane(xq_s[(b / (int)gridDim.x) * QK + lane], db, ov);
             p.qa[b * QK + lane] = (int8_t)q;
             if (lane == 0) p.da[b] = db;
         }
@@ -255,13 +258,14 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int H) {
     DecodeSmem L;
     size_t o = 0;
     L.gu = o;   o += al128((size_t)64 * nbH * Q4_BYTES);       // 32 gate + 32 up rows
-    L.dn = o;   o += al128((size_t)(H / CL) * DN_KB * Q4_BYTES); // H/8 rows x 8 blocks
+    o = (o + 1023) & ~size_t(1023);                               // swizzle pattern boundary
+    L.dn = o;   o += al128((size_t)H * DN_BOX_BYTES);              // H rows x 32 bytes
     L.qa = o;   o += al128((size_t)H);
     L.da = o;   o += al128((size_t)nbH * 4);
     L.dab = o;  o += al128((size_t)nbH * 2);
     L.qsum = o; o += al128((size_t)nbH * 4);
-    L.o = o;    o += al128((size_t)(H / CL) * 4);
-    L.total = o + 128;   // slack to align the map to 128 bytes
+    L.o = o;    o += al128((size_t)H * 4);
+    L.total = o + 1024;  // slack to align the map to 1024 bytes
     return L;
 }
 
@@ -317,11 +321,32 @@ __device__ __forceinline__ int topk_rounds(const float* __restrict__ logits, int
     return (int)__reduce_or_sync(0xffffffffu, fl);
 }
 
+// The down column of one h block: o[n] = wj * (I_n * (dW_n * dh)) for every
+// row n < H, I_n the integer dot of row n's block (at byte 4A + sh/8 of the
+// row's 32 copied bytes) with the h codes hv (sum hsum).
+template <int A>
+__device__ __forceinline__ void down_column(const uint8_t* dn_s, int H, uint32_t sh, const int (&hv)[8], int hsum,
+                                            float dh, float wj, float* o_s) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll 2
+    for (int n = warp * 32 + lane; n < H; n += FFN_THREADS) {
+        const int sw = (n >> 2) & 1;
+        const uint4 c0 = *reinterpret_cast<const uint4*>(dn_s + (size_t)n * DN_BOX_BYTES + 16 * sw);
+        const uint4 c1 = *reinterpret_cast<const uint4*>(dn_s + (size_t)n * DN_BOX_BYTES + 16 * (sw ^ 1));
+        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const uint32_t dbits = __funnelshift_r(w[A], w[A + 1], sh) & 0xffffu;
+        uint32_t qs[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) qs[i] = __funnelshift_rc(w[A + i], w[A + i + 1], 16u + sh);
+        o_s[n] = wj * ((float)q4_q8_dot(qs, hv, hsum) * (half_bits_to_float(dbits) * dh));
+    }
+}
+
 __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams p,
                                                                     const __grid_constant__ DecodeMaps maps) {
     extern __shared__ __align__(16) unsigned char dsm_raw[];
-    // tensor-copy destinations 128-byte aligned (the allocation has 128 bytes of slack)
-    unsigned char* dsm = dsm_raw + ((128u - (smem_u32(dsm_raw) & 127u)) & 127u);
+    // tensor-copy destinations 1024-byte aligned (the allocation has 1024 bytes of slack)
+    unsigned char* dsm = dsm_raw + ((1024u - (smem_u32(dsm_raw) & 1023u)) & 1023u);
     __shared__ __align__(8) uint64_t bar_gu[4];
     __shared__ __align__(8) uint64_t bar_dn;
     __shared__ int idx_s[16];
@@ -329,6 +354,8 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     __shared__ float w_s[16];
     __shared__ int slot_s[17];
     __shared__ float gs[32], us[32];
+    __shared__ __align__(16) int8_t hq_s[32];
+    __shared__ float dh_s;
     __shared__ int flags_s;
 
     unsigned long long t_entry = 0;
@@ -337,14 +364,13 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = p.H, F = p.F, E = p.E, k = p.k;
     const int nbH = H / QK, nbF = F / QK;
-    const int c = blockIdx.x / CL;                  // group
-    const int r = blockIdx.x % CL;                  // CTA within the group
-    const int j = c / p.nF;                         // expert of the token: rank j < k, or k = shared
-    const int fp = c % p.nF;                        // F part: h blocks 8 fp .. 8 fp + 7
-    const int hb = fp * CL + r;                     // this CTA's h block
+    const int j = blockIdx.x / p.nbF;               // expert of the token: rank j < k, or k = shared
+    const int hb = blockIdx.x % p.nbF;              // this CTA's h block
     const bool is_shared = (j == k);
-    const int Hs = H / CL;                          // down rows of this CTA
-    const int n0 = r * Hs;
+    // this CTA's column of the down matrix: block hb of every row, inside a
+    // 32-byte box from the 16-byte boundary at or below it
+    const int dn_x0 = (hb * Q4_BYTES) & ~15;
+    const int dn_off = hb * Q4_BYTES - dn_x0;       // 0, 2, .., 14
     const size_t row_gu = (size_t)nbH * Q4_BYTES;
     const size_t gu_stride = (size_t)F * row_gu;    // bytes of one expert's gate (or up) matrix
     const DecodeSmem SL = decode_smem_layout(H);
@@ -365,11 +391,11 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     }
     __syncthreads();
 
-    // copies of this CTA's weights, issued by lanes 0..4 of warp 0 at once:
-    // lane i < 4 gate/up chunk i = 8 gate rows + the same 8 up rows on
-    // bar_gu[i]; lane 4 the down slice = rows n0 .. n0 + Hs, blocks 8 fp ..
-    // 8 fp + 7, on bar_dn
+    // copies of this CTA's weights, issued by warp 0's lanes at once: lane
+    // i < 4 gate/up chunk i = 8 gate rows + the same 8 up rows on bar_gu[i];
+    // lanes 4, 5, .. one 256-row box each of the down column on bar_dn
     const uint32_t chunk_bytes = (uint32_t)(8 * row_gu);
+    const int n_dn_box = H / DN_BOX_ROWS;
     auto issue_copies = [&](const uint8_t* Wg, const uint8_t* Wu, const CUtensorMap* dmap, int drow0) {
         if (lane < 4) {
             const int ch = lane;
@@ -378,11 +404,13 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
             const size_t src = (size_t)(hb * 32 + 8 * ch) * row_gu;
             bulk_g2s(gu_s + (size_t)(8 * ch) * row_gu, Wg + src, chunk_bytes, &bar_gu[ch]);
             bulk_g2s(gu_s + (size_t)(32 + 8 * ch) * row_gu, Wu + src, chunk_bytes, &bar_gu[ch]);
-        } else if (lane == 4) {
-            mbar_arrive_expect_tx(&bar_dn, (uint32_t)(Hs * DN_KB * Q4_BYTES));
-            for (int r0 = 0; r0 < Hs; r0 += p.box_rows)
-                tma_load_2d(dn_s + (size_t)r0 * DN_KB * Q4_BYTES, dmap, fp * DN_KB * Q4_BYTES, drow0 + r0, &bar_dn);
         }
+        if (lane == 4) mbar_arrive_expect_tx(&bar_dn, (uint32_t)(H * DN_BOX_BYTES));
+        __syncwarp();
+        const int bx = lane - 4;
+        if (bx >= 0 && bx < n_dn_box)
+            tma_load_2d(dn_s + (size_t)bx * DN_BOX_ROWS * DN_BOX_BYTES, dmap, dn_x0, drow0 + bx * DN_BOX_ROWS,
+                        &bar_dn);
     };
 
     // ---- prologue: the shared expert's copies do not depend on the routing;
@@ -391,10 +419,12 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.down)) : "memory");
         if (p.S) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.sh_down)) : "memory");
     }
-    if (is_shared && warp == 0) issue_copies(p.sh_gate, p.sh_up, &maps.sh_down, n0);
+    if (is_shared && warp == 0) issue_copies(p.sh_gate, p.sh_up, &maps.sh_down, 0);
 
     pdl_wait();  // logits, Q8_0 of x and the zeroed y are visible
     pdl_launch_dependents();
+    unsigned long long t_ready = 0;
+    if (p.kernel_ns && blockIdx.x == 0 && threadIdx.x == 0) t_ready = global_ns();
 
     if (warp == 0) {
         // ---- top-k by warp 0, straight from the logits in L2 (a NaN ranks as
@@ -410,7 +440,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
             }
             if (!is_shared && rr == j) {
                 const size_t eo = (size_t)e * gu_stride;
-                issue_copies(p.w_gate + eo, p.w_up + eo, &maps.down, e * H + n0);
+                issue_copies(p.w_gate + eo, p.w_up + eo, &maps.down, e * H);
             }
         };
         const int fl = (E <= 128) ? topk_rounds<4>(p.logits, E, k, lane, on_round)
@@ -457,7 +487,69 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     }
     __syncthreads();
 
-    // inspection arrays of the workspace (the same as the grouped path's)
+    // ---- gate/up: warp w computes rows 4w .. 4w + 3 of the 64 (0..31 gate,
+    // 32..63 up), from chunk (w mod 8) / 2; lanes split the blocks along H
+    {
+        if (!mbar_wait_bounded(&bar_gu[(warp & 7) >> 1], 0, MBAR_LIMIT)) timed_out = true;
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        const uint8_t* rows4 = gu_s + (size_t)(warp * 4) * row_gu;
+#pragma unroll 1
+        for (int b = lane; b < nbH; b += 32)
+            block_rows<4>(rows4 + (size_t)b * Q4_BYTES, row_gu, qa_s + b * QK, qsum_s[b], da_s[b], acc);
+        const float s = butterfly<4, 32>(acc);
+        if (bf_owner<4, 32>(lane)) {
+            const int row64 = warp * 4 + bf_index<4, 32>(lane);
+            (row64 < 32 ? gs : us)[row64 & 31] = s;
+        }
+    }
+    __syncthreads();
+
+    // ---- SwiGLU + Q8_0 of this CTA's h block: into shared memory for the
+    // down column, and into the workspace (hq, dh) for inspection
+    const int slot = slot_s[j];
+    if (warp == 0) {
+        const float h = swiglu(gs[lane], us[lane]);
+        if (p.h_dbg) p.h_dbg[(size_t)slot * F + hb * QK + lane] = h;
+        uint16_t db;
+        bool ov;
+        const int q = q8_0_lane(h, db, ov);
+        hq_s[lane] = (int8_t)q;
+        p.hq[(size_t)slot * F + hb * QK + lane] = (int8_t)q;
+        if (lane == 0) {
+            dh_s = half_bits_to_float(db);
+            p.dh[(size_t)slot * nbF + hb] = db;
+            if (ov) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
+        }
+    }
+    __syncthreads();
+
+    // ---- down: o[n] = w_j * (block hb of row n against the h block), every
+    // row n < H; thread rows n = 32 w + lane + 512 i.  Row n's 32 bytes hold
+    // 16-byte chunk c at 32 n + 16 (c ^ bit 2 of n) (the copy's swizzle), so
+    // a warp's 16-byte loads of 32 consecutive rows hit distinct banks.
+    {
+        const int4 h0 = reinterpret_cast<const int4*>(hq_s)[0], h1 = reinterpret_cast<const int4*>(hq_s)[1];
+        const int hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+        const int hsum = q8_block_sum(hv);
+        const float dh = dh_s, wj = is_shared ? 1.0f : w_s[j];
+        if (!mbar_wait_bounded(&bar_dn, 0, MBAR_LIMIT)) timed_out = true;
+        const uint32_t sh = (uint32_t)(dn_off & 2) * 8u;
+        switch (dn_off >> 2) {
+            case 0: down_column<0>(dn_s, H, sh, hv, hsum, dh, wj, o_s); break;
+            case 1: down_column<1>(dn_s, H, sh, hv, hsum, dh, wj, o_s); break;
+            case 2: down_column<2>(dn_s, H, sh, hv, hsum, dh, wj, o_s); break;
+            default: down_column<3>(dn_s, H, sh, hv, hsum, dh, wj, o_s); break;
+        }
+    }
+    __syncthreads();
+    // ---- combine: y[n] += o[n], vector reductions at L2
+    for (int t = tid; t < H / 4; t += FFN_THREADS)
+        red_add_v4(p.y + 4 * t, reinterpret_cast<const float4*>(o_s)[t]);
+    if (timed_out) atomicOr(&flags_s, (int)STATUS_SPIN_TIMEOUT);
+    __syncthreads();
+    if (tid == 0 && flags_s) atomicOr(p.status, (uint32_t)flags_s);
+    // inspection arrays of the workspace (the same as the grouped path's),
+    // written last: nothing in the call reads them
     if (blockIdx.x == 0) {
         for (int e = tid; e <= E + 1; e += FFN_THREADS) {
             int o = 0, chosen = 0;
@@ -477,92 +569,11 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
         }
     }
 
-    // ---- gate/up: warp w computes rows 4w .. 4w + 3 of the 64 (0..31 gate,
-    // 32..63 up), from chunk (w mod 8) / 2; lanes split the blocks along H
-    {
-        if (!mbar_wait_bounded(&bar_gu[(warp & 7) >> 1], 0, MBAR_LIMIT)) timed_out = true;
-        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        const uint8_t* rows4 = gu_s + (size_t)(warp * 4) * row_gu;
-#pragma unroll 1
-        for (int b = lane; b < nbH; b += 32)
-            block_rows<4>(rows4 + (size_t)b * Q4_BYTES, row_gu, qa_s + b * QK, qsum_s[b], da_s[b], acc);
-        const float s = butterfly<4, 32>(acc);
-        if (bf_owner<4, 32>(lane)) {
-            const int row64 = warp * 4 + bf_index<4, 32>(lane);
-            (row64 < 32 ? gs : us)[row64 & 31] = s;
-        }
-    }
-    __syncthreads();
-
-    // ---- SwiGLU + Q8_0 of this CTA's h block into the workspace (hq, dh),
-    // announced on the group's counter
-    const int slot = slot_s[j];
-    if (warp == 0) {
-        const float h = swiglu(gs[lane], us[lane]);
-        if (p.h_dbg) p.h_dbg[(size_t)slot * F + hb * QK + lane] = h;
-        uint16_t db;
-        bool ov;
-        const int q = q8_0_lane(h, db, ov);
-        p.hq[(size_t)slot * F + hb * QK + lane] = (int8_t)q;
-        if (lane == 0) {
-            p.dh[(size_t)slot * nbF + hb] = db;
-            if (ov) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
-        }
-        // the warp barrier orders every lane's stores before lane 0's release
-        // (cumulative, device scope), which the readers acquire
-        __syncwarp();
-        if (lane == 0) red_release_add_gpu(p.group_cnt + c, 1u);
-    }
-    // ---- the group's 8 blocks: a bounded wait on its counter (every CTA of
-    // the cooperative grid is resident, so the 7 others get there)
-    if (tid == 0) {
-        const uint64_t t0 = global_ns();
-        while (ld_acquire_gpu(p.group_cnt + c) < (uint32_t)CL) {
-            if (global_ns() - t0 > 1000000000ull) {   // 1 s
-                timed_out = true;
-                break;
-            }
-            __nanosleep(32);
-        }
-    }
-    __syncthreads();
-
-    // ---- down: o[n] = sum over the group's 8 blocks, n < Hs.  A task is 4
-    // rows; 8 lanes share a task, one block each, and add with a butterfly.
-    // Lane block kb: its 32 codes and scale straight from L2 into registers.
-    {
-        const int kb = lane & 7, grp = lane >> 3;
-        const int4* hsrc = reinterpret_cast<const int4*>(p.hq + (size_t)slot * F + (fp * CL + kb) * QK);
-        const int4 h0 = __ldcg(hsrc), h1 = __ldcg(hsrc + 1);
-        const float dv = half_bits_to_float(__ldcg(p.dh + (size_t)slot * nbF + fp * CL + kb));
-        const int hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-        const int qsum = q8_block_sum(hv);
-        if (!mbar_wait_bounded(&bar_dn, 0, MBAR_LIMIT)) timed_out = true;
-        const size_t row_dn = (size_t)DN_KB * Q4_BYTES;
-        for (int t0 = 0; t0 < Hs; t0 += FFN_WARPS * 16) {
-            const int row0 = t0 + warp * 16 + grp * 4;
-            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            if (row0 < Hs)
-                block_rows_reg<4>(dn_s + (size_t)row0 * row_dn + (size_t)kb * Q4_BYTES, row_dn, hv, qsum, dv, acc);
-            const float s = butterfly<4, 8>(acc);
-            if (bf_owner<4, 8>(kb) && row0 < Hs) o_s[row0 + bf_index<4, 8>(kb)] = s;
-        }
-    }
-    __syncthreads();
-    // ---- combine: y[n0 + n] += w_j * o[n] (weight 1 for the shared expert)
-    {
-        const float wj = is_shared ? 1.0f : w_s[j];
-        for (int t = tid; t < Hs / 4; t += FFN_THREADS) {
-            const float4 o = reinterpret_cast<const float4*>(o_s)[t];
-            red_add_v4(p.y + n0 + 4 * t, make_float4(wj * o.x, wj * o.y, wj * o.z, wj * o.w));
-        }
-    }
-    if (timed_out) atomicOr(&flags_s, (int)STATUS_SPIN_TIMEOUT);
-    __syncthreads();
-    if (tid == 0 && flags_s) atomicOr(p.status, (uint32_t)flags_s);
     if (p.kernel_ns && blockIdx.x == 0 && tid == 0) {
-        atomicAdd(p.kernel_ns, global_ns() - t_entry);
+        const unsigned long long t_end = global_ns();
+        atomicAdd(p.kernel_ns, t_end - t_ready);
         atomicAdd(p.kernel_ns + 1, 1ull);
+        atomicAdd(p.kernel_ns + 2, t_end - t_entry);
     }
 }
 
@@ -607,30 +618,35 @@ PFN_cuTensorMapEncodeTiled_v12000 decode_encoder() {
     return fn;
 }
 
-// `rows` rows of F/32 blocks at `base` as bytes, copied as boxes of 144 bytes
-// (8 blocks) x `box_rows` rows.
-cudaError_t encode_down(CUtensorMap* map, const uint8_t* base, uint64_t rows, int F, uint32_t box_rows) {
+// Tensor map of a down matrix ([rows][F/32 blocks of 18 bytes], a row a
+// multiple of 16 bytes): boxes of 32 bytes x 256 rows, 32-byte swizzle.
+cudaError_t encode_down(CUtensorMap* map, const uint8_t* base, uint64_t rows, int F) {
     const PFN_cuTensorMapEncodeTiled_v12000 enc = decode_encoder();
     if (!enc) return cudaErrorNotSupported;
     const cuuint64_t row_bytes = (cuuint64_t)(F / QK) * Q4_BYTES;
     const cuuint64_t dims[2] = {row_bytes, rows};
     const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {(cuuint32_t)(DN_KB * Q4_BYTES), box_rows};
+    const cuuint32_t box[2] = {(cuuint32_t)DN_BOX_BYTES, (cuuint32_t)DN_BOX_ROWS};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-size_t router_smem(const LayerView& L) { return (size_t)L.H * 4; }
+// the router row, then the Q8_0 blocks of x the CTA quantises
+size_t router_smem(const LayerView& L) {
+    return (size_t)L.H * 4 + (size_t)((L.H / QK + L.E - 1) / L.E) * QK * 4;
+}
 
 }  // namespace
 
 bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev) {
     if (T != 1 || L.E > 256 || L.k > 16) return false;
-    // one CTA per SM, all resident (the cooperative launch)
-    if ((int64_t)(L.k + L.S) * (L.F / (CL * QK)) * CL > dev.sm_count) return false;
+    // one CTA per SM in a single wave
+    if ((int64_t)(L.k + L.S) * (L.F / QK) > dev.sm_count) return false;
+    // one lane of warp 0 per 256-row box of the down column (lanes 4..31)
+    if (L.H / DN_BOX_ROWS > 28) return false;
     const DecodeSmem SL = decode_smem_layout(L.H);
     // the FFN kernel must fit with room for the router kernel's CTA beside it
     return SL.total <= (size_t)std::min(dev.max_smem_optin - 4096, 200 * 1024) && router_smem(L) <= 96 * 1024;
@@ -642,26 +658,19 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
                           cudaStream_t s) {
     DecodeParams p;
     p.H = L.H; p.F = L.F; p.E = L.E; p.k = L.k; p.S = L.S;
-    p.nF = L.F / (CL * QK);
+    p.nbF = L.F / QK;
     p.clear_status = clear_status ? 1 : 0;
     p.force_timeout = force_timeout ? 1 : 0;
     p.x = x; p.w_router = L.w_router; p.bias = L.router_bias;
     p.w_gate = L.w_gate; p.w_up = L.w_up; p.sh_gate = L.sh_gate; p.sh_up = L.sh_up;
     p.logits = ws.logits; p.topk_idx = ws.topk_idx; p.topk_w = ws.topk_w; p.qa = ws.qa; p.da = ws.da;
     p.cnt = ws.cnt; p.off = ws.off; p.sorted = ws.sorted; p.pos = ws.pos; p.hq = ws.hq; p.dh = ws.dh;
-    p.h_dbg = h_dbg; p.y = y; p.status = ws.status; p.group_cnt = ws.sync; p.kernel_ns = kernel_ns;
+    p.h_dbg = h_dbg; p.y = y; p.status = ws.status; p.kernel_ns = kernel_ns;
 
-    // rows per tensor copy: a multiple of 32 that divides H/8 (a multiple of
-    // 32), so the copies tile the CTA's rows exactly
-    const int Hs = L.H / CL;
-    int box = DN_BOX_ROWS;
-    while (Hs % box) box -= 32;
-    const uint32_t box_rows = (uint32_t)box;
     DecodeMaps maps;
     std::memset(&maps, 0, sizeof(maps));
-    p.box_rows = box;
-    cudaError_t e = encode_down(&maps.down, L.w_down, (uint64_t)L.E * L.H, L.F, box_rows);
-    if (e == cudaSuccess && L.S) e = encode_down(&maps.sh_down, L.sh_down, (uint64_t)L.H, L.F, box_rows);
+    cudaError_t e = encode_down(&maps.down, L.w_down, (uint64_t)L.E * L.H, L.F);
+    if (e == cudaSuccess && L.S) e = encode_down(&maps.sh_down, L.sh_down, (uint64_t)L.H, L.F);
     if (e != cudaSuccess) return e;
 
     int per_sm = 0;
@@ -672,7 +681,7 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
     e = kernel_occupancy(reinterpret_cast<const void*>(decode_ffn_kernel), FFN_THREADS, SL.total, &per_sm);
     if (e != cudaSuccess) return e;
 
-    cudaLaunchAttribute attrs[2];
+    cudaLaunchAttribute attrs[1];
     attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attrs[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
@@ -696,12 +705,10 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
     if (e != cudaSuccess) return e;
 
     if (ev_start && (e = record_event(ev_start, s)) != cudaSuccess) return e;
-    attrs[1].id = cudaLaunchAttributeCooperative;
-    attrs[1].val.cooperative = 1;
-    cfg.gridDim = dim3((unsigned)((L.k + L.S) * p.nF * CL));
+    cfg.gridDim = dim3((unsigned)((L.k + L.S) * p.nbF));
     cfg.blockDim = dim3(FFN_THREADS);
     cfg.dynamicSmemBytes = SL.total;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, decode_ffn_kernel, p, maps);
     if (e != cudaSuccess) return e;
     if (ev_stop && (e = record_event(ev_stop, s)) != cudaSuccess) return e;

@@ -37,7 +37,6 @@ struct Workspace {
     int32_t* pos;
     int8_t* hq;
     uint16_t* dh;
-    uint32_t* sync;   // per-group counters of the fused T = 1 kernels
 };
 
 // Test capture of the per-block integer dot products I_b of one row block of
@@ -88,7 +87,7 @@ cudaError_t launch_gateup_tc(const LayerView& L, int64_t T, const Workspace& ws,
 cudaError_t launch_down_tc(const LayerView& L, int64_t T, const Workspace& ws, float* y, const DeviceInfo& dev,
                            int tile, const BlockDotCapture* cap, cudaStream_t s);
 
-// k_decode.cu: the fused T=1 path (router kernel + cooperative FFN kernel,
+// k_decode.cu: the fused T=1 path (router kernel + FFN kernel,
 // chained with programmatic dependent launch).  Events, if given, bracket the
 // FFN kernel.
 bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev);

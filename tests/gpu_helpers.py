@@ -59,6 +59,16 @@ def pairs_from_slots(lw, T, v, arr):
     return out
 
 
+# Two runs of the T = 1 path add the (k+S) x F/32 partial sums of an output
+# element of y (144 for the 2048/512 layer with 8 routed experts and a shared
+# one) in different orders.  Recursive summation of n binary32 terms errs by
+# at most (n - 1) u sum|t| (u = 2^-24), so two orders differ by at most
+# 2 (n - 1) u sum|t|: about 1.6e-4 of rule13's scale when sum|t| is ten times
+# the row's rms; rounding errors of random sign stay near sqrt(n) u of it
+# (about 1e-6).  The run-to-run comparisons take 1e-5, between the two.
+ORDER_REL = 1e-5
+
+
 def rule13(y, y_ref, rel=1e-3):
     """Per element |y - y_ref| <= rel * max(|y_ref|, rms of its row).
     Returns (ok, worst ratio)."""

@@ -108,9 +108,9 @@ def test_workspace_bytes_and_layout(lib):
     n947 = lib.moe_q4_ffn_workspace_bytes(ctypes.byref(L), 947)
     assert 0 < n1 < n947
     assert lib.moe_q4_ffn_workspace_bytes(ctypes.byref(make(top_k=0)), 4) == 0
-    offs = (ctypes.c_size_t * 17)()
+    offs = (ctypes.c_size_t * 16)()
     lib.moe_q4_workspace_layout.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int]
-    assert lib.moe_q4_workspace_layout(ctypes.byref(L), 947, offs, 17) == 0
+    assert lib.moe_q4_workspace_layout(ctypes.byref(L), 947, offs, 16) == 0
     o = list(offs)
     assert o[0] == 0 and all(b > a for a, b in zip(o, o[1:])) and all(v % 256 == 0 for v in o)
     assert o[-1] == n947
@@ -118,8 +118,8 @@ def test_workspace_bytes_and_layout(lib):
     P = T * k
     # hq spans (P + T) slots of F bytes
     assert o[14] - o[13] >= (P + T) * F
-    # the fused decode kernels' group counters: (k + S) x F / 256
-    assert o[16] - o[15] >= 4 * (k + 1) * (F // 256)
+    # dh: one binary16 scale per 32 values of hq
+    assert o[15] - o[14] >= 2 * (P + T) * (F // 32)
 
 
 def test_other_entry_points_reject_bad_args(lib):

@@ -9,7 +9,7 @@ import time
 import pytest
 import torch
 
-from gpu_helpers import rule13, workload
+from gpu_helpers import ORDER_REL, rule13, workload
 
 pytestmark = pytest.mark.gpu
 
@@ -37,11 +37,11 @@ def test_decode_wait_timeout_reported_and_recovered():
     status = int(m.workspace_views(L, 1, ws)["status"][0].item())
     assert status & m.STATUS_SPIN_TIMEOUT
     # the partial sums are added into y in no fixed order: equal to rounding
-    assert rule13(y.cpu().numpy(), y_ref.cpu().numpy(), 1e-6)[0]
+    assert rule13(y.cpu().numpy(), y_ref.cpu().numpy(), ORDER_REL)[0]
     assert elapsed < 60.0
 
     y2 = torch.empty_like(xt)
     m.moe_q4_ffn_forward_debug(L, xt, y2, ws, path=m.PATH_DECODE)
     torch.cuda.synchronize()
     assert int(m.workspace_views(L, 1, ws)["status"][0].item()) == 0
-    assert rule13(y2.cpu().numpy(), y_ref.cpu().numpy(), 1e-6)[0]
+    assert rule13(y2.cpu().numpy(), y_ref.cpu().numpy(), ORDER_REL)[0]

@@ -14,7 +14,7 @@ import torch
 
 import oracle
 import synth
-from gpu_helpers import (check_permutation, check_routing, expected_block_dots, free_running_report, rule13,
+from gpu_helpers import (ORDER_REL, check_permutation, check_routing, expected_block_dots, free_running_report, rule13,
                          run_forward, tile_boundary_tokens, teacher_forced_check, workload)
 
 pytestmark = pytest.mark.gpu
@@ -336,8 +336,29 @@ def test_forward_host_single_token(pinned):
         yh = yh.pin_memory() if pinned else yh
         m.moe_q4_ffn_forward_host(L, xh, yh, ws)
         torch.cuda.synchronize()
-        ok, worst = rule13(yh.numpy(), y_dev, 1e-6)
+        ok, worst = rule13(yh.numpy(), y_dev, ORDER_REL)
         assert ok, worst
+
+
+def test_decode_kernel_timer():
+    """The fused T = 1 path's device timer: one count per call, the span from
+    the dependency wait no longer than the span from the kernel's start, both
+    positive and below a millisecond a call; results unchanged by timing."""
+    x, lw = workload("decode_t1", T=8)
+    L = m.Layer.from_host(lw)
+    ws = m.alloc_workspace(m.moe_q4_ffn_workspace_bytes(L, 1))
+    timer = torch.zeros(3, dtype=torch.int64, device="cuda")
+    xd = torch.from_numpy(x).cuda()
+    y_t, y_u = torch.empty_like(xd), torch.empty_like(xd)
+    for t in range(8):
+        m.moe_q4_ffn_forward_debug(L, xd[t:t + 1], y_t[t:t + 1], ws, path=m.PATH_DECODE, decode_kernel_ns=timer)
+        m.moe_q4_ffn_forward_debug(L, xd[t:t + 1], y_u[t:t + 1], ws, path=m.PATH_DECODE)
+    torch.cuda.synchronize()
+    ready_ns, n, resident_ns = timer.cpu().tolist()
+    assert n == 8
+    assert 0 < ready_ns <= resident_ns < 8 * 1_000_000
+    ok, worst = rule13(y_t.cpu().numpy(), y_u.cpu().numpy(), ORDER_REL)
+    assert ok, worst
 
 
 def test_scale_overflow_reported_in_status():

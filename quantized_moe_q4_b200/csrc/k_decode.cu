@@ -133,34 +133,36 @@ __device__ __forceinline__ bool bf_owner(int lane) {
     return (lane & (W / V - 1)) == 0;
 }
 
-// acc[r] += W4A8 term of one block in NR rows (stride row_bytes) against one
-// staged Q8_0 block, the activation loaded once for all rows: NR independent
-// dependency chains per lane.
+// acc[r] += W4A8 terms of a pair of blocks (36 bytes from a 4-byte boundary:
+// the pair's first byte is at 36 p) in NR rows (stride row_bytes), against
+// the pair's two Q8_0 blocks in registers.  Nine 32-bit loads a row; lanes
+// taking consecutive pairs hit banks 9 l + i, all distinct.
 template <int NR>
-__device__ __forceinline__ void block_rows(const uint8_t* rows, size_t row_bytes, const int8_t* q_blk, int qsum,
-                                           float da, float (&acc)[NR]) {
-    const int4* qv = reinterpret_cast<const int4*>(q_blk);
-    const int4 a0 = qv[0], a1 = qv[1];
-    const int qa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+__device__ __forceinline__ void pair_rows(const uint8_t* rows, size_t row_bytes, const int (&qa0)[8],
+                                          const int (&qa1)[8], int qs0, int qs1, float da0, float da1,
+                                          float (&acc)[NR]) {
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
-        uint32_t qs[4], dbits;
-        load_q4_block_smem(rows + (size_t)r * row_bytes, qs, dbits);
-        acc[r] = fmaf((float)q4_q8_dot(qs, qa, qsum), half_bits_to_float(dbits) * da, acc[r]);
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(rows + (size_t)r * row_bytes);
+        uint32_t v[9];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) v[i] = w[i];
+        // block 0: scale in bytes 0-1, nibbles in 2-17; block 1: scale in 18-19, nibbles in 20-35
+        uint32_t q0[4], q1[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            q0[i] = __funnelshift_r(v[i], v[i + 1], 16);
+            q1[i] = v[5 + i];
+        }
+        acc[r] = fmaf((float)q4_q8_dot(q0, qa0, qs0), half_bits_to_float(v[0] & 0xffffu) * da0, acc[r]);
+        acc[r] = fmaf((float)q4_q8_dot(q1, qa1, qs1), half_bits_to_float(v[4] >> 16) * da1, acc[r]);
     }
 }
 
-// block_rows with the activation block already in registers.
-template <int NR>
-__device__ __forceinline__ void block_rows_reg(const uint8_t* rows, size_t row_bytes, const int (&qa)[8], int qsum,
-                                               float da, float (&acc)[NR]) {
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-        uint32_t qs[4], dbits;
-        load_q4_block_smem(rows + (size_t)r * row_bytes, qs, dbits);
-        acc[r] = fmaf((float)q4_q8_dot(qs, qa, qsum), half_bits_to_float(dbits) * da, acc[r]);
-    }
-}
+// Q8_0 codes of x in shared memory: the codes of block pair p (64 bytes) at
+// byte 80 p, so that 16-byte loads by lanes taking consecutive pairs fall in
+// distinct banks.
+__host__ __device__ constexpr int qa_pair_off(int p) { return 80 * p; }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
     asm volatile(
@@ -260,7 +262,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int H) {
     L.gu = o;   o += al128((size_t)64 * nbH * Q4_BYTES);       // 32 gate + 32 up rows
     o = (o + 1023) & ~size_t(1023);                               // swizzle pattern boundary
     L.dn = o;   o += al128((size_t)H * DN_BOX_BYTES);              // H rows x 32 bytes
-    L.qa = o;   o += al128((size_t)H);
+    L.qa = o;   o += al128((size_t)qa_pair_off(H / 64));
     L.da = o;   o += al128((size_t)nbH * 4);
     L.dab = o;  o += al128((size_t)nbH * 2);
     L.qsum = o; o += al128((size_t)nbH * 4);
@@ -328,7 +330,7 @@ template <int A>
 __device__ __forceinline__ void down_column(const uint8_t* dn_s, int H, uint32_t sh, const int (&hv)[8], int hsum,
                                             float dh, float wj, float* o_s) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll 2
+#pragma unroll 4
     for (int n = warp * 32 + lane; n < H; n += FFN_THREADS) {
         const int sw = (n >> 2) & 1;
         const uint4 c0 = *reinterpret_cast<const uint4*>(dn_s + (size_t)n * DN_BOX_BYTES + 16 * sw);
@@ -354,8 +356,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     __shared__ float w_s[16];
     __shared__ int slot_s[17];
     __shared__ float gs[32], us[32];
-    __shared__ __align__(16) int8_t hq_s[32];
-    __shared__ float dh_s;
+    __shared__ __align__(16) int8_t hq_w[FFN_WARPS * 32];
     __shared__ int flags_s;
 
     unsigned long long t_entry = 0;
@@ -470,7 +471,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
         // ---- warps 1..: the Q8_0 of x into shared memory by cp.async, then
         // its block scales and block sums (the -8 offset of the nibbles)
         const int t = tid - 32, nt = FFN_THREADS - 32;
-        for (int i = t; i < H / 16; i += nt) cp_async16(qa_s + 16 * i, p.qa + 16 * i);
+        for (int i = t; i < H / 16; i += nt) cp_async16(qa_s + qa_pair_off(i >> 2) + 16 * (i & 3), p.qa + 16 * i);
         for (int i = t; i < nbH / 8; i += nt) cp_async16(dab_s + 8 * i, p.da + 8 * i);
         cp_async_wait_all();
         asm volatile("bar.sync 1, %0;" ::"n"(FFN_THREADS - 32) : "memory");
@@ -478,7 +479,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
             const uint32_t bits = dab_s[b];
             if ((bits & 0x7fffu) == 0x7c00u) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
             da_s[b] = half_bits_to_float(bits);
-            const int* qw = reinterpret_cast<const int*>(qa_s + b * QK);
+            const int* qw = reinterpret_cast<const int*>(qa_s + qa_pair_off(b >> 1) + QK * (b & 1));
             int s = 0;
 #pragma unroll
             for (int q = 0; q < 8; ++q) s = __dp4a(qw[q], 0x01010101, s);
@@ -493,9 +494,16 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
         if (!mbar_wait_bounded(&bar_gu[(warp & 7) >> 1], 0, MBAR_LIMIT)) timed_out = true;
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         const uint8_t* rows4 = gu_s + (size_t)(warp * 4) * row_gu;
+        // lane l takes block pairs l, l + 32, ..
 #pragma unroll 1
-        for (int b = lane; b < nbH; b += 32)
-            block_rows<4>(rows4 + (size_t)b * Q4_BYTES, row_gu, qa_s + b * QK, qsum_s[b], da_s[b], acc);
+        for (int pr = lane; pr < nbH / 2; pr += 32) {
+            const int4* a = reinterpret_cast<const int4*>(qa_s + qa_pair_off(pr));
+            const int4 a0 = a[0], a1 = a[1], a2 = a[2], a3 = a[3];
+            const int qa0[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const int qa1[8] = {a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
+            pair_rows<4>(rows4 + (size_t)pr * 2 * Q4_BYTES, row_gu, qa0, qa1, qsum_s[2 * pr], qsum_s[2 * pr + 1],
+                         da_s[2 * pr], da_s[2 * pr + 1], acc);
+        }
         const float s = butterfly<4, 32>(acc);
         if (bf_owner<4, 32>(lane)) {
             const int row64 = warp * 4 + bf_index<4, 32>(lane);
@@ -504,34 +512,42 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     }
     __syncthreads();
 
-    // ---- SwiGLU + Q8_0 of this CTA's h block: into shared memory for the
-    // down column, and into the workspace (hq, dh) for inspection
+    // ---- SwiGLU + Q8_0 of this CTA's h block, by every warp (each needs all
+    // 32 codes for the down column; the arithmetic is the same in every warp):
+    // lane l's code into the warp's own 32 bytes of shared memory, read back as
+    // eight words.  Warp 0 writes h, the codes and the scale to the workspace.
     const int slot = slot_s[j];
-    if (warp == 0) {
+    int hv[8], hsum;
+    float dh;
+    {
         const float h = swiglu(gs[lane], us[lane]);
-        if (p.h_dbg) p.h_dbg[(size_t)slot * F + hb * QK + lane] = h;
         uint16_t db;
         bool ov;
         const int q = q8_0_lane(h, db, ov);
-        hq_s[lane] = (int8_t)q;
-        p.hq[(size_t)slot * F + hb * QK + lane] = (int8_t)q;
-        if (lane == 0) {
-            dh_s = half_bits_to_float(db);
-            p.dh[(size_t)slot * nbF + hb] = db;
-            if (ov) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
+        int8_t* hw = hq_w + 32 * warp;
+        hw[lane] = (int8_t)q;
+        __syncwarp();
+        const int4 h0 = reinterpret_cast<const int4*>(hw)[0], h1 = reinterpret_cast<const int4*>(hw)[1];
+        hv[0] = h0.x; hv[1] = h0.y; hv[2] = h0.z; hv[3] = h0.w;
+        hv[4] = h1.x; hv[5] = h1.y; hv[6] = h1.z; hv[7] = h1.w;
+        hsum = q8_block_sum(hv);
+        dh = half_bits_to_float(db);
+        if (warp == 0) {
+            if (p.h_dbg) p.h_dbg[(size_t)slot * F + hb * QK + lane] = h;
+            p.hq[(size_t)slot * F + hb * QK + lane] = (int8_t)q;
+            if (lane == 0) {
+                p.dh[(size_t)slot * nbF + hb] = db;
+                if (ov) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
+            }
         }
     }
-    __syncthreads();
 
     // ---- down: o[n] = w_j * (block hb of row n against the h block), every
     // row n < H; thread rows n = 32 w + lane + 512 i.  Row n's 32 bytes hold
     // 16-byte chunk c at 32 n + 16 (c ^ bit 2 of n) (the copy's swizzle), so
     // a warp's 16-byte loads of 32 consecutive rows hit distinct banks.
     {
-        const int4 h0 = reinterpret_cast<const int4*>(hq_s)[0], h1 = reinterpret_cast<const int4*>(hq_s)[1];
-        const int hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-        const int hsum = q8_block_sum(hv);
-        const float dh = dh_s, wj = is_shared ? 1.0f : w_s[j];
+        const float wj = is_shared ? 1.0f : w_s[j];
         if (!mbar_wait_bounded(&bar_dn, 0, MBAR_LIMIT)) timed_out = true;
         const uint32_t sh = (uint32_t)(dn_off & 2) * 8u;
         switch (dn_off >> 2) {
@@ -541,12 +557,11 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
             default: down_column<3>(dn_s, H, sh, hv, hsum, dh, wj, o_s); break;
         }
     }
+    if (timed_out) atomicOr(&flags_s, (int)STATUS_SPIN_TIMEOUT);
     __syncthreads();
     // ---- combine: y[n] += o[n], vector reductions at L2
     for (int t = tid; t < H / 4; t += FFN_THREADS)
         red_add_v4(p.y + 4 * t, reinterpret_cast<const float4*>(o_s)[t]);
-    if (timed_out) atomicOr(&flags_s, (int)STATUS_SPIN_TIMEOUT);
-    __syncthreads();
     if (tid == 0 && flags_s) atomicOr(p.status, (uint32_t)flags_s);
     // inspection arrays of the workspace (the same as the grouped path's),
     // written last: nothing in the call reads them

@@ -9,9 +9,9 @@
 // chained with programmatic dependent launch (PDL):
 //
 //   decode_router_kernel: one CTA per expert.  Before waiting on the previous
-//     kernel it bulk-copies its router row into shared memory; then the logit
-//     (four independent FMA chains); the first H/32 CTAs quantise one Q8_0
-//     block of x each; y is zeroed (the FFN kernel accumulates into it).
+//     kernel it bulk-copies its router row into shared memory and prefetches
+//     x into L2; then the logit (four independent FMA chains); y is zeroed
+//     (the FFN kernel accumulates into it).
 //   decode_ffn_kernel: a grid of (k+S) x F/32 CTAs (one wave), one per (expert
 //     of the token, 32-row block of h).  The shared expert's weights are
 //     copied before the wait on the router (they do not depend on the
@@ -19,11 +19,11 @@
 //     max and one warp min per round); the CTA of rank j issues its copies as
 //     soon as round j names its expert: the block's 32 gate rows and 32 up
 //     rows (bulk copies) and its column of the down matrix (block hb of all H
-//     rows, 2D tensor copies of 32 bytes x 256 rows) at once, while the other
-//     warps stage the Q8_0 of x.  Gate/up dot products, SwiGLU and the Q8_0
-//     requantisation give the CTA's h block; the down column against that
-//     block gives its share of every output row, added into y with vector
-//     reductions (red.v4.f32).
+//     rows, 2D tensor copies of 32 bytes x 256 rows) at once, while the
+//     other warps quantise x (Q8_0) themselves.  Gate/up dot products,
+//     SwiGLU and the Q8_0 requantisation give the CTA's h block; the down
+//     column against that block gives its share of every output row, added
+//     into y with vector reductions (red.v4.f32).
 //
 // No CTA waits for another: a CTA's h block is all its down column needs, so
 // nothing is exchanged between CTAs and y collects (k+S) x F/32 partial sums
@@ -204,6 +204,7 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
     // them (each CTA fetches its share of the 128-byte lines)
     for (int i = e * 128 + tid; i < H / 32; i += (int)gridDim.x * 128)
         asm volatile("prefetch.global.L2 [%0];" ::"l"(p.x + 32 * i));
+    const float bias = p.bias ? __ldg(p.bias + e) : 0.0f;   // a weight: read before the wait
     pdl_launch_dependents();
     pdl_wait();  // x and the workspace are now the previous kernels' results
     if (e == 0 && tid == 0 && p.clear_status) p.status[0] = 0u;
@@ -211,13 +212,9 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
     const bool ok = mbar_wait_bounded(&bar, 0, MBAR_LIMIT);
     const float4* x4 = reinterpret_cast<const float4*>(p.x);
     const float4* w4 = reinterpret_cast<const float4*>(wr_s);
-    float* xq_s = wr_s + H;   // the Q8_0 blocks b = e, e + E, ... of x, kept for the quantisation below
     float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;  // four independent chains
     for (int h4 = tid; h4 < H / 4; h4 += 128) {
         const float4 a = __ldcg(x4 + h4), b = w4[h4];
-        const int blk = h4 / (QK / 4);
-        if (blk % (int)gridDim.x == e)
-            reinterpret_cast<float4*>(xq_s)[(blk / (int)gridDim.x) * (QK / 4) + h4 % (QK / 4)] = a;
         a0 = fmaf(a.x, b.x, a0);
         a1 = fmaf(a.y, b.y, a1);
         a2 = fmaf(a.z, b.z, a2);
@@ -229,20 +226,8 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
     if (lane == 0) red[warp] = acc;
     __syncthreads();
     if (tid == 0) {
-        const float l = (red[0] + red[1]) + (red[2] + red[3]) + (p.bias ? __ldg(p.bias + e) : 0.0f);
+        const float l = (red[0] + red[1]) + (red[2] + red[3]) + bias;
         p.logits[e] = ok ? l : __uint_as_float(TIMEOUT_NAN);
-    }
-    // Q8_0 of x: block b by warp 0 of CTA b (and CTA b + E, ... when H/32 > E),
-    // from the copy in shared memory (the barrier above orders its stores).
-    // A binary16 scale overflow is visible to the next kernel as an infinite scale.
-    if (warp == 0) {
-        for (int b = e; b < H / QK; b += gridDim.x) {
-            uint16_t db;
-            bool ov;
-            const int q = q8_0_lane(xq_s[(b / (int)gridDim.x) * QK + lane], db, ov);
-            p.qa[b * QK + lane] = (int8_t)q;
-            if (lane == 0) p.da[b] = db;
-        }
     }
 }
 
@@ -250,7 +235,7 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
 // K2: gate/up + SwiGLU + requant, exchange within a group, down + combine.
 // ---------------------------------------------------------------------------
 struct DecodeSmem {
-    size_t gu, dn, qa, da, dab, qsum, o, total;  // byte offsets
+    size_t gu, dn, qa, da, qsum, o, total;  // byte offsets
 };
 
 __host__ __device__ inline size_t al128(size_t v) { return (v + 127) & ~size_t(127); }
@@ -264,7 +249,6 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int H) {
     L.dn = o;   o += al128((size_t)H * DN_BOX_BYTES);              // H rows x 32 bytes
     L.qa = o;   o += al128((size_t)qa_pair_off(H / 64));
     L.da = o;   o += al128((size_t)nbH * 4);
-    L.dab = o;  o += al128((size_t)nbH * 2);
     L.qsum = o; o += al128((size_t)nbH * 4);
     L.o = o;    o += al128((size_t)H * 4);
     L.total = o + 1024;  // slack to align the map to 1024 bytes
@@ -379,7 +363,6 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     uint8_t* dn_s = dsm + SL.dn;
     int8_t* qa_s = reinterpret_cast<int8_t*>(dsm + SL.qa);
     float* da_s = reinterpret_cast<float*>(dsm + SL.da);
-    uint16_t* dab_s = reinterpret_cast<uint16_t*>(dsm + SL.dab);
     int* qsum_s = reinterpret_cast<int*>(dsm + SL.qsum);
     float* o_s = reinterpret_cast<float*>(dsm + SL.o);
     bool timed_out = false;
@@ -468,22 +451,43 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
         }
         if (lane == 0) slot_s[k] = k;  // the shared expert's slot: P + t
     } else {
-        // ---- warps 1..: the Q8_0 of x into shared memory by cp.async, then
-        // its block scales and block sums (the -8 offset of the nibbles)
-        const int t = tid - 32, nt = FFN_THREADS - 32;
-        for (int i = t; i < H / 16; i += nt) cp_async16(qa_s + qa_pair_off(i >> 2) + 16 * (i & 3), p.qa + 16 * i);
-        for (int i = t; i < nbH / 8; i += nt) cp_async16(dab_s + 8 * i, p.da + 8 * i);
-        cp_async_wait_all();
-        asm volatile("bar.sync 1, %0;" ::"n"(FFN_THREADS - 32) : "memory");
-        for (int b = t; b < nbH; b += nt) {
-            const uint32_t bits = dab_s[b];
-            if ((bits & 0x7fffu) == 0x7c00u) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
-            da_s[b] = half_bits_to_float(bits);
-            const int* qw = reinterpret_cast<const int*>(qa_s + qa_pair_off(b >> 1) + QK * (b & 1));
-            int s = 0;
+        // ---- warps 1..: the Q8_0 of x, all blocks in one pass: thread t
+        // quantises values 4t .. 4t + 3 (8 threads a block: the block's
+        // absolute maximum over 8 lanes, then per value the arithmetic of
+        // every Q8_0 step: d = amax / 127, q = round half away from zero of
+        // x / d, clamped to +-127); codes into shared memory (pair layout),
+        // scales and code sums beside them; CTA 0 also writes them to the
+        // workspace.  A binary16 scale overflow is reported.
+        for (int t4 = tid - 32; t4 < H / 4; t4 += FFN_THREADS - 32) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(p.x) + t4);
+            float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 #pragma unroll
-            for (int q = 0; q < 8; ++q) s = __dp4a(qw[q], 0x01010101, s);
-            qsum_s[b] = s;
+            for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            const float d = __fdiv_rn(a, 127.0f);
+            int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+            if (d != 0.0f) {
+                q0 = max(-127, min(127, round_half_away(__fdiv_rn(v.x, d))));
+                q1 = max(-127, min(127, round_half_away(__fdiv_rn(v.y, d))));
+                q2 = max(-127, min(127, round_half_away(__fdiv_rn(v.z, d))));
+                q3 = max(-127, min(127, round_half_away(__fdiv_rn(v.w, d))));
+            }
+            const uint32_t word = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) |
+                                  ((uint32_t)(q2 & 0xff) << 16) | ((uint32_t)(q3 & 0xff) << 24);
+            const int b = t4 >> 3, part = t4 & 7;   // block, word within it
+            *reinterpret_cast<uint32_t*>(qa_s + qa_pair_off(b >> 1) + QK * (b & 1) + 4 * part) = word;
+            int qs = (q0 + q1) + (q2 + q3);
+#pragma unroll
+            for (int o = 4; o > 0; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+            const uint16_t db = __half_as_ushort(__float2half_rn(d));
+            if (part == 0) {
+                da_s[b] = half_bits_to_float(db);
+                qsum_s[b] = qs;
+                if ((db & 0x7fffu) == 0x7c00u) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
+            }
+            if (blockIdx.x == 0) {
+                reinterpret_cast<uint32_t*>(p.qa)[t4] = word;
+                if (part == 0) p.da[b] = db;
+            }
         }
     }
     __syncthreads();
@@ -519,6 +523,9 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     const int slot = slot_s[j];
     int hv[8], hsum;
     float dh;
+    float h_mine = 0.0f;      // warp 0: lane's h value, code and the scale, written out at the end
+    int q_mine = 0;
+    uint16_t db_mine = 0;
     {
         const float h = swiglu(gs[lane], us[lane]);
         uint16_t db;
@@ -533,12 +540,10 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
         hsum = q8_block_sum(hv);
         dh = half_bits_to_float(db);
         if (warp == 0) {
-            if (p.h_dbg) p.h_dbg[(size_t)slot * F + hb * QK + lane] = h;
-            p.hq[(size_t)slot * F + hb * QK + lane] = (int8_t)q;
-            if (lane == 0) {
-                p.dh[(size_t)slot * nbF + hb] = db;
-                if (ov) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
-            }
+            h_mine = h;
+            q_mine = q;
+            db_mine = db;
+            if (ov && lane == 0) atomicOr(&flags_s, (int)STATUS_SCALE_OVERFLOW);
         }
     }
 
@@ -563,8 +568,14 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
     for (int t = tid; t < H / 4; t += FFN_THREADS)
         red_add_v4(p.y + 4 * t, reinterpret_cast<const float4*>(o_s)[t]);
     if (tid == 0 && flags_s) atomicOr(p.status, (uint32_t)flags_s);
-    // inspection arrays of the workspace (the same as the grouped path's),
-    // written last: nothing in the call reads them
+    // the h block, its codes and scale, and the inspection arrays of the
+    // workspace (the same as the grouped path's), written last: nothing in
+    // the call reads them
+    if (warp == 0) {
+        if (p.h_dbg) p.h_dbg[(size_t)slot * F + hb * QK + lane] = h_mine;
+        p.hq[(size_t)slot * F + hb * QK + lane] = (int8_t)q_mine;
+        if (lane == 0) p.dh[(size_t)slot * nbF + hb] = db_mine;
+    }
     if (blockIdx.x == 0) {
         for (int e = tid; e <= E + 1; e += FFN_THREADS) {
             int o = 0, chosen = 0;
@@ -649,10 +660,8 @@ cudaError_t encode_down(CUtensorMap* map, const uint8_t* base, uint64_t rows, in
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// the router row, then the Q8_0 blocks of x the CTA quantises
-size_t router_smem(const LayerView& L) {
-    return (size_t)L.H * 4 + (size_t)((L.H / QK + L.E - 1) / L.E) * QK * 4;
-}
+// the router row
+size_t router_smem(const LayerView& L) { return (size_t)L.H * 4; }
 
 }  // namespace
 

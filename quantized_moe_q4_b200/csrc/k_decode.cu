@@ -9,9 +9,9 @@
 // chained with programmatic dependent launch (PDL):
 //
 //   decode_router_kernel: one CTA per expert.  Before waiting on the previous
-//     kernel it bulk-copies its router row into shared memory and prefetches
-//     x into L2; then the logit (four independent FMA chains); y is zeroed
-//     (the FFN kernel accumulates into it).
+//     kernel it loads its router row into registers and prefetches x into
+//     L2; then the logit (four independent FMA chains); y is zeroed (the FFN
+//     kernel accumulates into it).
 //   decode_ffn_kernel: a grid of (k+S) x F/32 CTAs (one wave), one per (expert
 //     of the token, 32-row block of h).  The shared expert's weights are
 //     copied before the wait on the router (they do not depend on the
@@ -53,9 +53,7 @@ constexpr int FFN_THREADS = 512;            // 16 warps
 constexpr int FFN_WARPS = FFN_THREADS / 32;
 constexpr int DN_BOX_BYTES = 32;            // bytes of each down row per tensor copy (holds the 18-byte block)
 constexpr int DN_BOX_ROWS = 256;            // rows per 2D tensor copy of the down column
-// The router kernel's timeout report: a NaN logit with this payload (arithmetic
-// on data never produces it).
-constexpr uint32_t TIMEOUT_NAN = 0x7fc0deadu;
+constexpr int ROUTER_STEPS = 5;             // float4 steps of 128 in a router row: H <= 2560
 
 struct DecodeParams {
     int H, F, E, k, S;
@@ -184,41 +182,37 @@ __device__ __forceinline__ void red_add_v4(float* y, float4 v) {
 // K1: router logits (one CTA per expert), Q8_0 of x, y zeroed.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
-    extern __shared__ __align__(16) unsigned char dsm_router[];
-    float* wr_s = reinterpret_cast<float*>(dsm_router);
-    __shared__ __align__(8) uint64_t bar;
     __shared__ float red[4];
     const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = p.H;
-    if (tid == 0) {
-        mbar_init(&bar, 1);
-        mbar_fence_init();
-    }
-    __syncthreads();
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&bar, (uint32_t)H * 4u);
-        bulk_g2s(wr_s, p.w_router + (size_t)e * H, (uint32_t)H * 4u, &bar);
-    }
+    // the router row (a weight: read before the wait) into registers, float4
+    // steps tid, tid + 128, .. (at most ROUTER_STEPS of them)
+    const float4* w4 = reinterpret_cast<const float4*>(p.w_router + (size_t)e * H);
+    float4 w[ROUTER_STEPS];
+#pragma unroll
+    for (int i = 0; i < ROUTER_STEPS; ++i)
+        w[i] = (tid + 128 * i < H / 4) ? __ldg(w4 + tid + 128 * i) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     // x into L2 ahead of the wait: a prefetch returns no data, and L2 is where
     // the previous kernel's stores land, so the loads after the wait still see
     // them (each CTA fetches its share of the 128-byte lines)
     for (int i = e * 128 + tid; i < H / 32; i += (int)gridDim.x * 128)
         asm volatile("prefetch.global.L2 [%0];" ::"l"(p.x + 32 * i));
-    const float bias = p.bias ? __ldg(p.bias + e) : 0.0f;   // a weight: read before the wait
+    const float bias = p.bias ? __ldg(p.bias + e) : 0.0f;
     pdl_launch_dependents();
     pdl_wait();  // x and the workspace are now the previous kernels' results
     if (e == 0 && tid == 0 && p.clear_status) p.status[0] = 0u;
     for (int i = e * 128 + tid; i < H; i += (int)gridDim.x * 128) p.y[i] = 0.0f;
-    const bool ok = mbar_wait_bounded(&bar, 0, MBAR_LIMIT);
     const float4* x4 = reinterpret_cast<const float4*>(p.x);
-    const float4* w4 = reinterpret_cast<const float4*>(wr_s);
     float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;  // four independent chains
-    for (int h4 = tid; h4 < H / 4; h4 += 128) {
-        const float4 a = __ldcg(x4 + h4), b = w4[h4];
-        a0 = fmaf(a.x, b.x, a0);
-        a1 = fmaf(a.y, b.y, a1);
-        a2 = fmaf(a.z, b.z, a2);
-        a3 = fmaf(a.w, b.w, a3);
+#pragma unroll
+    for (int i = 0; i < ROUTER_STEPS; ++i) {
+        if (tid + 128 * i < H / 4) {
+            const float4 a = __ldcg(x4 + tid + 128 * i), b = w[i];
+            a0 = fmaf(a.x, b.x, a0);
+            a1 = fmaf(a.y, b.y, a1);
+            a2 = fmaf(a.z, b.z, a2);
+            a3 = fmaf(a.w, b.w, a3);
+        }
     }
     float acc = (a0 + a1) + (a2 + a3);
 #pragma unroll
@@ -226,8 +220,7 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
     if (lane == 0) red[warp] = acc;
     __syncthreads();
     if (tid == 0) {
-        const float l = (red[0] + red[1]) + (red[2] + red[3]) + bias;
-        p.logits[e] = ok ? l : __uint_as_float(TIMEOUT_NAN);
+        p.logits[e] = (red[0] + red[1]) + (red[2] + red[3]) + bias;
     }
 }
 
@@ -284,8 +277,7 @@ __device__ __forceinline__ int topk_rounds(const float* __restrict__ logits, int
         key[i] = 0u;
         if (e < E) {
             const float l = __ldcg(logits + e);
-            if (!isfinite(l))
-                fl |= (__float_as_uint(l) == TIMEOUT_NAN) ? STATUS_SPIN_TIMEOUT : STATUS_NONFINITE_LOGIT;
+            if (!isfinite(l)) fl |= STATUS_NONFINITE_LOGIT;
             key[i] = logit_key(l != l ? -INFINITY : l);
         }
     }
@@ -660,8 +652,7 @@ cudaError_t encode_down(CUtensorMap* map, const uint8_t* base, uint64_t rows, in
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// the router row
-size_t router_smem(const LayerView& L) { return (size_t)L.H * 4; }
+
 
 }  // namespace
 
@@ -673,7 +664,7 @@ bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev) {
     if (L.H / DN_BOX_ROWS > 28) return false;
     const DecodeSmem SL = decode_smem_layout(L.H);
     // the FFN kernel must fit with room for the router kernel's CTA beside it
-    return SL.total <= (size_t)std::min(dev.max_smem_optin - 4096, 200 * 1024) && router_smem(L) <= 96 * 1024;
+    return L.H / 4 <= 128 * ROUTER_STEPS && SL.total <= (size_t)std::min(dev.max_smem_optin - 4096, 200 * 1024);
 }
 
 cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Workspace& ws, float* h_dbg,
@@ -698,8 +689,7 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
     if (e != cudaSuccess) return e;
 
     int per_sm = 0;
-    const size_t smem1 = router_smem(L);
-    e = kernel_occupancy(reinterpret_cast<const void*>(decode_router_kernel), 128, smem1, &per_sm);
+    e = kernel_occupancy(reinterpret_cast<const void*>(decode_router_kernel), 128, 0, &per_sm);
     if (e != cudaSuccess) return e;
     const DecodeSmem SL = decode_smem_layout(L.H);
     e = kernel_occupancy(reinterpret_cast<const void*>(decode_ffn_kernel), FFN_THREADS, SL.total, &per_sm);
@@ -721,7 +711,7 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
     }
     cfg.gridDim = dim3((unsigned)L.E);
     cfg.blockDim = dim3(128);
-    cfg.dynamicSmemBytes = smem1;
+    cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
     cfg.attrs = attrs;
     cfg.numAttrs = 1;

@@ -648,12 +648,12 @@ def run_ours(args):
     del g2
 
     # algorithmic bytes of one launch of the dominant kernel (the fused T=1 FFN
-    # kernel: gate/up, SwiGLU, requant, down, combine): the three Q4_0 matrices
-    # of the k routed experts and the shared expert, the router logits and the
-    # token's Q8_0 row read, y written
+    # kernel: top-k, Q8_0 of x, gate/up, SwiGLU, requant, down, combine): the
+    # three Q4_0 matrices of the k routed experts and the shared expert, the
+    # router logits and x read, y written
     nb, nbF = H // 32, F // 32
     experts = k + 1
-    ffn_bytes = experts * 3 * F * nb * 18 + E * 4 + (H + 2 * nb) + H * 4
+    ffn_bytes = experts * 3 * F * nb * 18 + E * 4 + H * 4 + H * 4
     peak, peak_src = measured_peaks()
     achieved = ffn_bytes / (dom_us * 1e-6) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,

@@ -42,7 +42,6 @@
 #include "common.cuh"
 #include "launch.h"
 #include "ptx.cuh"
-#include "tc.cuh"
 
 namespace moeq4 {
 

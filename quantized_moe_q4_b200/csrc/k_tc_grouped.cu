@@ -20,32 +20,34 @@
 // bound the kernel.
 //
 // Tile: 128 weight rows (gate/up: 64 gate rows + the same 64 up rows; down:
-// 128 rows of H) x 128 slots of one expert (MMA M = 128, N = 128), so one MMA
-// pair covers 128 x 128 x 32 and a weight block converted once serves 128
-// slots.
+// 128 rows of H) x TN slots of one expert (MMA M = 128, N = TN), TN = 32, 64
+// or 128, chosen per call from the routed slots per expert (tc_tile_tokens):
+// a weight block converted once serves TN slots.
 //
-// Warp roles (22 warps):
+// Warp roles (10 warps for TN = 32, 14 for 64 and 128):
 //   0      producer: 2D tensor copies (TMA) of the packed weight rows (a box
 //          of 64 or 128 rows x 144 B = 8 blocks), two input stages in flight;
-//   1..4   converters: nibbles -> binary16 (nib - 8) for the A operand, and
-//          the slots' int8 activations, read from L2 with 16-byte loads
-//          issued before the wait for a free operand stage, -> binary16 for
-//          the B operand; both into the K-major shared-memory layout (8-row x
-//          16-byte core matrices); two operand stages of 2 blocks; block
-//          scales into a ring read by the epilogue;
+//   1..4   converters, a weight row and a slot each: nibbles -> binary16
+//          (nib - 8) for the A operand; the slot's int8 activations and
+//          block scales come through a 4-entry ring of cp.async copies issued
+//          three operand stages ahead, then -> binary16 for the B operand;
+//          both into the K-major shared-memory layout (8-row x 16-byte core
+//          matrices); two operand stages of 2 blocks; block scales into a
+//          ring read by the epilogue;
 //   5      MMA issuer (one thread): two MMAs per block (A and B from shared
 //          memory); one wait and one commit per operand stage, for its pair
 //          of accumulators;
-//   6..21  epilogue: 4 TMEM lane quarters x 4 column quarters; per operand
-//          stage one wait, two TMEM loads of 32 columns and the
-//          rescale-accumulate; after the last block of a tile gate/up ->
-//          SwiGLU + Q8_0 requantisation, down -> y += w_slot * o with vector
+//   6..    epilogue: 4 TMEM lane quarters x TN / CW column groups (CW = 32,
+//          or 64 for TN = 128); per operand stage one wait, TMEM loads of 16
+//          columns software-pipelined against the rescale-accumulate, the
+//          accumulator pair released as soon as its last chunk is in
+//          registers; after the last block of a tile gate/up -> SwiGLU +
+//          Q8_0 requantisation, down -> y += w_slot * o with vector
 //          reductions (red.v4.f32) of 4 consecutive rows of H of one token.
-// TMEM: four accumulators of 128 columns (all 512 columns), handed between
-// the MMA issuer and the epilogue a pair (one operand stage) at a time;
-// full/empty mbarriers between every pair of roles; every wait bounded, and
-// one that runs out makes every role leave its loop and records
-// STATUS_SPIN_TIMEOUT.
+// TMEM: four accumulators of TN columns, handed between the MMA issuer and the
+// epilogue a pair (one operand stage) at a time; full/empty mbarriers between
+// every pair of roles; every wait bounded, and one that runs out makes every
+// role leave its loop and records STATUS_SPIN_TIMEOUT.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -64,32 +66,37 @@ namespace {
 
 constexpr int TM = 128;            // MMA M: weight rows per tile
 constexpr int IN_KB = 8;           // Q4_0 blocks per input stage (144-byte rows: a 16-byte multiple)
-constexpr int OP_KB = 2;           // blocks per operand stage
 constexpr int NIN = 2, NOP = 2, NSC = 4;  // input, operand and scale-ring stages
-constexpr int NACC = 2 * OP_KB;    // accumulators: two pairs
 constexpr int IN_ROW = IN_KB * Q4_BYTES;          // 144
 constexpr int N_CONV = 128;        // converter threads: one weight row (and one slot) each
 constexpr int W_PROD = 0, W_CONV0 = 1, W_MMA = 5, W_EPI0 = 6;
 constexpr uint32_t LIMIT = 1u << 22;
 constexpr size_t SZ_IN_W = (size_t)TM * IN_ROW;           // one input stage of packed weight rows
-constexpr size_t SZ_OP_A = (size_t)OP_KB * 2 * TM * 32;   // one operand stage of A (K-steps of 16 x binary16)
-// Activation prefetch ring of the converters: NPF operand stages, a slot's 2
-// blocks of int8 codes (64 B) and their 2 binary16 scales (4 B) per entry,
-// copied by the thread that converts them (cp.async), PF stages ahead.
+// Activation prefetch ring of the converters: NPF operand stages, a slot's
+// OP_KB blocks of int8 codes and their binary16 scales per entry, copied by
+// the thread that converts them (cp.async), PF stages ahead.
 constexpr int NPF = 4, PF = 3;
-constexpr size_t BPF_SLOT = 80;
 
-// Per tile width TN (slots, the MMA N): the epilogue has TN/32 column groups
-// of 4 warps (one per TMEM lane quarter), and the shared-memory map.
+// Per tile width TN (slots, the MMA N): the blocks per operand stage, the
+// epilogue's column groups of 4 warps (one per TMEM lane quarter), and the
+// shared-memory map.
 template <int TN>
 struct TcCfg {
     static_assert(TN == 32 || TN == 64 || TN == 128, "tile widths");
+    // blocks per operand stage: each stage is one hand-off between the roles,
+    // so narrower tiles (less epilogue work a block) take four blocks a stage,
+    // 128-slot tiles two (their eight accumulators would need 1024 columns)
+    static constexpr int OP_KB = (TN == 128) ? 2 : 4;
+    static constexpr int NACC = 2 * OP_KB;                // accumulators: two sets of OP_KB
+    static constexpr size_t SZ_OP_A = (size_t)OP_KB * 2 * TM * 32;   // one operand stage of A (K-steps of 16 x binary16)
+    // a ring entry: OP_KB x 32 codes, OP_KB binary16 scales, padded to 16 bytes
+    static constexpr size_t BPF_SLOT = ((size_t)OP_KB * (QK + 2) + 15) & ~size_t(15);
     // epilogue: a thread owns one accumulator row x CW columns; 4 warps (the
     // TMEM lane quarters) per CW-wide column group
     static constexpr int CW = (TN == 128) ? 64 : 32;
     static constexpr int N_EPI = 4 * (TN / CW) * 32;
     static constexpr int THREADS = 6 * 32 + N_EPI;        // at most 14 warps: up to 128 registers a thread
-    static constexpr uint32_t TMEM_COLS = NACC * TN;      // 512 or 128 columns
+    static constexpr uint32_t TMEM_COLS = NACC * TN;      // 512, 512 or 256 columns
     static constexpr size_t SZ_OP_B = (size_t)OP_KB * 2 * TN * 32;
     static constexpr int XCH_LD = TN + 1;
     static constexpr size_t OFF_IN_W = 0;
@@ -101,7 +108,8 @@ struct TcCfg {
     static constexpr size_t OFF_BPF = OFF_XCH + (size_t)TM * XCH_LD * 4;
     static constexpr size_t SMEM_BYTES = OFF_BPF + (size_t)NPF * TN * BPF_SLOT;
     static constexpr size_t SMEM_ALLOC = SMEM_BYTES + 1024;   // slack to align the map to 1024 B
-    static_assert(SMEM_ALLOC <= 220 * 1024, "shared memory map too large");
+    static_assert(SMEM_ALLOC <= 226 * 1024, "shared memory map too large");
+    static_assert(TMEM_COLS <= 512, "TMEM budget");
 };
 
 enum { GATEUP = 0, DOWN = 1 };
@@ -177,6 +185,9 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 
 __device__ __forceinline__ void cp_async4(void* dst_smem, const void* src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* dst_smem, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 // this thread's copies of all but the newest N committed groups have landed
@@ -343,6 +354,8 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
     tc_grouped_kernel(TcParams p, const __grid_constant__ TcMaps maps) {
     using C = TcCfg<TN>;
     constexpr int N_EPI = C::N_EPI, THREADS = C::THREADS, XCH_LD = C::XCH_LD, CW = C::CW, NCH = CW / 16;
+    constexpr int OP_KB = C::OP_KB;
+    constexpr size_t SZ_OP_A = C::SZ_OP_A, BPF_SLOT = C::BPF_SLOT;
     constexpr uint32_t TMEM_COLS = C::TMEM_COLS;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -467,8 +480,9 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 uint8_t* dst = bpf + ((size_t)(i_pf % NPF) * TN + ct) * BPF_SLOT;
                 const int8_t* src = pf_arow + (size_t)pf_c * OP_KB * QK;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) cp_async16(dst + 16 * i, src + 16 * i);
-                cp_async4(dst + 64, pf_ascale + pf_c * OP_KB);
+                for (int i = 0; i < 2 * OP_KB; ++i) cp_async16(dst + 16 * i, src + 16 * i);
+                if (OP_KB == 4) cp_async8(dst + OP_KB * QK, pf_ascale + pf_c * OP_KB);
+                else cp_async4(dst + OP_KB * QK, pf_ascale + pf_c * OP_KB);
             }
             cp_async_commit();
             ++i_pf;
@@ -496,29 +510,33 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 if (!wait_phase(&op_empty[o], ((i_op / NOP) & 1) ^ 1, abort)) { ok = false; break; }
                 tc_fence_after_sync();
 
-                // weights: this row's 2 blocks, 36 bytes at a 4-byte boundary
-                uint32_t w[9];
+                // weights: this row's OP_KB blocks, pairs of 36 bytes at 4-byte
+                // boundaries
+                uint32_t w[9 * OP_KB / 2];
                 const uint32_t* wsrc = reinterpret_cast<const uint32_t*>(in_w + (size_t)s * SZ_IN_W + (size_t)ct * IN_ROW +
                                                                          sub * OP_KB * Q4_BYTES);
 #pragma unroll
-                for (int i = 0; i < 9; ++i) w[i] = wsrc[i];
+                for (int i = 0; i < 9 * OP_KB / 2; ++i) w[i] = wsrc[i];
                 uint8_t* oa = op_a + (size_t)o * SZ_OP_A;
                 uint8_t* ob = op_b + (size_t)o * C::SZ_OP_B;
                 float dws[OP_KB];
-                {
-                    // block 0 starts at byte 0 (scale, then 16 nibble bytes), block 1 at byte 18
+#pragma unroll
+                for (int pq = 0; pq < OP_KB / 2; ++pq) {
+                    // a pair's first block starts at its byte 0 (scale, then 16
+                    // nibble bytes), the second at byte 18
+                    const uint32_t* v = w + 9 * pq;
                     uint32_t qs[4];
-                    dws[0] = half_bits_to_float(w[0] & 0xffffu);
+                    dws[2 * pq] = half_bits_to_float(v[0] & 0xffffu);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) qs[i] = __funnelshift_r(w[i], w[i + 1], 16);
-                    store_weights(oa, 0, ct, qs);
-                    dws[1] = half_bits_to_float(w[4] >> 16);
+                    for (int i = 0; i < 4; ++i) qs[i] = __funnelshift_r(v[i], v[i + 1], 16);
+                    store_weights(oa, 2 * pq, ct, qs);
+                    dws[2 * pq + 1] = half_bits_to_float(v[4] >> 16);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) qs[i] = w[5 + i];
-                    store_weights(oa, 1, ct, qs);
+                    for (int i = 0; i < 4; ++i) qs[i] = v[5 + i];
+                    store_weights(oa, 2 * pq + 1, ct, qs);
                 }
                 // activations of slot ct from the ring (zeros past the tile's slots)
-                uint32_t dab = 0;
+                uint32_t dab[OP_KB / 2] = {};
                 cp_async_wait_group<PF>();                    // this thread's stage i_op has landed
                 if (ct < TN) {
                     const uint8_t* src = bpf + ((size_t)(i_op % NPF) * TN + ct) * BPF_SLOT;
@@ -530,7 +548,10 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                                                   : make_uint4(0, 0, 0, 0);
                             store_act16(ob, TN, kb, ks, ct, a);
                         }
-                    if (valid) dab = *reinterpret_cast<const uint32_t*>(src + 64);
+                    if (valid) {
+#pragma unroll
+                        for (int i = 0; i < OP_KB / 2; ++i) dab[i] = *reinterpret_cast<const uint32_t*>(src + OP_KB * QK + 4 * i);
+                    }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
@@ -543,7 +564,8 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 for (int kb = 0; kb < OP_KB; ++kb) {
                     dw_ring[(sc * OP_KB + kb) * TM + ct] = dws[kb];
                     if (ct < TN)
-                        da_ring[(sc * OP_KB + kb) * TN + ct] = valid ? half_bits_to_float(kb ? (dab >> 16) : dab) : 0.0f;
+                        da_ring[(sc * OP_KB + kb) * TN + ct] =
+                            valid ? half_bits_to_float((kb & 1) ? (dab[kb >> 1] >> 16) : dab[kb >> 1]) : 0.0f;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sc_full[sc]);
@@ -621,7 +643,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     break;
                 }
                 tc_fence_after_sync();
-                // chunks of 16 columns (2 blocks x CW / 16), software pipelined:
+                // chunks of 16 columns (OP_KB blocks x CW / 16), software pipelined:
                 // the TMEM load of chunk qc + 1 is in flight while chunk qc is
                 // rescaled; the accumulator pair is released as soon as its
                 // last chunk is in registers
@@ -845,7 +867,7 @@ int tc_tile_tokens(const LayerView& L, int64_t T, int force) {
     // routed slots per expert on average, against the measured crossovers of
     // the three widths (one 2048/512 layer, 128 experts top-8): 32 slots up to
     // 27 per expert (T <= 384), 64 from 28 (T = 512; a 947-token prompt's 59),
-    // 128 from 96
+    // 128 from 96 (a 16384-token batch's 1024)
     const int64_t per_expert = T * L.k / L.E;
     return per_expert >= 96 ? 128 : per_expert >= 28 ? 64 : 32;
 }

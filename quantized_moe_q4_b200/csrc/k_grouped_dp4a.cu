@@ -43,7 +43,12 @@ namespace {
 
 constexpr int SR = 64;                 // weight rows per item
 constexpr int ST = DP4A_TT;            // slots per tile (8)
-constexpr int KCMAX = 32;              // blocks per chunk
+constexpr int KCMAX = 32;              // blocks per chunk, at most
+// Blocks per chunk for rows of nb blocks (nb a multiple of 8): the largest of
+// 32, 24, 16, 8 that divides nb, so the chunks tile the row exactly.
+__host__ __device__ constexpr int chunk_blocks(int nb) {
+    return nb % 32 == 0 ? 32 : nb % 24 == 0 ? 24 : nb % 16 == 0 ? 16 : 8;
+}
 constexpr int NST = 3;                 // chunks in flight
 constexpr int NCW = 16;                // compute warps
 constexpr int RPL = 2;                 // weight rows per lane
@@ -240,7 +245,7 @@ __global__ void __maxnreg__(96) stream_dp4a_kernel(StreamParams p, const __grid_
     const int H = p.H, F = p.F, E = p.E;
     const int K = (MODE == DOWN) ? F : H;
     const int nb = K / QK;
-    const int KC = min(KCMAX, nb);          // nb is a multiple of 8
+    const int KC = chunk_blocks(nb);
     const int nchunk = nb / KC;
     const int n_rb = (MODE == GATEUP) ? F / 32 : ((MODE == DOWN) ? H / SR : (p.N + SR - 1) / SR);
     const int ngroups = E + 1;
@@ -494,13 +499,13 @@ cudaError_t launch_stream(const LayerView& L, int64_t T, const Workspace& ws, fl
     std::memset(&maps, 0, sizeof(maps));
     const uint64_t E = (uint64_t)L.E, F = (uint64_t)L.F, H = (uint64_t)L.H;
     if (MODE == GATEUP) {
-        const int nb = L.H / QK, KC = std::min(KCMAX, nb);
+        const int nb = L.H / QK, KC = chunk_blocks(nb);
         e = encode_rows_2d(&maps.m[0], L.w_gate, E * F, nb, KC, 32);
         if (e == cudaSuccess) e = encode_rows_2d(&maps.m[1], L.w_up, E * F, nb, KC, 32);
         if (e == cudaSuccess && L.S) e = encode_rows_2d(&maps.m[2], L.sh_gate, F, nb, KC, 32);
         if (e == cudaSuccess && L.S) e = encode_rows_2d(&maps.m[3], L.sh_up, F, nb, KC, 32);
     } else {
-        const int nb = L.F / QK, KC = std::min(KCMAX, nb);
+        const int nb = L.F / QK, KC = chunk_blocks(nb);
         e = encode_rows_2d(&maps.m[0], L.w_down, E * H, nb, KC, SR);
         if (e == cudaSuccess && L.S) e = encode_rows_2d(&maps.m[2], L.sh_down, H, nb, KC, SR);
     }
@@ -530,7 +535,7 @@ cudaError_t launch_gemv_dp4a(const uint8_t* W, int64_t N, int H, const int8_t* q
     if (e != cudaSuccess) return e;
     StreamMaps maps;
     std::memset(&maps, 0, sizeof(maps));
-    const int nb = H / QK, KC = std::min(KCMAX, nb);
+    const int nb = H / QK, KC = chunk_blocks(nb);
     e = encode_rows_2d(&maps.m[0], W, (uint64_t)N, nb, KC, SR);
     if (e != cudaSuccess) return e;
     StreamParams p;

@@ -24,7 +24,9 @@ def _matrix(seed, N, H):
 
 
 @pytest.mark.parametrize("N,H,T", [(131072, 2048, 1), (131072, 2048, 5), (1000, 512, 8), (4096, 4096, 3),
-                                   (64, 256, 2)])
+                                   (64, 256, 2),
+                                   # rows of 48, 56, 72, 80 blocks: chunks of 24, 8, 24, 16 blocks
+                                   (700, 1536, 2), (300, 1792, 1), (520, 2304, 4), (128, 2560, 3)])
 def test_gemv_matches_oracle(N, H, T):
     W = _matrix(N + H, N, H)
     x = np.random.default_rng(T).standard_normal((T, H)).astype(np.float32)

@@ -8,6 +8,8 @@ routing and requantised h.  Sizes: every workload the benchmark and the
 design use, at full size on the GPU, checked on all tokens where the oracle
 is fast and on sampled tokens where it is not (tokens are independent).
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -265,11 +267,15 @@ def test_block_dots_extreme_values(path, R):
     (3, 512, 768, 5, 2, True),        # F = 3*256
     (40, 768, 256, 256, 16, False),   # E = 256, k = 16
     (1, 768, 768, 5, 2, True),        # decode path: odd H and F
-    (1, 4096, 512, 16, 4, True),      # decode path: wide H
-    (1, 512, 1024, 8, 8, True),       # decode path: more gate/up items than CTAs
+    (1, 4096, 512, 16, 4, True),      # H above the decode path's 2560: falls back
+    (1, 2560, 512, 16, 4, True),      # decode path: the widest H
+    (1, 512, 1024, 8, 8, True),       # 288 h blocks, more than one wave: falls back
     (1, 2048, 2048, 64, 8, True),     # too large for the decode path: falls back
-    (1, 256, 512, 256, 16, False),    # decode path: E = 256, k = 16
+    (1, 256, 256, 256, 16, False),    # decode path: E = 256 (8 logits a lane in the top-k), k = 16
+    (1, 512, 256, 200, 8, True),      # decode path: E = 200, not a multiple of 32
     (17, 4096, 256, 8, 2, True),      # wide H
+    (5, 1536, 1792, 12, 3, True),     # rows of 48 and 56 blocks (streaming chunks of 24 and 8)
+    (3, 2304, 2560, 6, 2, False),     # rows of 72 and 80 blocks (chunks of 24 and 16)
 ])
 def test_shapes_and_degenerate_cases(path, T, H, F, E, k, shared):
     x, lw = synth.random_layer(seed=T + H + F + E, H=H, F=F, E=E, k=k, shared=shared, T=T)
@@ -279,10 +285,33 @@ def test_shapes_and_degenerate_cases(path, T, H, F, E, k, shared):
     teacher_forced_check(lw, x, v, np.arange(T))
 
 
+@pytest.mark.parametrize("path", PATHS)
+def test_routing_with_exact_ties(path):
+    """Ten experts with identical router rows get identical logits on every
+    path (the same products summed in the same order), at the top of the
+    ranking: with k = 8 the top-k takes the eight lowest of their indices, in
+    index order, exactly as the oracle's top-k of the device's own logits."""
+    T = 1 if path == m.PATH_DECODE else 24
+    x, lw = synth.random_layer(seed=99, H=256, F=256, E=64, k=8, shared=True, T=T)
+    tied = [1, 3, 7, 12, 20, 30, 41, 50, 55, 63]
+    row = lw.w_router[41].copy()
+    if float(np.dot(x[0].astype(np.float64), row)) < 0:
+        row = -row                                   # token 0 ranks the tied experts first
+    Wr = lw.w_router.copy()
+    for e in tied:
+        Wr[e] = 10 * row
+    lw = dataclasses.replace(lw, w_router=Wr)
+    v = run_forward(lw, x, path=path, L=m.Layer.from_host(lw))
+    check_routing(lw, x, v)
+    check_permutation(lw, v)
+    assert v["topk_idx"][0].tolist() == tied[:8]
+    teacher_forced_check(lw, x, v, np.arange(T))
+
+
 def test_kernel_shared_memory_sizes_in_any_order():
     # the same kernels at a large, a small and again the large shared-memory
     # size: the per-kernel dynamic shared-memory limit must cover all of them
-    cases = [(1, 4096, 512, 16, 4, True), (1, 256, 256, 4, 2, True), (1, 4096, 512, 16, 4, True),
+    cases = [(1, 2560, 512, 16, 4, True), (1, 256, 256, 4, 2, True), (1, 2560, 512, 16, 4, True),
              (9, 4096, 256, 8, 2, True), (9, 256, 256, 4, 2, True), (9, 4096, 256, 8, 2, True)]
     for T, H, F, E, k, shared in cases:
         x, lw = synth.random_layer(seed=H + T, H=H, F=F, E=E, k=k, shared=shared, T=T)

@@ -454,9 +454,27 @@ def gemv_lines(m, torch, stream):
 def streamed_lines(m, torch, stream):
     """Host-streamed experts (expert matrices in page-locked host memory,
     the selected experts copied per call): decode T = 1 and the 947-token
-    prefill; link GB/s over the expert bytes that cross per call."""
+    prefill; link GB/s over the expert bytes that cross per call, beside a
+    plain page-locked host-to-device copy of the same bytes (the link's
+    rate for one large copy)."""
     import synth
     out = {}
+    ref_bytes = 129 * 3 * 512 * (2048 // 32) * 18
+    src = torch.empty(ref_bytes, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(ref_bytes, dtype=torch.uint8, device="cuda")
+    times = []
+    for rep in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            dst.copy_(src, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if rep >= 1:
+            times.append(e0.elapsed_time(e1))
+    out["link_copy"] = {"bytes": ref_bytes, "ms": float(np.median(times)),
+                        "gbs": ref_bytes / (float(np.median(times)) * 1e-3) / 1e9}
+    del src, dst
     for name, T in (("decode_t1", 1), ("prefill_t947", 947)):
         x_np, lw = synth.workload_inputs(name, seed=0, T=T if name == "decode_t1" else None)
         Lh = m.Layer.from_host_pinned(lw)

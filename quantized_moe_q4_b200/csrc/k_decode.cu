@@ -178,7 +178,7 @@ __device__ __forceinline__ void red_add_v4(float* y, float4 v) {
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// K1: router logits (one CTA per expert), Q8_0 of x, y zeroed.
+// K1: router logits (one CTA per expert), y zeroed.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
     __shared__ float red[4];
@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(128) decode_router_kernel(DecodeParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// K2: gate/up + SwiGLU + requant, exchange within a group, down + combine.
+// K2: top-k, Q8_0 of x, gate/up + SwiGLU + requant, down column + combine.
 // ---------------------------------------------------------------------------
 struct DecodeSmem {
     size_t gu, dn, qa, da, qsum, o, total;  // byte offsets

@@ -88,16 +88,20 @@ __device__ __forceinline__ int dp4a_u8s8(uint32_t a, int b, int c) {
 }
 
 // Exact sum_i (nibble_i - 8) * q_i of one Q4_0 block (nibble bytes qs as four
-// little-endian words) against 32 int8 activations (eight words).  The -8
-// offset is applied once through the activations' block sum qsum.
+// little-endian words) against 32 int8 activations (eight words).  The low
+// nibbles (weights 0..15) go through dp4a as they are; the high nibbles
+// (weights 16..31) are masked in place, so each byte holds 16 x the nibble,
+// and their chain is divided by 16 once at the end (exact: every term is a
+// multiple of 16, and the sum stays below 2^20).  The -8 offset is applied
+// once through the activations' block sum qsum.
 __device__ __forceinline__ int q4_q8_dot(const uint32_t qs[4], const int qa[8], int qsum) {
-    int s = 0;
+    int lo = 0, hi = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        s = dp4a_u8s8(qs[j] & 0x0f0f0f0fu, qa[j], s);          // weights 4j..4j+3
-        s = dp4a_u8s8((qs[j] >> 4) & 0x0f0f0f0fu, qa[4 + j], s);  // weights 16+4j..
+        lo = dp4a_u8s8(qs[j] & 0x0f0f0f0fu, qa[j], lo);       // weights 4j..4j+3
+        hi = dp4a_u8s8(qs[j] & 0xf0f0f0f0u, qa[4 + j], hi);   // 16 x weights 16+4j..
     }
-    return s - 8 * qsum;
+    return lo + (hi >> 4) - 8 * qsum;
 }
 
 // Sum of the 32 int8 values held as eight words.

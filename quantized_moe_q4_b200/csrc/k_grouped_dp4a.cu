@@ -213,12 +213,15 @@ __device__ __forceinline__ void block_slots(float (&acc)[RPL_][ST_], int s0, con
     for (int r = 0; r < RPL_; ++r) {
 #pragma unroll
         for (int j = 0; j < SPW; ++j) {
-            int I = base[j];
+            // low nibbles as they are; high nibbles masked in place (16 x the
+            // nibble), their chain divided by 16 once (exact)
+            int lo = base[j], hi = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                I = dp4a_u8s8(qs[r][i] & 0x0f0f0f0fu, qa[j][i], I);
-                I = dp4a_u8s8((qs[r][i] >> 4) & 0x0f0f0f0fu, qa[j][4 + i], I);
+                lo = dp4a_u8s8(qs[r][i] & 0x0f0f0f0fu, qa[j][i], lo);
+                hi = dp4a_u8s8(qs[r][i] & 0xf0f0f0f0u, qa[j][4 + i], hi);
             }
+            const int I = lo + (hi >> 4);
             if (CAP && cap.out) cap.out[((size_t)(cap.slot_rel + s0 + j) * SR + cap.row0 + r) * cap.nb + cap.blk] = I;
             acc[r][s0 + j] = fmaf(int_to_float_exact(I), dW[r] * dA[j], acc[r][s0 + j]);
         }

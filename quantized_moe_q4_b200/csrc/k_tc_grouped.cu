@@ -72,10 +72,9 @@ constexpr int N_CONV = 128;        // converter threads: one weight row (and one
 constexpr int W_PROD = 0, W_CONV0 = 1, W_MMA = 5, W_EPI0 = 6;
 constexpr uint32_t LIMIT = 1u << 22;
 constexpr size_t SZ_IN_W = (size_t)TM * IN_ROW;           // one input stage of packed weight rows
-// Activation prefetch ring of the converters: NPF operand stages, a slot's
-// OP_KB blocks of int8 codes and their binary16 scales per entry, copied by
-// the thread that converts them (cp.async), PF stages ahead.
-constexpr int NPF = 4, PF = 3;
+// Activation ring: NPF operand stages, a slot's OP_KB blocks of int8 codes and
+// their binary16 scales per entry, copied by the producer warp (cp.async).
+constexpr int NPF = 4;
 
 // Per tile width TN (slots, the MMA N): the blocks per operand stage, the
 // epilogue's column groups of 4 warps (one per TMEM lane quarter), and the
@@ -189,10 +188,11 @@ __device__ __forceinline__ void cp_async4(void* dst_smem, const void* src) {
 __device__ __forceinline__ void cp_async8(void* dst_smem, const void* src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// this thread's copies of all but the newest N committed groups have landed
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// arrive on bar once this thread's earlier cp.async copies have landed (the
+// barrier's count includes the arrival)
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 // y[0..3] += v (one vector reduction at L2; y 16-byte aligned)
 __device__ __forceinline__ void red_add_v4(float* y, float4 v) {
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __shared__ __align__(8) uint64_t in_full[NIN], in_empty[NIN], op_full[NOP], op_empty[NOP], tm_full[2],
-        tm_empty[2], sc_full[NSC], sc_empty[NSC], epi_bar;
+        tm_empty[2], sc_full[NSC], sc_empty[NSC], epi_bar, b_full[NPF], b_empty[NPF];
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ int tile_off_s[258], off_s[258];
@@ -405,6 +405,10 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
             mbar_init(&sc_full[i], N_CONV / 32);
             mbar_init(&sc_empty[i], N_EPI / 32);
         }
+        for (int i = 0; i < NPF; ++i) {
+            mbar_init(&b_full[i], 32);              // the producer's 32 lanes, after their copies land
+            mbar_init(&b_empty[i], N_CONV / 32);    // the converter warps, after reading the entry
+        }
         mbar_init(&epi_bar, N_EPI / 32);
         mbar_fence_init();
     }
@@ -420,10 +424,37 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
 
     if (warp == W_PROD) {
         // ------------------------------------------------------------ producer
-        uint32_t i_in = 0;
+        // weights: TMA copies of each input stage; activations: for each of
+        // its operand stages, the codes and scales of every slot of the tile
+        // (lane l: slots l, l + 32, ..) into a ring entry by cp.async, whose
+        // landing the lane reports on the entry's barrier
+        uint8_t* bpf = smem + C::OFF_BPF;
+        constexpr int SPL = (TN + 31) / 32;          // slots per lane
+        uint32_t i_in = 0, i_b = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const Tile T = tile_of<TN>(item, n_rb, tile_off_s, off_s, ngroups);
+            const int8_t* arow[SPL];
+            const uint16_t* ascale[SPL];
+#pragma unroll
+            for (int q = 0; q < SPL; ++q) {
+                arow[q] = nullptr;
+                ascale[q] = nullptr;
+                const int n = lane + 32 * q;
+                if (n < TN && n < T.nslots) {
+                    const int sl = T.slot0 + n;
+                    int tok;
+                    float w;
+                    slot_info(p, T.g, sl, tok, w);
+                    if (MODE == GATEUP) {
+                        arow[q] = p.qa + (size_t)tok * H;
+                        ascale[q] = p.da + (size_t)tok * (H / QK);
+                    } else {
+                        arow[q] = p.hq + (size_t)sl * F;
+                        ascale[q] = p.dh + (size_t)sl * nbF;
+                    }
+                }
+            }
             // weight rows of this item: one box of 64 gate + one of 64 up rows, or 128 down rows
             const bool shared_g = T.g >= E;
             const CUtensorMap* map0 = &maps.m[shared_g ? 2 : 0];
@@ -439,70 +470,41 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     if (MODE == GATEUP) tma_load_2d(dw + 64 * IN_ROW, map1, c * IN_ROW, wy, &in_full[s]);
                 }
                 __syncwarp();
+                for (int sb = 0; sb < IN_KB / OP_KB; ++sb, ++i_b) {
+                    const int r = i_b % NPF;
+                    if (!wait_phase(&b_empty[r], ((i_b / NPF) & 1) ^ 1, abort)) { ok = false; break; }
+                    const int cb = c * (IN_KB / OP_KB) + sb;   // operand stage within the item
+#pragma unroll
+                    for (int q = 0; q < SPL; ++q) {
+                        if (!arow[q]) continue;
+                        uint8_t* dst = bpf + ((size_t)r * TN + lane + 32 * q) * BPF_SLOT;
+                        const int8_t* src = arow[q] + (size_t)cb * OP_KB * QK;
+#pragma unroll
+                        for (int i = 0; i < 2 * OP_KB; ++i) cp_async16(dst + 16 * i, src + 16 * i);
+                        if (OP_KB == 4) cp_async8(dst + OP_KB * QK, ascale[q] + cb * OP_KB);
+                        else cp_async4(dst + OP_KB * QK, ascale[q] + cb * OP_KB);
+                    }
+                    cp_async_arrive_noinc(&b_full[r]);
+                }
+                if (!ok) break;
             }
         }
         // let the copies in flight land before the CTA can exit
+        cp_async_wait_all();
         if (i_in > 0) mbar_wait_bounded(&in_full[(i_in - 1) % NIN], ((i_in - 1) / NIN) & 1, LIMIT);
     } else if (warp >= W_CONV0 && warp < W_CONV0 + 4) {
         // ------------------------------------------------------------ converters
         // thread ct converts weight row ct and (ct < TN) the activations of
-        // slot ct; it copies those activations PF operand stages ahead into
-        // its own entries of the prefetch ring (cp.async: no registers held,
-        // no wait on L2 in the loop)
+        // slot ct, which the producer has copied into the ring
         const int ct = tid - W_CONV0 * 32;
-        uint8_t* bpf = smem + C::OFF_BPF;
+        const uint8_t* bpf = smem + C::OFF_BPF;
         const int nst = nbK / OP_KB;                      // operand stages per item
-        // the prefetch cursor: item, stage, and this slot's rows (NULL: no slot)
-        int pf_item = blockIdx.x, pf_c = 0;
-        const int8_t* pf_arow = nullptr;
-        const uint16_t* pf_ascale = nullptr;
-        auto pf_rows = [&](int item) {
-            pf_arow = nullptr;
-            pf_ascale = nullptr;
-            if (item >= n_items || ct >= TN) return;
-            const Tile Tn = tile_of<TN>(item, n_rb, tile_off_s, off_s, ngroups);
-            if (ct >= Tn.nslots) return;
-            const int sl = Tn.slot0 + ct;
-            int tok;
-            float w;
-            slot_info(p, Tn.g, sl, tok, w);
-            if (MODE == GATEUP) {
-                pf_arow = p.qa + (size_t)tok * H;
-                pf_ascale = p.da + (size_t)tok * (H / QK);
-            } else {
-                pf_arow = p.hq + (size_t)sl * F;
-                pf_ascale = p.dh + (size_t)sl * nbF;
-            }
-        };
-        uint32_t i_pf = 0;
-        auto pf_issue = [&]() {   // one operand stage ahead, always one commit group
-            if (pf_item < n_items && pf_arow) {
-                uint8_t* dst = bpf + ((size_t)(i_pf % NPF) * TN + ct) * BPF_SLOT;
-                const int8_t* src = pf_arow + (size_t)pf_c * OP_KB * QK;
-#pragma unroll
-                for (int i = 0; i < 2 * OP_KB; ++i) cp_async16(dst + 16 * i, src + 16 * i);
-                if (OP_KB == 4) cp_async8(dst + OP_KB * QK, pf_ascale + pf_c * OP_KB);
-                else cp_async4(dst + OP_KB * QK, pf_ascale + pf_c * OP_KB);
-            }
-            cp_async_commit();
-            ++i_pf;
-            if (++pf_c == nst) {
-                pf_c = 0;
-                pf_item += gridDim.x;
-                pf_rows(pf_item);
-            }
-        };
-        pf_rows(pf_item);
-#pragma unroll 1
-        for (int i = 0; i < PF; ++i) pf_issue();
-
         uint32_t i_op = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const Tile T = tile_of<TN>(item, n_rb, tile_off_s, off_s, ngroups);
             const bool valid = ct < T.nslots;
             for (int c = 0; c < nst && ok; ++c, ++i_op) {
-                pf_issue();                                   // stage i_op + PF
                 const uint32_t i_in = i_op / (IN_KB / OP_KB);
                 const int s = i_in % NIN, sub = i_op % (IN_KB / OP_KB);
                 if (sub == 0 && !wait_phase(&in_full[s], (i_in / NIN) & 1, abort)) { ok = false; break; }
@@ -537,7 +539,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 }
                 // activations of slot ct from the ring (zeros past the tile's slots)
                 uint32_t dab[OP_KB / 2] = {};
-                cp_async_wait_group<PF>();                    // this thread's stage i_op has landed
+                if (!wait_phase(&b_full[i_op % NPF], (i_op / NPF) & 1, abort)) { ok = false; break; }
                 if (ct < TN) {
                     const uint8_t* src = bpf + ((size_t)(i_op % NPF) * TN + ct) * BPF_SLOT;
 #pragma unroll
@@ -553,6 +555,8 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                         for (int i = 0; i < OP_KB / 2; ++i) dab[i] = *reinterpret_cast<const uint32_t*>(src + OP_KB * QK + 4 * i);
                     }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&b_empty[i_op % NPF]);   // the ring entry is free again
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 mbar_arrive(&op_full[o]);
@@ -571,7 +575,6 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 if (lane == 0) mbar_arrive(&sc_full[sc]);
             }
         }
-        cp_async_wait_all();   // the prefetches past the last stage land before the CTA exits
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -605,7 +608,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                         mma_f16_ss(d, ad + (uint64_t)(kb * 2) * KA, bd + (uint64_t)(kb * 2) * KB, idesc, false);
                         mma_f16_ss(d, ad + (uint64_t)(kb * 2 + 1) * KA, bd + (uint64_t)(kb * 2 + 1) * KB, idesc, true);
                     }
-                    mma_commit(&tm_full[o]);  // covers the pair's four MMAs
+                    mma_commit(&tm_full[o]);  // covers the set's MMAs
                     mma_commit(&op_empty[o]);
                 }
             }

@@ -345,6 +345,13 @@ __device__ __forceinline__ void slot_info(const TcParams& p, int g, int s, int& 
     }
 }
 
+// w[i] = win[i + OFS] (zero past the window)
+template <int OFS, int N, int M>
+__device__ __forceinline__ void take_words(uint32_t (&w)[N], const uint32_t (&win)[M]) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) w[i] = (i + OFS < M) ? win[i + OFS] : 0u;
+}
+
 }  // namespace
 
 // CAP: also write the per-block integer sums (the MMA accumulators before the
@@ -512,13 +519,31 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 if (!wait_phase(&op_empty[o], ((i_op / NOP) & 1) ^ 1, abort)) { ok = false; break; }
                 tc_fence_after_sync();
 
-                // weights: this row's OP_KB blocks, pairs of 36 bytes at 4-byte
-                // boundaries
+                // weights: this row's OP_KB blocks (pairs of 36 bytes at 4-byte
+                // boundaries), read as 16-byte loads of the window from the
+                // 16-byte boundary at or below them: rows are 144 bytes apart,
+                // so a quarter-warp's loads fall in distinct banks
                 uint32_t w[9 * OP_KB / 2];
-                const uint32_t* wsrc = reinterpret_cast<const uint32_t*>(in_w + (size_t)s * SZ_IN_W + (size_t)ct * IN_ROW +
-                                                                         sub * OP_KB * Q4_BYTES);
+                {
+                    // the blocks start at word 0..3 of the window (0 or 2 for OP_KB = 4)
+                    constexpr int MAXOFS = (OP_KB == 4) ? 2 : 3;
+                    constexpr int NW = (4 * MAXOFS + OP_KB * Q4_BYTES + 15) / 16;   // 16-byte loads, in the row
+                    const int gb = sub * OP_KB * Q4_BYTES;
+                    const uint4* wsrc = reinterpret_cast<const uint4*>(in_w + (size_t)s * SZ_IN_W + (size_t)ct * IN_ROW +
+                                                                       (gb & ~15));
+                    uint32_t win[4 * NW];
 #pragma unroll
-                for (int i = 0; i < 9 * OP_KB / 2; ++i) w[i] = wsrc[i];
+                    for (int i = 0; i < NW; ++i) {
+                        const uint4 v = wsrc[i];
+                        win[4 * i] = v.x; win[4 * i + 1] = v.y; win[4 * i + 2] = v.z; win[4 * i + 3] = v.w;
+                    }
+                    switch ((gb & 15) >> 2) {   // the same in every lane of the warp
+                        case 0: take_words<0>(w, win); break;
+                        case 1: take_words<1>(w, win); break;
+                        case 2: take_words<2>(w, win); break;
+                        default: take_words<3>(w, win); break;
+                    }
+                }
                 uint8_t* oa = op_a + (size_t)o * SZ_OP_A;
                 uint8_t* ob = op_b + (size_t)o * C::SZ_OP_B;
                 float dws[OP_KB];

@@ -68,8 +68,7 @@ constexpr int TM = 128;            // MMA M: weight rows per tile
 constexpr int IN_KB = 8;           // Q4_0 blocks per input stage (144-byte rows: a 16-byte multiple)
 constexpr int NIN = 2, NOP = 2, NSC = 4;  // input, operand and scale-ring stages
 constexpr int IN_ROW = IN_KB * Q4_BYTES;          // 144
-constexpr int N_CONV = 128;        // converter threads: one weight row (and one slot) each
-constexpr int W_PROD = 0, W_CONV0 = 1, W_MMA = 5, W_EPI0 = 6;
+constexpr int W_PROD = 0, W_CONV0 = 1;
 constexpr uint32_t LIMIT = 1u << 22;
 constexpr size_t SZ_IN_W = (size_t)TM * IN_ROW;           // one input stage of packed weight rows
 // Activation ring: NPF operand stages, a slot's OP_KB blocks of int8 codes and
@@ -94,7 +93,11 @@ struct TcCfg {
     // TMEM lane quarters) per CW-wide column group
     static constexpr int CW = (TN == 128) ? 64 : 32;
     static constexpr int N_EPI = 4 * (TN / CW) * 32;
-    static constexpr int THREADS = 6 * 32 + N_EPI;        // at most 14 warps: up to 128 registers a thread
+    // converters: one pair of blocks of a weight row (and of a slot) per
+    // thread, so OP_KB / 2 threads a row: 8 warps for 4-block stages, 4 for 2
+    static constexpr int N_CONV = TM * OP_KB / 2;
+    static constexpr int W_MMA = W_CONV0 + N_CONV / 32, W_EPI0 = W_MMA + 1;
+    static constexpr int THREADS = (W_EPI0 * 32) + N_EPI;  // 10, 18 or 14 warps
     static constexpr uint32_t TMEM_COLS = NACC * TN;      // 512, 512 or 256 columns
     static constexpr size_t SZ_OP_B = (size_t)OP_KB * 2 * TN * 32;
     static constexpr int XCH_LD = TN + 1;
@@ -361,6 +364,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
     tc_grouped_kernel(TcParams p, const __grid_constant__ TcMaps maps) {
     using C = TcCfg<TN>;
     constexpr int N_EPI = C::N_EPI, THREADS = C::THREADS, XCH_LD = C::XCH_LD, CW = C::CW, NCH = CW / 16;
+    constexpr int N_CONV = C::N_CONV, W_MMA = C::W_MMA, W_EPI0 = C::W_EPI0;
     constexpr int OP_KB = C::OP_KB;
     constexpr size_t SZ_OP_A = C::SZ_OP_A, BPF_SLOT = C::BPF_SLOT;
     constexpr uint32_t TMEM_COLS = C::TMEM_COLS;
@@ -499,18 +503,20 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
         // let the copies in flight land before the CTA can exit
         cp_async_wait_all();
         if (i_in > 0) mbar_wait_bounded(&in_full[(i_in - 1) % NIN], ((i_in - 1) / NIN) & 1, LIMIT);
-    } else if (warp >= W_CONV0 && warp < W_CONV0 + 4) {
+    } else if (warp >= W_CONV0 && warp < W_MMA) {
         // ------------------------------------------------------------ converters
-        // thread ct converts weight row ct and (ct < TN) the activations of
-        // slot ct, which the producer has copied into the ring
+        // thread ct converts one pair of blocks (kb0, kb0 + 1) of weight row
+        // ct mod 128 and (row < TN) of the activations of that slot, which the
+        // producer has copied into the ring
         const int ct = tid - W_CONV0 * 32;
+        const int row = ct % TM, kb0 = 2 * (ct / TM);
         const uint8_t* bpf = smem + C::OFF_BPF;
         const int nst = nbK / OP_KB;                      // operand stages per item
         uint32_t i_op = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const Tile T = tile_of<TN>(item, n_rb, tile_off_s, off_s, ngroups);
-            const bool valid = ct < T.nslots;
+            const bool valid = row < T.nslots;
             for (int c = 0; c < nst && ok; ++c, ++i_op) {
                 const uint32_t i_in = i_op / (IN_KB / OP_KB);
                 const int s = i_in % NIN, sub = i_op % (IN_KB / OP_KB);
@@ -519,17 +525,15 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 if (!wait_phase(&op_empty[o], ((i_op / NOP) & 1) ^ 1, abort)) { ok = false; break; }
                 tc_fence_after_sync();
 
-                // weights: this row's OP_KB blocks (pairs of 36 bytes at 4-byte
-                // boundaries), read as 16-byte loads of the window from the
-                // 16-byte boundary at or below them: rows are 144 bytes apart,
-                // so a quarter-warp's loads fall in distinct banks
-                uint32_t w[9 * OP_KB / 2];
+                // weights: this thread's pair of blocks (36 bytes at a 4-byte
+                // boundary), read as 16-byte loads of the window from the
+                // 16-byte boundary at or below it: rows are 144 bytes apart, so
+                // a quarter-warp's loads fall in distinct banks
+                uint32_t w[9];
                 {
-                    // the blocks start at word 0..3 of the window (0 or 2 for OP_KB = 4)
-                    constexpr int MAXOFS = (OP_KB == 4) ? 2 : 3;
-                    constexpr int NW = (4 * MAXOFS + OP_KB * Q4_BYTES + 15) / 16;   // 16-byte loads, in the row
-                    const int gb = sub * OP_KB * Q4_BYTES;
-                    const uint4* wsrc = reinterpret_cast<const uint4*>(in_w + (size_t)s * SZ_IN_W + (size_t)ct * IN_ROW +
+                    constexpr int NW = (4 * 3 + 2 * Q4_BYTES + 15) / 16;   // 3 loads, inside the row
+                    const int gb = (sub * OP_KB + kb0) * Q4_BYTES;
+                    const uint4* wsrc = reinterpret_cast<const uint4*>(in_w + (size_t)s * SZ_IN_W + (size_t)row * IN_ROW +
                                                                        (gb & ~15));
                     uint32_t win[4 * NW];
 #pragma unroll
@@ -546,39 +550,34 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 }
                 uint8_t* oa = op_a + (size_t)o * SZ_OP_A;
                 uint8_t* ob = op_b + (size_t)o * C::SZ_OP_B;
-                float dws[OP_KB];
-#pragma unroll
-                for (int pq = 0; pq < OP_KB / 2; ++pq) {
-                    // a pair's first block starts at its byte 0 (scale, then 16
-                    // nibble bytes), the second at byte 18
-                    const uint32_t* v = w + 9 * pq;
+                float dws[2];
+                {
+                    // the pair's first block starts at its byte 0 (scale, then
+                    // 16 nibble bytes), the second at byte 18
                     uint32_t qs[4];
-                    dws[2 * pq] = half_bits_to_float(v[0] & 0xffffu);
+                    dws[0] = half_bits_to_float(w[0] & 0xffffu);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) qs[i] = __funnelshift_r(v[i], v[i + 1], 16);
-                    store_weights(oa, 2 * pq, ct, qs);
-                    dws[2 * pq + 1] = half_bits_to_float(v[4] >> 16);
+                    for (int i = 0; i < 4; ++i) qs[i] = __funnelshift_r(w[i], w[i + 1], 16);
+                    store_weights(oa, kb0, row, qs);
+                    dws[1] = half_bits_to_float(w[4] >> 16);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) qs[i] = v[5 + i];
-                    store_weights(oa, 2 * pq + 1, ct, qs);
+                    for (int i = 0; i < 4; ++i) qs[i] = w[5 + i];
+                    store_weights(oa, kb0 + 1, row, qs);
                 }
-                // activations of slot ct from the ring (zeros past the tile's slots)
-                uint32_t dab[OP_KB / 2] = {};
+                // activations of slot `row` from the ring (zeros past the tile's slots)
+                uint32_t dab = 0;
                 if (!wait_phase(&b_full[i_op % NPF], (i_op / NPF) & 1, abort)) { ok = false; break; }
-                if (ct < TN) {
-                    const uint8_t* src = bpf + ((size_t)(i_op % NPF) * TN + ct) * BPF_SLOT;
+                if (row < TN) {
+                    const uint8_t* src = bpf + ((size_t)(i_op % NPF) * TN + row) * BPF_SLOT;
 #pragma unroll
-                    for (int kb = 0; kb < OP_KB; ++kb)
+                    for (int kb = kb0; kb < kb0 + 2; ++kb)
 #pragma unroll
                         for (int ks = 0; ks < 2; ++ks) {
                             const uint4 a = valid ? *reinterpret_cast<const uint4*>(src + 16 * (2 * kb + ks))
                                                   : make_uint4(0, 0, 0, 0);
-                            store_act16(ob, TN, kb, ks, ct, a);
+                            store_act16(ob, TN, kb, ks, row, a);
                         }
-                    if (valid) {
-#pragma unroll
-                        for (int i = 0; i < OP_KB / 2; ++i) dab[i] = *reinterpret_cast<const uint32_t*>(src + OP_KB * QK + 4 * i);
-                    }
+                    if (valid) dab = *reinterpret_cast<const uint32_t*>(src + OP_KB * QK + 2 * kb0);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&b_empty[i_op % NPF]);   // the ring entry is free again
@@ -590,11 +589,11 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 const int sc = i_op % NSC;
                 if (!wait_phase(&sc_empty[sc], ((i_op / NSC) & 1) ^ 1, abort)) { ok = false; break; }
 #pragma unroll
-                for (int kb = 0; kb < OP_KB; ++kb) {
-                    dw_ring[(sc * OP_KB + kb) * TM + ct] = dws[kb];
-                    if (ct < TN)
-                        da_ring[(sc * OP_KB + kb) * TN + ct] =
-                            valid ? half_bits_to_float((kb & 1) ? (dab[kb >> 1] >> 16) : dab[kb >> 1]) : 0.0f;
+                for (int i = 0; i < 2; ++i) {
+                    dw_ring[(sc * OP_KB + kb0 + i) * TM + row] = dws[i];
+                    if (row < TN)
+                        da_ring[(sc * OP_KB + kb0 + i) * TN + row] =
+                            valid ? half_bits_to_float(i ? (dab >> 16) : dab) : 0.0f;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sc_full[sc]);

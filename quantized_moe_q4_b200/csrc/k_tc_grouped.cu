@@ -9,43 +9,49 @@
 // Arithmetic.  Every Q4_0 block (32 weights along K) carries its own binary16
 // scale, and so does every Q8_0 block of the activations, so the sum over K is
 // sum_b dW[row,b] * dA[slot,b] * I_b with I_b the exact integer block dot
-// product.  The tensor core computes I_b: operands hold the exact small
-// integers (nibble - 8 in [-8, 7], q in [-127, 127]) as binary16, products and
-// 32-term sums are exact in the fp32 accumulator, so each 32-wide block is two
-// K=16 MMAs into its own TMEM buffer.  The epilogue then accumulates
-// acc += I_b * (dW * dA) in fp32 registers (packed f32x2 FMUL + FFMA; the
-// product of two binary16 scales is exact in binary32).  Binary16 rather than
-// int8 operands spare an int32 -> fp32 conversion per accumulator element per
-// block, which on B200 issues at about a quarter of the FMA rate and would
-// bound the kernel.
+// product.  The tensor core computes I_b into its own TMEM buffer, from the
+// exact small integers (nibble - 8 in [-8, 7], q in [-127, 127]) held either
+// as int8 (kind::i8, one K = 32 MMA a block, int32 accumulator started at a
+// bias that makes its bits an fp32 1.5 * 2^23 + I_b) or as binary16
+// (kind::f16, two K = 16 MMAs a block; products and 32-term sums are exact in
+// the fp32 accumulator).  The epilogue then accumulates acc += I_b * (dW * dA)
+// in fp32 registers (packed f32x2 FMUL + FFMA, plus one packed FADD taking
+// the bias off for int8; the product of two binary16 scales is exact in
+// binary32).  int8 operands halve the converters' shared-memory traffic (the
+// activation codes go in as they are) but cost the epilogue the FADD and the
+// TMEM reset: they win on 32-slot tiles, where the converters bound the
+// kernel, and lose on 64- and 128-slot tiles, where the epilogue does.
 //
 // Tile: 128 weight rows (gate/up: 64 gate rows + the same 64 up rows; down:
 // 128 rows of H) x TN slots of one expert (MMA M = 128, N = TN), TN = 32, 64
 // or 128, chosen per call from the routed slots per expert (tc_tile_tokens):
 // a weight block converted once serves TN slots.
 //
-// Warp roles (10 warps for TN = 32, 14 for 64 and 128):
+// Warp roles (14 warps for TN = 32, 18 for 64, 14 for 128):
 //   0      producer: 2D tensor copies (TMA) of the packed weight rows (a box
-//          of 64 or 128 rows x 144 B = 8 blocks), two input stages in flight;
-//   1..4   converters, a weight row and a slot each: nibbles -> binary16
-//          (nib - 8) for the A operand; the slot's int8 activations and
-//          block scales come through a 4-entry ring of cp.async copies issued
-//          three operand stages ahead, then -> binary16 for the B operand;
-//          both into the K-major shared-memory layout (8-row x 16-byte core
-//          matrices); two operand stages of 2 blocks; block scales into a
-//          ring read by the epilogue;
-//   5      MMA issuer (one thread): two MMAs per block (A and B from shared
-//          memory); one wait and one commit per operand stage, for its pair
-//          of accumulators;
-//   6..    epilogue: 4 TMEM lane quarters x TN / CW column groups (CW = 32,
+//          of 64 or 128 rows x 144 B = 8 blocks), two input stages in flight,
+//          and the activation ring's cp.async copies;
+//   1..    converters (8 warps for 4-block operand stages, 4 for 2), a pair
+//          of blocks of a weight row and of a slot each: nibbles -> nib - 8
+//          (int8 or binary16) for the A operand, read as 16-byte loads of the
+//          window around the pair; the slot's int8 activations and block
+//          scales come through a 4-entry ring of cp.async copies the producer
+//          issues three operand stages ahead, then go into the B operand (as
+//          they are, or as binary16); both in the K-major shared-memory layout
+//          (8-row x 16-byte core matrices); two operand stages; block scales
+//          into a ring read by the epilogue;
+//   then   the MMA issuer (one thread): one (int8) or two (binary16) MMAs per
+//          block, A and B from shared memory; one wait and one commit per
+//          operand stage, for its set of accumulators;
+//   last   epilogue: 4 TMEM lane quarters x TN / CW column groups (CW = 32,
 //          or 64 for TN = 128); per operand stage one wait, TMEM loads of 16
 //          columns software-pipelined against the rescale-accumulate, the
 //          accumulator pair released as soon as its last chunk is in
 //          registers; after the last block of a tile gate/up -> SwiGLU +
 //          Q8_0 requantisation, down -> y += w_slot * o with vector
 //          reductions (red.v4.f32) of 4 consecutive rows of H of one token.
-// TMEM: four accumulators of TN columns, handed between the MMA issuer and the
-// epilogue a pair (one operand stage) at a time; full/empty mbarriers between
+// TMEM: two sets of OP_KB accumulators of TN columns, handed between the MMA
+// issuer and the epilogue a set (one operand stage) at a time; full/empty mbarriers between
 // every pair of roles; every wait bounded, and one that runs out makes every
 // role leave its loop and records STATUS_SPIN_TIMEOUT.
 #include <cuda.h>
@@ -86,7 +92,11 @@ struct TcCfg {
     // 128-slot tiles two (their eight accumulators would need 1024 columns)
     static constexpr int OP_KB = (TN == 128) ? 2 : 4;
     static constexpr int NACC = 2 * OP_KB;                // accumulators: two sets of OP_KB
-    static constexpr size_t SZ_OP_A = (size_t)OP_KB * 2 * TM * 32;   // one operand stage of A (K-steps of 16 x binary16)
+    // operand type: int8 (kind::i8, one K = 32 MMA a block) for 32-slot tiles,
+    // binary16 (kind::f16, two K = 16 MMAs a block) for wider ones
+    static constexpr bool I8 = (TN == 32);
+    static constexpr int OPB = I8 ? 1 : 2;                // bytes per operand element
+    static constexpr size_t SZ_OP_A = (size_t)OP_KB * OPB * TM * 32;   // one operand stage of A
     // a ring entry: OP_KB x 32 codes, OP_KB binary16 scales, padded to 16 bytes
     static constexpr size_t BPF_SLOT = ((size_t)OP_KB * (QK + 2) + 15) & ~size_t(15);
     // epilogue: a thread owns one accumulator row x CW columns; 4 warps (the
@@ -99,7 +109,7 @@ struct TcCfg {
     static constexpr int W_MMA = W_CONV0 + N_CONV / 32, W_EPI0 = W_MMA + 1;
     static constexpr int THREADS = (W_EPI0 * 32) + N_EPI;  // 10, 18 or 14 warps
     static constexpr uint32_t TMEM_COLS = NACC * TN;      // 512, 512 or 256 columns
-    static constexpr size_t SZ_OP_B = (size_t)OP_KB * 2 * TN * 32;
+    static constexpr size_t SZ_OP_B = (size_t)OP_KB * OPB * TN * 32;
     static constexpr int XCH_LD = TN + 1;
     static constexpr size_t OFF_IN_W = 0;
     static constexpr size_t OFF_OP_A = (OFF_IN_W + NIN * SZ_IN_W + 1023) & ~size_t(1023);
@@ -214,8 +224,36 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "memory");
 }
 
+// 16 consecutive 32-bit columns of this warp's 32 TMEM lanes, all set to v.
+__device__ __forceinline__ void tmem_st16_fill(uint32_t taddr, uint32_t v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+        "r"(v)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// int8 operands: every accumulator starts at ACC_BIAS and the MMAs add the
+// int32 block dot I (|I| <= 8 * 127 * 32 < 2^22) to it.  The int32
+// ACC_BIAS + I read as binary32 is exactly 1.5 * 2^23 + I (the significand
+// field of ACC_BIAS is 2^22, so adding I never carries into the exponent),
+// and one packed subtraction of 1.5 * 2^23 gives I exactly, with no
+// int32 -> fp32 conversion.
+constexpr uint32_t ACC_BIAS = 0x4B400000u;
+constexpr float ACC_BIAS_F = 12582912.0f;   // 1.5 * 2^23
+
+// The 16 block dots of one chunk as fp32 pairs: binary16 operands leave
+// exact fp32 integers; int8 operands leave them offset by ACC_BIAS.
+template <bool I8>
+__device__ __forceinline__ float2 block_dots2(uint32_t a, uint32_t b) {
+    const float2 v = make_float2(__uint_as_float(a), __uint_as_float(b));
+    if constexpr (I8) return __fadd2_rn(v, make_float2(-ACC_BIAS_F, -ACC_BIAS_F));
+    return v;
+}
+
 // acc[slot pair h8 + j] += I (16 columns of one block) * dW * dA[slot].
-template <int NA>
+template <bool I8, int NA>
 __device__ __forceinline__ void rescale_acc16(float2 (&acc)[NA], int h8, const uint32_t (&r)[16], float dwv,
                                               const float* da) {
     const float4* da4 = reinterpret_cast<const float4*>(da);
@@ -225,10 +263,8 @@ __device__ __forceinline__ void rescale_acc16(float2 (&acc)[NA], int h8, const u
         const float4 d = da4[j];
         const float2 s0 = __fmul2_rn(dw2, make_float2(d.x, d.y));
         const float2 s1 = __fmul2_rn(dw2, make_float2(d.z, d.w));
-        acc[h8 + 2 * j] =
-            __ffma2_rn(make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), s0, acc[h8 + 2 * j]);
-        acc[h8 + 2 * j + 1] = __ffma2_rn(make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), s1,
-                                         acc[h8 + 2 * j + 1]);
+        acc[h8 + 2 * j] = __ffma2_rn(block_dots2<I8>(r[4 * j], r[4 * j + 1]), s0, acc[h8 + 2 * j]);
+        acc[h8 + 2 * j + 1] = __ffma2_rn(block_dots2<I8>(r[4 * j + 2], r[4 * j + 3]), s1, acc[h8 + 2 * j + 1]);
     }
 }
 
@@ -252,6 +288,16 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
            | ((uint32_t)(M >> 4) << 24);    // M / 16
 }
 
+// Byte offset of the 16-byte core-matrix piece `core` (0/1) of row r in K-step
+// `ks` of block `kb` of an operand stage of `rows` rows.  A K-step is one
+// 32-byte slab per row (int8: the whole block, K = 32; binary16: half of it,
+// K = 16, so OPB = 2 K-steps a block); inside it, 8-row groups are 256 B
+// apart and the two pieces of a row 128 B apart (the descriptor's SBO and LBO).
+template <int OPB>
+__device__ __forceinline__ uint32_t op_off(int rows, int kb, int ks, int r, int core) {
+    return (uint32_t)((kb * OPB + ks) * rows * 32 + (r >> 3) * 256 + core * 128 + (r & 7) * 16);
+}
+
 // Four unsigned bytes u_i of w -> binary16 (1024 + u_i) - bias, two per word:
 // 1024 + u has the bit pattern 0x6400 | u for u < 256, and the subtraction of
 // two exact small integers is exact.
@@ -267,47 +313,59 @@ __device__ __forceinline__ uint2 bytes_to_f16(uint32_t w, uint32_t bias2) {
 constexpr uint32_t BIAS_NIB = 0x64086408u;   // binary16 1032, twice: 1024 + n - 1032 = n - 8
 constexpr uint32_t BIAS_ACT = 0x64806480u;   // binary16 1152, twice: 1024 + (q ^ 0x80) - 1152 = q
 
-// Byte offset of the 16-byte core-matrix piece `core` (0/1) of row r in K-step
-// `ks` of block `kb` of an operand stage of `rows` rows: K-steps are 32-byte
-// (16 x binary16) slabs; inside one, 8-row groups are 256 B apart and the two
-// pieces of a row 128 B apart (the descriptor's SBO and LBO).
-__device__ __forceinline__ uint32_t op_off(int rows, int kb, int ks, int r, int core) {
-    return (uint32_t)((kb * 2 + ks) * rows * 32 + (r >> 3) * 256 + core * 128 + (r & 7) * 16);
-}
+// Four nibbles n (one per byte, high bits clear) -> the bytes n - 8 as int8:
+// n + 0x78 stays below 0x88 (no carry between bytes) and flipping its top bit
+// subtracts 0x80.
+__device__ __forceinline__ uint32_t nib_to_s8(uint32_t w) { return (w + 0x78787878u) ^ 0x80808080u; }
 
-// 16 activation codes (one 16-byte load) -> the two core-matrix pieces of one
-// K-step of slot n.
-__device__ __forceinline__ void store_act16(uint8_t* ob, int rows, int kb, int ks, int n, uint4 a) {
-    const uint2 a0 = bytes_to_f16(a.x ^ 0x80808080u, BIAS_ACT);
-    const uint2 a1 = bytes_to_f16(a.y ^ 0x80808080u, BIAS_ACT);
-    const uint2 a2 = bytes_to_f16(a.z ^ 0x80808080u, BIAS_ACT);
-    const uint2 a3 = bytes_to_f16(a.w ^ 0x80808080u, BIAS_ACT);
-    *reinterpret_cast<uint4*>(ob + op_off(rows, kb, ks, n, 0)) = make_uint4(a0.x, a0.y, a1.x, a1.y);
-    *reinterpret_cast<uint4*>(ob + op_off(rows, kb, ks, n, 1)) = make_uint4(a2.x, a2.y, a3.x, a3.y);
-}
-
-// One Q4_0 block (qs as four words) -> the four core-matrix pieces of weight
-// row r: columns 0..7 of a K-step pair are the low nibbles (weights 0..15),
-// 8..15 the high nibbles (16..31).
+// One Q4_0 block (qs as four words) -> weight row r of block kb in the A
+// operand: the low nibbles are weights 0..15 of the block, the high nibbles
+// 16..31, each minus 8.
+template <bool I8>
 __device__ __forceinline__ void store_weights(uint8_t* oa, int kb, int r, const uint32_t (&qs)[4]) {
-    uint32_t v[16];
+    if constexpr (I8) {
+        *reinterpret_cast<uint4*>(oa + op_off<1>(TM, kb, 0, r, 0)) =
+            make_uint4(nib_to_s8(qs[0] & 0x0f0f0f0fu), nib_to_s8(qs[1] & 0x0f0f0f0fu),
+                       nib_to_s8(qs[2] & 0x0f0f0f0fu), nib_to_s8(qs[3] & 0x0f0f0f0fu));
+        *reinterpret_cast<uint4*>(oa + op_off<1>(TM, kb, 0, r, 1)) =
+            make_uint4(nib_to_s8((qs[0] >> 4) & 0x0f0f0f0fu), nib_to_s8((qs[1] >> 4) & 0x0f0f0f0fu),
+                       nib_to_s8((qs[2] >> 4) & 0x0f0f0f0fu), nib_to_s8((qs[3] >> 4) & 0x0f0f0f0fu));
+    } else {
+        uint32_t v[16];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint2 lo = bytes_to_f16(qs[i] & 0x0f0f0f0fu, BIAS_NIB);
-        const uint2 hi = bytes_to_f16((qs[i] >> 4) & 0x0f0f0f0fu, BIAS_NIB);
-        v[2 * i] = lo.x;
-        v[2 * i + 1] = lo.y;
-        v[8 + 2 * i] = hi.x;
-        v[8 + 2 * i + 1] = hi.y;
-    }
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks)
-#pragma unroll
-        for (int core = 0; core < 2; ++core) {
-            const int c0 = 8 * ks + 4 * core;
-            *reinterpret_cast<uint4*>(oa + op_off(TM, kb, ks, r, core)) =
-                make_uint4(v[c0], v[c0 + 1], v[c0 + 2], v[c0 + 3]);
+        for (int i = 0; i < 4; ++i) {
+            const uint2 lo = bytes_to_f16(qs[i] & 0x0f0f0f0fu, BIAS_NIB);
+            const uint2 hi = bytes_to_f16((qs[i] >> 4) & 0x0f0f0f0fu, BIAS_NIB);
+            v[2 * i] = lo.x;
+            v[2 * i + 1] = lo.y;
+            v[8 + 2 * i] = hi.x;
+            v[8 + 2 * i + 1] = hi.y;
         }
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+            for (int core = 0; core < 2; ++core) {
+                const int c0 = 8 * ks + 4 * core;
+                *reinterpret_cast<uint4*>(oa + op_off<2>(TM, kb, ks, r, core)) =
+                    make_uint4(v[c0], v[c0 + 1], v[c0 + 2], v[c0 + 3]);
+            }
+    }
+}
+
+// 16 activation codes (one 16-byte load: half `h` of block kb) -> slot n of
+// the B operand: as they are (int8), or as binary16 (one K-step).
+template <bool I8>
+__device__ __forceinline__ void store_act16(uint8_t* ob, int rows, int kb, int h, int n, uint4 a) {
+    if constexpr (I8) {
+        *reinterpret_cast<uint4*>(ob + op_off<1>(rows, kb, 0, n, h)) = a;
+    } else {
+        const uint2 a0 = bytes_to_f16(a.x ^ 0x80808080u, BIAS_ACT);
+        const uint2 a1 = bytes_to_f16(a.y ^ 0x80808080u, BIAS_ACT);
+        const uint2 a2 = bytes_to_f16(a.z ^ 0x80808080u, BIAS_ACT);
+        const uint2 a3 = bytes_to_f16(a.w ^ 0x80808080u, BIAS_ACT);
+        *reinterpret_cast<uint4*>(ob + op_off<2>(rows, kb, h, n, 0)) = make_uint4(a0.x, a0.y, a1.x, a1.y);
+        *reinterpret_cast<uint4*>(ob + op_off<2>(rows, kb, h, n, 1)) = make_uint4(a2.x, a2.y, a3.x, a3.y);
+    }
 }
 
 __device__ __forceinline__ int find_group(const int* tile_off, int ngroups, int tile) {
@@ -367,6 +425,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
     constexpr int N_CONV = C::N_CONV, W_MMA = C::W_MMA, W_EPI0 = C::W_EPI0;
     constexpr int OP_KB = C::OP_KB;
     constexpr size_t SZ_OP_A = C::SZ_OP_A, BPF_SLOT = C::BPF_SLOT;
+    constexpr bool I8 = C::I8;
     constexpr uint32_t TMEM_COLS = C::TMEM_COLS;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -558,11 +617,11 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     dws[0] = half_bits_to_float(w[0] & 0xffffu);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) qs[i] = __funnelshift_r(w[i], w[i + 1], 16);
-                    store_weights(oa, kb0, row, qs);
+                    store_weights<I8>(oa, kb0, row, qs);
                     dws[1] = half_bits_to_float(w[4] >> 16);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) qs[i] = w[5 + i];
-                    store_weights(oa, kb0 + 1, row, qs);
+                    store_weights<I8>(oa, kb0 + 1, row, qs);
                 }
                 // activations of slot `row` from the ring (zeros past the tile's slots)
                 uint32_t dab = 0;
@@ -572,11 +631,10 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
 #pragma unroll
                     for (int kb = kb0; kb < kb0 + 2; ++kb)
 #pragma unroll
-                        for (int ks = 0; ks < 2; ++ks) {
-                            const uint4 a = valid ? *reinterpret_cast<const uint4*>(src + 16 * (2 * kb + ks))
-                                                  : make_uint4(0, 0, 0, 0);
-                            store_act16(ob, TN, kb, ks, row, a);
-                        }
+                        for (int h = 0; h < 2; ++h)
+                            store_act16<I8>(ob, TN, kb, h, row,
+                                            valid ? *reinterpret_cast<const uint4*>(src + 16 * (2 * kb + h))
+                                                  : make_uint4(0, 0, 0, 0));
                     if (valid) dab = *reinterpret_cast<const uint32_t*>(src + OP_KB * QK + 2 * kb0);
                 }
                 __syncwarp();
@@ -602,9 +660,9 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_f16(TM, TN);
-            // descriptors of the first K-step of each operand stage; a later
-            // K-step adds its byte offset / 16 to the start-address field
+            constexpr uint32_t idesc = I8 ? idesc_i8(TM, TN) : idesc_f16(TM, TN);
+            // descriptors of the first block of each operand stage; a later
+            // block adds its byte offset / 16 to the start-address field
             const uint64_t b0 = smem_desc_kmajor(op_b, 128, 256), b1 = smem_desc_kmajor(op_b + C::SZ_OP_B, 128, 256);
             const uint64_t a0 = smem_desc_kmajor(op_a, 128, 256), a1 = smem_desc_kmajor(op_a + SZ_OP_A, 128, 256);
             static_assert(NOP == 2, "two operand stages");
@@ -617,9 +675,10 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                         ok = false;
                         break;
                     }
-                    // the pair of accumulators of this operand stage: buffers
-                    // 2o, 2o + 1, freed by the epilogue two stages ago
-                    if (!wait_phase(&tm_empty[o], ((i_op / 2) & 1) ^ 1, abort)) {
+                    // the set of accumulators of this operand stage, released by
+                    // the epilogue (int8 operands: reset to ACC_BIAS); its first
+                    // phase is the epilogue's start-up arrival
+                    if (!wait_phase(&tm_empty[o], (i_op / 2) & 1, abort)) {
                         ok = false;
                         break;
                     }
@@ -629,8 +688,13 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     for (int kb = 0; kb < OP_KB; ++kb) {
                         const uint32_t d = tmem + (uint32_t)(OP_KB * o + kb) * TN;
                         constexpr uint64_t KA = (uint64_t)TM * 32 >> 4, KB = (uint64_t)TN * 32 >> 4;  // K-step / 16
-                        mma_f16_ss(d, ad + (uint64_t)(kb * 2) * KA, bd + (uint64_t)(kb * 2) * KB, idesc, false);
-                        mma_f16_ss(d, ad + (uint64_t)(kb * 2 + 1) * KA, bd + (uint64_t)(kb * 2 + 1) * KB, idesc, true);
+                        if constexpr (I8) {
+                            mma_i8(d, ad + (uint64_t)kb * KA, bd + (uint64_t)kb * KB, idesc, true);  // onto ACC_BIAS
+                        } else {
+                            mma_f16_ss(d, ad + (uint64_t)(kb * 2) * KA, bd + (uint64_t)(kb * 2) * KB, idesc, false);
+                            mma_f16_ss(d, ad + (uint64_t)(kb * 2 + 1) * KA, bd + (uint64_t)(kb * 2 + 1) * KB, idesc,
+                                       true);
+                        }
                     }
                     mma_commit(&tm_full[o]);  // covers the set's MMAs
                     mma_commit(&op_empty[o]);
@@ -648,6 +712,20 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
         const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + CW * cq;
         uint32_t i_op = 0, epi_phase = 0;
         bool ok = true;
+        // both sets of accumulators start at ACC_BIAS (int8 operands)
+        if constexpr (I8) {
+#pragma unroll
+            for (int a = 0; a < C::NACC; ++a)
+#pragma unroll
+                for (int hf = 0; hf < NCH; ++hf) tmem_st16_fill(taddr + a * TN + 16 * hf, ACC_BIAS);
+            tmem_wait_st();
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&tm_empty[0]);
+            mbar_arrive(&tm_empty[1]);
+        }
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const Tile T = tile_of<TN>(item, n_rb, tile_off_s, off_s, ngroups);
             if (MODE == DOWN && et < TN) {
@@ -672,11 +750,13 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 tc_fence_after_sync();
                 // chunks of 16 columns (OP_KB blocks x CW / 16), software pipelined:
                 // the TMEM load of chunk qc + 1 is in flight while chunk qc is
-                // rescaled; the accumulator pair is released as soon as its
-                // last chunk is in registers
+                // rescaled; int8 operands: each chunk is reset to ACC_BIAS
+                // once it is in registers, and the set is released once every
+                // reset landed
                 uint32_t rA[16], rB[16];
                 tmem_ld16(taddr + (OP_KB * pr) * TN, rA);
                 tmem_wait_ld();
+                if constexpr (I8) tmem_st16_fill(taddr + (OP_KB * pr) * TN, ACC_BIAS);
 #pragma unroll
                 for (int qc = 0; qc < NCH * OP_KB; ++qc) {
                     const int kb = qc / NCH, hf = qc % NCH;
@@ -686,20 +766,26 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     }
                     const uint32_t(&r)[16] = (qc & 1) ? rB : rA;
                     if (CAP && T.g == p.cap_group && T.rb == p.cap_rb) {
-                        // exact integers held in binary32: convert back without rounding
+                        // the int32 block dots as the tensor cores left them
                         const size_t s0 = (size_t)(T.slot0 - off_s[T.g]);
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int n = CW * cq + 16 * hf + j;
                             if (n < T.nslots)
-                                p.cap_out[((s0 + n) * TM + row) * nbK + b + kb] = __float2int_rn(__uint_as_float(r[j]));
+                                p.cap_out[((s0 + n) * TM + row) * nbK + b + kb] =
+                                    I8 ? (int)(r[j] - ACC_BIAS) : __float2int_rn(__uint_as_float(r[j]));
                         }
                     }
-                    rescale_acc16(acc, 8 * hf, r, dw_ring[(sc * OP_KB + kb) * TM + row],
+                    rescale_acc16<I8>(acc, 8 * hf, r, dw_ring[(sc * OP_KB + kb) * TM + row],
                                   da_ring + (sc * OP_KB + kb) * TN + CW * cq + 16 * hf);
-                    if (qc + 1 < NCH * OP_KB) tmem_wait_ld();
+                    if (qc + 1 < NCH * OP_KB) {
+                        tmem_wait_ld();
+                        const int kb1 = (qc + 1) / NCH, hf1 = (qc + 1) % NCH;
+                        if constexpr (I8) tmem_st16_fill(taddr + (OP_KB * pr + kb1) * TN + 16 * hf1, ACC_BIAS);
+                    }
                     if (qc + 2 == NCH * OP_KB) {
-                        // every chunk of the pair is loaded: the accumulators are free
+                        // every chunk of the set is loaded and reset: the accumulators are free
+                        if constexpr (I8) tmem_wait_st();
                         tc_fence_before_sync();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&tm_empty[pr]);
@@ -777,6 +863,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
             }
             if (!epi_sync(&epi_bar, epi_phase++, abort)) break;  // xch is free for the next tile
         }
+        if constexpr (I8) tmem_wait_st();   // no reset may still be in flight when TMEM is freed
     }
 
     tc_fence_before_sync();

@@ -72,14 +72,10 @@ namespace {
 
 constexpr int TM = 128;            // MMA M: weight rows per tile
 constexpr int IN_KB = 8;           // Q4_0 blocks per input stage (144-byte rows: a 16-byte multiple)
-constexpr int NIN = 2, NOP = 2, NSC = 4;  // input, operand and scale-ring stages
 constexpr int IN_ROW = IN_KB * Q4_BYTES;          // 144
 constexpr int W_PROD = 0, W_CONV0 = 1;
 constexpr uint32_t LIMIT = 1u << 22;
 constexpr size_t SZ_IN_W = (size_t)TM * IN_ROW;           // one input stage of packed weight rows
-// Activation ring: NPF operand stages, a slot's OP_KB blocks of int8 codes and
-// their binary16 scales per entry, copied by the producer warp (cp.async).
-constexpr int NPF = 4;
 
 // Per tile width TN (slots, the MMA N): the blocks per operand stage, the
 // epilogue's column groups of 4 warps (one per TMEM lane quarter), and the
@@ -91,7 +87,17 @@ struct TcCfg {
     // so narrower tiles (less epilogue work a block) take four blocks a stage,
     // 128-slot tiles two (their eight accumulators would need 1024 columns)
     static constexpr int OP_KB = (TN == 128) ? 2 : 4;
-    static constexpr int NACC = 2 * OP_KB;                // accumulators: two sets of OP_KB
+    // pipeline depths: input stages of weight rows (NIN), operand stages
+    // (NOP), accumulator sets in TMEM (NTS), the scale ring (NSC) and the
+    // activation ring (NPF: operand stages of a slot's OP_KB blocks of int8
+    // codes and their binary16 scales, copied by the producer warp); the
+    // narrow tiles have the shared memory to run deeper
+    static constexpr int NIN = (TN == 32) ? 4 : 2;
+    static constexpr int NOP = (TN == 32) ? 3 : 2;
+    static constexpr int NTS = (TN == 32) ? 3 : 2;
+    static constexpr int NSC = (TN == 32) ? 8 : 4;
+    static constexpr int NPF = (TN == 32) ? 6 : 4;
+    static constexpr int NACC = NTS * OP_KB;              // accumulators: NTS sets of OP_KB
     // operand type: int8 (kind::i8, one K = 32 MMA a block) for 32-slot tiles,
     // binary16 (kind::f16, two K = 16 MMAs a block) for wider ones
     static constexpr bool I8 = (TN == 32);
@@ -108,7 +114,7 @@ struct TcCfg {
     static constexpr int N_CONV = TM * OP_KB / 2;
     static constexpr int W_MMA = W_CONV0 + N_CONV / 32, W_EPI0 = W_MMA + 1;
     static constexpr int THREADS = (W_EPI0 * 32) + N_EPI;  // 10, 18 or 14 warps
-    static constexpr uint32_t TMEM_COLS = NACC * TN;      // 512, 512 or 256 columns
+    static constexpr uint32_t TMEM_COLS = (NACC * TN <= 256) ? 256 : 512;   // a power of two
     static constexpr size_t SZ_OP_B = (size_t)OP_KB * OPB * TN * 32;
     static constexpr int XCH_LD = TN + 1;
     static constexpr size_t OFF_IN_W = 0;
@@ -429,8 +435,9 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
     constexpr uint32_t TMEM_COLS = C::TMEM_COLS;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t in_full[NIN], in_empty[NIN], op_full[NOP], op_empty[NOP], tm_full[2],
-        tm_empty[2], sc_full[NSC], sc_empty[NSC], epi_bar, b_full[NPF], b_empty[NPF];
+    constexpr int NIN = C::NIN, NOP = C::NOP, NTS = C::NTS, NSC = C::NSC, NPF = C::NPF;
+    __shared__ __align__(8) uint64_t in_full[NIN], in_empty[NIN], op_full[NOP], op_empty[NOP], tm_full[NTS],
+        tm_empty[NTS], sc_full[NSC], sc_empty[NSC], epi_bar, b_full[NPF], b_empty[NPF];
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ int tile_off_s[258], off_s[258];
@@ -467,7 +474,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
             mbar_init(&op_full[i], N_CONV);
             mbar_init(&op_empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {  // one pair of accumulators each
+        for (int i = 0; i < NTS; ++i) {  // one set of accumulators each
             mbar_init(&tm_full[i], 1);
             mbar_init(&tm_empty[i], N_EPI / 32);
         }
@@ -661,16 +668,15 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = I8 ? idesc_i8(TM, TN) : idesc_f16(TM, TN);
-            // descriptors of the first block of each operand stage; a later
-            // block adds its byte offset / 16 to the start-address field
-            const uint64_t b0 = smem_desc_kmajor(op_b, 128, 256), b1 = smem_desc_kmajor(op_b + C::SZ_OP_B, 128, 256);
-            const uint64_t a0 = smem_desc_kmajor(op_a, 128, 256), a1 = smem_desc_kmajor(op_a + SZ_OP_A, 128, 256);
-            static_assert(NOP == 2, "two operand stages");
+            // descriptors of the first K-step of operand stage 0; a later
+            // stage or K-step adds its byte offset / 16 to the start-address
+            // field (shared-memory offsets stay below 2^18: no carry out)
+            const uint64_t b00 = smem_desc_kmajor(op_b, 128, 256), a00 = smem_desc_kmajor(op_a, 128, 256);
             uint32_t i_op = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 for (int c = 0; c < nbK / OP_KB; ++c, ++i_op) {
-                    const int o = i_op & 1;
+                    const int o = i_op % NOP, ts = i_op % NTS;
                     if (!wait_phase(&op_full[o], (i_op / NOP) & 1, abort)) {
                         ok = false;
                         break;
@@ -678,15 +684,15 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     // the set of accumulators of this operand stage, released by
                     // the epilogue (int8 operands: reset to ACC_BIAS); its first
                     // phase is the epilogue's start-up arrival
-                    if (!wait_phase(&tm_empty[o], (i_op / 2) & 1, abort)) {
+                    if (!wait_phase(&tm_empty[ts], (i_op / NTS) & 1, abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint64_t bd = o ? b1 : b0, ad = o ? a1 : a0;
+                    const uint64_t bd = b00 + (uint64_t)((o * C::SZ_OP_B) >> 4), ad = a00 + (uint64_t)((o * SZ_OP_A) >> 4);
 #pragma unroll
                     for (int kb = 0; kb < OP_KB; ++kb) {
-                        const uint32_t d = tmem + (uint32_t)(OP_KB * o + kb) * TN;
+                        const uint32_t d = tmem + (uint32_t)(OP_KB * ts + kb) * TN;
                         constexpr uint64_t KA = (uint64_t)TM * 32 >> 4, KB = (uint64_t)TN * 32 >> 4;  // K-step / 16
                         if constexpr (I8) {
                             mma_i8(d, ad + (uint64_t)kb * KA, bd + (uint64_t)kb * KB, idesc, true);  // onto ACC_BIAS
@@ -696,7 +702,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                                        true);
                         }
                     }
-                    mma_commit(&tm_full[o]);  // covers the set's MMAs
+                    mma_commit(&tm_full[ts]);  // covers the set's MMAs
                     mma_commit(&op_empty[o]);
                 }
             }
@@ -723,8 +729,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) {
-            mbar_arrive(&tm_empty[0]);
-            mbar_arrive(&tm_empty[1]);
+            for (int i = 0; i < NTS; ++i) mbar_arrive(&tm_empty[i]);
         }
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const Tile T = tile_of<TN>(item, n_rb, tile_off_s, off_s, ngroups);
@@ -741,7 +746,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < CW / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
             for (int b = 0; b < nbK; b += OP_KB, ++i_op) {
-                const uint32_t pr = i_op & 1, ppar = (i_op >> 1) & 1;
+                const uint32_t pr = i_op % NTS, ppar = (i_op / NTS) & 1;
                 const uint32_t sc = i_op % NSC, spar = (i_op / NSC) & 1;
                 if (!wait_phase(&tm_full[pr], ppar, abort) || !wait_phase(&sc_full[sc], spar, abort)) {
                     ok = false;

@@ -272,13 +272,44 @@ def int8_peak_tops():
     return 1590.0 * 2.0, "fallback bf16 x nominal int8/bf16 ratio 2"
 
 
+def rescale_ceiling(m, torch, stream, peak):
+    """The tensor-core epilogue's per-block rescale alone (moe_q4_rescale_ceiling):
+    accumulator elements per second for binary16 and int8 operands, and the
+    int8 rate that bounds (64 ops an element: 32 multiply-adds)."""
+    sink = torch.zeros(1, dtype=torch.float32, device="cuda")
+    out = {}
+    for name, i8 in (("binary16_operands", False), ("int8_operands", True)):
+        times = []
+        n = 0
+        for rep in range(7):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            n = m.moe_q4_rescale_ceiling(i8, 4096, sink, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 2:
+                times.append(e0.elapsed_time(e1))
+        ms = float(np.median(times))
+        eps = n / (ms * 1e-3)
+        out[name] = {"ms": ms, "elements_per_s": eps, "int8_tops_bound": eps * 64 / 1e12,
+                     "frac_of_int8_peak": eps * 64 / 1e12 / peak}
+    out["how"] = ("one CTA per SM, 16 warps, 4096 operand stages of the epilogue's inner loop over all of TMEM "
+                  "(4 blocks x 32 columns a thread a stage), no other role")
+    return out
+
+
 def prefill_lines(m, torch, stream, names=("prefill_t947", "zipf_t16384")):
     """Single-pass prefill of the two prefill workloads on the automatic path
     (tensor cores at these sizes): tokens/s over whole forwards and the int8
-    ops/s of the gate/up kernel, L2 flushed (256 MB written) before each rep."""
+    ops/s of the gate/up kernel, L2 flushed (256 MB written) before each rep;
+    the gate/up rate also as a fraction of the epilogue-rescale ceiling of its
+    operand type (binary16 on 64- and 128-slot tiles, the automatic choice at
+    these sizes; int8 on 32-slot ones)."""
     import synth
     out = {}
     peak, peak_src = int8_peak_tops()
+    ceil = rescale_ceiling(m, torch, stream, peak)
+    out["rescale_ceiling"] = ceil
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     variants = (("auto", m.PATH_AUTO), ("tc_n32", m.PATH_TENSOR_CORE_N32), ("tc_n64", m.PATH_TENSOR_CORE_N64),
                 ("tc_n128", m.PATH_TENSOR_CORE_N128))
@@ -310,6 +341,8 @@ def prefill_lines(m, torch, stream, names=("prefill_t947", "zipf_t16384")):
             rec = {"tokens_per_s": T / (ms * 1e-3), "ms": ms, "gateup_ms": gu_ms,
                    "gateup_int8_tops": gu_ops / (gu_ms * 1e-3) / 1e12,
                    "gateup_frac_of_int8_peak": gu_ops / (gu_ms * 1e-3) / 1e12 / peak,
+                   "gateup_frac_of_rescale_ceiling": gu_ops / (gu_ms * 1e-3) / 1e12 / ceil[
+                       "int8_operands" if vname == "tc_n32" else "binary16_operands"]["int8_tops_bound"],
                    "layer_int8_tops": all_ops / (ms * 1e-3) / 1e12,
                    "layer_frac_of_int8_peak": all_ops / (ms * 1e-3) / 1e12 / peak}
             if vname == "auto":

@@ -345,6 +345,21 @@ int moe_q4_test_override_device(int32_t enable, int32_t major, int32_t minor);
 int moe_q4_block_dots(const uint8_t* w_blocks, const int8_t* qa, int64_t n, int32_t* out,
                       moe_q4_stream_t stream);
 
+/* Measurement aid: the tensor-core projections' epilogue rescale on its own
+ * (the per-block step acc += I_b * dW * dA that follows every 32-wide block's
+ * MMA; "Methodologie 1" of the Dutch technical summary page, the W4A8 block
+ * arithmetic).  One CTA per SM runs `iters` (1 .. 2^20) operand stages of the
+ * epilogue's inner loop -- TMEM loads, block scales from shared memory, the
+ * packed fp32 rescale, and with int8_operands != 0 the int8 path's bias
+ * removal and TMEM reset -- over its whole TMEM, with no other role, so its
+ * rate is the ceiling the rescale puts on the projection kernels.  Writes one
+ * float (a checksum that keeps the work live) to sink (device, 4-byte
+ * aligned) and the number of accumulator elements rescaled to *elements
+ * (host); each element stands for 32 int8 multiply-adds.  Asynchronous on
+ * `stream`; time it with events around the call. */
+int moe_q4_rescale_ceiling(int32_t int8_operands, int32_t iters, float* sink, int64_t* elements,
+                           moe_q4_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -48,7 +48,8 @@ EXPORTS = ["moe_q4_quantize_act", "moe_q4_route", "moe_q4_ffn_workspace_bytes", 
            "moe_q4_workspace_layout", "moe_q4_ffn_forward_debug", "moe_q4_block_dots",
            "moe_q4_ffn_forward_noalloc", "moe_q4_last_cuda_error", "moe_q4_residual_rmsnorm",
            "moe_q4_stack_workspace_bytes", "moe_q4_stack_forward", "moe_q4_gemv_workspace_bytes", "moe_q4_gemv",
-           "moe_q4_staging_bytes", "moe_q4_ffn_forward_streamed", "moe_q4_test_override_device"]
+           "moe_q4_staging_bytes", "moe_q4_ffn_forward_streamed", "moe_q4_test_override_device",
+           "moe_q4_rescale_ceiling"]
 
 
 class MoeQ4Error(RuntimeError):
@@ -106,6 +107,7 @@ def _load() -> ctypes.CDLL:
         "moe_q4_staging_bytes": ([P], sz),
         "moe_q4_ffn_forward_streamed": ([P, P, i64, P, P, sz, P, sz, P], ctypes.c_int),
         "moe_q4_test_override_device": ([i32, i32, i32], ctypes.c_int),
+        "moe_q4_rescale_ceiling": ([i32, i32, P, P, P], ctypes.c_int),
     }
     for name, (args, res) in sigs.items():
         f = getattr(lib, name)
@@ -301,6 +303,16 @@ def moe_q4_block_dots(w_blocks: torch.Tensor, qa: torch.Tensor, out=None, stream
     out = torch.empty(n, dtype=torch.int32, device=w_blocks.device) if out is None else out
     _check(_lib.moe_q4_block_dots(_p(w_blocks), _p(qa), n, _p(out), _stream(stream)), "moe_q4_block_dots")
     return out
+
+
+def moe_q4_rescale_ceiling(int8_operands: bool, iters: int, sink: torch.Tensor, stream=None) -> int:
+    """Launch the epilogue-rescale measurement kernel (include/moe_q4.h) on
+    `stream`; returns the number of accumulator elements it rescales (each
+    one 32 int8 multiply-adds).  sink: a device float32 tensor of >= 1."""
+    n = ctypes.c_int64(0)
+    _check(_lib.moe_q4_rescale_ceiling(int(bool(int8_operands)), int(iters), _p(sink), ctypes.byref(n),
+                                       _stream(stream)), "moe_q4_rescale_ceiling")
+    return n.value
 
 
 def moe_q4_ffn_forward_noalloc(layer: Layer, x: torch.Tensor, y=None, stream=None):

@@ -610,4 +610,15 @@ int moe_q4_block_dots(const uint8_t* w_blocks, const int8_t* qa, int64_t n, int3
     return cuda_rc(launch_block_dots(w_blocks, qa, n, out, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int moe_q4_rescale_ceiling(int32_t int8_operands, int32_t iters, float* sink, int64_t* elements,
+                           moe_q4_stream_t stream) {
+    if (iters < 1 || iters > (1 << 20) || !sink || !elements) return MOE_Q4_ERR_INVALID_ARG;
+    if (!aligned(sink, 4)) return MOE_Q4_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    return cuda_rc(launch_rescale_ceiling(int8_operands != 0, iters, sink, dev, elements,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

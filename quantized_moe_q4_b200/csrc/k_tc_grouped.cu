@@ -419,6 +419,78 @@ __device__ __forceinline__ void take_words(uint32_t (&w)[N], const uint32_t (&wi
     for (int i = 0; i < N; ++i) w[i] = (i + OFS < M) ? win[i + OFS] : 0u;
 }
 
+// ---------------------------------------------------------------------------
+// The epilogue's per-block rescale on its own (a measurement aid): one CTA per
+// SM of RC_WARPS warps, each owning TMEM lane quarter warp % 4 and 128 of the
+// 512 columns, runs `iters` operand stages of the epilogue's inner loop over
+// them -- 16-column TMEM loads software-pipelined against rescale_acc16, the
+// block scales read from shared memory, and for int8 operands the reset of
+// every chunk to ACC_BIAS and the wait for it -- with nothing handed between
+// roles, so its rate bounds the rescale of the projection kernels.  A stage
+// is 4 blocks x 32 columns per thread, as in the 32- and 64-slot tiles.
+constexpr int RC_WARPS = 16;
+
+template <bool I8>
+__global__ void __launch_bounds__(RC_WARPS * 32, 1) rescale_ceiling_kernel(int iters, float* sink) {
+    __shared__ uint32_t tmem_base_s;
+    __shared__ __align__(16) float da_s[4 * 4 * 32];     // 4 scale-ring entries x 4 blocks x 32 slots
+    __shared__ float dw_s[4 * 4 * 128];                  // 4 entries x 4 blocks x 128 rows
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < 4 * 4 * 32; i += RC_WARPS * 32) da_s[i] = 1.0f + (float)(i & 63) * (1.0f / 1024.0f);
+    for (int i = tid; i < 4 * 4 * 128; i += RC_WARPS * 32) dw_s[i] = 1.0f / 4096.0f + (float)(i & 31) * 1e-6f;
+    if (warp == 0) {
+        tmem_alloc(&tmem_base_s, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const int q = warp & 3, cg = warp >> 2;            // lane quarter, group of 128 columns
+    const int row = 32 * q + lane;
+    const uint32_t taddr = tmem_base_s + ((uint32_t)(32 * q) << 16) + 128u * cg;
+    // small exact integers (1 + the column) as the accumulators' contents
+#pragma unroll
+    for (int c = 0; c < 8; ++c) tmem_st16_fill(taddr + 16 * c, I8 ? ACC_BIAS + 1u + c : __float_as_uint(1.0f + c));
+    tmem_wait_st();
+    tc_fence_before_sync();
+    __syncwarp();
+    tc_fence_after_sync();
+    float2 acc[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc[j] = make_float2(0.0f, 0.0f);
+    for (int it = 0; it < iters; ++it) {
+        const int sc = it & 3;
+        uint32_t rA[16], rB[16];
+        tmem_ld16(taddr, rA);
+        tmem_wait_ld();
+        if constexpr (I8) tmem_st16_fill(taddr, ACC_BIAS + 1u);
+#pragma unroll
+        for (int qc = 0; qc < 8; ++qc) {           // 4 blocks x 2 chunks of 16 columns
+            const int kb = qc >> 1, hf = qc & 1;
+            if (qc + 1 < 8) tmem_ld16(taddr + 16 * (qc + 1), (qc & 1) ? rA : rB);
+            const uint32_t(&r)[16] = (qc & 1) ? rB : rA;
+            rescale_acc16<I8>(acc, 8 * hf, r, dw_s[(sc * 4 + kb) * 128 + row], da_s + (sc * 4 + kb) * 32 + 16 * hf);
+            if (qc + 1 < 8) {
+                tmem_wait_ld();
+                if constexpr (I8) tmem_st16_fill(taddr + 16 * (qc + 1), ACC_BIAS + 1u + (qc + 1));
+            }
+            if (qc + 2 == 8) {
+                if constexpr (I8) tmem_wait_st();
+                tc_fence_before_sync();
+                __syncwarp();
+                tc_fence_after_sync();
+            }
+        }
+    }
+    float t = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) t += acc[j].x + acc[j].y;
+    if (blockIdx.x == 0 && tid == 0) *sink = t;
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem_base_s, 512);
+}
+
 }  // namespace
 
 // CAP: also write the per-block integer sums (the MMA accumulators before the
@@ -999,6 +1071,17 @@ cudaError_t launch_gateup_tc(const LayerView& L, int64_t T, const Workspace& ws,
 cudaError_t launch_down_tc(const LayerView& L, int64_t T, const Workspace& ws, float* y, const DeviceInfo& dev,
                            int tile, const BlockDotCapture* cap, cudaStream_t s) {
     return launch_tc<DOWN>(L, T, ws, nullptr, y, dev, tile, cap, s);
+}
+
+cudaError_t launch_rescale_ceiling(bool int8_operands, int iters, float* sink, const DeviceInfo& dev,
+                                   int64_t* elements, cudaStream_t s) {
+    const dim3 grid((unsigned)dev.sm_count), block(RC_WARPS * 32);
+    if (int8_operands)
+        rescale_ceiling_kernel<true><<<grid, block, 0, s>>>(iters, sink);
+    else
+        rescale_ceiling_kernel<false><<<grid, block, 0, s>>>(iters, sink);
+    *elements = (int64_t)dev.sm_count * RC_WARPS * 32 * 128 * (int64_t)iters;
+    return cudaGetLastError();
 }
 
 }  // namespace moeq4

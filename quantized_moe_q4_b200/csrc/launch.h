@@ -106,6 +106,12 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
 cudaError_t launch_block_dots(const uint8_t* w, const int8_t* qa, int64_t n, int32_t* out,
                               cudaStream_t s);
 
+// k_tc_grouped.cu: the tensor-core epilogue's per-block rescale on its own
+// (one CTA per SM, iters operand stages); *elements = accumulator elements
+// rescaled (each one 32 int8 multiply-adds of the projection).
+cudaError_t launch_rescale_ceiling(bool int8_operands, int iters, float* sink, const DeviceInfo& dev,
+                                   int64_t* elements, cudaStream_t s);
+
 // k_stage.cu: copy the experts with cnt[g] > 0 (and the shared expert) from
 // pinned host memory (h_*) into the device staging copy (d_*).
 struct StageParams {

@@ -138,6 +138,14 @@ def test_other_entry_points_reject_bad_args(lib):
     b.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
     assert b(FAKE, FAKE, 7, FAKE, None) == -1                # n not a multiple of 8
     assert b(FAKE + 2, FAKE, 8, FAKE, None) == -3
+    rc = lib.moe_q4_rescale_ceiling
+    rc.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    n = ctypes.c_int64(0)
+    assert rc(0, 0, FAKE, ctypes.byref(n), None) == -1           # no stages
+    assert rc(1, (1 << 20) + 1, FAKE, ctypes.byref(n), None) == -1
+    assert rc(0, 8, None, ctypes.byref(n), None) == -1           # no sink
+    assert rc(0, 8, FAKE, None, None) == -1                      # no element count
+    assert rc(1, 8, FAKE + 2, ctypes.byref(n), None) == -3       # sink not 4-byte aligned
     d = lib.moe_q4_ffn_forward_debug
     d.argtypes = [ctypes.c_void_p] * 2 + [ctypes.c_int64] + [ctypes.c_void_p] * 2 + [ctypes.c_size_t] + \
                  [ctypes.c_void_p] * 2

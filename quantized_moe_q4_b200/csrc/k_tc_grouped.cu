@@ -115,7 +115,13 @@ struct TcCfg {
     static constexpr int W_MMA = W_CONV0 + N_CONV / 32, W_EPI0 = W_MMA + 1;
     static constexpr int THREADS = (W_EPI0 * 32) + N_EPI;  // 10, 18 or 14 warps
     static constexpr uint32_t TMEM_COLS = (NACC * TN <= 256) ? 256 : 512;   // a power of two
-    static constexpr size_t SZ_OP_B = (size_t)OP_KB * OPB * TN * 32;
+    // binary16 tiles convert the activations into B operand stages; int8
+    // tiles read B straight from the activation ring, whose entries then hold
+    // the codes in the MMA's core-matrix layout followed by the scales
+    static constexpr size_t SZ_OP_B = I8 ? 0 : (size_t)OP_KB * OPB * TN * 32;
+    static constexpr size_t BPF_CODES = (size_t)OP_KB * TN * 32;
+    static constexpr size_t BPF_ENTRY = I8 ? ((BPF_CODES + (size_t)TN * OP_KB * 2 + 15) & ~size_t(15))
+                                           : (size_t)TN * BPF_SLOT;
     static constexpr int XCH_LD = TN + 1;
     static constexpr size_t OFF_IN_W = 0;
     static constexpr size_t OFF_OP_A = (OFF_IN_W + NIN * SZ_IN_W + 1023) & ~size_t(1023);
@@ -124,7 +130,7 @@ struct TcCfg {
     static constexpr size_t OFF_DA = OFF_DW + (size_t)NSC * OP_KB * TM * 4;
     static constexpr size_t OFF_XCH = OFF_DA + (size_t)NSC * OP_KB * TN * 4;
     static constexpr size_t OFF_BPF = OFF_XCH + (size_t)TM * XCH_LD * 4;
-    static constexpr size_t SMEM_BYTES = OFF_BPF + (size_t)NPF * TN * BPF_SLOT;
+    static constexpr size_t SMEM_BYTES = OFF_BPF + (size_t)NPF * BPF_ENTRY;
     static constexpr size_t SMEM_ALLOC = SMEM_BYTES + 1024;   // slack to align the map to 1024 B
     static_assert(SMEM_ALLOC <= 226 * 1024, "shared memory map too large");
     static_assert(TMEM_COLS <= 512, "TMEM budget");
@@ -556,7 +562,9 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
         }
         for (int i = 0; i < NPF; ++i) {
             mbar_init(&b_full[i], 32);              // the producer's 32 lanes, after their copies land
-            mbar_init(&b_empty[i], N_CONV / 32);    // the converter warps, after reading the entry
+            // binary16: the converter warps, after reading the entry; int8:
+            // the MMAs' commit and the converter warp that takes the scales
+            mbar_init(&b_empty[i], I8 ? 2 : N_CONV / 32);
         }
         mbar_init(&epi_bar, N_EPI / 32);
         mbar_fence_init();
@@ -626,12 +634,25 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
 #pragma unroll
                     for (int q = 0; q < SPL; ++q) {
                         if (!arow[q]) continue;
-                        uint8_t* dst = bpf + ((size_t)r * TN + lane + 32 * q) * BPF_SLOT;
+                        const int n = lane + 32 * q;
                         const int8_t* src = arow[q] + (size_t)cb * OP_KB * QK;
+                        if constexpr (I8) {
+                            // codes into the B operand layout (block kb: a K = 32
+                            // slab of TN rows), scales after them
+                            uint8_t* ent = bpf + (size_t)r * C::BPF_ENTRY;
 #pragma unroll
-                        for (int i = 0; i < 2 * OP_KB; ++i) cp_async16(dst + 16 * i, src + 16 * i);
-                        if (OP_KB == 4) cp_async8(dst + OP_KB * QK, ascale[q] + cb * OP_KB);
-                        else cp_async4(dst + OP_KB * QK, ascale[q] + cb * OP_KB);
+                            for (int kb = 0; kb < OP_KB; ++kb)
+#pragma unroll
+                                for (int h = 0; h < 2; ++h)
+                                    cp_async16(ent + op_off<1>(TN, kb, 0, n, h), src + 32 * kb + 16 * h);
+                            cp_async8(ent + C::BPF_CODES + 8 * n, ascale[q] + cb * OP_KB);
+                        } else {
+                            uint8_t* dst = bpf + (size_t)r * C::BPF_ENTRY + (size_t)n * BPF_SLOT;
+#pragma unroll
+                            for (int i = 0; i < 2 * OP_KB; ++i) cp_async16(dst + 16 * i, src + 16 * i);
+                            if (OP_KB == 4) cp_async8(dst + OP_KB * QK, ascale[q] + cb * OP_KB);
+                            else cp_async4(dst + OP_KB * QK, ascale[q] + cb * OP_KB);
+                        }
                     }
                     cp_async_arrive_noinc(&b_full[r]);
                 }
@@ -687,7 +708,6 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     }
                 }
                 uint8_t* oa = op_a + (size_t)o * SZ_OP_A;
-                uint8_t* ob = op_b + (size_t)o * C::SZ_OP_B;
                 float dws[2];
                 {
                     // the pair's first block starts at its byte 0 (scale, then
@@ -702,22 +722,40 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     for (int i = 0; i < 4; ++i) qs[i] = w[5 + i];
                     store_weights<I8>(oa, kb0 + 1, row, qs);
                 }
-                // activations of slot `row` from the ring (zeros past the tile's slots)
-                uint32_t dab = 0;
-                if (!wait_phase(&b_full[i_op % NPF], (i_op / NPF) & 1, abort)) { ok = false; break; }
-                if (row < TN) {
-                    const uint8_t* src = bpf + ((size_t)(i_op % NPF) * TN + row) * BPF_SLOT;
+                // activations.  binary16 tiles: slot `row`'s codes from the ring
+                // into the B operand (zeros past the tile's slots).  int8 tiles:
+                // the MMA reads the codes in the ring; the first converter warp
+                // takes the scales of slot `lane` (all OP_KB blocks)
+                uint32_t dab = 0, dab2 = 0;
+                if constexpr (I8) {
+                    if (ct < 32) {
+                        if (!wait_phase(&b_full[i_op % NPF], (i_op / NPF) & 1, abort)) { ok = false; break; }
+                        if (valid) {
+                            const uint2 v = *reinterpret_cast<const uint2*>(bpf + (size_t)(i_op % NPF) * C::BPF_ENTRY +
+                                                                            C::BPF_CODES + 8 * lane);
+                            dab = v.x;
+                            dab2 = v.y;
+                        }
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&b_empty[i_op % NPF]);   // with the MMAs' commit: entry free
+                    }
+                } else {
+                    uint8_t* ob = op_b + (size_t)o * C::SZ_OP_B;
+                    if (!wait_phase(&b_full[i_op % NPF], (i_op / NPF) & 1, abort)) { ok = false; break; }
+                    if (row < TN) {
+                        const uint8_t* src = bpf + (size_t)(i_op % NPF) * C::BPF_ENTRY + (size_t)row * BPF_SLOT;
 #pragma unroll
-                    for (int kb = kb0; kb < kb0 + 2; ++kb)
+                        for (int kb = kb0; kb < kb0 + 2; ++kb)
 #pragma unroll
-                        for (int h = 0; h < 2; ++h)
-                            store_act16<I8>(ob, TN, kb, h, row,
-                                            valid ? *reinterpret_cast<const uint4*>(src + 16 * (2 * kb + h))
-                                                  : make_uint4(0, 0, 0, 0));
-                    if (valid) dab = *reinterpret_cast<const uint32_t*>(src + OP_KB * QK + 2 * kb0);
+                            for (int h = 0; h < 2; ++h)
+                                store_act16<I8>(ob, TN, kb, h, row,
+                                                valid ? *reinterpret_cast<const uint4*>(src + 16 * (2 * kb + h))
+                                                      : make_uint4(0, 0, 0, 0));
+                        if (valid) dab = *reinterpret_cast<const uint32_t*>(src + OP_KB * QK + 2 * kb0);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&b_empty[i_op % NPF]);   // the ring entry is free again
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&b_empty[i_op % NPF]);   // the ring entry is free again
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 mbar_arrive(&op_full[o]);
@@ -726,11 +764,21 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 const int sc = i_op % NSC;
                 if (!wait_phase(&sc_empty[sc], ((i_op / NSC) & 1) ^ 1, abort)) { ok = false; break; }
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    dw_ring[(sc * OP_KB + kb0 + i) * TM + row] = dws[i];
-                    if (row < TN)
-                        da_ring[(sc * OP_KB + kb0 + i) * TN + row] =
-                            valid ? half_bits_to_float(i ? (dab >> 16) : dab) : 0.0f;
+                for (int i = 0; i < 2; ++i) dw_ring[(sc * OP_KB + kb0 + i) * TM + row] = dws[i];
+                if constexpr (I8) {
+                    static_assert(!I8 || OP_KB == 4, "int8 tiles: 4-block stages");
+                    if (ct < 32) {
+                        const uint32_t d4[4] = {dab & 0xffffu, dab >> 16, dab2 & 0xffffu, dab2 >> 16};
+#pragma unroll
+                        for (int kb = 0; kb < 4; ++kb)
+                            da_ring[(sc * OP_KB + kb) * TN + lane] = valid ? half_bits_to_float(d4[kb]) : 0.0f;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 2; ++i)
+                        if (row < TN)
+                            da_ring[(sc * OP_KB + kb0 + i) * TN + row] =
+                                valid ? half_bits_to_float(i ? (dab >> 16) : dab) : 0.0f;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sc_full[sc]);
@@ -743,7 +791,8 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
             // descriptors of the first K-step of operand stage 0; a later
             // stage or K-step adds its byte offset / 16 to the start-address
             // field (shared-memory offsets stay below 2^18: no carry out)
-            const uint64_t b00 = smem_desc_kmajor(op_b, 128, 256), a00 = smem_desc_kmajor(op_a, 128, 256);
+            const uint64_t b00 = smem_desc_kmajor(I8 ? smem + C::OFF_BPF : op_b, 128, 256);
+            const uint64_t a00 = smem_desc_kmajor(op_a, 128, 256);
             uint32_t i_op = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -760,8 +809,20 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                         ok = false;
                         break;
                     }
+                    if constexpr (I8) {
+                        // the B operand is the ring entry the producer's
+                        // cp.async copies filled (generic proxy): order them
+                        // before the MMA's reads (async proxy)
+                        if (!wait_phase(&b_full[i_op % NPF], (i_op / NPF) & 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        fence_proxy_async_smem();
+                    }
                     tc_fence_after_sync();
-                    const uint64_t bd = b00 + (uint64_t)((o * C::SZ_OP_B) >> 4), ad = a00 + (uint64_t)((o * SZ_OP_A) >> 4);
+                    const uint64_t bd = I8 ? b00 + (uint64_t)(((i_op % NPF) * C::BPF_ENTRY) >> 4)
+                                           : b00 + (uint64_t)((o * C::SZ_OP_B) >> 4);
+                    const uint64_t ad = a00 + (uint64_t)((o * SZ_OP_A) >> 4);
 #pragma unroll
                     for (int kb = 0; kb < OP_KB; ++kb) {
                         const uint32_t d = tmem + (uint32_t)(OP_KB * ts + kb) * TN;
@@ -776,10 +837,12 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     }
                     mma_commit(&tm_full[ts]);  // covers the set's MMAs
                     mma_commit(&op_empty[o]);
+                    if constexpr (I8) mma_commit(&b_empty[i_op % NPF]);
                 }
             }
             // the last commit's arrival must land before the CTA can exit
             if (i_op > 0) mbar_wait_bounded(&op_empty[(i_op - 1) % NOP], ((i_op - 1) / NOP) & 1, LIMIT);
+            if (I8 && i_op > 0) mbar_wait_bounded(&b_empty[(i_op - 1) % NPF], ((i_op - 1) / NPF) & 1, LIMIT);
         }
     } else {
         // ------------------------------------------------------------ epilogue

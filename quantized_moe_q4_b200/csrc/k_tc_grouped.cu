@@ -84,18 +84,18 @@ template <int TN>
 struct TcCfg {
     static_assert(TN == 32 || TN == 64 || TN == 128, "tile widths");
     // blocks per operand stage: each stage is one hand-off between the roles,
-    // so narrower tiles (less epilogue work a block) take four blocks a stage,
-    // 128-slot tiles two (their eight accumulators would need 1024 columns)
-    static constexpr int OP_KB = (TN == 128) ? 2 : 4;
+    // so narrower tiles (less epilogue work a block) take more blocks a stage:
+    // eight for 32 slots, four for 64, two for 128 (TMEM holds 512 columns)
+    static constexpr int OP_KB = (TN == 128) ? 2 : (TN == 64) ? 4 : 8;
     // pipeline depths: input stages of weight rows (NIN), operand stages
     // (NOP), accumulator sets in TMEM (NTS), the scale ring (NSC) and the
     // activation ring (NPF: operand stages of a slot's OP_KB blocks of int8
     // codes and their binary16 scales, copied by the producer warp); the
     // narrow tiles have the shared memory to run deeper
-    static constexpr int NIN = (TN == 32) ? 4 : 2;
-    static constexpr int NOP = (TN == 32) ? 3 : 2;
-    static constexpr int NTS = (TN == 32) ? 3 : 2;
-    static constexpr int NSC = (TN == 32) ? 8 : 4;
+    static constexpr int NIN = (TN == 32) ? 3 : 2;
+    static constexpr int NOP = 2;
+    static constexpr int NTS = 2;
+    static constexpr int NSC = 4;
     static constexpr int NPF = (TN == 32) ? 6 : 4;
     static constexpr int NACC = NTS * OP_KB;              // accumulators: NTS sets of OP_KB
     // operand type: int8 (kind::i8, one K = 32 MMA a block) for 32-slot tiles,
@@ -109,11 +109,13 @@ struct TcCfg {
     // TMEM lane quarters) per CW-wide column group
     static constexpr int CW = (TN == 128) ? 64 : 32;
     static constexpr int N_EPI = 4 * (TN / CW) * 32;
-    // converters: one pair of blocks of a weight row (and of a slot) per
-    // thread, so OP_KB / 2 threads a row: 8 warps for 4-block stages, 4 for 2
-    static constexpr int N_CONV = TM * OP_KB / 2;
+    // converters: PPT pairs of blocks of a weight row (and on binary16 tiles
+    // of a slot) per thread, OP_KB / 2 / PPT threads a row: 8 warps for 8- and
+    // 4-block stages, 4 for 2
+    static constexpr int PPT = (OP_KB == 8) ? 2 : 1;
+    static constexpr int N_CONV = TM * OP_KB / 2 / PPT;
     static constexpr int W_MMA = W_CONV0 + N_CONV / 32, W_EPI0 = W_MMA + 1;
-    static constexpr int THREADS = (W_EPI0 * 32) + N_EPI;  // 10, 18 or 14 warps
+    static constexpr int THREADS = (W_EPI0 * 32) + N_EPI;  // 14, 18 or 14 warps
     static constexpr uint32_t TMEM_COLS = (NACC * TN <= 256) ? 256 : 512;   // a power of two
     // binary16 tiles convert the activations into B operand stages; int8
     // tiles read B straight from the activation ring, whose entries then hold
@@ -645,7 +647,10 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
 #pragma unroll
                                 for (int h = 0; h < 2; ++h)
                                     cp_async16(ent + op_off<1>(TN, kb, 0, n, h), src + 32 * kb + 16 * h);
-                            cp_async8(ent + C::BPF_CODES + 8 * n, ascale[q] + cb * OP_KB);
+                            if constexpr (OP_KB == 8)
+                                cp_async16(ent + C::BPF_CODES + 16 * n, ascale[q] + cb * OP_KB);
+                            else
+                                cp_async8(ent + C::BPF_CODES + 8 * n, ascale[q] + cb * OP_KB);
                         } else {
                             uint8_t* dst = bpf + (size_t)r * C::BPF_ENTRY + (size_t)n * BPF_SLOT;
 #pragma unroll
@@ -664,9 +669,11 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
         if (i_in > 0) mbar_wait_bounded(&in_full[(i_in - 1) % NIN], ((i_in - 1) / NIN) & 1, LIMIT);
     } else if (warp >= W_CONV0 && warp < W_MMA) {
         // ------------------------------------------------------------ converters
-        // thread ct converts one pair of blocks (kb0, kb0 + 1) of weight row
-        // ct mod 128 and (row < TN) of the activations of that slot, which the
-        // producer has copied into the ring
+        // thread ct converts PPT pairs of blocks (kb0 + 2 G j, kb0 + 2 G j + 1;
+        // G = N_CONV / 128 threads a row) of weight row ct mod 128 and, on
+        // binary16 tiles, (row < TN) of the activations of that slot, which
+        // the producer has copied into the ring
+        constexpr int PPT = C::PPT, G = N_CONV / TM;
         const int ct = tid - W_CONV0 * 32;
         const int row = ct % TM, kb0 = 2 * (ct / TM);
         const uint8_t* bpf = smem + C::OFF_BPF;
@@ -684,57 +691,66 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 if (!wait_phase(&op_empty[o], ((i_op / NOP) & 1) ^ 1, abort)) { ok = false; break; }
                 tc_fence_after_sync();
 
-                // weights: this thread's pair of blocks (36 bytes at a 4-byte
-                // boundary), read as 16-byte loads of the window from the
+                // weights: each of this thread's pairs of blocks (36 bytes at a
+                // 4-byte boundary), read as 16-byte loads of the window from the
                 // 16-byte boundary at or below it: rows are 144 bytes apart, so
                 // a quarter-warp's loads fall in distinct banks
-                uint32_t w[9];
-                {
-                    constexpr int NW = (4 * 3 + 2 * Q4_BYTES + 15) / 16;   // 3 loads, inside the row
-                    const int gb = (sub * OP_KB + kb0) * Q4_BYTES;
-                    const uint4* wsrc = reinterpret_cast<const uint4*>(in_w + (size_t)s * SZ_IN_W + (size_t)row * IN_ROW +
-                                                                       (gb & ~15));
-                    uint32_t win[4 * NW];
-#pragma unroll
-                    for (int i = 0; i < NW; ++i) {
-                        const uint4 v = wsrc[i];
-                        win[4 * i] = v.x; win[4 * i + 1] = v.y; win[4 * i + 2] = v.z; win[4 * i + 3] = v.w;
-                    }
-                    switch ((gb & 15) >> 2) {   // the same in every lane of the warp
-                        case 0: take_words<0>(w, win); break;
-                        case 1: take_words<1>(w, win); break;
-                        case 2: take_words<2>(w, win); break;
-                        default: take_words<3>(w, win); break;
-                    }
-                }
                 uint8_t* oa = op_a + (size_t)o * SZ_OP_A;
-                float dws[2];
-                {
+                float dws[2 * PPT];
+#pragma unroll
+                for (int j = 0; j < PPT; ++j) {
+                    const int kp = kb0 + 2 * G * j;               // first block of the pair
+                    uint32_t w[9];
+                    {
+                        constexpr int NW = (4 * 3 + 2 * Q4_BYTES + 15) / 16;   // 3 loads, inside the row
+                        const int gb = (sub * OP_KB + kp) * Q4_BYTES;
+                        const uint4* wsrc = reinterpret_cast<const uint4*>(in_w + (size_t)s * SZ_IN_W +
+                                                                           (size_t)row * IN_ROW + (gb & ~15));
+                        uint32_t win[4 * NW];
+#pragma unroll
+                        for (int i = 0; i < NW; ++i) {
+                            const uint4 v = wsrc[i];
+                            win[4 * i] = v.x; win[4 * i + 1] = v.y; win[4 * i + 2] = v.z; win[4 * i + 3] = v.w;
+                        }
+                        switch ((gb & 15) >> 2) {   // the same in every lane of the warp
+                            case 0: take_words<0>(w, win); break;
+                            case 1: take_words<1>(w, win); break;
+                            case 2: take_words<2>(w, win); break;
+                            default: take_words<3>(w, win); break;
+                        }
+                    }
                     // the pair's first block starts at its byte 0 (scale, then
                     // 16 nibble bytes), the second at byte 18
                     uint32_t qs[4];
-                    dws[0] = half_bits_to_float(w[0] & 0xffffu);
+                    dws[2 * j] = half_bits_to_float(w[0] & 0xffffu);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) qs[i] = __funnelshift_r(w[i], w[i + 1], 16);
-                    store_weights<I8>(oa, kb0, row, qs);
-                    dws[1] = half_bits_to_float(w[4] >> 16);
+                    store_weights<I8>(oa, kp, row, qs);
+                    dws[2 * j + 1] = half_bits_to_float(w[4] >> 16);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) qs[i] = w[5 + i];
-                    store_weights<I8>(oa, kb0 + 1, row, qs);
+                    store_weights<I8>(oa, kp + 1, row, qs);
                 }
                 // activations.  binary16 tiles: slot `row`'s codes from the ring
                 // into the B operand (zeros past the tile's slots).  int8 tiles:
                 // the MMA reads the codes in the ring; the first converter warp
                 // takes the scales of slot `lane` (all OP_KB blocks)
-                uint32_t dab = 0, dab2 = 0;
+                uint32_t dab = 0;
+                uint32_t dsl[OP_KB / 2];                          // int8: the slot's OP_KB scales
+#pragma unroll
+                for (int i = 0; i < OP_KB / 2; ++i) dsl[i] = 0;
                 if constexpr (I8) {
                     if (ct < 32) {
                         if (!wait_phase(&b_full[i_op % NPF], (i_op / NPF) & 1, abort)) { ok = false; break; }
                         if (valid) {
-                            const uint2 v = *reinterpret_cast<const uint2*>(bpf + (size_t)(i_op % NPF) * C::BPF_ENTRY +
-                                                                            C::BPF_CODES + 8 * lane);
-                            dab = v.x;
-                            dab2 = v.y;
+                            const uint8_t* sp = bpf + (size_t)(i_op % NPF) * C::BPF_ENTRY + C::BPF_CODES + 2 * OP_KB * lane;
+                            if constexpr (OP_KB == 8) {
+                                const uint4 v = *reinterpret_cast<const uint4*>(sp);
+                                dsl[0] = v.x; dsl[1] = v.y; dsl[2] = v.z; dsl[3] = v.w;
+                            } else {
+                                const uint2 v = *reinterpret_cast<const uint2*>(sp);
+                                dsl[0] = v.x; dsl[1] = v.y;
+                            }
                         }
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&b_empty[i_op % NPF]);   // with the MMAs' commit: entry free
@@ -764,16 +780,20 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 const int sc = i_op % NSC;
                 if (!wait_phase(&sc_empty[sc], ((i_op / NSC) & 1) ^ 1, abort)) { ok = false; break; }
 #pragma unroll
-                for (int i = 0; i < 2; ++i) dw_ring[(sc * OP_KB + kb0 + i) * TM + row] = dws[i];
-                if constexpr (I8) {
-                    static_assert(!I8 || OP_KB == 4, "int8 tiles: 4-block stages");
-                    if (ct < 32) {
-                        const uint32_t d4[4] = {dab & 0xffffu, dab >> 16, dab2 & 0xffffu, dab2 >> 16};
+                for (int j = 0; j < PPT; ++j)
 #pragma unroll
-                        for (int kb = 0; kb < 4; ++kb)
-                            da_ring[(sc * OP_KB + kb) * TN + lane] = valid ? half_bits_to_float(d4[kb]) : 0.0f;
+                    for (int i = 0; i < 2; ++i) dw_ring[(sc * OP_KB + kb0 + 2 * G * j + i) * TM + row] = dws[2 * j + i];
+                if constexpr (I8) {
+                    static_assert(!I8 || OP_KB == 4 || OP_KB == 8, "int8 tiles: 4- or 8-block stages");
+                    if (ct < 32) {
+#pragma unroll
+                        for (int kb = 0; kb < OP_KB; ++kb)
+                            da_ring[(sc * OP_KB + kb) * TN + lane] =
+                                valid ? half_bits_to_float((kb & 1) ? (dsl[kb >> 1] >> 16) : (dsl[kb >> 1] & 0xffffu))
+                                      : 0.0f;
                     }
                 } else {
+                    static_assert(I8 || PPT == 1, "binary16 tiles: a pair a thread");
 #pragma unroll
                     for (int i = 0; i < 2; ++i)
                         if (row < TN)
@@ -1119,11 +1139,12 @@ static cudaError_t launch_tc(const LayerView& L, int64_t T, const Workspace& ws,
 int tc_tile_tokens(const LayerView& L, int64_t T, int force) {
     if (force == 32 || force == 64 || force == 128) return force;
     // routed slots per expert on average, against the measured crossovers of
-    // the three widths (one 2048/512 layer, 128 experts top-8): 32 slots up to
-    // 27 per expert (T <= 384), 64 from 28 (T = 512; a 947-token prompt's 59),
+    // the three widths (one 2048/512 layer, 128 experts top-8): 32 slots still
+    // lead at 32 per expert (T = 512: 351 against 372 us) and 64 at 59 (a
+    // 947-token prompt: 0.475 against 0.521 ms), so 64 from 44, between them;
     // 128 from 96 (a 16384-token batch's 1024)
     const int64_t per_expert = T * L.k / L.E;
-    return per_expert >= 96 ? 128 : per_expert >= 28 ? 64 : 32;
+    return per_expert >= 96 ? 128 : per_expert >= 44 ? 64 : 32;
 }
 
 cudaError_t launch_gateup_tc(const LayerView& L, int64_t T, const Workspace& ws, float* h_dbg, const DeviceInfo& dev,

@@ -27,7 +27,7 @@
 // or 128, chosen per call from the routed slots per expert (tc_tile_tokens):
 // a weight block converted once serves TN slots.
 //
-// Warp roles (14 warps for TN = 32, 18 for 64, 14 for 128):
+// Warp roles (18 warps for TN = 32 and 64, 14 for 128):
 //   0      producer: 2D tensor copies (TMA) of the packed weight rows (a box
 //          of 64 or 128 rows x 144 B = 8 blocks), two input stages in flight,
 //          and the activation ring's cp.async copies;
@@ -43,16 +43,17 @@
 //   then   the MMA issuer (one thread): one (int8) or two (binary16) MMAs per
 //          block, A and B from shared memory; one wait and one commit per
 //          operand stage, for its set of accumulators;
-//   last   epilogue: 4 TMEM lane quarters x TN / CW column groups (CW = 32,
-//          or 64 for TN = 128); per operand stage one wait, TMEM loads of 16
-//          columns software-pipelined against the rescale-accumulate, the
-//          accumulator pair released as soon as its last chunk is in
-//          registers; after the last block of a tile gate/up -> SwiGLU +
-//          Q8_0 requantisation, down -> y += w_slot * o with vector
-//          reductions (red.v4.f32) of 4 consecutive rows of H of one token.
+//   last   epilogue: 4 TMEM lane quarters x TN / CW column groups (CW = 16,
+//          32 or 64 for TN = 32, 64, 128); per operand stage one wait, TMEM
+//          loads of 16 columns software-pipelined against the
+//          rescale-accumulate, the accumulator set released as soon as its
+//          last chunk is in registers; after the last block of a tile
+//          gate/up -> SwiGLU + Q8_0 requantisation, down -> y += w_slot * o
+//          with vector reductions (red.v4.f32) of 4 consecutive rows of H of
+//          one token.
 // TMEM: two sets of OP_KB accumulators of TN columns, handed between the MMA
-// issuer and the epilogue a set (one operand stage) at a time; full/empty mbarriers between
-// every pair of roles; every wait bounded, and one that runs out makes every
+// issuer and the epilogue a set (one operand stage) at a time; full/empty
+// mbarriers between every pair of roles; every wait bounded, and one that runs out makes every
 // role leave its loop and records STATUS_SPIN_TIMEOUT.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -106,8 +107,9 @@ struct TcCfg {
     // a ring entry: OP_KB x 32 codes, OP_KB binary16 scales, padded to 16 bytes
     static constexpr size_t BPF_SLOT = ((size_t)OP_KB * (QK + 2) + 15) & ~size_t(15);
     // epilogue: a thread owns one accumulator row x CW columns; 4 warps (the
-    // TMEM lane quarters) per CW-wide column group
-    static constexpr int CW = (TN == 128) ? 64 : 32;
+    // TMEM lane quarters) per CW-wide column group: 8 warps at every width
+    // (16 on 64-slot tiles or on 128-slot ones measured slower)
+    static constexpr int CW = (TN == 128) ? 64 : (TN == 64) ? 32 : 16;
     static constexpr int N_EPI = 4 * (TN / CW) * 32;
     // converters: PPT pairs of blocks of a weight row (and on binary16 tiles
     // of a slot) per thread, OP_KB / 2 / PPT threads a row: 8 warps for 8- and
@@ -115,7 +117,7 @@ struct TcCfg {
     static constexpr int PPT = (OP_KB == 8) ? 2 : 1;
     static constexpr int N_CONV = TM * OP_KB / 2 / PPT;
     static constexpr int W_MMA = W_CONV0 + N_CONV / 32, W_EPI0 = W_MMA + 1;
-    static constexpr int THREADS = (W_EPI0 * 32) + N_EPI;  // 14, 18 or 14 warps
+    static constexpr int THREADS = (W_EPI0 * 32) + N_EPI;  // 18, 18 or 14 warps
     static constexpr uint32_t TMEM_COLS = (NACC * TN <= 256) ? 256 : 512;   // a power of two
     // binary16 tiles convert the activations into B operand stages; int8
     // tiles read B straight from the activation ring, whose entries then hold

@@ -568,7 +568,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
             mbar_init(&b_full[i], 32);              // the producer's 32 lanes, after their copies land
             // binary16: the converter warps, after reading the entry; int8:
             // the MMAs' commit and the converter warp that takes the scales
-            mbar_init(&b_empty[i], I8 ? 2 : N_CONV / 32);
+            mbar_init(&b_empty[i], I8 ? 1 + TN / 32 : N_CONV / 32);
         }
         mbar_init(&epi_bar, N_EPI / 32);
         mbar_fence_init();
@@ -735,17 +735,17 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 }
                 // activations.  binary16 tiles: slot `row`'s codes from the ring
                 // into the B operand (zeros past the tile's slots).  int8 tiles:
-                // the MMA reads the codes in the ring; the first converter warp
-                // takes the scales of slot `lane` (all OP_KB blocks)
+                // the MMA reads the codes in the ring; the first TN / 32
+                // converter warps take the scales of slot ct (all OP_KB blocks)
                 uint32_t dab = 0;
                 uint32_t dsl[OP_KB / 2];                          // int8: the slot's OP_KB scales
 #pragma unroll
                 for (int i = 0; i < OP_KB / 2; ++i) dsl[i] = 0;
                 if constexpr (I8) {
-                    if (ct < 32) {
+                    if (ct < TN) {   // slot ct: warp-uniform
                         if (!wait_phase(&b_full[i_op % NPF], (i_op / NPF) & 1, abort)) { ok = false; break; }
                         if (valid) {
-                            const uint8_t* sp = bpf + (size_t)(i_op % NPF) * C::BPF_ENTRY + C::BPF_CODES + 2 * OP_KB * lane;
+                            const uint8_t* sp = bpf + (size_t)(i_op % NPF) * C::BPF_ENTRY + C::BPF_CODES + 2 * OP_KB * ct;
                             if constexpr (OP_KB == 8) {
                                 const uint4 v = *reinterpret_cast<const uint4*>(sp);
                                 dsl[0] = v.x; dsl[1] = v.y; dsl[2] = v.z; dsl[3] = v.w;
@@ -787,10 +787,10 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     for (int i = 0; i < 2; ++i) dw_ring[(sc * OP_KB + kb0 + 2 * G * j + i) * TM + row] = dws[2 * j + i];
                 if constexpr (I8) {
                     static_assert(!I8 || OP_KB == 4 || OP_KB == 8, "int8 tiles: 4- or 8-block stages");
-                    if (ct < 32) {
+                    if (ct < TN) {
 #pragma unroll
                         for (int kb = 0; kb < OP_KB; ++kb)
-                            da_ring[(sc * OP_KB + kb) * TN + lane] =
+                            da_ring[(sc * OP_KB + kb) * TN + ct] =
                                 valid ? half_bits_to_float((kb & 1) ? (dsl[kb >> 1] >> 16) : (dsl[kb >> 1] & 0xffffu))
                                       : 0.0f;
                     }

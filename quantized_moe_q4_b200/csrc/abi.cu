@@ -4,6 +4,8 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
+#include <utility>
 
 #include "moe_q4.h"
 #include "common.cuh"
@@ -260,7 +262,7 @@ static int forward_impl(const moe_q4_layer* Lp, const float* x, int64_t T, float
     if ((path == MOE_Q4_PATH_AUTO || path == MOE_Q4_PATH_DECODE) && decode_eligible(L, T, dev))
         return cuda_rc(launch_decode(L, x, y, w, dbg ? dbg->h_out : nullptr, dev, ev0, ev1,
                                      dbg && dbg->force_spin_timeout, clear_status,
-                                     dbg ? dbg->decode_kernel_ns : nullptr, nullptr, nullptr, s));
+                                     dbg ? dbg->decode_kernel_ns : nullptr, nullptr, nullptr, false, s));
 
     // grouped paths: tensor cores once experts see tens of tokens, else dp4a
     const bool tc = (path == MOE_Q4_PATH_TENSOR_CORE) || (path == MOE_Q4_PATH_TENSOR_CORE_N32) ||
@@ -384,6 +386,37 @@ int moe_q4_ffn_forward_debug(const moe_q4_layer* L, const float* x, int64_t T, f
     return forward_impl(L, x, T, y, workspace, ws_bytes, dbg, reinterpret_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+// The one-token host path's copy-in kernel may read x_host before the work
+// ahead of it on the stream has finished (see decode_copy_in_kernel).  The
+// only such work that can still be writing host memory is the previous
+// call's copy-out kernel on the same stream (it lets the next kernel launch
+// early); every other predecessor completes before the launch.  So x_host is
+// read early unless it overlaps that call's y_host, tracked per stream here.
+namespace {
+std::mutex g_host_y_mu;
+std::unordered_map<cudaStream_t, std::pair<uintptr_t, uintptr_t>> g_host_y;   // [begin, end)
+}  // namespace
+
+static bool x_host_read_early(cudaStream_t s, const float* x_host, const float* y_host, size_t bytes) {
+    const uintptr_t xb = reinterpret_cast<uintptr_t>(x_host), yb = reinterpret_cast<uintptr_t>(y_host);
+    std::lock_guard<std::mutex> lk(g_host_y_mu);
+    auto it = g_host_y.find(s);
+    const bool early = it == g_host_y.end() || xb + bytes <= it->second.first || it->second.second <= xb;
+    g_host_y[s] = {yb, yb + bytes};
+    return early;
+}
+
+// Any other kind of call on the stream ends with a copy or kernel that does
+// not release the next launch early.
+static void forget_host_y(cudaStream_t s) {
+    std::lock_guard<std::mutex> lk(g_host_y_mu);
+    g_host_y.erase(s);
+}
+
+extern "C" {
+
 size_t moe_q4_ffn_host_workspace_bytes(const moe_q4_layer* L, int64_t T_max) {
     const size_t base = moe_q4_ffn_workspace_bytes(L, T_max);
     if (!base) return 0;
@@ -418,9 +451,11 @@ int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t 
     if (T == 1 && decode_eligible(Lv, T, dev) && aligned(x_host, 16) && aligned(y_host, 16) && pinned_host(x_host) &&
         pinned_host(y_host)) {
         const Workspace w = carve(workspace, off);
+        const bool early = x_host_read_early(s, x_host, y_host, bytes);
         return cuda_rc(launch_decode(Lv, x_dev, y_dev, w, nullptr, dev, nullptr, nullptr, false, true, nullptr,
-                                     x_host, y_host, s));
+                                     x_host, y_host, early, s));
     }
+    forget_host_y(s);
     MOE_TRY(cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s));
     rc = forward_impl(L, x_dev, T, y_dev, workspace, off[WS_TOTAL], nullptr, s);
     if (rc) return rc;

@@ -600,12 +600,31 @@ __global__ void __launch_bounds__(FFN_THREADS, 1) decode_ffn_kernel(DecodeParams
 // copy node in it (one CTA reads x over the bus once; the router's CTAs then
 // read the device copy).
 // ---------------------------------------------------------------------------
+constexpr int COPY_IN_VEC = 4;   // float4 loads a thread: H <= 4 * 4 * 256
+
+// EARLY: x_host is read into registers before the dependency wait, so the
+// bus round trip overlaps the previous call's tail; only the store into the
+// device copy (which the previous call's kernels may still read) waits.  The
+// host side uses it unless x_host overlaps the previous call's y_host on the
+// same stream (whose copy-out may still be writing it).
+template <bool EARLY>
 __global__ void __launch_bounds__(256) decode_copy_in_kernel(const float* __restrict__ x_host, float* __restrict__ x,
                                                              int H) {
     pdl_launch_dependents();
-    pdl_wait();  // the previous call's kernels no longer read x
-    for (int i = threadIdx.x; i < H / 4; i += blockDim.x)
-        reinterpret_cast<float4*>(x)[i] = reinterpret_cast<const float4*>(x_host)[i];
+    const float4* src = reinterpret_cast<const float4*>(x_host);
+    float4 v[COPY_IN_VEC];
+    if (!EARLY) pdl_wait();  // the previous call's kernels no longer read x, nor write x_host
+#pragma unroll
+    for (int j = 0; j < COPY_IN_VEC; ++j) {
+        const int i = threadIdx.x + 256 * j;
+        if (i < H / 4) v[j] = src[i];
+    }
+    if (EARLY) pdl_wait();  // the previous call's kernels no longer read x
+#pragma unroll
+    for (int j = 0; j < COPY_IN_VEC; ++j) {
+        const int i = threadIdx.x + 256 * j;
+        if (i < H / 4) reinterpret_cast<float4*>(x)[i] = v[j];
+    }
 }
 
 __global__ void __launch_bounds__(256) decode_copy_out_kernel(const float* __restrict__ y, float* __restrict__ y_host,
@@ -669,7 +688,7 @@ bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev) {
 cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Workspace& ws, float* h_dbg,
                           const DeviceInfo& dev, cudaEvent_t ev_start, cudaEvent_t ev_stop, bool force_timeout,
                           bool clear_status, unsigned long long* kernel_ns, const float* x_host, float* y_host,
-                          cudaStream_t s) {
+                          bool x_host_early, cudaStream_t s) {
     DecodeParams p;
     p.H = L.H; p.F = L.F; p.E = L.E; p.k = L.k; p.S = L.S;
     p.nbF = L.F / QK;
@@ -701,11 +720,13 @@ cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Wo
     cfg.stream = s;
     cfg.attrs = attrs;
     if (x_host) {
+        if (L.H / 4 > 256 * COPY_IN_VEC) return cudaErrorInvalidValue;
         cfg.gridDim = dim3(1);
         cfg.blockDim = dim3(256);
         cfg.dynamicSmemBytes = 0;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, decode_copy_in_kernel, x_host, const_cast<float*>(x), L.H);
+        e = x_host_early ? cudaLaunchKernelEx(&cfg, decode_copy_in_kernel<true>, x_host, const_cast<float*>(x), L.H)
+                         : cudaLaunchKernelEx(&cfg, decode_copy_in_kernel<false>, x_host, const_cast<float*>(x), L.H);
         if (e != cudaSuccess) return e;
     }
     cfg.gridDim = dim3((unsigned)L.E);

@@ -101,7 +101,7 @@ bool decode_eligible(const LayerView& L, int64_t T, const DeviceInfo& dev);
 cudaError_t launch_decode(const LayerView& L, const float* x, float* y, const Workspace& ws, float* h_dbg,
                           const DeviceInfo& dev, cudaEvent_t ev_start, cudaEvent_t ev_stop, bool force_timeout,
                           bool clear_status, unsigned long long* kernel_ns, const float* x_host, float* y_host,
-                          cudaStream_t s);
+                          bool x_host_early, cudaStream_t s);
 
 cudaError_t launch_block_dots(const uint8_t* w, const int8_t* qa, int64_t n, int32_t* out,
                               cudaStream_t s);

@@ -369,6 +369,32 @@ def test_forward_host_single_token(pinned):
         assert ok, worst
 
 
+def test_forward_host_back_to_back():
+    """One-token host calls enqueued with no synchronisation between them: a
+    call whose x is the previous call's y (the entry must not read it before
+    that y has landed), then calls on distinct buffers (x read early, while
+    the previous call finishes).  Each output must be the device forward of
+    the input it was given; outputs start as NaN so a stale read shows."""
+    x, lw = workload("decode_t1", T=1000)
+    L = m.Layer.from_host(lw)
+    ws = m.alloc_workspace(m.moe_q4_ffn_host_workspace_bytes(L, 1))
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).pin_memory()
+    nan = lambda: torch.full((1, lw.hidden), float("nan")).pin_memory()
+    x0, x1, x2 = pin(x[0:1]), pin(x[1:2]), pin(x[2:3])
+    ya, yb, yc, yd, ye = nan(), nan(), nan(), nan(), nan()
+    m.moe_q4_ffn_forward_host(L, x0, ya, ws)
+    m.moe_q4_ffn_forward_host(L, ya, yb, ws)        # x = the previous call's y
+    m.moe_q4_ffn_forward_host(L, x1, yc, ws)        # distinct buffers from here on
+    m.moe_q4_ffn_forward_host(L, x2, yd, ws)
+    m.moe_q4_ffn_forward_host(L, yd, ye, ws)        # aliasing again
+    torch.cuda.synchronize()
+    for xin, yout in ((x0, ya), (ya, yb), (x1, yc), (x2, yd), (yd, ye)):
+        assert np.all(np.isfinite(yout.numpy()))
+        y_dev = m.moe_q4_ffn_forward(L, xin.cuda()).cpu().numpy()
+        ok, worst = rule13(yout.numpy(), y_dev, ORDER_REL)
+        assert ok, worst
+
+
 def test_decode_kernel_timer():
     """The fused T = 1 path's device timer: one count per call, the span from
     the dependency wait no longer than the span from the kernel's start, both

@@ -17,44 +17,48 @@
 // the fp32 accumulator).  The epilogue then accumulates acc += I_b * (dW * dA)
 // in fp32 registers (packed f32x2 FMUL + FFMA, plus one packed FADD taking
 // the bias off for int8; the product of two binary16 scales is exact in
-// binary32).  int8 operands halve the converters' shared-memory traffic (the
-// activation codes go in as they are) but cost the epilogue the FADD and the
-// TMEM reset: they win on 32-slot tiles, where the converters bound the
-// kernel, and lose on 64- and 128-slot tiles, where the epilogue does.
+// binary32).  int8 operands spare the converters the activations altogether
+// (the MMA reads the codes where the producer copied them) and halve the
+// weight bytes, but cost the epilogue the FADD and the TMEM reset: they win
+// on 32-slot tiles, which also take 8 blocks per operand stage, and lose on
+// 64- and 128-slot tiles, whose epilogues have more columns per block.
 //
 // Tile: 128 weight rows (gate/up: 64 gate rows + the same 64 up rows; down:
 // 128 rows of H) x TN slots of one expert (MMA M = 128, N = TN), TN = 32, 64
 // or 128, chosen per call from the routed slots per expert (tc_tile_tokens):
 // a weight block converted once serves TN slots.
 //
-// Warp roles (18 warps for TN = 32 and 64, 14 for 128):
+// Warp roles (18 warps for TN = 32 and 64, 14 for 128); the pipeline depths
+// and stage sizes per width are in TcCfg:
 //   0      producer: 2D tensor copies (TMA) of the packed weight rows (a box
-//          of 64 or 128 rows x 144 B = 8 blocks), two input stages in flight,
-//          and the activation ring's cp.async copies;
-//   1..    converters (8 warps for 4-block operand stages, 4 for 2), a pair
-//          of blocks of a weight row and of a slot each: nibbles -> nib - 8
+//          of 64 or 128 rows x 144 B = 8 blocks), and the activation ring's
+//          cp.async copies (a slot's codes and scales per operand stage),
+//          issued as far ahead as the ring allows;
+//   1..    converters (8 warps, 4 for TN = 128): a pair of blocks of a weight
+//          row per thread (two pairs on 32-slot tiles): nibbles -> nib - 8
 //          (int8 or binary16) for the A operand, read as 16-byte loads of the
-//          window around the pair; the slot's int8 activations and block
-//          scales come through a 4-entry ring of cp.async copies the producer
-//          issues three operand stages ahead, then go into the B operand (as
-//          they are, or as binary16); both in the K-major shared-memory layout
-//          (8-row x 16-byte core matrices); two operand stages; block scales
-//          into a ring read by the epilogue;
+//          window around the pair.  binary16 tiles: the threads of rows < TN
+//          also turn the same pair of that slot's codes from the ring into
+//          binary16 for the B operand.  int8 tiles: the MMA reads B in the
+//          ring, and the first TN / 32 warps take the slots' scales.  Operands
+//          are K-major (8-row x 16-byte core matrices); block scales go into a
+//          ring read by the epilogue;
 //   then   the MMA issuer (one thread): one (int8) or two (binary16) MMAs per
 //          block, A and B from shared memory; one wait and one commit per
 //          operand stage, for its set of accumulators;
-//   last   epilogue: 4 TMEM lane quarters x TN / CW column groups (CW = 16,
-//          32 or 64 for TN = 32, 64, 128); per operand stage one wait, TMEM
-//          loads of 16 columns software-pipelined against the
+//   last   epilogue (8 warps): 4 TMEM lane quarters x TN / CW column groups
+//          (CW = 16, 32 or 64 for TN = 32, 64, 128); per operand stage one
+//          wait, TMEM loads of 16 columns software-pipelined against the
 //          rescale-accumulate, the accumulator set released as soon as its
 //          last chunk is in registers; after the last block of a tile
 //          gate/up -> SwiGLU + Q8_0 requantisation, down -> y += w_slot * o
 //          with vector reductions (red.v4.f32) of 4 consecutive rows of H of
 //          one token.
-// TMEM: two sets of OP_KB accumulators of TN columns, handed between the MMA
-// issuer and the epilogue a set (one operand stage) at a time; full/empty
-// mbarriers between every pair of roles; every wait bounded, and one that runs out makes every
-// role leave its loop and records STATUS_SPIN_TIMEOUT.
+// TMEM: two sets of OP_KB accumulators of TN columns (all 512 columns),
+// handed between the MMA issuer and the epilogue a set (one operand stage) at
+// a time; full/empty mbarriers between every pair of roles; every wait
+// bounded, and one that runs out makes every role leave its loop and records
+// STATUS_SPIN_TIMEOUT.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

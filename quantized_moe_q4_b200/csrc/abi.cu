@@ -15,7 +15,7 @@ namespace moeq4 {
 
 static constexpr int64_t T_LIMIT = int64_t(1) << 24;
 // Token count from which the automatic choice uses the tensor-core kernels.
-static constexpr int64_t TC_MIN_TOKENS = 64;   // measured crossover of the dp4a and tensor-core paths
+static constexpr int64_t TC_MIN_TOKENS = 48;   // measured crossover of the dp4a and tensor-core paths
 static constexpr int MAX_DEVICES = 64;
 
 struct DeviceState {

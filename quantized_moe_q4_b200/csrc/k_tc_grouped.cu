@@ -764,7 +764,20 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                 } else {
                     uint8_t* ob = op_b + (size_t)o * C::SZ_OP_B;
                     if (!wait_phase(&b_full[i_op % NPF], (i_op / NPF) & 1, abort)) { ok = false; break; }
-                    if (row < TN) {
+                    if constexpr (TN * 2 == TM) {
+                        // 64-slot tiles: one block of one slot per thread (slot
+                        // row mod 64, block kb0 + row / 64), so every converter
+                        // thread carries the same share of the activations
+                        const int sl = row % TN, kb = kb0 + row / TN;
+                        const uint8_t* src = bpf + (size_t)(i_op % NPF) * C::BPF_ENTRY + (size_t)sl * BPF_SLOT;
+                        const bool v = sl < T.nslots;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            store_act16<I8>(ob, TN, kb, h, sl,
+                                            v ? *reinterpret_cast<const uint4*>(src + 16 * (2 * kb + h))
+                                              : make_uint4(0, 0, 0, 0));
+                        if (v) dab = *reinterpret_cast<const uint16_t*>(src + OP_KB * QK + 2 * kb);
+                    } else if (row < TN) {
                         const uint8_t* src = bpf + (size_t)(i_op % NPF) * C::BPF_ENTRY + (size_t)row * BPF_SLOT;
 #pragma unroll
                         for (int kb = kb0; kb < kb0 + 2; ++kb)
@@ -800,11 +813,16 @@ __global__ void __launch_bounds__(TcCfg<TN>::THREADS, 1)
                     }
                 } else {
                     static_assert(I8 || PPT == 1, "binary16 tiles: a pair a thread");
+                    if constexpr (TN * 2 == TM) {
+                        const int sl = row % TN, kb = kb0 + row / TN;
+                        da_ring[(sc * OP_KB + kb) * TN + sl] = sl < T.nslots ? half_bits_to_float(dab) : 0.0f;
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < 2; ++i)
-                        if (row < TN)
-                            da_ring[(sc * OP_KB + kb0 + i) * TN + row] =
-                                valid ? half_bits_to_float(i ? (dab >> 16) : dab) : 0.0f;
+                        for (int i = 0; i < 2; ++i)
+                            if (row < TN)
+                                da_ring[(sc * OP_KB + kb0 + i) * TN + row] =
+                                    valid ? half_bits_to_float(i ? (dab >> 16) : dab) : 0.0f;
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sc_full[sc]);

@@ -37,9 +37,10 @@
 //   1..    converters (8 warps, 4 for TN = 128): a pair of blocks of a weight
 //          row per thread (two pairs on 32-slot tiles): nibbles -> nib - 8
 //          (int8 or binary16) for the A operand, read as 16-byte loads of the
-//          window around the pair.  binary16 tiles: the threads of rows < TN
-//          also turn the same pair of that slot's codes from the ring into
-//          binary16 for the B operand.  int8 tiles: the MMA reads B in the
+//          window around the pair.  binary16 tiles: the threads also turn
+//          slots' codes from the ring into binary16 for the B operand (128
+//          slots: the pair of slot `row`; 64 slots: one block each, so every
+//          thread has the same share).  int8 tiles: the MMA reads B in the
 //          ring, and the first TN / 32 warps take the slots' scales.  Operands
 //          are K-major (8-row x 16-byte core matrices); block scales go into a
 //          ring read by the epilogue;

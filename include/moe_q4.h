@@ -134,7 +134,12 @@ size_t moe_q4_ffn_host_workspace_bytes(const moe_q4_layer* L, int64_t T_max);
  * synchronises the stream.  For one token with both x and y page-locked (and
  * 16-byte aligned) the copies are made by kernels of the decode chain (a
  * first one reads x, a last one writes y over the bus), with no copy node
- * between the kernels. */
+ * between the kernels.  That first kernel is a programmatic dependent launch
+ * and reads x before its dependency wait: x may be read as soon as the kernel
+ * enqueued just before the call lets its dependents launch.  A kernel of the
+ * caller's that writes x must therefore not release its dependents early
+ * (the default).  The previous one-token host call's y on the same stream is
+ * tracked by the library: when x overlaps it, x is read after the wait. */
 int moe_q4_ffn_forward_host(const moe_q4_layer* L, const float* x_host, int64_t T, float* y_host,
                             void* workspace, size_t ws_bytes, moe_q4_stream_t stream);
 

@@ -388,12 +388,14 @@ int moe_q4_ffn_forward_debug(const moe_q4_layer* L, const float* x, int64_t T, f
 
 }  // extern "C"
 
-// The one-token host path's copy-in kernel may read x_host before the work
-// ahead of it on the stream has finished (see decode_copy_in_kernel).  The
-// only such work that can still be writing host memory is the previous
-// call's copy-out kernel on the same stream (it lets the next kernel launch
-// early); every other predecessor completes before the launch.  So x_host is
-// read early unless it overlaps that call's y_host, tracked per stream here.
+// The one-token host path's copy-in kernel may read x_host before the kernel
+// ahead of it on the stream has finished (see decode_copy_in_kernel), if that
+// kernel lets its dependents launch early.  Of this library's kernels, the
+// one that can then still be writing host memory is the previous call's
+// copy-out kernel on the same stream; a caller's kernel that writes x_host
+// must not release its dependents early (include/moe_q4.h).  So x_host is
+// read early unless it overlaps the previous host call's y_host, tracked per
+// stream here.
 namespace {
 std::mutex g_host_y_mu;
 std::unordered_map<cudaStream_t, std::pair<uintptr_t, uintptr_t>> g_host_y;   // [begin, end)
